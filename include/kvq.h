@@ -1,0 +1,256 @@
+/*
+ * kvq.h — C ABI of the 2-bit mixed-precision KV cache with fused decode attention.
+ *
+ * What the library computes
+ * -------------------------
+ * Keys are quantized asymmetrically (min/max, scale + zero point) per channel over
+ * groups of consecutive tokens; values are quantized per token over the head
+ * dimension.  This split of quantization axes is the KIVI scheme (aibr.jp article on
+ * "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache", section 3 "core
+ * technical elements": Keys per channel, Values per token, asymmetric quantization,
+ * a full-precision residual of recent tokens, and streaming append into the
+ * quantized cache).  On top of it sits Kitty's Dynamic Channel-wise Precision Boost
+ * (fugumt.com summary of "Kitty: Accurate and Efficient 2-bit KV Cache Quantization
+ * with Dynamic Channel-wise Precision Boost", Abstract; and the notes.yuuk.io wiki
+ * page "KVキャッシュ量子化", open questions): the Key channels are ranked by magnitude,
+ * a small fraction of them is kept at 4 bits, and every mixed-precision Key page is
+ * stored as two uniform 2-bit tensors so that dequantization stays uniform and the
+ * page stays coalesced.  Decode attention reads the packed pages directly and
+ * dequantizes inside the attention kernel (MiniKV summary on f-binder, section
+ * "proposed method": 2-bit KV expanded inside the fused attention matmul).
+ *
+ * Where the pages leave a step open the library takes one fixed reading; every
+ * such reading is listed in this header next to the call it affects.
+ *
+ * Quantizer (shared by keys, boosted keys and values)
+ * ---------------------------------------------------
+ * For a group x[0..n) of dtype values and a bit width b:
+ *   mn = min x, mx = max x                         (exact; compared after widening to fp32)
+ *   s32 = fp32(mx - mn) / (2^b - 1)                (fp32, round-to-nearest-even divide)
+ *   scale = s32 rounded toward +infinity to dtype   (so scale*(2^b-1) >= mx-mn)
+ *   zero  = mn                                      (stored in dtype, exact)
+ *   code  = clamp(rint(fp32(x - zero) / fp32(scale)), 0, 2^b-1)
+ *           (fp32 subtract, fp32 divide, rint = round half to even); code = 0 if scale == 0
+ *   dequantized value = code * scale + zero
+ * Inputs are assumed finite.
+ *
+ * Boost-channel selection (per physical page and KV head)
+ *   score_c = max over the page's tokens of |K[t][c]|; the num_boost channels with the
+ *   largest score are boosted, ties going to the lower channel index; the indices are
+ *   stored in ascending order.
+ *
+ * Keys (per channel c, per group g of key_group consecutive tokens of the page)
+ *   normal channel : 2-bit code -> plane A; plane-A scale = scale, plane-A zero = mn.
+ *   boosted channel: 4-bit code4 with scale s4 and zero mn; hi = code4 >> 2 -> plane A,
+ *                    lo = code4 & 3 -> plane B row j (j = rank of c in boost_idx);
+ *                    plane-A scale = 4*s4 (exact), plane-A zero = mn; plane-B scale = s4,
+ *                    plane-B zero = 0.  Hence K^ = hi*(4*s4) + mn + lo*s4 = code4*s4 + mn.
+ * Values (per token t): 2-bit code over the head_dim channels of that token.
+ *
+ * Page record (one per physical page and KV head), P = page_tokens, D = head_dim,
+ * k = num_boost, G = key_group, S = dtype (2 bytes).  Sections follow one another
+ * without gaps, in this order:
+ *   k_codes   uint32 [P][D/16]   plane A, token-major; word (t, w) = channels 16w..16w+15 of token t
+ *   kb_codes  uint32 [P][k/16]   plane B, token-major; word (t, w) = boosted rows 16w..16w+15
+ *   v_codes   uint32 [D][P/16]   values, channel-major; word (c, w) = tokens 16w..16w+15 of channel c
+ *   k_scale   S [P/G][D]         plane-A scale per (group, channel)
+ *   k_zero    S [P/G][D]         plane-A zero  per (group, channel)
+ *   kb_scale  S [P/G][k]         plane-B scale per (group, boosted row)
+ *   v_scale   S [P]              value scale per token
+ *   v_zero    S [P]              value zero  per token
+ *   boost_idx uint8 [k]          boosted channels, ascending
+ * The record stride (kvq_page_bytes) rounds the payload up to a multiple of 128 bytes;
+ * the padding bytes are never read.
+ * Inside a 32-bit code word the 16 two-bit elements e = 0..15 are interleaved:
+ * element e sits at bit 16*(e & 1) + 2*(e >> 1), i.e. even elements fill the low
+ * half-word and odd elements the high half-word, each half little-endian in 2-bit steps.
+ * Keys are packed along channels and values along tokens — the contraction axis of
+ * q.K^T and of p.V respectively — so that the decode kernel can feed codes straight
+ * into its matrix products with the scales folded into the other operand.
+ *
+ * Pool: uint8 pool[pool_pages][num_kv_heads][kvq_page_bytes(cfg)], 256-byte aligned base.
+ * Residual window: dtype res_k/res_v[batch][num_kv_heads][page_tokens][head_dim];
+ *   res_len[b] tokens of sequence b are valid (0 <= res_len[b] <= page_tokens).
+ * Page table: int32 page_table[batch][max_pages]; the first num_pages[b] entries are
+ *   the physical pages of sequence b in token order.
+ *
+ * Ownership, streams and errors
+ * -----------------------------
+ * Every buffer is allocated and owned by the caller.  Pointers named *_h are host
+ * pointers; every other pointer is a device pointer.  Every call is enqueued on the
+ * given stream and returns before the device work finishes.  Arguments are checked
+ * on the host before any launch; on a failed check nothing is enqueued and the
+ * status says why.  Faults that only the device can see (a page id outside the pool,
+ * a full residual window, a full page table) set bits of the optional device word
+ * *err (KVQ_DEV_ERR_* flags, OR-ed atomically; pass NULL to ignore) and the offending
+ * work item is skipped; outputs of a call that raised a device error are undefined.
+ * No kernel traps.  The library holds no global state.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,  /* null pointer, inconsistent sizes, bad page count         */
+  KVQ_ERR_UNSUPPORTED = 2,  /* a shape or precision this build has no kernel for         */
+  KVQ_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed                */
+  KVQ_ERR_CAPACITY = 4      /* workspace too small                                        */
+} kvq_status;
+
+typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+/* Device-side error flags OR-ed into *err. */
+#define KVQ_DEV_ERR_PAGE_RANGE   1  /* a page id in a table or destination list is outside the pool */
+#define KVQ_DEV_ERR_RESIDUAL     2  /* append into a full residual window                            */
+#define KVQ_DEV_ERR_TABLE_FULL   4  /* flush with no free page-table slot or no destination page      */
+#define KVQ_DEV_ERR_TIMEOUT      8  /* a bounded wait for an asynchronous copy gave up                */
+#define KVQ_DEV_ERR_LENGTH      16  /* num_pages[b] or res_len[b] outside its valid range             */
+
+/* Shape and precision of one attention layer's KV cache.
+ * Supported: head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8};
+ * page_tokens in {32, 64, 128}; key_group 32; key_bits 2, boost_bits 4, value_bits 2;
+ * num_boost a multiple of 16 in [0, head_dim]; dtype KVQ_F16 or KVQ_BF16
+ * (keys, values, queries, residual, scales and zeros all use dtype). */
+typedef struct {
+  int32_t head_dim;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t page_tokens;
+  int32_t key_group;
+  int32_t key_bits;
+  int32_t boost_bits;
+  int32_t value_bits;
+  int32_t num_boost;
+  int32_t dtype;
+} kvq_config;
+
+/* Byte offsets of the sections of one page record (see the layout above). */
+typedef struct {
+  size_t k_codes, kb_codes, v_codes, k_scale, k_zero, kb_scale, v_scale, v_zero, boost_idx;
+  size_t payload_bytes;  /* bytes actually used by the sections                 */
+  size_t record_bytes;   /* stride between records = payload rounded up to 128  */
+} kvq_layout;
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* kvq_status_string(kvq_status s);
+
+/* Checks a configuration without touching the GPU. */
+kvq_status kvq_check_config(const kvq_config* cfg);
+
+/* Fills *out with the record layout of cfg. Host only; no CUDA call. */
+kvq_status kvq_page_layout(const kvq_config* cfg, kvq_layout* out);
+
+/* Record stride in bytes for cfg, or 0 if cfg is not supported. */
+size_t kvq_page_bytes(const kvq_config* cfg);
+
+/* Source of whole pages for the quantize calls.  Element (page i, token t, kv head h,
+ * channel c) is read at src[i*page_stride + t*token_stride + h*head_stride + c]
+ * (strides in elements of dtype).  For a token-major prompt [tokens][Hkv][D] use
+ * page_stride = P*Hkv*D, token_stride = Hkv*D, head_stride = D. */
+typedef struct {
+  const void* src;
+  int64_t page_stride;
+  int64_t token_stride;
+  int64_t head_stride;
+} kvq_source;
+
+/* a1 — Dynamic Channel-wise Precision Boost selection (Kitty abstract; wiki open
+ * question on the magnitude-based channel heuristic).  For each of the n_pages pages
+ * of k and each KV head, ranks the channels by max |K| over the page and writes the
+ * num_boost highest (ties to the lower index) in ascending order into the boost_idx
+ * section of record (dst_pages[i], h).  dst_pages: device int32[n_pages]. */
+kvq_status kvq_select_boost_channels(const kvq_config* cfg, kvq_source k,
+                                     const int32_t* dst_pages, int32_t n_pages,
+                                     void* pool, int64_t pool_pages, int32_t* err,
+                                     cudaStream_t stream);
+
+/* a2 — per-channel Key quantization with the two-plane split (KIVI per-channel keys;
+ * Kitty abstract: each mixed-precision Key page becomes two unified 2-bit tensors).
+ * Reads boost_idx from the destination records (written by
+ * kvq_select_boost_channels) and writes k_codes, kb_codes, k_scale, k_zero, kb_scale. */
+kvq_status kvq_quantize_page_keys(const kvq_config* cfg, kvq_source k,
+                                  const int32_t* dst_pages, int32_t n_pages,
+                                  void* pool, int64_t pool_pages, int32_t* err,
+                                  cudaStream_t stream);
+
+/* a3 — per-token Value quantization (KIVI section 3).  Writes v_codes, v_scale, v_zero. */
+kvq_status kvq_quantize_values(const kvq_config* cfg, kvq_source v,
+                               const int32_t* dst_pages, int32_t n_pages,
+                               void* pool, int64_t pool_pages, int32_t* err,
+                               cudaStream_t stream);
+
+/* a1+a2+a3 in one pass over each page: the same bytes as the three calls above. */
+kvq_status kvq_quantize_pages(const kvq_config* cfg, kvq_source k, kvq_source v,
+                              const int32_t* dst_pages, int32_t n_pages,
+                              void* pool, int64_t pool_pages, int32_t* err,
+                              cudaStream_t stream);
+
+/* a4 — streaming append into the full-precision residual window (KIVI section 3:
+ * recent tokens stay in full precision and new tokens are appended without touching
+ * quantized pages).  k_new, v_new: dtype [batch][Hkv][D].  For every b, writes the
+ * token at position res_len[b] of res_k/res_v and increments res_len[b].  A sequence
+ * whose window is already full (res_len[b] == page_tokens) is skipped and raises
+ * KVQ_DEV_ERR_RESIDUAL: flush first. */
+kvq_status kvq_append_token(const kvq_config* cfg, int32_t batch,
+                            const void* k_new, const void* v_new,
+                            void* res_k, void* res_v, int32_t* res_len,
+                            int32_t* err, cudaStream_t stream);
+
+/* a5 — residual flush.  Reading: the window is flushed when it holds a whole page
+ * (res_len[b] == page_tokens); the flush quantizes the window as one page (a1-a3)
+ * into physical page new_page[b], appends that page to the page table
+ * (page_table[b][num_pages[b]] = new_page[b], num_pages[b] += 1) and empties the
+ * window (res_len[b] = 0).  Sequences whose window is not full are left untouched.
+ * new_page: device int32[batch], the page the host reserves for b (ignored unless b
+ * flushes; a negative id or a full table raises KVQ_DEV_ERR_TABLE_FULL and skips b).
+ * The caller decides which sequences will flush (it issued the appends), so the call
+ * needs no device-to-host read and can be captured in a CUDA graph. */
+kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
+                              const void* res_k, const void* res_v, int32_t* res_len,
+                              const int32_t* new_page, int32_t* page_table,
+                              int32_t max_pages, int32_t* num_pages,
+                              void* pool, int64_t pool_pages, int32_t* err,
+                              cudaStream_t stream);
+
+/* Scratch bytes kvq_decode_attention needs for (cfg, batch, max_pages).  The
+ * workspace holds split-K partial results and one arrival counter per
+ * (sequence, KV head).  The counters must be zero before the first call (clear the
+ * whole workspace once after allocating it); every call leaves them zero again. */
+size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages);
+
+/* a6 + a7 — decode attention over the paged, packed cache plus the residual window
+ * (Kitty abstract: page dequantization kernels over a page-centric layout; MiniKV
+ * proposed method: dequantization fused into the attention matmuls).  For every
+ * sequence b and query head h (KV head h / (Hq/Hkv)):
+ *   out[b][h] = softmax(sm_scale * q[b][h] . K^T) V
+ * over the num_pages[b] quantized pages of page_table[b] (dequantized inside the
+ * kernel) followed by the res_len[b] residual tokens.  The token range of a sequence
+ * is split across CTAs and the partial softmax states are merged by log-sum-exp in
+ * the same launch (no second kernel).
+ * q: dtype [batch][Hq][D]; out: fp32 [batch][Hq][D]; sm_scale normally 1/sqrt(D).
+ * workspace: device, >= kvq_decode_workspace_bytes(cfg, batch, max_pages) bytes,
+ * see kvq_decode_workspace_bytes for its zero-counter contract.
+ * A sequence with no tokens at all (num_pages[b] == 0 and res_len[b] == 0) gets an
+ * all-zero output row. */
+kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t pool_pages,
+                                const void* q, int32_t batch,
+                                const int32_t* page_table, int32_t max_pages,
+                                const int32_t* num_pages,
+                                const void* res_k, const void* res_v, const int32_t* res_len,
+                                float sm_scale, float* out,
+                                void* workspace, size_t workspace_bytes,
+                                int32_t* err, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,421 @@
+/*
+ * kvq_oracle.c — TEST INFRASTRUCTURE, not part of the product.
+ *
+ * A plain, slow CPU restatement of the 2-bit mixed-precision KV cache and of decode
+ * attention over it.  Only the tests, the smoke check and the benchmark's CPU
+ * baseline may load this library; the product path never does.  It shares no code,
+ * header, table or constant with the CUDA library: the record layout, the packing
+ * and every formula are written out again here from their definitions.
+ *
+ * Sources (web pages on the method):
+ *  - aibr.jp article on KIVI, section 3 (core technical elements): asymmetric
+ *    quantization, Keys per channel, Values per token, full-precision residual of
+ *    recent tokens, streaming append.
+ *  - fugumt.com summary of Kitty (arXiv 2511.18643), Abstract: channels of the Key
+ *    cache are ranked and a small fraction kept at higher precision; each
+ *    mixed-precision Key page is stored as two uniform 2-bit tensors.
+ *  - notes.yuuk.io wiki page "KVキャッシュ量子化", open questions: the ranking is a
+ *    magnitude heuristic; boost ratios 12.5% and 25%.
+ *  - f-binder summary of MiniKV, section "proposed method": keys grouped along
+ *    channels, values per token, 2-bit codes expanded inside the attention matmul.
+ * The pages print no formula.  The readings taken here (min/max asymmetric
+ * quantizer with scale = (max-min)/(2^b-1) rounded up to the storage type, zero =
+ * min, round half to even, clamp; magnitude = max |x| over the page; ties to the
+ * lower channel; 4-bit code = 4*hi + lo) are the plainest ones and are the same
+ * readings the library documents.
+ *
+ * Arithmetic: the quantizer works in fp32 with one rounding per operation, in the
+ * order written (build with -ffp-contract=off, no fast-math), because its fp32
+ * decisions fix integer codes.  Dequantization and attention work in fp64, where
+ * code*scale + zero of two 16-bit values is exact.
+ *
+ * Every function below states which part of the method it follows.  Parity pins for
+ * each function live in the tests (brute force, closed forms, library routines).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define DT_F16 0
+#define DT_BF16 1
+
+/* ---------------------------------------------------------------- 16-bit float types */
+
+/* IEEE binary16 bits -> value (exact). */
+static double f16_value(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0)
+    v = ldexp((double)m, -24);
+  else if (e == 31)
+    v = m ? NAN : INFINITY;
+  else
+    v = ldexp((double)(m + 1024), e - 25);
+  return sign ? -v : v;
+}
+
+/* bfloat16 bits -> value (exact): the upper half of an IEEE binary32. */
+static double bf16_value(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+static double dt_value(uint16_t bits, int dtype) {
+  return dtype == DT_BF16 ? bf16_value(bits) : f16_value(bits);
+}
+
+/* Rounds a finite double to the 16-bit type.  mode 0: nearest, ties to even;
+ * mode 1: toward +infinity.  Written from the format definitions: a value is an
+ * integer multiple of the quantum of its binade (or of the subnormal quantum). */
+static uint16_t dt_round(double x, int dtype, int mode) {
+  const int man_bits = dtype == DT_BF16 ? 7 : 10;
+  const int emin = dtype == DT_BF16 ? -126 : -14;  /* exponent of the smallest normal */
+  const int emax = dtype == DT_BF16 ? 127 : 15;
+  const int bias = dtype == DT_BF16 ? 127 : 15;
+  const int exp_field_max = dtype == DT_BF16 ? 255 : 31;
+  uint16_t sign = 0;
+  double a = x;
+  if (x < 0 || (x == 0 && signbit(x))) {
+    sign = 1;
+    a = -x;
+  }
+  if (a == 0) return (uint16_t)(sign << 15);
+  int e2;
+  frexp(a, &e2);          /* a = f * 2^e2 with f in [0.5, 1) */
+  int e = e2 - 1;         /* a in [2^e, 2^(e+1)) */
+  if (e < emin) e = emin; /* subnormal range shares the quantum of the smallest binade */
+  double quantum = ldexp(1.0, e - man_bits);
+  double n = a / quantum; /* exact: scaling by a power of two */
+  double r;
+  if (mode == 0) {
+    r = nearbyint(n);     /* default rounding mode: half to even */
+  } else {
+    /* toward +inf: magnitude up for positive numbers, down for negative ones */
+    r = sign ? floor(n) : ceil(n);
+  }
+  double v = r * quantum;
+  double maxv = ldexp((double)((2 << man_bits) - 1), emax - man_bits);
+  if (v > maxv) {
+    /* overflow: nearest gives inf beyond the halfway point; upward gives +inf for
+     * positive values (negative values cannot round up in magnitude here) */
+    return (uint16_t)((sign << 15) | (exp_field_max << man_bits));
+  }
+  if (v == 0) return (uint16_t)(sign << 15);
+  /* encode the exact value v */
+  frexp(v, &e2);
+  e = e2 - 1;
+  uint16_t bits;
+  if (e < emin) {
+    bits = (uint16_t)(v / ldexp(1.0, emin - man_bits));
+  } else {
+    uint32_t m = (uint32_t)(v / ldexp(1.0, e - man_bits)) - (1u << man_bits);
+    bits = (uint16_t)(((uint32_t)(e + bias) << man_bits) | m);
+  }
+  return (uint16_t)((sign << 15) | bits);
+}
+
+double kvqo_value(uint16_t bits, int dtype) { return dt_value(bits, dtype); }
+uint16_t kvqo_round_nearest(double x, int dtype) { return dt_round(x, dtype, 0); }
+uint16_t kvqo_round_up(double x, int dtype) { return dt_round(x, dtype, 1); }
+
+/* ------------------------------------------------------------------------ quantizer */
+
+/* Asymmetric min/max quantization of one group (KIVI section 3: asymmetric
+ * quantization).  x: n values given as 16-bit patterns of dtype, read with stride.
+ * Writes n codes, the stored scale and zero (16-bit patterns).  fp32 arithmetic,
+ * one rounding per operation:
+ *   mn, mx       = min and max of the group
+ *   s32          = (mx - mn) / (2^bits - 1)
+ *   scale        = s32 rounded toward +inf to dtype
+ *   zero         = mn (a zero minimum is stored as +0)
+ *   code         = clamp(rint((x - zero) / scale), 0, 2^bits - 1); 0 when scale == 0 */
+void kvqo_quant_group(const uint16_t* x, int n, long stride, int bits, int dtype,
+                      uint8_t* codes, uint16_t* scale_bits, uint16_t* zero_bits) {
+  float mn = (float)dt_value(x[0], dtype);
+  float mx = mn;
+  for (int i = 1; i < n; ++i) {
+    float v = (float)dt_value(x[i * stride], dtype);
+    if (v < mn) mn = v;
+    if (v > mx) mx = v;
+  }
+  const int qmax = (1 << bits) - 1;
+  volatile float range = mx - mn;
+  volatile float s32 = range / (float)qmax;
+  uint16_t sb = dt_round((double)s32, dtype, 1);
+  float scale = (float)dt_value(sb, dtype);
+  uint16_t zb = mn == 0.0f ? 0 : dt_round((double)mn, dtype, 0);
+  float zero = (float)dt_value(zb, dtype);
+  for (int i = 0; i < n; ++i) {
+    int code = 0;
+    if (scale != 0.0f) {
+      float v = (float)dt_value(x[i * stride], dtype);
+      volatile float d = v - zero;
+      volatile float t = d / scale;
+      float r = rintf(t);
+      if (r < 0.0f) r = 0.0f;
+      if (r > (float)qmax) r = (float)qmax;
+      code = (int)r;
+    }
+    codes[i] = (uint8_t)code;
+  }
+  *scale_bits = sb;
+  *zero_bits = zb;
+}
+
+/* --------------------------------------------------------------------- page layout */
+
+typedef struct {
+  long k_codes, kb_codes, v_codes, k_scale, k_zero, kb_scale, v_scale, v_zero, boost_idx;
+  long payload, record;
+} layout_t;
+
+/* Section order and sizes of one (page, KV head) record; see the library's ABI
+ * description of the page record.  P tokens, D channels, k boosted rows, G group. */
+static layout_t make_layout(int P, int D, int k, int G) {
+  layout_t L;
+  long off = 0;
+  L.k_codes = off;   off += (long)P * (D / 16) * 4;
+  L.kb_codes = off;  off += (long)P * (k / 16) * 4;
+  L.v_codes = off;   off += (long)D * (P / 16) * 4;
+  L.k_scale = off;   off += (long)(P / G) * D * 2;
+  L.k_zero = off;    off += (long)(P / G) * D * 2;
+  L.kb_scale = off;  off += (long)(P / G) * k * 2;
+  L.v_scale = off;   off += (long)P * 2;
+  L.v_zero = off;    off += (long)P * 2;
+  L.boost_idx = off; off += k;
+  L.payload = off;
+  L.record = (off + 127) / 128 * 128;
+  return L;
+}
+
+void kvqo_layout(int P, int D, int k, int G, long* out /* 11 entries */) {
+  layout_t L = make_layout(P, D, k, G);
+  long v[11] = {L.k_codes, L.kb_codes, L.v_codes, L.k_scale, L.k_zero, L.kb_scale,
+                L.v_scale, L.v_zero, L.boost_idx, L.payload, L.record};
+  memcpy(out, v, sizeof v);
+}
+
+/* Position of element e (0..15) inside a 32-bit code word: even elements in the low
+ * half-word, odd elements in the high half-word, 2 bits apart. */
+static int elem_shift(int e) { return 16 * (e & 1) + 2 * (e >> 1); }
+
+static void put2(uint32_t* words, int word, int e, unsigned code) {
+  words[word] |= (uint32_t)(code & 3u) << elem_shift(e);
+}
+
+static unsigned get2(const uint32_t* words, int word, int e) {
+  return (words[word] >> elem_shift(e)) & 3u;
+}
+
+/* -------------------------------------------------------------- boost selection (a1) */
+
+/* Dynamic Channel-wise Precision Boost selection (Kitty abstract; wiki: magnitude
+ * heuristic).  score_c = max_t |K[t][c]| over the page; the k channels with the
+ * highest score, ties to the lower index, returned in ascending channel order. */
+void kvqo_select_boost(const uint16_t* K, long tok_stride, int P, int D, int k, int dtype,
+                       uint8_t* idx) {
+  double* score = (double*)malloc(sizeof(double) * D);
+  char* taken = (char*)calloc(D, 1);
+  for (int c = 0; c < D; ++c) {
+    double s = 0.0;
+    for (int t = 0; t < P; ++t) {
+      double a = fabs(dt_value(K[t * tok_stride + c], dtype));
+      if (a > s) s = a;
+    }
+    score[c] = s;
+  }
+  /* k rounds of "pick the best remaining channel" */
+  for (int r = 0; r < k; ++r) {
+    int best = -1;
+    for (int c = 0; c < D; ++c) {
+      if (taken[c]) continue;
+      if (best < 0 || score[c] > score[best]) best = c;  /* strict: lower index wins ties */
+    }
+    taken[best] = 1;
+  }
+  int j = 0;
+  for (int c = 0; c < D; ++c)
+    if (taken[c]) idx[j++] = (uint8_t)c;
+  free(score);
+  free(taken);
+}
+
+/* ------------------------------------------------------------- page quantization */
+
+/* Quantizes one page of one KV head into a record (a1 + a2 + a3).
+ * K, V: [P][D] 16-bit patterns with token stride tok_stride (elements).
+ * rec: record_bytes bytes; padding is left zero. */
+void kvqo_quantize_page(const uint16_t* K, const uint16_t* V, long tok_stride, int P, int D,
+                        int G, int k, int dtype, uint8_t* rec) {
+  layout_t L = make_layout(P, D, k, G);
+  memset(rec, 0, (size_t)L.record);
+  uint32_t* kA = (uint32_t*)(rec + L.k_codes);
+  uint32_t* kB = (uint32_t*)(rec + L.kb_codes);
+  uint32_t* vq = (uint32_t*)(rec + L.v_codes);
+  uint16_t* ks = (uint16_t*)(rec + L.k_scale);
+  uint16_t* kz = (uint16_t*)(rec + L.k_zero);
+  uint16_t* kbs = (uint16_t*)(rec + L.kb_scale);
+  uint16_t* vs = (uint16_t*)(rec + L.v_scale);
+  uint16_t* vz = (uint16_t*)(rec + L.v_zero);
+  uint8_t* bidx = rec + L.boost_idx;
+
+  /* a1: boosted channels */
+  kvqo_select_boost(K, tok_stride, P, D, k, dtype, bidx);
+  int* row_of = (int*)malloc(sizeof(int) * D); /* plane-B row of a boosted channel, else -1 */
+  for (int c = 0; c < D; ++c) row_of[c] = -1;
+  for (int j = 0; j < k; ++j) row_of[bidx[j]] = j;
+
+  /* a2: keys, per channel and per group of G tokens */
+  uint8_t* codes = (uint8_t*)malloc((size_t)(P > D ? P : D));
+  const int kw = D / 16, kbw = k / 16;
+  for (int g = 0; g < P / G; ++g) {
+    for (int c = 0; c < D; ++c) {
+      const uint16_t* col = K + (long)g * G * tok_stride + c;
+      uint16_t sb, zb;
+      int j = row_of[c];
+      if (j < 0) {
+        kvqo_quant_group(col, G, tok_stride, 2, dtype, codes, &sb, &zb);
+        for (int t = 0; t < G; ++t) put2(kA, (g * G + t) * kw + c / 16, c % 16, codes[t]);
+        ks[g * D + c] = sb;
+      } else {
+        kvqo_quant_group(col, G, tok_stride, 4, dtype, codes, &sb, &zb);
+        for (int t = 0; t < G; ++t) {
+          put2(kA, (g * G + t) * kw + c / 16, c % 16, codes[t] >> 2);
+          put2(kB, (g * G + t) * kbw + j / 16, j % 16, codes[t] & 3);
+        }
+        /* plane A carries the high bits with four times the 4-bit scale (exact) */
+        ks[g * D + c] = dt_round(4.0 * dt_value(sb, dtype), dtype, 0);
+        kbs[g * k + j] = sb;
+      }
+      kz[g * D + c] = zb;
+    }
+  }
+
+  /* a3: values, per token over all D channels */
+  const int vw = P / 16;
+  for (int t = 0; t < P; ++t) {
+    uint16_t sb, zb;
+    kvqo_quant_group(V + (long)t * tok_stride, D, 1, 2, dtype, codes, &sb, &zb);
+    for (int c = 0; c < D; ++c) put2(vq, c * vw + t / 16, t % 16, codes[c]);
+    vs[t] = sb;
+    vz[t] = zb;
+  }
+  free(codes);
+  free(row_of);
+}
+
+/* Dequantizes a record in fp64: Khat, Vhat [P][D].  K^ = A-code * A-scale + A-zero
+ * (+ B-code * B-scale for boosted channels); V^ = code * scale + zero. */
+void kvqo_dequantize_page(const uint8_t* rec, int P, int D, int G, int k, int dtype,
+                          double* Khat, double* Vhat) {
+  layout_t L = make_layout(P, D, k, G);
+  const uint32_t* kA = (const uint32_t*)(rec + L.k_codes);
+  const uint32_t* kB = (const uint32_t*)(rec + L.kb_codes);
+  const uint32_t* vq = (const uint32_t*)(rec + L.v_codes);
+  const uint16_t* ks = (const uint16_t*)(rec + L.k_scale);
+  const uint16_t* kz = (const uint16_t*)(rec + L.k_zero);
+  const uint16_t* kbs = (const uint16_t*)(rec + L.kb_scale);
+  const uint16_t* vs = (const uint16_t*)(rec + L.v_scale);
+  const uint16_t* vz = (const uint16_t*)(rec + L.v_zero);
+  const uint8_t* bidx = rec + L.boost_idx;
+  const int kw = D / 16, kbw = k / 16, vw = P / 16;
+  if (Khat) {
+    for (int t = 0; t < P; ++t) {
+      int g = t / G;
+      for (int c = 0; c < D; ++c) {
+        unsigned a = get2(kA, t * kw + c / 16, c % 16);
+        Khat[t * D + c] = a * dt_value(ks[g * D + c], dtype) + dt_value(kz[g * D + c], dtype);
+      }
+      for (int j = 0; j < k; ++j) {
+        unsigned b = get2(kB, t * kbw + j / 16, j % 16);
+        Khat[t * D + bidx[j]] += b * dt_value(kbs[g * k + j], dtype);
+      }
+    }
+  }
+  if (Vhat) {
+    for (int t = 0; t < P; ++t)
+      for (int c = 0; c < D; ++c) {
+        unsigned v = get2(vq, c * vw + t / 16, t % 16);
+        Vhat[t * D + c] = v * dt_value(vs[t], dtype) + dt_value(vz[t], dtype);
+      }
+  }
+}
+
+/* ------------------------------------------------------------------ decode attention */
+
+/* Decode attention for one sequence and one KV head (fp64): the quantized pages
+ * listed in pages[0..n_pages) (token order) followed by res_len residual tokens;
+ * q: [gqa][D] 16-bit patterns of the query heads sharing this KV head.
+ *   out[h] = sum_t softmax_t(sm_scale * q_h . K^_t) V^_t
+ * Two plain passes: scores over every token, then the weighted sum of values.
+ * pool is the base of record (0, head) layout: record (p, head) lives at
+ * pool + (p * Hkv + head) * record_bytes.  out: [gqa][D]. */
+void kvqo_decode_unit(const uint8_t* pool, int Hkv, int head, const int32_t* pages, int n_pages,
+                      const uint16_t* res_k, const uint16_t* res_v, int res_len,
+                      const uint16_t* q, int gqa, int P, int D, int G, int k, int dtype,
+                      double sm_scale, double* out) {
+  layout_t L = make_layout(P, D, k, G);
+  long n_tok = (long)n_pages * P + res_len;
+  for (int i = 0; i < gqa * D; ++i) out[i] = 0.0;
+  if (n_tok == 0) return;
+  double* scores = (double*)malloc(sizeof(double) * gqa * n_tok);
+  double* Kh = (double*)malloc(sizeof(double) * P * D);
+  double* Vh = (double*)malloc(sizeof(double) * P * D);
+  double* qd = (double*)malloc(sizeof(double) * gqa * D);
+  for (int i = 0; i < gqa * D; ++i) qd[i] = dt_value(q[i], dtype);
+
+  /* pass 1: scores */
+  for (int p = 0; p < n_pages; ++p) {
+    const uint8_t* rec = pool + ((long)pages[p] * Hkv + head) * L.record;
+    kvqo_dequantize_page(rec, P, D, G, k, dtype, Kh, NULL);
+    for (int t = 0; t < P; ++t)
+      for (int h = 0; h < gqa; ++h) {
+        double s = 0.0;
+        for (int c = 0; c < D; ++c) s += qd[h * D + c] * Kh[t * D + c];
+        scores[h * n_tok + (long)p * P + t] = s * sm_scale;
+      }
+  }
+  for (int t = 0; t < res_len; ++t)
+    for (int h = 0; h < gqa; ++h) {
+      double s = 0.0;
+      for (int c = 0; c < D; ++c) s += qd[h * D + c] * dt_value(res_k[(long)t * D + c], dtype);
+      scores[h * n_tok + (long)n_pages * P + t] = s * sm_scale;
+    }
+  /* softmax with the maximum subtracted */
+  for (int h = 0; h < gqa; ++h) {
+    double* s = scores + (long)h * n_tok;
+    double m = s[0];
+    for (long t = 1; t < n_tok; ++t)
+      if (s[t] > m) m = s[t];
+    double l = 0.0;
+    for (long t = 0; t < n_tok; ++t) {
+      s[t] = exp(s[t] - m);
+      l += s[t];
+    }
+    for (long t = 0; t < n_tok; ++t) s[t] /= l;
+  }
+  /* pass 2: probability-weighted values */
+  for (int p = 0; p < n_pages; ++p) {
+    const uint8_t* rec = pool + ((long)pages[p] * Hkv + head) * L.record;
+    kvqo_dequantize_page(rec, P, D, G, k, dtype, NULL, Vh);
+    for (int h = 0; h < gqa; ++h)
+      for (int t = 0; t < P; ++t) {
+        double pt = scores[h * n_tok + (long)p * P + t];
+        for (int c = 0; c < D; ++c) out[h * D + c] += pt * Vh[t * D + c];
+      }
+  }
+  for (int h = 0; h < gqa; ++h)
+    for (int t = 0; t < res_len; ++t) {
+      double pt = scores[h * n_tok + (long)n_pages * P + t];
+      for (int c = 0; c < D; ++c) out[h * D + c] += pt * dt_value(res_v[(long)t * D + c], dtype);
+    }
+  free(scores);
+  free(Kh);
+  free(Vh);
+  free(qd);
+}
