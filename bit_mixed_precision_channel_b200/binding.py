@@ -1,1 +1,261 @@
-__all__ = []
+"""ctypes binding of libkvq.so — argument marshalling only.
+
+Every function has the name of the C entry point it calls (without the ``kvq_``
+prefix) and passes device pointers (``tensor.data_ptr()``), sizes and the current
+PyTorch CUDA stream straight through.  All computation happens in the library's
+CUDA kernels; there is no fallback of any kind: if the library is missing, was not
+built, or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "KVQError", "Config", "Source", "library_path", "load", "status_string", "check_config",
+    "page_layout", "page_bytes", "select_boost_channels", "quantize_page_keys",
+    "quantize_values", "quantize_pages", "append_token", "flush_residual",
+    "decode_workspace_bytes", "decode_attention", "F16", "BF16", "torch_dtype",
+    "DEV_ERR_PAGE_RANGE", "DEV_ERR_RESIDUAL", "DEV_ERR_TABLE_FULL", "DEV_ERR_TIMEOUT",
+    "DEV_ERR_LENGTH",
+]
+
+F16 = 0
+BF16 = 1
+DEV_ERR_PAGE_RANGE = 1
+DEV_ERR_RESIDUAL = 2
+DEV_ERR_TABLE_FULL = 4
+DEV_ERR_TIMEOUT = 8
+DEV_ERR_LENGTH = 16
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libkvq.so")
+
+
+class KVQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "head_dim", "num_q_heads", "num_kv_heads", "page_tokens", "key_group", "key_bits",
+        "boost_bits", "value_bits", "num_boost", "dtype")]
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "k_codes", "kb_codes", "v_codes", "k_scale", "k_zero", "kb_scale", "v_scale", "v_zero",
+        "boost_idx", "payload_bytes", "record_bytes")]
+
+
+class _Source(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("page_stride", ctypes.c_int64),
+                ("token_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64)]
+
+
+@dataclass(frozen=True)
+class Config:
+    """Cache shape of one attention layer (mirrors kvq_config)."""
+    head_dim: int = 128
+    num_q_heads: int = 32
+    num_kv_heads: int = 8
+    page_tokens: int = 128
+    key_group: int = 32
+    num_boost: int = 32
+    dtype: int = F16
+    key_bits: int = 2
+    boost_bits: int = 4
+    value_bits: int = 2
+
+    @property
+    def gqa(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    def c(self) -> _Config:
+        return _Config(self.head_dim, self.num_q_heads, self.num_kv_heads, self.page_tokens,
+                       self.key_group, self.key_bits, self.boost_bits, self.value_bits,
+                       self.num_boost, self.dtype)
+
+
+def torch_dtype(dtype: int) -> torch.dtype:
+    return torch.bfloat16 if dtype == BF16 else torch.float16
+
+
+@dataclass
+class Source:
+    """Pages of a 16-bit tensor: element (page i, token t, kv head h, channel c) is at
+    tensor.flatten()[i*page_stride + t*token_stride + h*head_stride + c]."""
+    tensor: torch.Tensor
+    page_stride: int
+    token_stride: int
+    head_stride: int
+
+    @staticmethod
+    def token_major(x: torch.Tensor, cfg: Config, first_token: int = 0) -> "Source":
+        """x: [tokens][Hkv][D] contiguous; pages start at token `first_token`."""
+        assert x.is_contiguous() and x.dim() == 3
+        H, D, P = cfg.num_kv_heads, cfg.head_dim, cfg.page_tokens
+        return Source(x[first_token:] if first_token else x, P * H * D, H * D, D)
+
+    def c(self) -> _Source:
+        return _Source(self.tensor.data_ptr(), self.page_stride, self.token_stride, self.head_stride)
+
+
+_lib = None
+
+
+def load():
+    """Loads libkvq.so once; raises if it is missing."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"libkvq.so not found at {path}; build it with "
+                               "`python -m bit_mixed_precision_channel_b200.build`")
+        L = ctypes.CDLL(path)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        cfgp = ctypes.POINTER(_Config)
+        L.kvq_status_string.restype = ctypes.c_char_p
+        L.kvq_status_string.argtypes = [ctypes.c_int]
+        L.kvq_check_config.restype = ctypes.c_int
+        L.kvq_check_config.argtypes = [cfgp]
+        L.kvq_page_layout.restype = ctypes.c_int
+        L.kvq_page_layout.argtypes = [cfgp, ctypes.POINTER(_Layout)]
+        L.kvq_page_bytes.restype = sz
+        L.kvq_page_bytes.argtypes = [cfgp]
+        for name in ("kvq_select_boost_channels", "kvq_quantize_page_keys", "kvq_quantize_values"):
+            f = getattr(L, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [cfgp, _Source, vp, i32, vp, i64, vp, vp]
+        L.kvq_quantize_pages.restype = ctypes.c_int
+        L.kvq_quantize_pages.argtypes = [cfgp, _Source, _Source, vp, i32, vp, i64, vp, vp]
+        L.kvq_append_token.restype = ctypes.c_int
+        L.kvq_append_token.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.kvq_flush_residual.restype = ctypes.c_int
+        L.kvq_flush_residual.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, i32, vp, vp, i64, vp, vp]
+        L.kvq_decode_workspace_bytes.restype = sz
+        L.kvq_decode_workspace_bytes.argtypes = [cfgp, i32, i32]
+        L.kvq_decode_attention.restype = ctypes.c_int
+        L.kvq_decode_attention.argtypes = [cfgp, vp, i64, vp, i32, vp, i32, vp, vp, vp, vp,
+                                           ctypes.c_float, vp, vp, sz, vp, vp]
+        _lib = L
+    return _lib
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise KVQError(fn, status)
+
+
+def _cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("kvq calls take CUDA tensors (device memory)")
+
+
+def status_string(status: int) -> str:
+    return load().kvq_status_string(status).decode()
+
+
+def check_config(cfg: Config) -> int:
+    return load().kvq_check_config(ctypes.byref(cfg.c()))
+
+
+def page_layout(cfg: Config) -> dict:
+    out = _Layout()
+    _check("kvq_page_layout", load().kvq_page_layout(ctypes.byref(cfg.c()), ctypes.byref(out)))
+    return {n: int(getattr(out, n)) for n, _ in _Layout._fields_}
+
+
+def page_bytes(cfg: Config) -> int:
+    return int(load().kvq_page_bytes(ctypes.byref(cfg.c())))
+
+
+def _quant(fn, cfg, src_k, src_v, dst_pages, pool, err, stream):
+    _cuda(dst_pages, pool, err)
+    pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
+    L = load()
+    n = dst_pages.numel()
+    if fn == "kvq_quantize_pages":
+        st = L.kvq_quantize_pages(ctypes.byref(cfg.c()), src_k.c(), src_v.c(), dst_pages.data_ptr(), n,
+                                  pool.data_ptr(), pool_pages, _ptr(err), _stream(stream))
+    else:
+        src = src_k if src_k is not None else src_v
+        st = getattr(L, fn)(ctypes.byref(cfg.c()), src.c(), dst_pages.data_ptr(), n, pool.data_ptr(),
+                            pool_pages, _ptr(err), _stream(stream))
+    _check(fn, st)
+
+
+def select_boost_channels(cfg: Config, k: Source, dst_pages: torch.Tensor, pool: torch.Tensor,
+                          err: torch.Tensor | None = None, stream=None):
+    _quant("kvq_select_boost_channels", cfg, k, None, dst_pages, pool, err, stream)
+
+
+def quantize_page_keys(cfg: Config, k: Source, dst_pages: torch.Tensor, pool: torch.Tensor,
+                       err: torch.Tensor | None = None, stream=None):
+    _quant("kvq_quantize_page_keys", cfg, k, None, dst_pages, pool, err, stream)
+
+
+def quantize_values(cfg: Config, v: Source, dst_pages: torch.Tensor, pool: torch.Tensor,
+                    err: torch.Tensor | None = None, stream=None):
+    _quant("kvq_quantize_values", cfg, None, v, dst_pages, pool, err, stream)
+
+
+def quantize_pages(cfg: Config, k: Source, v: Source, dst_pages: torch.Tensor, pool: torch.Tensor,
+                   err: torch.Tensor | None = None, stream=None):
+    _quant("kvq_quantize_pages", cfg, k, v, dst_pages, pool, err, stream)
+
+
+def append_token(cfg: Config, k_new, v_new, res_k, res_v, res_len, err=None, stream=None):
+    _cuda(k_new, v_new, res_k, res_v, res_len, err)
+    batch = res_len.numel()
+    _check("kvq_append_token", load().kvq_append_token(
+        ctypes.byref(cfg.c()), batch, k_new.data_ptr(), v_new.data_ptr(), res_k.data_ptr(),
+        res_v.data_ptr(), res_len.data_ptr(), _ptr(err), _stream(stream)))
+
+
+def flush_residual(cfg: Config, res_k, res_v, res_len, new_page, page_table, num_pages, pool,
+                   err=None, stream=None):
+    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err)
+    batch, max_pages = page_table.shape
+    pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
+    _check("kvq_flush_residual", load().kvq_flush_residual(
+        ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
+        new_page.data_ptr(), page_table.data_ptr(), max_pages, num_pages.data_ptr(), pool.data_ptr(),
+        pool_pages, _ptr(err), _stream(stream)))
+
+
+def decode_workspace_bytes(cfg: Config, batch: int, max_pages: int) -> int:
+    return int(load().kvq_decode_workspace_bytes(ctypes.byref(cfg.c()), batch, max_pages))
+
+
+def decode_attention(cfg: Config, pool, q, page_table, num_pages, res_k, res_v, res_len, out,
+                     workspace, sm_scale: float | None = None, err=None, stream=None):
+    _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, workspace, err)
+    batch, max_pages = page_table.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(cfg.head_dim)
+    pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
+    _check("kvq_decode_attention", load().kvq_decode_attention(
+        ctypes.byref(cfg.c()), pool.data_ptr(), pool_pages, q.data_ptr(), batch, page_table.data_ptr(),
+        max_pages, num_pages.data_ptr(), res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
+        float(sm_scale), out.data_ptr(), workspace.data_ptr(), workspace.numel(), _ptr(err),
+        _stream(stream)))

@@ -1,0 +1,262 @@
+// kvq_api.cu — the C ABI of include/kvq.h: host-side argument checks and launches.
+#include <algorithm>
+#include <cstdint>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+struct Plan {
+  SplitPlan split;
+  size_t part_bytes, cnt_bytes;
+};
+
+static Plan decode_plan(const kvq_config* cfg, int batch, int max_pages) {
+  const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  const int units = batch * cfg->num_kv_heads;
+  Plan pl;
+  pl.split = plan_splits(units, max_pages, sm_count());
+  pl.part_bytes = size_t(units) * pl.split.max_splits * gqa * (2 + kHeadDim) * sizeof(float);
+  pl.part_bytes = (pl.part_bytes + 255) / 256 * 256;
+  pl.cnt_bytes = size_t(units) * sizeof(uint32_t);
+  return pl;
+}
+
+}  // namespace kvq
+
+using namespace kvq;
+
+static kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument (null pointer, inconsistent sizes or misaligned buffer)";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration (shape or precision without a kernel)";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+    case KVQ_ERR_CAPACITY: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_check_config(const kvq_config* cfg) {
+  if (!cfg) return KVQ_ERR_INVALID_ARG;
+  if (cfg->head_dim <= 0 || cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->page_tokens <= 0 ||
+      cfg->key_group <= 0 || cfg->num_boost < 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (cfg->num_q_heads % cfg->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  if (cfg->page_tokens % cfg->key_group != 0) return KVQ_ERR_INVALID_ARG;
+  if (cfg->num_boost > cfg->head_dim || cfg->num_boost % 16 != 0) return KVQ_ERR_INVALID_ARG;
+  const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  if (cfg->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if (gqa != 1 && gqa != 2 && gqa != 4 && gqa != 8) return KVQ_ERR_UNSUPPORTED;
+  if (cfg->page_tokens != 32 && cfg->page_tokens != 64 && cfg->page_tokens != 128) return KVQ_ERR_UNSUPPORTED;
+  if (cfg->key_group != 32) return KVQ_ERR_UNSUPPORTED;
+  if (cfg->key_bits != 2 || cfg->boost_bits != 4 || cfg->value_bits != 2) return KVQ_ERR_UNSUPPORTED;
+  if (cfg->dtype != KVQ_F16 && cfg->dtype != KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+kvq_status kvq_page_layout(const kvq_config* cfg, kvq_layout* out) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  const Layout L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
+  out->k_codes = L.k_codes;
+  out->kb_codes = L.kb_codes;
+  out->v_codes = L.v_codes;
+  out->k_scale = L.k_scale;
+  out->k_zero = L.k_zero;
+  out->kb_scale = L.kb_scale;
+  out->v_scale = L.v_scale;
+  out->v_zero = L.v_zero;
+  out->boost_idx = L.boost_idx;
+  out->payload_bytes = L.payload;
+  out->record_bytes = L.record;
+  return KVQ_OK;
+}
+
+size_t kvq_page_bytes(const kvq_config* cfg) {
+  if (kvq_check_config(cfg) != KVQ_OK) return 0;
+  return make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group).record;
+}
+
+static kvq_status quantize_common(const kvq_config* cfg, kvq_source k, kvq_source v, int mode,
+                                  const int32_t* dst_pages, int32_t n_pages, void* pool, int64_t pool_pages,
+                                  int32_t* err, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (n_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (n_pages == 0) return KVQ_OK;
+  if (!dst_pages || !pool || pool_pages <= 0 || !aligned16(pool)) return KVQ_ERR_INVALID_ARG;
+  auto bad_src = [](const kvq_source& x) {
+    return !x.src || !aligned16(x.src) || x.page_stride % 8 || x.token_stride % 8 || x.head_stride % 8 ||
+           x.page_stride < 0 || x.token_stride < 0 || x.head_stride < 0;
+  };
+  if ((mode & (kModeSelect | kModeKeys)) && bad_src(k)) return KVQ_ERR_INVALID_ARG;
+  if ((mode & kModeValues) && bad_src(v)) return KVQ_ERR_INVALID_ARG;
+  QuantParams p{};
+  p.k_src = static_cast<const uint16_t*>(k.src);
+  p.v_src = static_cast<const uint16_t*>(v.src);
+  p.k_page_stride = k.page_stride;
+  p.k_tok_stride = k.token_stride;
+  p.k_head_stride = k.head_stride;
+  p.v_page_stride = v.page_stride;
+  p.v_tok_stride = v.token_stride;
+  p.v_head_stride = v.head_stride;
+  p.dst_pages = dst_pages;
+  p.pool = static_cast<uint8_t*>(pool);
+  p.pool_pages = pool_pages;
+  p.Hkv = cfg->num_kv_heads;
+  p.P = cfg->page_tokens;
+  p.k = cfg->num_boost;
+  p.L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
+  p.err = err;
+  p.mode = mode;
+  p.flush = 0;
+  return cuda_status(launch_quantize(p, n_pages, cfg->dtype, stream));
+}
+
+kvq_status kvq_select_boost_channels(const kvq_config* cfg, kvq_source k, const int32_t* dst_pages,
+                                     int32_t n_pages, void* pool, int64_t pool_pages, int32_t* err,
+                                     cudaStream_t stream) {
+  return quantize_common(cfg, k, kvq_source{}, kModeSelect, dst_pages, n_pages, pool, pool_pages, err, stream);
+}
+
+kvq_status kvq_quantize_page_keys(const kvq_config* cfg, kvq_source k, const int32_t* dst_pages, int32_t n_pages,
+                                  void* pool, int64_t pool_pages, int32_t* err, cudaStream_t stream) {
+  return quantize_common(cfg, k, kvq_source{}, kModeKeys, dst_pages, n_pages, pool, pool_pages, err, stream);
+}
+
+kvq_status kvq_quantize_values(const kvq_config* cfg, kvq_source v, const int32_t* dst_pages, int32_t n_pages,
+                               void* pool, int64_t pool_pages, int32_t* err, cudaStream_t stream) {
+  return quantize_common(cfg, kvq_source{}, v, kModeValues, dst_pages, n_pages, pool, pool_pages, err, stream);
+}
+
+kvq_status kvq_quantize_pages(const kvq_config* cfg, kvq_source k, kvq_source v, const int32_t* dst_pages,
+                              int32_t n_pages, void* pool, int64_t pool_pages, int32_t* err, cudaStream_t stream) {
+  return quantize_common(cfg, k, v, kModeSelect | kModeKeys | kModeValues, dst_pages, n_pages, pool, pool_pages,
+                         err, stream);
+}
+
+kvq_status kvq_append_token(const kvq_config* cfg, int32_t batch, const void* k_new, const void* v_new,
+                            void* res_k, void* res_v, int32_t* res_len, int32_t* err, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (batch < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!k_new || !v_new || !res_k || !res_v || !res_len) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(res_k) || !aligned16(res_v)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_append(k_new, v_new, res_k, res_v, res_len, batch, cfg->num_kv_heads,
+                                   cfg->page_tokens, err, stream));
+}
+
+kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch, const void* res_k, const void* res_v,
+                              int32_t* res_len, const int32_t* new_page, int32_t* page_table, int32_t max_pages,
+                              int32_t* num_pages, void* pool, int64_t pool_pages, int32_t* err,
+                              cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!res_k || !res_v || !res_len || !new_page || !page_table || !num_pages || !pool || pool_pages <= 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(res_k) || !aligned16(res_v) || !aligned16(pool)) return KVQ_ERR_INVALID_ARG;
+  const int P = cfg->page_tokens, Hkv = cfg->num_kv_heads, D = cfg->head_dim;
+  QuantParams p{};
+  p.k_src = static_cast<const uint16_t*>(res_k);
+  p.v_src = static_cast<const uint16_t*>(res_v);
+  p.k_page_stride = p.v_page_stride = (long long)Hkv * P * D;
+  p.k_tok_stride = p.v_tok_stride = D;
+  p.k_head_stride = p.v_head_stride = (long long)P * D;
+  p.dst_pages = new_page;
+  p.pool = static_cast<uint8_t*>(pool);
+  p.pool_pages = pool_pages;
+  p.Hkv = Hkv;
+  p.P = P;
+  p.k = cfg->num_boost;
+  p.L = make_layout(P, D, cfg->num_boost, cfg->key_group);
+  p.err = err;
+  p.mode = kModeSelect | kModeKeys | kModeValues;
+  p.flush = 1;
+  p.res_len = res_len;
+  p.num_pages = num_pages;
+  p.max_pages = max_pages;
+  cudaError_t e = launch_quantize(p, batch, cfg->dtype, stream);
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  return cuda_status(launch_flush_commit(res_len, new_page, page_table, max_pages, num_pages, pool_pages, batch, P,
+                                         stream));
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages) {
+  if (kvq_check_config(cfg) != KVQ_OK || batch < 0 || max_pages < 0) return 0;
+  const Plan pl = decode_plan(cfg, batch, max_pages);
+  return pl.part_bytes + pl.cnt_bytes;
+}
+
+kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t pool_pages, const void* q,
+                                int32_t batch, const int32_t* page_table, int32_t max_pages,
+                                const int32_t* num_pages, const void* res_k, const void* res_v,
+                                const int32_t* res_len, float sm_scale, float* out, void* workspace,
+                                size_t workspace_bytes, int32_t* err, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!pool || pool_pages <= 0 || !q || !num_pages || !res_k || !res_v || !res_len || !out || !workspace)
+    return KVQ_ERR_INVALID_ARG;
+  if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(q) || !aligned16(res_k) || !aligned16(res_v) || !aligned16(workspace))
+    return KVQ_ERR_INVALID_ARG;
+  const Plan pl = decode_plan(cfg, batch, max_pages);
+  if (workspace_bytes < pl.part_bytes + pl.cnt_bytes) return KVQ_ERR_CAPACITY;
+  const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  DecodeParams p{};
+  p.pool = static_cast<const uint8_t*>(pool);
+  p.pool_pages = pool_pages;
+  p.Hkv = cfg->num_kv_heads;
+  p.P = cfg->page_tokens;
+  p.k = cfg->num_boost;
+  p.KB = cfg->num_boost / 16;
+  p.L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
+  p.rec_bytes = p.L.record;
+  p.payload = p.L.payload;
+  p.stage_bytes = uint32_t(128 / p.P) * p.L.record;
+  p.main_bytes = uint32_t(decode_main_bytes(p.P, gqa, p.L.record));
+  p.q = static_cast<const uint16_t*>(q);
+  p.batch = batch;
+  p.Hq = cfg->num_q_heads;
+  p.page_table = page_table;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.res_k = static_cast<const uint16_t*>(res_k);
+  p.res_v = static_cast<const uint16_t*>(res_v);
+  p.res_len = res_len;
+  p.c_log2 = sm_scale * 1.4426950408889634f;
+  p.out = out;
+  p.part = static_cast<float*>(workspace);
+  p.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.part_bytes);
+  p.pps = pl.split.pps;
+  p.max_splits = pl.split.max_splits;
+  p.err = err;
+  return cuda_status(launch_decode(p, gqa, cfg->dtype, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,255 @@
+// kvq_internal.cuh — shared device/host helpers of the kvq CUDA library (sm_100a).
+//
+// Record layout, launch helpers and thin inline-PTX wrappers used by the quantize
+// and decode kernels.  Nothing here is exported; the C ABI lives in include/kvq.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kKeyGroup = 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Byte offsets of one (page, kv head) record.  Section order and sizes follow the
+// page-record description in kvq.h: plane A codes, plane B codes, value codes, plane-A
+// scale and zero, plane-B scale, value scale and zero, boost indices; the stride rounds
+// the payload up to 128 bytes so records stay aligned for 16-byte vector access and
+// for bulk copies.
+struct Layout {
+  uint32_t k_codes, kb_codes, v_codes, k_scale, k_zero, kb_scale, v_scale, v_zero, boost_idx;
+  uint32_t payload, record;
+};
+
+inline Layout make_layout(int P, int D, int k, int G) {
+  Layout L;
+  uint32_t off = 0;
+  L.k_codes = off;   off += uint32_t(P) * uint32_t(D / 16) * 4u;
+  L.kb_codes = off;  off += uint32_t(P) * uint32_t(k / 16) * 4u;
+  L.v_codes = off;   off += uint32_t(D) * uint32_t(P / 16) * 4u;
+  L.k_scale = off;   off += uint32_t(P / G) * uint32_t(D) * 2u;
+  L.k_zero = off;    off += uint32_t(P / G) * uint32_t(D) * 2u;
+  L.kb_scale = off;  off += uint32_t(P / G) * uint32_t(k) * 2u;
+  L.v_scale = off;   off += uint32_t(P) * 2u;
+  L.v_zero = off;    off += uint32_t(P) * 2u;
+  L.boost_idx = off; off += uint32_t(k);
+  L.payload = off;
+  L.record = (off + 127u) / 128u * 128u;
+  return L;
+}
+
+__device__ __forceinline__ void flag_error(int32_t* err, int bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ------------------------------------------------------------------ 16-bit helpers
+
+template <typename T> struct Pair;
+template <> struct Pair<__half> { using type = __half2; };
+template <> struct Pair<__nv_bfloat16> { using type = __nv_bfloat162; };
+
+__device__ __forceinline__ float bits_to_float(uint16_t b, __half) { return __half2float(__ushort_as_half(b)); }
+__device__ __forceinline__ float bits_to_float(uint16_t b, __nv_bfloat16) {
+  return __uint_as_float(uint32_t(b) << 16);
+}
+// Rounds a float toward +infinity to the 16-bit type; returns the bits.
+__device__ __forceinline__ uint16_t round_up_bits(float x, __half) { return __half_as_ushort(__float2half_ru(x)); }
+__device__ __forceinline__ uint16_t round_up_bits(float x, __nv_bfloat16) {
+  return __bfloat16_as_ushort(__float2bfloat16_ru(x));
+}
+// Exact conversion of a representable float to the 16-bit type.
+__device__ __forceinline__ uint16_t exact_bits(float x, __half) { return __half_as_ushort(__float2half_rn(x)); }
+__device__ __forceinline__ uint16_t exact_bits(float x, __nv_bfloat16) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// ------------------------------------------------------------------ shared memory access
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t lds32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
+__device__ __forceinline__ uint2 lds64(const void* p) { return *reinterpret_cast<const uint2*>(p); }
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// ------------------------------------------------------------------ mbarrier + bulk copy
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of `parity` to complete; gives up after ~2^32 SM cycles
+// (about two seconds) and returns false so the caller can flag an error and leave.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > (1ll << 32)) return false;
+  }
+  return true;
+}
+// One contiguous global -> shared copy through the bulk-copy engine, completing on `bar`.
+// Both addresses 16-byte aligned, bytes a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+// L2 policy for data read once per launch: evicted first.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes < 16 zero-fills the rest.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ warp-level matrix ops
+
+// D += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                          __half) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                          __nv_bfloat16) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// 2^x (hardware approximation, relative error ~2^-22; -inf -> 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two 2-bit codes of a packed word as an fp16 pair for the tensor cores: pair j holds
+// elements 2j (low half) and 2j+1 (high half).  Each half keeps its code in the two
+// lowest mantissa bits of an fp16 with a zero exponent, i.e. the exact value
+// code * 2^-24; products with the other operand stay exact in fp32 and the 2^24
+// factor is restored after the contraction.  One shift and one AND per pair.
+constexpr float kCodeUnitInv = 16777216.0f;  // 2^24
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, int j) { return (w >> (2 * j)) & 0x00030003u; }
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ uint32_t bf2_as_u32(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// ------------------------------------------------------------------ launch parameters
+
+enum : int { kModeSelect = 1, kModeKeys = 2, kModeValues = 4 };
+
+// Page quantization (a1..a3) over n items; in flush mode item = sequence b and only
+// sequences whose residual window is full are quantized.
+struct QuantParams {
+  const uint16_t* k_src;
+  const uint16_t* v_src;
+  long long k_page_stride, k_tok_stride, k_head_stride;  // elements
+  long long v_page_stride, v_tok_stride, v_head_stride;
+  const int32_t* dst_pages;  // page id per item, or new_page[b] in flush mode
+  uint8_t* pool;
+  long long pool_pages;
+  int Hkv, P, k;
+  Layout L;
+  int32_t* err;
+  int mode;
+  int flush;
+  const int32_t* res_len;
+  const int32_t* num_pages;
+  int max_pages;
+};
+
+// Decode attention (a6 + a7).
+struct DecodeParams {
+  const uint8_t* pool;
+  long long pool_pages;
+  int Hkv, P, k, KB;  // KB = k / 16
+  uint32_t rec_bytes, payload, stage_bytes, main_bytes;
+  Layout L;
+  const uint16_t* q;
+  int batch, Hq;
+  const int32_t* page_table;
+  int max_pages;
+  const int32_t* num_pages;
+  const uint16_t* res_k;
+  const uint16_t* res_v;
+  const int32_t* res_len;
+  float c_log2;   // sm_scale * log2(e)
+  float* out;
+  float* part;    // [B][Hkv][max_splits][GQA][2 + 128]: max, sum, unnormalised output
+  uint32_t* cnt;  // [B][Hkv] arrival counters
+  int pps, max_splits;
+  int32_t* err;
+};
+
+struct SplitPlan {
+  int pps, max_splits;
+};
+
+cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream);
+cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, void* res_v, int32_t* res_len,
+                          int batch, int Hkv, int P, int32_t* err, cudaStream_t stream);
+cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32_t* page_table, int max_pages,
+                                int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int gqa, int dtype, cudaStream_t stream);
+SplitPlan plan_splits(int units, int max_pages, int sm_count);
+size_t decode_main_bytes(int P, int GQA, uint32_t rec_bytes);
+
+}  // namespace kvq

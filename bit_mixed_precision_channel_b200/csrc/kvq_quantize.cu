@@ -1,0 +1,326 @@
+// kvq_quantize.cu — page quantization (boost selection, two-plane keys, per-token
+// values), residual append and residual flush for sm_100a.
+//
+// One CTA quantizes one (page, kv head): it stages the page's K and V tiles
+// ([P][128] each) in shared memory with 16-byte loads, then
+//   a1  ranks channels by max |K| over the page (Kitty, Dynamic Channel-wise
+//       Precision Boost; magnitude heuristic per the notes.yuuk.io wiki page),
+//   a2  quantizes every (key group, channel) asymmetrically — 4 bits for boosted
+//       channels, split into a high plane and a low plane of 2-bit codes, 2 bits
+//       otherwise (KIVI per-channel keys; Kitty two uniform 2-bit tensors),
+//   a3  quantizes every token's values over the head dimension (KIVI per-token values),
+// and writes the packed record.  The quantizer's fp32 operations use explicit
+// round-to-nearest intrinsics in the order the ABI documents, so codes, scales and
+// zeros are bit-identical to any implementation of that definition.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+constexpr int kQThreads = 256;
+
+// Shared memory of one quantize CTA.
+struct QSmem {
+  static size_t bytes(int P, int k) {
+    return size_t(P) * kHeadDim * 2 * 2    // K and V tiles
+           + size_t(P) * kHeadDim          // plane-A codes [P][128]
+           + size_t(P) * (k > 0 ? k : 16)  // plane-B codes [P][k]
+           + size_t(P) * kHeadDim          // value codes [P][128]
+           + kHeadDim * 4 * 2 + 16 * 4;    // scores, plane-B row of each channel, warp counts
+  }
+};
+
+__device__ __forceinline__ uint32_t pack16(const uint8_t* c) {
+  // 16 codes -> one word: element e at bit 16*(e & 1) + 2*(e >> 1).
+  const uint4 v = lds128(c);
+  const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t x = q[i];  // elements 4i .. 4i+3, one per byte
+    const uint32_t part = (x & 0x3u) | ((x >> 14) & 0xCu) | ((x << 8) & 0x30000u) | ((x >> 6) & 0xC0000u);
+    w |= part << (4 * i);
+  }
+  return w;
+}
+
+// Quantizes one group with the documented fp32 op order; returns the scale as float
+// and writes scale/zero bits.  min/max are exact; a zero minimum is stored as +0.
+template <typename T>
+__device__ __forceinline__ float quant_params(float mn, float mx, int qmax, uint16_t& sbits, uint16_t& zbits,
+                                              float& zero) {
+  const float range = __fsub_rn(mx, mn);
+  const float s32 = __fdiv_rn(range, float(qmax));
+  sbits = round_up_bits(s32, T());
+  zero = __fadd_rn(mn, 0.0f);  // -0 -> +0
+  zbits = exact_bits(zero, T());
+  return bits_to_float(sbits, T());
+}
+
+__device__ __forceinline__ int quant_code(float x, float zero, float scale, int qmax) {
+  if (scale == 0.0f) return 0;
+  const float t = __fdiv_rn(__fsub_rn(x, zero), scale);
+  float r = rintf(t);
+  r = fminf(fmaxf(r, 0.0f), float(qmax));
+  return int(r);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p) {
+  const int item = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int P = p.P, k = p.k;
+  int dst;
+  if (p.flush) {
+    if (p.res_len[item] != P) return;
+    dst = p.dst_pages[item];
+    const int np = p.num_pages[item];
+    if (dst < 0 || np < 0 || np >= p.max_pages) {
+      if (tid == 0 && h == 0) flag_error(p.err, KVQ_DEV_ERR_TABLE_FULL);
+      return;
+    }
+  } else {
+    dst = p.dst_pages[item];
+  }
+  if (dst < 0 || dst >= p.pool_pages) {
+    if (tid == 0) flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
+    return;
+  }
+  uint8_t* rec = p.pool + (size_t(dst) * p.Hkv + h) * p.L.record;
+
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* Vs = Ks + P * kHeadDim;
+  uint8_t* cA = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);
+  uint8_t* cB = cA + P * kHeadDim;
+  uint8_t* cV = cB + P * (k > 0 ? k : 16);
+  float* score = reinterpret_cast<float*>(cV + P * kHeadDim);
+  int* row_of = reinterpret_cast<int*>(score + kHeadDim);
+  int* warp_cnt = row_of + kHeadDim;
+
+  const bool need_k = p.mode & (kModeSelect | kModeKeys);
+  const bool need_v = p.mode & kModeValues;
+
+  // ---- stage the page tiles (rows of 128 x 16-bit = 16 x 16 bytes)
+  if (need_k) {
+    const uint16_t* src = p.k_src + item * p.k_page_stride + h * p.k_head_stride;
+    for (int i = tid; i < P * 16; i += kQThreads) {
+      const int t = i >> 4, c = i & 15;
+      reinterpret_cast<uint4*>(Ks)[i] = __ldg(reinterpret_cast<const uint4*>(src + t * p.k_tok_stride) + c);
+    }
+  }
+  if (need_v) {
+    const uint16_t* src = p.v_src + item * p.v_page_stride + h * p.v_head_stride;
+    for (int i = tid; i < P * 16; i += kQThreads) {
+      const int t = i >> 4, c = i & 15;
+      reinterpret_cast<uint4*>(Vs)[i] = __ldg(reinterpret_cast<const uint4*>(src + t * p.v_tok_stride) + c);
+    }
+  }
+  __syncthreads();
+
+  // ---- a1: boosted channels (or read them back from the record)
+  if (p.mode & kModeSelect) {
+    if (tid < kHeadDim) {
+      float m = 0.0f;
+      for (int t = 0; t < P; ++t) m = fmaxf(m, fabsf(bits_to_float(Ks[t * kHeadDim + tid], T())));
+      score[tid] = m;
+    }
+    __syncthreads();
+    if (tid < kHeadDim) {
+      const float s = score[tid];
+      int rank = 0;
+      for (int c = 0; c < kHeadDim; ++c) {
+        const float o = score[c];
+        rank += (o > s) || (o == s && c < tid);
+      }
+      const bool boosted = rank < k;
+      const unsigned ballot = __ballot_sync(kFull, boosted);
+      if ((tid & 31) == 0) warp_cnt[tid >> 5] = __popc(ballot);
+      __syncwarp();
+      row_of[tid] = boosted ? int(__popc(ballot & ((1u << (tid & 31)) - 1u))) : -1;
+    }
+    __syncthreads();
+    if (tid < kHeadDim && row_of[tid] >= 0) {
+      int before = 0;
+      for (int w = 0; w < (tid >> 5); ++w) before += warp_cnt[w];
+      row_of[tid] += before;
+      rec[p.L.boost_idx + row_of[tid]] = uint8_t(tid);
+    }
+    __syncthreads();
+  } else if (p.mode & kModeKeys) {
+    if (tid < kHeadDim) row_of[tid] = -1;
+    __syncthreads();
+    if (tid < k) {
+      const int c = rec[p.L.boost_idx + tid];
+      if (c < kHeadDim) row_of[c] = tid;
+    }
+    __syncthreads();
+  }
+
+  // ---- a2: keys, one task per (group, channel)
+  if (p.mode & kModeKeys) {
+    const int n_groups = P / kKeyGroup;
+    uint16_t* ks_out = reinterpret_cast<uint16_t*>(rec + p.L.k_scale);
+    uint16_t* kz_out = reinterpret_cast<uint16_t*>(rec + p.L.k_zero);
+    uint16_t* kbs_out = reinterpret_cast<uint16_t*>(rec + p.L.kb_scale);
+    for (int task = tid; task < n_groups * kHeadDim; task += kQThreads) {
+      const int g = task / kHeadDim, c = task % kHeadDim;
+      const uint16_t* col = Ks + g * kKeyGroup * kHeadDim + c;
+      float mn = bits_to_float(col[0], T()), mx = mn;
+      for (int t = 1; t < kKeyGroup; ++t) {
+        const float v = bits_to_float(col[t * kHeadDim], T());
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+      }
+      const int j = row_of[c];
+      const int qmax = j >= 0 ? 15 : 3;
+      uint16_t sb, zb;
+      float zero;
+      const float scale = quant_params<T>(mn, mx, qmax, sb, zb, zero);
+      for (int t = 0; t < kKeyGroup; ++t) {
+        const int tok = g * kKeyGroup + t;
+        const int code = quant_code(bits_to_float(col[t * kHeadDim], T()), zero, scale, qmax);
+        if (j >= 0) {
+          cA[tok * kHeadDim + c] = uint8_t(code >> 2);
+          cB[tok * k + j] = uint8_t(code & 3);
+        } else {
+          cA[tok * kHeadDim + c] = uint8_t(code);
+        }
+      }
+      // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
+      ks_out[g * kHeadDim + c] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
+      kz_out[g * kHeadDim + c] = zb;
+      if (j >= 0) kbs_out[g * k + j] = sb;
+    }
+  }
+
+  // ---- a3: values, one warp per token
+  if (need_v) {
+    const int warp = tid >> 5, lane = tid & 31;
+    uint16_t* vs_out = reinterpret_cast<uint16_t*>(rec + p.L.v_scale);
+    uint16_t* vz_out = reinterpret_cast<uint16_t*>(rec + p.L.v_zero);
+    for (int t = warp; t < P; t += kQThreads / 32) {
+      const uint2 raw = lds64(Vs + t * kHeadDim + 4 * lane);
+      float x[4] = {bits_to_float(uint16_t(raw.x & 0xffff), T()), bits_to_float(uint16_t(raw.x >> 16), T()),
+                    bits_to_float(uint16_t(raw.y & 0xffff), T()), bits_to_float(uint16_t(raw.y >> 16), T())};
+      float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+      }
+      uint16_t sb, zb;
+      float zero;
+      const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
+      uint32_t four = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) four |= uint32_t(quant_code(x[i], zero, scale, 3)) << (8 * i);
+      *reinterpret_cast<uint32_t*>(cV + t * kHeadDim + 4 * lane) = four;
+      if (lane == 0) {
+        vs_out[t] = sb;
+        vz_out[t] = zb;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- pack the code planes into the record
+  if (p.mode & kModeKeys) {
+    uint32_t* kA = reinterpret_cast<uint32_t*>(rec + p.L.k_codes);
+    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) kA[i] = pack16(cA + 16 * i);
+    const int kbw = k / 16;
+    uint32_t* kB = reinterpret_cast<uint32_t*>(rec + p.L.kb_codes);
+    for (int i = tid; i < P * kbw; i += kQThreads) kB[i] = pack16(cB + 16 * i);
+  }
+  if (need_v) {
+    uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
+    const int vw = P / 16;
+    for (int i = tid; i < kHeadDim * vw; i += kQThreads) {
+      // word (channel c, w) holds tokens 16w .. 16w+15 of channel c
+      const int c = i / vw, w = i % vw;
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        word |= uint32_t(cV[(16 * w + e) * kHeadDim + c] & 3u) << (16 * (e & 1) + 2 * (e >> 1));
+      vq[i] = word;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ residual window
+
+// a4: append one token per sequence at position res_len[b], then res_len[b] += 1.
+// One CTA per sequence; every head's K and V row is 256 bytes (16 x 16 bytes).
+__global__ void __launch_bounds__(256) append_kernel(const uint4* k_new, const uint4* v_new, uint4* res_k,
+                                                     uint4* res_v, int32_t* res_len, int Hkv, int P,
+                                                     int32_t* err) {
+  const int b = blockIdx.x;
+  __shared__ int s_r;
+  if (threadIdx.x == 0) s_r = res_len[b];
+  __syncthreads();
+  const int r = s_r;
+  if (r < 0 || r >= P) {
+    if (threadIdx.x == 0) flag_error(err, r >= P ? KVQ_DEV_ERR_RESIDUAL : KVQ_DEV_ERR_LENGTH);
+    return;
+  }
+  const int n = Hkv * 16;
+  for (int i = threadIdx.x; i < 2 * n; i += blockDim.x) {
+    const int which = i / n, j = i % n, h = j >> 4, c = j & 15;
+    const uint4* src = which ? v_new : k_new;
+    uint4* dst = which ? res_v : res_k;
+    dst[((size_t(b) * Hkv + h) * P + r) * 16 + c] = src[(size_t(b) * Hkv + h) * 16 + c];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) res_len[b] = r + 1;
+}
+
+// a5 (second half): after the full windows were quantized into their new pages, link
+// the pages and empty the windows.  Uses the same predicate as the quantize launch, so a
+// sequence skipped there (bad page id, full table) is skipped here too.
+__global__ void flush_commit_kernel(int32_t* res_len, const int32_t* new_page, int32_t* page_table,
+                                    int max_pages, int32_t* num_pages, long long pool_pages, int batch,
+                                    int P) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+    if (res_len[b] != P) continue;
+    const int dst = new_page[b], np = num_pages[b];
+    if (dst < 0 || np < 0 || np >= max_pages || dst >= pool_pages) continue;
+    page_table[size_t(b) * max_pages + np] = dst;
+    num_pages[b] = np + 1;
+    res_len[b] = 0;
+  }
+}
+
+// ------------------------------------------------------------------ host launchers
+
+cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream) {
+  if (n_items <= 0) return cudaSuccess;
+  const size_t smem = QSmem::bytes(p.P, p.k);
+  const dim3 grid(n_items, p.Hkv);
+  if (dtype == KVQ_BF16) {
+    cudaFuncSetAttribute(quantize_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    quantize_kernel<__nv_bfloat16><<<grid, kQThreads, smem, stream>>>(p);
+  } else {
+    cudaFuncSetAttribute(quantize_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    quantize_kernel<__half><<<grid, kQThreads, smem, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, void* res_v, int32_t* res_len,
+                          int batch, int Hkv, int P, int32_t* err, cudaStream_t stream) {
+  if (batch <= 0) return cudaSuccess;
+  append_kernel<<<batch, 256, 0, stream>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                                           static_cast<uint4*>(res_k), static_cast<uint4*>(res_v), res_len, Hkv,
+                                           P, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32_t* page_table, int max_pages,
+                                int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream) {
+  if (batch <= 0) return cudaSuccess;
+  const int threads = 256, blocks = (batch + threads - 1) / threads;
+  flush_commit_kernel<<<blocks, threads, 0, stream>>>(res_len, new_page, page_table, max_pages, num_pages,
+                                                      pool_pages, batch, P);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

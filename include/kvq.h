@@ -28,7 +28,7 @@
  *   mn = min x, mx = max x                         (exact; compared after widening to fp32)
  *   s32 = fp32(mx - mn) / (2^b - 1)                (fp32, round-to-nearest-even divide)
  *   scale = s32 rounded toward +infinity to dtype   (so scale*(2^b-1) >= mx-mn)
- *   zero  = mn                                      (stored in dtype, exact)
+ *   zero  = mn                                      (stored in dtype, exact; a zero minimum as +0)
  *   code  = clamp(rint(fp32(x - zero) / fp32(scale)), 0, 2^b-1)
  *           (fp32 subtract, fp32 divide, rint = round half to even); code = 0 if scale == 0
  *   dequantized value = code * scale + zero
@@ -76,8 +76,8 @@
  *
  * Ownership, streams and errors
  * -----------------------------
- * Every buffer is allocated and owned by the caller.  Pointers named *_h are host
- * pointers; every other pointer is a device pointer.  Every call is enqueued on the
+ * Every buffer is allocated and owned by the caller; every pointer argument is a
+ * device pointer (16-byte aligned where it is read in vectors).  Every call is enqueued on the
  * given stream and returns before the device work finishes.  Arguments are checked
  * on the host before any launch; on a failed check nothing is enqueued and the
  * status says why.  Faults that only the device can see (a page id outside the pool,
@@ -92,6 +92,13 @@
 #include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
+
+/* Every entry point is exported with default visibility; the rest of the library is hidden. */
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
 
 #ifdef __cplusplus
 extern "C" {
@@ -140,16 +147,16 @@ typedef struct {
 } kvq_layout;
 
 /* Human-readable text for a status code (static storage, never NULL). */
-const char* kvq_status_string(kvq_status s);
+KVQ_API const char* kvq_status_string(kvq_status s);
 
 /* Checks a configuration without touching the GPU. */
-kvq_status kvq_check_config(const kvq_config* cfg);
+KVQ_API kvq_status kvq_check_config(const kvq_config* cfg);
 
 /* Fills *out with the record layout of cfg. Host only; no CUDA call. */
-kvq_status kvq_page_layout(const kvq_config* cfg, kvq_layout* out);
+KVQ_API kvq_status kvq_page_layout(const kvq_config* cfg, kvq_layout* out);
 
 /* Record stride in bytes for cfg, or 0 if cfg is not supported. */
-size_t kvq_page_bytes(const kvq_config* cfg);
+KVQ_API size_t kvq_page_bytes(const kvq_config* cfg);
 
 /* Source of whole pages for the quantize calls.  Element (page i, token t, kv head h,
  * channel c) is read at src[i*page_stride + t*token_stride + h*head_stride + c]
@@ -167,7 +174,7 @@ typedef struct {
  * of k and each KV head, ranks the channels by max |K| over the page and writes the
  * num_boost highest (ties to the lower index) in ascending order into the boost_idx
  * section of record (dst_pages[i], h).  dst_pages: device int32[n_pages]. */
-kvq_status kvq_select_boost_channels(const kvq_config* cfg, kvq_source k,
+KVQ_API kvq_status kvq_select_boost_channels(const kvq_config* cfg, kvq_source k,
                                      const int32_t* dst_pages, int32_t n_pages,
                                      void* pool, int64_t pool_pages, int32_t* err,
                                      cudaStream_t stream);
@@ -176,19 +183,19 @@ kvq_status kvq_select_boost_channels(const kvq_config* cfg, kvq_source k,
  * Kitty abstract: each mixed-precision Key page becomes two unified 2-bit tensors).
  * Reads boost_idx from the destination records (written by
  * kvq_select_boost_channels) and writes k_codes, kb_codes, k_scale, k_zero, kb_scale. */
-kvq_status kvq_quantize_page_keys(const kvq_config* cfg, kvq_source k,
+KVQ_API kvq_status kvq_quantize_page_keys(const kvq_config* cfg, kvq_source k,
                                   const int32_t* dst_pages, int32_t n_pages,
                                   void* pool, int64_t pool_pages, int32_t* err,
                                   cudaStream_t stream);
 
 /* a3 — per-token Value quantization (KIVI section 3).  Writes v_codes, v_scale, v_zero. */
-kvq_status kvq_quantize_values(const kvq_config* cfg, kvq_source v,
+KVQ_API kvq_status kvq_quantize_values(const kvq_config* cfg, kvq_source v,
                                const int32_t* dst_pages, int32_t n_pages,
                                void* pool, int64_t pool_pages, int32_t* err,
                                cudaStream_t stream);
 
 /* a1+a2+a3 in one pass over each page: the same bytes as the three calls above. */
-kvq_status kvq_quantize_pages(const kvq_config* cfg, kvq_source k, kvq_source v,
+KVQ_API kvq_status kvq_quantize_pages(const kvq_config* cfg, kvq_source k, kvq_source v,
                               const int32_t* dst_pages, int32_t n_pages,
                               void* pool, int64_t pool_pages, int32_t* err,
                               cudaStream_t stream);
@@ -199,7 +206,7 @@ kvq_status kvq_quantize_pages(const kvq_config* cfg, kvq_source k, kvq_source v,
  * token at position res_len[b] of res_k/res_v and increments res_len[b].  A sequence
  * whose window is already full (res_len[b] == page_tokens) is skipped and raises
  * KVQ_DEV_ERR_RESIDUAL: flush first. */
-kvq_status kvq_append_token(const kvq_config* cfg, int32_t batch,
+KVQ_API kvq_status kvq_append_token(const kvq_config* cfg, int32_t batch,
                             const void* k_new, const void* v_new,
                             void* res_k, void* res_v, int32_t* res_len,
                             int32_t* err, cudaStream_t stream);
@@ -213,7 +220,7 @@ kvq_status kvq_append_token(const kvq_config* cfg, int32_t batch,
  * flushes; a negative id or a full table raises KVQ_DEV_ERR_TABLE_FULL and skips b).
  * The caller decides which sequences will flush (it issued the appends), so the call
  * needs no device-to-host read and can be captured in a CUDA graph. */
-kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
+KVQ_API kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
                               const void* res_k, const void* res_v, int32_t* res_len,
                               const int32_t* new_page, int32_t* page_table,
                               int32_t max_pages, int32_t* num_pages,
@@ -224,7 +231,7 @@ kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
  * workspace holds split-K partial results and one arrival counter per
  * (sequence, KV head).  The counters must be zero before the first call (clear the
  * whole workspace once after allocating it); every call leaves them zero again. */
-size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages);
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages);
 
 /* a6 + a7 — decode attention over the paged, packed cache plus the residual window
  * (Kitty abstract: page dequantization kernels over a page-centric layout; MiniKV
@@ -239,8 +246,11 @@ size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t 
  * workspace: device, >= kvq_decode_workspace_bytes(cfg, batch, max_pages) bytes,
  * see kvq_decode_workspace_bytes for its zero-counter contract.
  * A sequence with no tokens at all (num_pages[b] == 0 and res_len[b] == 0) gets an
- * all-zero output row. */
-kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t pool_pages,
+ * all-zero output row.
+ * Precision: inside the kernel q*scale (keys) and p*scale (values) are carried as an
+ * fp16 high part plus an fp16 low part, so |q| * key scale must stay below the fp16
+ * maximum (65504); codes are exact.  Accumulation is fp32. */
+KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t pool_pages,
                                 const void* q, int32_t batch,
                                 const int32_t* page_table, int32_t max_pages,
                                 const int32_t* num_pages,
