@@ -1,0 +1,502 @@
+"""Benchmark of the 2-bit mixed-precision KV cache decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+Workload (one GPU): the Llama-3-8B-shaped decode layer — batch 16, 32 query / 8 KV
+heads, head_dim 128, 4096-token prompts in pages of 128, 32 boosted key channels of
+128 (25%), fp16 — replicated over 32 layers, as a decode step of that model walks its
+32 layers.  The 32 layer caches (1.6 GB of packed KV) are far larger than the 126 MB
+L2, so every step reads its pages from HBM.  Inputs are seeded synthetic tensors
+(see bit_mixed_precision_channel_b200/synthetic.py).
+
+A step = for every layer: append the new token to the residual window, flush full
+windows, decode attention over pages + window (all rows of the hot path; the prompt
+pages were quantized once at prefill, whose rate is reported as "quantize").  The step
+is captured once in a CUDA graph and replayed.
+
+value: decode-attention algorithmic bytes of all layers / step time (GB/s), whole job
+(summed over ranks for N > 1, each rank running its own batch: weak scaling).
+roofline: the decode kernel alone, timed over L launches per replay in its own loop.
+e2e: the same step driven from host buffers: q, k_new, v_new copied in from pinned
+memory and the output copied back, inside the timed region.
+cpu_baseline / --impl reference: the CPU oracle (oracle/, fp64 attention) timed on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOAD = "llama3_8b"
+LAYERS = 32
+METRIC = "2-bit KV decode-attn GB/s & % of HBM peak; quantize tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ workload bytes
+
+def decode_bytes(w, payload, n_pages, res_len):
+    """Algorithmic bytes of one decode-attention launch (one layer): packed pages
+    (codes + scales + zeros + boost indices), the fp16 residual K and V, the query,
+    the fp32 output and the page table entries."""
+    B, Hkv, Hq, D = w.batch, w.Hkv, w.Hq, w.D
+    return (B * Hkv * n_pages * payload + B * Hkv * res_len * 2 * D * 2 + B * Hq * D * 2 + B * Hq * D * 4
+            + 4 * B * n_pages + 8 * B)
+
+
+# ------------------------------------------------------------------ clocks during timing
+
+_CLOCK_POLLER = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+out = open(sys.argv[2], "w")
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+while True:
+    try:
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        out.write(f"{time.time():.4f} {sm} {mx} {r}\n"); out.flush()
+    except Exception as e:
+        out.write(f"# {e}\n"); out.flush()
+    time.sleep(0.002)
+"""
+
+REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+           0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle", 0x2: "applications_clocks_setting",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, uuid: str):
+        self.path = tempfile.mktemp(prefix="kvq_clocks_", suffix=".txt")
+        self.proc = subprocess.Popen([sys.executable, "-c", _CLOCK_POLLER, uuid, self.path],
+                                     stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        self.t0 = self.t1 = None
+
+    def wait_ready(self, timeout=20.0):
+        t = time.time()
+        while time.time() - t < timeout:
+            if os.path.exists(self.path) and os.path.getsize(self.path) > 0:
+                return True
+            time.sleep(0.05)
+        return False
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    if line.startswith("#"):
+                        continue
+                    t, sm, mx, r = line.split()
+                    rows.append((float(t), int(sm), int(mx), int(r)))
+            os.unlink(self.path)
+        except OSError:
+            pass
+        sel = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": rows[0][2] if rows else None, "reasons": [], "samples": 0}
+        mask = 0
+        for r in sel:
+            mask |= r[3]
+        reasons = [name for bit, name in REASONS.items() if mask & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": sel[0][2], "reasons": reasons,
+                "samples": len(sel)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_baseline(w, K, V, res_k_host, res_v_host, res_len, q_host, budget_s=12.0, threads=None):
+    """The oracle (oracle/, plain C, fp64 attention) on the host cores: decode attention
+    of whole units (sequence, kv head) of one layer, repeated over the units of the
+    step until ~budget_s of wall time; returns GB/s over the same algorithmic bytes."""
+    import concurrent.futures as cf
+
+    import oracle
+
+    oc = oracle.Cfg(D=w.D, Hq=w.Hq, Hkv=w.Hkv, P=w.P, G=w.G, k=w.k, dtype=w.dtype)
+    P = w.P
+    n_pages = K.shape[1] // P
+    payload = oracle.layout(P, w.D, w.k, w.G)["payload_bytes"]
+    threads = threads or max(1, min(os.cpu_count() or 1, 32))
+    units = [(b, h) for b in range(w.batch) for h in range(w.Hkv)]
+    pools = {}
+
+    def quant(b):
+        pool = np.zeros((n_pages, w.Hkv, oc.record_bytes), np.uint8)
+        for i in range(n_pages):
+            for h in range(w.Hkv):
+                pool[i, h] = oracle.quantize_page(K[b, i * P:(i + 1) * P, h], V[b, i * P:(i + 1) * P, h], oc)
+        return b, pool
+
+    with cf.ThreadPoolExecutor(threads) as ex:
+        for b, pool in ex.map(quant, range(w.batch)):
+            pools[b] = pool
+    g = w.gqa
+    sm = 1.0 / math.sqrt(w.D)
+
+    def unit(bh):
+        b, h = bh
+        return oracle.decode_unit(pools[b], oc, h, list(range(n_pages)), res_k_host[b, h, :res_len],
+                                  res_v_host[b, h, :res_len], q_host[b, h * g:(h + 1) * g], sm)
+
+    per_unit = payload * n_pages + res_len * 2 * w.D * 2 + g * w.D * 6 + 4 * n_pages
+    done = 0
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(threads) as ex:
+        while time.perf_counter() - t0 < budget_s:
+            list(ex.map(unit, units))
+            done += len(units)
+    dt = time.perf_counter() - t0
+    return {"value": per_unit * done / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} (sequence, kv head) decode units of one layer ({done // len(units)} full "
+                      f"passes over the {len(units)} units), fp64 attention over {n_pages} pages + "
+                      f"{res_len} residual tokens each, {dt:.1f} s on {threads} threads"}
+
+
+# ------------------------------------------------------------------ GPU benchmark
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_mixed_precision_channel_b200 import binding as kb
+    from bit_mixed_precision_channel_b200 import synthetic as syn
+    from bit_mixed_precision_channel_b200.cache import PagedKVCache
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = syn.WORKLOADS[WORKLOAD]
+    L_layers = args.layers
+    cfg = kb.Config(head_dim=w.D, num_q_heads=w.Hq, num_kv_heads=w.Hkv, page_tokens=w.P, key_group=w.G,
+                    num_boost=w.k, dtype=w.dtype)
+    B, P, D = w.batch, w.P, w.D
+    n_pages = w.context // P
+    total_steps = args.warmup + args.steps + 3
+    max_pages = n_pages + total_steps // P + 2
+    pool_pages = B * max_pages
+    payload = kb.page_layout(cfg)["payload_bytes"]
+    tdt = kb.torch_dtype(w.dtype)
+
+    def dev_bits(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(tdt).to(dev)
+
+    # -------- prompts (the same synthetic prompt for every layer replica; each layer has its own cache)
+    sigma = syn.key_channel_sigma(w)
+    Kh = np.stack([syn.keys(w, b + 1000 * rank, 0, w.context, sigma) for b in range(B)])
+    Vh = np.stack([syn.values(w, b + 1000 * rank, 0, w.context) for b in range(B)])
+    Kd, Vd = dev_bits(Kh), dev_bits(Vh)
+    caches = [PagedKVCache(cfg, B, max_pages, pool_pages, device=dev) for _ in range(L_layers)]
+
+    # quantize leg: prefill of every layer, one launch per layer, timed
+    caches[0].prefill_batch(Kd, Vd)  # warm-up launch (first-call attribute setup)
+    caches[0] = PagedKVCache(cfg, B, max_pages, pool_pages, device=dev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for c in caches:
+        c.prefill_batch(Kd, Vd)
+    e1.record()
+    torch.cuda.synchronize()
+    q_ms = e0.elapsed_time(e1) / L_layers
+    quant_tokens_per_s = B * w.context / (q_ms * 1e-3)
+    quant_bytes = B * w.context * w.Hkv * D * 2 * 2 + B * n_pages * w.Hkv * payload
+    for c in caches:
+        assert c.check_errors() == 0
+
+    # -------- per-layer decode inputs (static buffers the graph reads)
+    kn, vn = syn.step_tokens(w, 0, sigma)
+    qh = syn.queries(w, 0)
+    qs = [dev_bits(qh) for _ in range(L_layers)]
+    kns = [dev_bits(kn) for _ in range(L_layers)]
+    vns = [dev_bits(vn) for _ in range(L_layers)]
+    outs = [torch.empty(B, w.Hq, D, device=dev) for _ in range(L_layers)]
+
+    def device_step():
+        for i, c in enumerate(caches):
+            c.append(kns[i], vns[i])
+            c.flush()
+            c.attend(qs[i], outs[i])
+
+    def attend_only():
+        for i, c in enumerate(caches):
+            c.attend(qs[i], outs[i])
+
+    def host_step(flag_list):
+        for i, c in enumerate(caches):
+            flag_list[i] = c.reserve_flush_pages()
+
+    def host_commit(flag_list):
+        for i, c in enumerate(caches):
+            c.commit_host(flag_list[i])
+
+    flags = [None] * L_layers
+    # eager warm-up (also sets kernel attributes before capture)
+    for _ in range(2):
+        host_step(flags)
+        device_step()
+        host_commit(flags)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    g_step, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        device_step()
+    with torch.cuda.graph(g_attn, stream=stream):
+        attend_only()
+    # e2e: host buffers in pinned memory, copies inside the graph
+    q_pin = [torch.from_numpy(qh.view(np.int16)).view(tdt).pin_memory() for _ in range(L_layers)]
+    kn_pin = [torch.from_numpy(kn.view(np.int16)).view(tdt).pin_memory() for _ in range(L_layers)]
+    vn_pin = [torch.from_numpy(vn.view(np.int16)).view(tdt).pin_memory() for _ in range(L_layers)]
+    out_pin = [torch.empty(B, w.Hq, D).pin_memory() for _ in range(L_layers)]
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=stream):
+        for i, c in enumerate(caches):
+            qs[i].copy_(q_pin[i], non_blocking=True)
+            kns[i].copy_(kn_pin[i], non_blocking=True)
+            vns[i].copy_(vn_pin[i], non_blocking=True)
+            c.append(kns[i], vns[i])
+            c.flush()
+            c.attend(qs[i], outs[i])
+            out_pin[i].copy_(outs[i], non_blocking=True)
+    h2d_bytes = L_layers * (qh.nbytes + kn.nbytes + vn.nbytes)
+    d2h_bytes = L_layers * B * w.Hq * D * 4
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(graph, n, warm, advance):
+        for _ in range(warm):
+            if advance:
+                host_step(flags)
+            graph.replay()
+            if advance:
+                host_commit(flags)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            if advance:
+                host_step(flags)
+            graph.replay()
+            if advance:
+                host_commit(flags)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return a.elapsed_time(b) / n  # ms per replay
+
+    def snapshot():
+        return ([c.res_len.clone() for c in caches], [list(c.host_res_len) for c in caches])
+
+    def restore(s):
+        for c, r, h in zip(caches, s[0], s[1]):
+            c.res_len.copy_(r)
+            c.host_res_len = list(h)
+
+    snap = snapshot()
+    res0 = caches[0].host_res_len[0]
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    clocks.wait_ready()
+    with torch.cuda.stream(stream):
+        # main timed region: K decode steps over all layers
+        for _ in range(args.warmup):
+            host_step(flags)
+            g_step.replay()
+            host_commit(flags)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        clocks.mark_start()
+        ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_a.record(stream)
+        for _ in range(args.steps):
+            host_step(flags)
+            g_step.replay()
+            host_commit(flags)
+        ev_b.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark_end()
+        barrier()
+        step_ms = ev_a.elapsed_time(ev_b) / args.steps
+    clock_info = clocks.stop()
+    res_avg = res0 + args.warmup + (args.steps - 1) / 2 + 1  # residual length during the timed steps
+    res_end = caches[0].host_res_len[0]
+    for c in caches:
+        assert c.check_errors() == 0, "device error flags set"
+
+    with torch.cuda.stream(stream):
+        attn_ms = timed(g_attn, max(args.steps, 20), 3, advance=False) / L_layers
+        restore(snap)
+        e2e_ms = timed(g_e2e, args.steps, args.warmup, advance=True)
+    restore(snap)
+
+    bytes_step = L_layers * decode_bytes(w, payload, n_pages, res_avg)
+    bytes_attn = decode_bytes(w, payload, n_pages, res_end)
+    t = torch.tensor([step_ms, e2e_ms, attn_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, e2e_ms, attn_ms = [float(x) for x in t.tolist()]
+    peak, peak_kind = peaks()
+    value = world * bytes_step / (step_ms * 1e-3) / 1e9
+    e2e_value = world * bytes_step / (e2e_ms * 1e-3) / 1e9
+    achieved = bytes_attn / (attn_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": f"Llama-3-8B-shaped decode: batch {B} per GPU, {w.Hq} q / {w.Hkv} kv heads, "
+                               f"head_dim {D}, {w.context}-token prompts in pages of {P}, {w.k} of {D} key "
+                               f"channels boosted to 4 bit, residual window {P}, {L_layers} layers per step",
+                   "global_batch": B * world, "layers": L_layers, "seq_len": w.context,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {L_layers} layer caches, "
+                         f"{L_layers * B * w.Hkv * n_pages * payload / 1e9:.2f} GB of packed pages per GPU"},
+        "hbm_frac": round(value / world / peak, 4),
+        "quantize": {"tokens_per_s": round(quant_tokens_per_s, 1), "ms_per_layer": round(q_ms, 4),
+                     "gbs": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
+                     "what": f"prefill of {B} x {w.context} tokens into pages (select + keys + values), per layer"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "decode_kernel<__half,4>", "peak_source": peak_kind,
+                     "per_launch_bytes": bytes_attn, "ms_per_launch": round(attn_ms, 5)},
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": args.steps * L_layers * 4,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # every step appended the same k_new / v_new, so the windows hold copies of them
+        rk = np.repeat(kn[:, :, None, :], res_end, axis=2)
+        rv = np.repeat(vn[:, :, None, :], res_end, axis=2)
+        result["cpu_baseline"] = cpu_baseline(w, Kh, Vh, rk, rv, res_end, qh)
+    if world > 1:
+        dist.barrier()
+        del g_step, g_attn, g_e2e
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    """The oracle as the reference implementation: each step decodes a bounded sample
+    (8 sequence x kv-head units) of the same workload on the host cores."""
+    import concurrent.futures as cf
+
+    import oracle
+    from bit_mixed_precision_channel_b200 import synthetic as syn
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    w = syn.WORKLOADS[WORKLOAD]
+    oc = oracle.Cfg(D=w.D, Hq=w.Hq, Hkv=w.Hkv, P=w.P, G=w.G, k=w.k, dtype=w.dtype)
+    P, D, g = w.P, w.D, w.gqa
+    n_pages = w.context // P
+    sigma = syn.key_channel_sigma(w)
+    threads = max(1, min(os.cpu_count() or 1, 32))
+    units = [(b, h) for b in range(2) for h in range(w.Hkv)][:8]
+    Ks = {b: syn.keys(w, b, 0, w.context, sigma) for b in {u[0] for u in units}}
+    Vs = {b: syn.values(w, b, 0, w.context) for b in Ks}
+    pools = {}
+    for b in Ks:
+        pool = np.zeros((n_pages, w.Hkv, oc.record_bytes), np.uint8)
+        for i in range(n_pages):
+            for h in range(w.Hkv):
+                pool[i, h] = oracle.quantize_page(Ks[b][i * P:(i + 1) * P, h], Vs[b][i * P:(i + 1) * P, h], oc)
+        pools[b] = pool
+    kn, _ = syn.step_tokens(w, 0, sigma)
+    q = syn.queries(w, 0)
+    sm = 1.0 / math.sqrt(D)
+    payload = oracle.layout(P, D, w.k, w.G)["payload_bytes"]
+    res_len = 1
+
+    def unit(bh):
+        b, h = bh
+        rk = kn[b, h][None]
+        return oracle.decode_unit(pools[b], oc, h, list(range(n_pages)), rk, rk, q[b, h * g:(h + 1) * g], sm)
+
+    per_unit = payload * n_pages + res_len * 2 * D * 2 + g * D * 6 + 4 * n_pages
+    with cf.ThreadPoolExecutor(threads) as ex:
+        for _ in range(args.warmup):
+            list(ex.map(unit, units))
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            list(ex.map(unit, units))
+        dt = time.perf_counter() - t0
+    value = per_unit * len(units) * args.steps / dt / 1e9
+    sample = (f"{len(units)} (sequence, kv head) decode units of one layer per step, fp64 attention over "
+              f"{n_pages} pages + {res_len} residual token, {threads} threads")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Llama-3-8B-shaped decode layer (batch 16, 32 q / 8 kv heads, head_dim 128, "
+                                   "4096-token prompts, pages of 128, 25% boost), CPU oracle on a sample of units"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

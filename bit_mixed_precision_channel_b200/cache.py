@@ -40,9 +40,12 @@ class PagedKVCache:
         self.new_page = torch.full((batch,), -1, dtype=torch.int32, device=self.device)
         # host mirrors used to hand out pages
         order = list(range(pool_pages)) if page_order is None else [int(x) for x in page_order]
+        if sorted(order) != list(range(pool_pages)):
+            raise ValueError("page_order must be a permutation of range(pool_pages)")
         self.free = order[::-1]  # pop() hands out order[0] first
         self.host_pages = [[] for _ in range(batch)]
         self.host_res_len = [0] * batch
+        self.host_new_page = [-1] * batch  # what the device new_page buffer holds
 
     # ---------------------------------------------------------------- allocation
     def take_pages(self, n: int) -> list:
@@ -75,25 +78,47 @@ class PagedKVCache:
         self.res_len[b] = r
         self.host_res_len[b] = r
 
+    def prefill_batch(self, k: torch.Tensor, v: torch.Tensor, stream=None):
+        """All sequences at once with the same prompt length L (a multiple of P):
+        k, v: [B][L][Hkv][D] contiguous.  One quantize launch for every page."""
+        B, L = k.shape[0], k.shape[1]
+        P = self.cfg.page_tokens
+        assert B == self.batch and L % P == 0 and k.is_contiguous() and v.is_contiguous()
+        n = L // P
+        pages = self.take_pages(B * n)
+        dst = torch.tensor(pages, dtype=torch.int32, device=self.device)
+        flat_k, flat_v = k.view(B * L, *k.shape[2:]), v.view(B * L, *v.shape[2:])
+        kb.quantize_pages(self.cfg, kb.Source.token_major(flat_k, self.cfg), kb.Source.token_major(flat_v, self.cfg),
+                          dst, self.pool, self.err, stream)
+        self.page_table[:, :n] = dst.view(B, n)
+        self.num_pages.fill_(n)
+        self.res_len.zero_()
+        for b in range(B):
+            self.host_pages[b] += pages[b * n:(b + 1) * n]
+            self.host_res_len[b] = 0
+        return dst
+
     # ---------------------------------------------------------------- decode step
     def reserve_flush_pages(self) -> list:
         """Before a step: a fresh page for every sequence whose window will be full
-        after this step's append; returns the sequences that will flush."""
+        after this step's append; returns the sequences that will flush.  The device
+        buffer is only written when its contents change."""
         P = self.cfg.page_tokens
         flushing = [b for b in range(self.batch) if self.host_res_len[b] + 1 == P]
         ids = [-1] * self.batch
         for b in flushing:
             ids[b] = self.take_pages(1)[0]
-        self.new_page.copy_(torch.tensor(ids, dtype=torch.int32), non_blocking=False)
+        if ids != self.host_new_page:
+            self.new_page.copy_(torch.tensor(ids, dtype=torch.int32), non_blocking=False)
+            self.host_new_page = ids
         return flushing
 
     def commit_host(self, flushing: list):
         P = self.cfg.page_tokens
         for b in range(self.batch):
             self.host_res_len[b] += 1
-        new = self.new_page.tolist() if flushing else None
         for b in flushing:
-            self.host_pages[b].append(new[b])
+            self.host_pages[b].append(self.host_new_page[b])
             self.host_res_len[b] = 0
         assert all(r < P for r in self.host_res_len)
 

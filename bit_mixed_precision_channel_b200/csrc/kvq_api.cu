@@ -8,16 +8,22 @@ namespace kvq {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// SM count of the current device, looked up once per device (148 when no device is
+// visible, so that workspace sizes can be computed on a machine without a GPU).
 static int sm_count() {
+  static int cached[64];
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return 148;
   }
+  n = __atomic_load_n(&cached[dev], __ATOMIC_ACQUIRE);
+  if (n > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
     cudaGetLastError();
     return 148;
   }
+  __atomic_store_n(&cached[dev], n, __ATOMIC_RELEASE);
   return n;
 }
 

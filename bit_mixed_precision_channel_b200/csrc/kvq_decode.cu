@@ -213,7 +213,6 @@ __device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t*
     }
   }
   // -- logits (log2 units) --
-  const float c24 = p.c_log2 * kCodeUnitInv;
   float L[2][4];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -221,10 +220,10 @@ __device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t*
     for (int i = 0; i < 4; ++i) {
       float v;
       if constexpr (NT == 1) {
-        v = fmaf(acc[mt][0][i], c24, z[i & 1] * p.c_log2);
+        v = (acc[mt][0][i] + z[i & 1]) * p.c_log2;
         v += __shfl_xor_sync(kFull, v, 2);
       } else {
-        v = fmaf(acc[mt][0][i] + acc[mt][1][i], c24, z[i & 1] * p.c_log2);
+        v = (acc[mt][0][i] + acc[mt][1][i] + z[i & 1]) * p.c_log2;
       }
       L[mt][i] = v;
     }
@@ -459,16 +458,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     __syncthreads();
     return;
   }
-  // page results are in units of code * 2^-24; bring them to real units
-  if (npg > 0) {
-#pragma unroll
-    for (int mc = 0; mc < 8; ++mc)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= kCodeUnitInv;
-  }
-
   // ---------------------------------------------------------------- residual window
   if (own_res) {
     const int rows = (rl + 31) & ~31;
@@ -618,7 +607,8 @@ size_t decode_main_bytes(int P, int GQA, uint32_t rec_bytes) {
 template <typename T, int GQA>
 cudaError_t launch_decode_t(DecodeParams p, cudaStream_t stream) {
   const size_t smem = size_t(p.main_bytes) + size_t(p.pps) * 4;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, GQA>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  static int seen[64];
+  cudaError_t e = ensure_dynamic_smem(decode_kernel<T, GQA>, int(smem), seen);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.max_splits, p.Hkv, p.batch);
   decode_kernel<T, GQA><<<grid, kDecodeThreads, smem, stream>>>(p);

@@ -180,16 +180,19 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Two 2-bit codes of a packed word as an fp16 pair for the tensor cores: pair j holds
-// elements 2j (low half) and 2j+1 (high half).  Each half keeps its code in the two
-// lowest mantissa bits of an fp16 with a zero exponent, i.e. the exact value
-// code * 2^-24; products with the other operand stay exact in fp32 and the 2^24
-// factor is restored after the contraction.  One shift and one AND per pair.
-constexpr float kCodeUnitInv = 16777216.0f;  // 2^24
-__device__ __forceinline__ uint32_t code_pair(uint32_t w, int j) { return (w >> (2 * j)) & 0x00030003u; }
-
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Two 2-bit codes of a packed word as an exact fp16 pair for the tensor cores: pair j
+// holds elements 2j (low half) and 2j+1 (high half).  OR-ing a code into the mantissa
+// of 1024.0 (0x6400) gives the fp16 value 1024 + code exactly; subtracting 1024 leaves
+// the code.  (Feeding the masked bits directly as fp16 subnormals, code * 2^-24, saves
+// the subtraction but was measured to lose the small products of the low operand part
+// inside the tensor core, ~1e-3 output error; the integers keep every product exact.)
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, int j) {
+  const uint32_t x = ((w >> (2 * j)) & 0x00030003u) | 0x64006400u;
+  return h2_as_u32(__hsub2(u32_as_h2(x), __half2(__half(1024.0f), __half(1024.0f))));
+}
 __device__ __forceinline__ uint32_t bf2_as_u32(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
 // ------------------------------------------------------------------ launch parameters
@@ -250,6 +253,26 @@ cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32
                                 int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int gqa, int dtype, cudaStream_t stream);
 SplitPlan plan_splits(int units, int max_pages, int sm_count);
+
+// Raises a kernel's dynamic shared-memory limit once per device and size, so that
+// later calls (and calls made while a stream is being captured into a graph) issue
+// no attribute call.  `seen` holds the largest size already set, per device.
+template <typename Kernel>
+inline cudaError_t ensure_dynamic_smem(Kernel kernel, int bytes, int (&seen)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (bytes <= __atomic_load_n(&seen[dev], __ATOMIC_ACQUIRE)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) {
+    int cur = __atomic_load_n(&seen[dev], __ATOMIC_ACQUIRE);
+    while (cur < bytes && !__atomic_compare_exchange_n(&seen[dev], &cur, bytes, false, __ATOMIC_ACQ_REL,
+                                                        __ATOMIC_ACQUIRE)) {
+    }
+  }
+  return e;
+}
 size_t decode_main_bytes(int P, int GQA, uint32_t rec_bytes);
 
 }  // namespace kvq

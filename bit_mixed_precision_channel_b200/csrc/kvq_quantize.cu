@@ -295,11 +295,14 @@ cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaSt
   if (n_items <= 0) return cudaSuccess;
   const size_t smem = QSmem::bytes(p.P, p.k);
   const dim3 grid(n_items, p.Hkv);
+  static int seen_bf16[64], seen_f16[64];
   if (dtype == KVQ_BF16) {
-    cudaFuncSetAttribute(quantize_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__nv_bfloat16>, int(smem), seen_bf16);
+    if (e != cudaSuccess) return e;
     quantize_kernel<__nv_bfloat16><<<grid, kQThreads, smem, stream>>>(p);
   } else {
-    cudaFuncSetAttribute(quantize_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__half>, int(smem), seen_f16);
+    if (e != cudaSuccess) return e;
     quantize_kernel<__half><<<grid, kQThreads, smem, stream>>>(p);
   }
   return cudaGetLastError();

@@ -84,7 +84,8 @@
  * a full residual window, a full page table) set bits of the optional device word
  * *err (KVQ_DEV_ERR_* flags, OR-ed atomically; pass NULL to ignore) and the offending
  * work item is skipped; outputs of a call that raised a device error are undefined.
- * No kernel traps.  The library holds no global state.
+ * No kernel traps.  The library's only global state is a per-device record of the
+ * SM count and of the kernel attributes it has already set (thread-safe).
  */
 #ifndef KVQ_H
 #define KVQ_H

@@ -28,13 +28,14 @@ def _inputs(rng, L, cfg, outlier_scale=(8.0, 20.0)):
     return K, V
 
 
-def _run(cfg, lens, seed, max_pages=None, page_order=None, q_scale=1.0):
+def _run(cfg, lens, seed, max_pages=None, shuffle=False, q_scale=1.0):
     """Prefill sequences of the given lengths, attend once; returns (out, oracle out)."""
     rng = np.random.default_rng(seed)
     P = cfg.page_tokens
     B = len(lens)
     max_pages = max_pages or max(1, max(L // P for L in lens))
     pool_pages = sum(L // P for L in lens) + 4
+    page_order = np.random.default_rng(seed + 1).permutation(pool_pages) if shuffle else None
     cache = PagedKVCache(cfg, B, max_pages, pool_pages, page_order=page_order)
     inputs = []
     for b, L in enumerate(lens):
@@ -111,8 +112,8 @@ def test_empty_and_residual_only_sequences():
 
 def test_shuffled_physical_pages():
     cfg = kb.Config(num_q_heads=4, num_kv_heads=2, page_tokens=128, num_boost=16)
-    order = np.random.default_rng(1).permutation(40)
-    got, want, _ = _run(cfg, [128 * 20 + 50, 128 * 15], seed=13, page_order=order)
+    got, want, cache = _run(cfg, [128 * 20 + 50, 128 * 15], seed=13, shuffle=True)
+    assert cache.host_pages[0] != sorted(cache.host_pages[0])
     assert_attention_close(got, want, "shuffled")
 
 
