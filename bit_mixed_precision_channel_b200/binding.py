@@ -19,7 +19,8 @@ __all__ = [
     "KVQError", "Config", "Source", "library_path", "load", "status_string", "check_config",
     "page_layout", "page_bytes", "select_boost_channels", "quantize_page_keys",
     "quantize_values", "quantize_pages", "append_token", "flush_residual",
-    "decode_workspace_bytes", "decode_attention", "F16", "BF16", "torch_dtype",
+    "decode_workspace_bytes", "decode_attention", "decode_attention_static", "STATIC_SCRATCH_BYTES",
+    "F16", "BF16", "torch_dtype",
     "DEV_ERR_PAGE_RANGE", "DEV_ERR_RESIDUAL", "DEV_ERR_TABLE_FULL", "DEV_ERR_TIMEOUT",
     "DEV_ERR_LENGTH",
 ]
@@ -31,6 +32,7 @@ DEV_ERR_RESIDUAL = 2
 DEV_ERR_TABLE_FULL = 4
 DEV_ERR_TIMEOUT = 8
 DEV_ERR_LENGTH = 16
+STATIC_SCRATCH_BYTES = 16 << 20  # KVQ_STATIC_SCRATCH_BYTES
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -147,6 +149,9 @@ def load():
         L.kvq_decode_attention.restype = ctypes.c_int
         L.kvq_decode_attention.argtypes = [cfgp, vp, i64, vp, i32, vp, i32, vp, vp, vp, vp,
                                            ctypes.c_float, vp, vp, sz, vp, vp]
+        L.kvq_decode_attention_static.restype = ctypes.c_int
+        L.kvq_decode_attention_static.argtypes = [cfgp, vp, i64, vp, i32, vp, i32, vp, vp, vp, vp,
+                                                  ctypes.c_float, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -259,3 +264,20 @@ def decode_attention(cfg: Config, pool, q, page_table, num_pages, res_k, res_v, 
         max_pages, num_pages.data_ptr(), res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
         float(sm_scale), out.data_ptr(), workspace.data_ptr(), workspace.numel(), _ptr(err),
         _stream(stream)))
+
+
+def decode_attention_static(cfg: Config, pool, q, page_table, num_pages, res_k, res_v, res_len, out,
+                            sm_scale: float | None = None, err=None, stream=None):
+    """decode_attention for callers that cannot allocate device memory: the split-K
+    scratch is the library's own static 16 MiB device buffer (no workspace argument).
+    Calls on one device share that buffer, so they must not overlap on the GPU; the
+    first call on a device must not be made during stream capture."""
+    _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
+    batch, max_pages = page_table.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(cfg.head_dim)
+    pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
+    _check("kvq_decode_attention_static", load().kvq_decode_attention_static(
+        ctypes.byref(cfg.c()), pool.data_ptr(), pool_pages, q.data_ptr(), batch, page_table.data_ptr(),
+        max_pages, num_pages.data_ptr(), res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
+        float(sm_scale), out.data_ptr(), _ptr(err), _stream(stream)))

@@ -260,6 +260,35 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool,
                                 void* workspace, size_t workspace_bytes,
                                 int32_t* err, cudaStream_t stream);
 
+/* Size of the library's built-in decode scratch (see kvq_decode_attention_static). */
+#define KVQ_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Decode attention without a caller workspace, for callers that cannot allocate
+ * device memory: a serving engine whose memory pool already holds all of the GPU, a
+ * plugin whose host framework owns every device allocation, or a latency-critical
+ * path that must not call cudaMalloc because it may synchronize the device.  (The
+ * web pages on the method have no counterpart of this call; it is a property of this
+ * library's interface only.)
+ * Same arguments, results and error behaviour as kvq_decode_attention, minus the
+ * workspace: the split-K partials and arrival counters live in a static device buffer
+ * of KVQ_STATIC_SCRATCH_BYTES (16 MiB) inside the library, which every GPU that loads
+ * the library keeps until the process exits.  Shapes that need more than that
+ * (kvq_decode_workspace_bytes(cfg, batch, max_pages) > KVQ_STATIC_SCRATCH_BYTES) are
+ * rejected with KVQ_ERR_CAPACITY before anything is enqueued.
+ * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * The first call on each device looks up the buffer's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call outside any
+ * stream capture.  Each call clears the buffer's arrival counters on `stream` before
+ * the kernel runs; the rest keeps the previous call's contents.  All calls on a device
+ * share the one buffer, so two calls whose executions overlap on the GPU (different
+ * streams without ordering between them) race and give undefined results. */
+KVQ_API kvq_status kvq_decode_attention_static(const kvq_config* cfg, const void* pool, int64_t pool_pages,
+                                               const void* q, int32_t batch,
+                                               const int32_t* page_table, int32_t max_pages,
+                                               const int32_t* num_pages,
+                                               const void* res_k, const void* res_v, const int32_t* res_len,
+                                               float sm_scale, float* out, int32_t* err, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
