@@ -36,7 +36,10 @@ static Plan decode_plan(const kvq_config* cfg, int batch, int max_pages) {
   const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
   const int units = batch * cfg->num_kv_heads;
   Plan pl;
-  pl.split = plan_splits(units, max_pages, sm_count());
+  // resident CTAs per SM, evaluated with a page-id list of 256 entries
+  const Layout L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
+  const size_t smem = decode_main_bytes(cfg->page_tokens, gqa, L.record) + 256 * 4;
+  pl.split = plan_splits(units, max_pages, sm_count() * decode_ctas_per_sm(gqa, cfg->dtype, cfg->num_boost / 16, smem));
   pl.part_bytes = size_t(units) * pl.split.max_splits * gqa * (2 + kHeadDim) * sizeof(float);
   pl.part_bytes = (pl.part_bytes + 255) / 256 * 256;
   pl.cnt_bytes = size_t(units) * sizeof(uint32_t);
@@ -76,6 +79,9 @@ kvq_status kvq_check_config(const kvq_config* cfg) {
   if (cfg->page_tokens != 32 && cfg->page_tokens != 64 && cfg->page_tokens != 128) return KVQ_ERR_UNSUPPORTED;
   if (cfg->key_group != 32) return KVQ_ERR_UNSUPPORTED;
   if (cfg->key_bits != 2 || cfg->boost_bits != 4 || cfg->value_bits != 2) return KVQ_ERR_UNSUPPORTED;
+  if (cfg->num_boost != 0 && cfg->num_boost != 16 && cfg->num_boost != 32 && cfg->num_boost != 64 &&
+      cfg->num_boost != 128)
+    return KVQ_ERR_UNSUPPORTED;
   if (cfg->dtype != KVQ_F16 && cfg->dtype != KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }

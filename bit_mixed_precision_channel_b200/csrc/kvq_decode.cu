@@ -1,12 +1,13 @@
 // kvq_decode.cu — decode attention over the paged 2-bit cache, sm_100a.
 //
 // One CTA = (sequence b, kv head, split of the page list); 4 warps.  Pages stream
-// through a 6-stage shared-memory ring filled by the bulk-copy engine (one
-// cp.async.bulk per page record, completion on an mbarrier, L2 evict-first hint);
-// a stage holds 128 tokens (1, 2 or 4 pages).  Each warp owns one 32-token key
-// group of the stage and keeps its own online-softmax state; the warps' states are
-// merged in shared memory at the end, and the splits of a sequence are merged by the
-// last CTA to finish (log-sum-exp merge, no second launch).
+// through a 4-stage shared-memory ring filled by the bulk-copy engine (one
+// cp.async.bulk per page record, completion on a "full" mbarrier, L2 evict-first
+// hint); a stage holds 128 tokens (1, 2 or 4 pages).  Each warp owns one 32-token key
+// group of the stage, keeps its own online-softmax state and releases the stage on an
+// "empty" mbarrier, so warps run decoupled; thread 0 refills released stages.  The
+// warps' states are merged in shared memory at the end, and the splits of a sequence
+// are merged by the last CTA to finish (log-sum-exp merge, no second launch).
 //
 // The 2-bit codes never become floating-point values with a scale applied.  The
 // scales are folded into the other operand of each product, and the codes go to the
@@ -16,10 +17,11 @@
 //             + sum_c q_c * zA_{g,c}
 //   sum_t p_t v_t[c] = sum_t code_V[t,c] * (p_t * sV_t) + sum_t p_t * zV_t
 // With the 4-bit boosted channels stored as two 2-bit planes, the boosted low bits
-// are simply 16*(k/16) more rows of the same contraction.  The folded operands are
-// carried as a high and a low fp16 part (hi = fp16(x), lo = fp16(x - hi)), so the
-// products keep ~22 bits; codes are exact in fp16.  Matrix shapes per warp and
-// 32-token group: QK^T = [32 tokens x (128 + k) channels] x [(128 + k) x 8 columns],
+// are simply k more rows of the same contraction.  The folded operands are carried
+// as a high and a low fp16 part (hi = fp16(x), lo = fp16(x - hi)), so the products
+// keep ~22 bits; codes reach the tensor cores exactly (as 0.5 * code through the FP4
+// conversion, the 0.5 undone afterwards).  Matrix shapes per warp and 32-token group:
+// QK^T = [32 tokens x (128 + k) channels] x [(128 + k) x 8 columns],
 // PV = [128 channels x 32 tokens] x [32 tokens x 8 columns], where the 8 columns hold
 // the hi and lo parts of up to 4 query heads (two column tiles for 8 heads).
 #include <algorithm>
@@ -28,15 +30,16 @@
 
 namespace kvq {
 
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kDecodeThreads = 128;
-constexpr int kResRowBytes = 272;  // residual row in shared memory: 256 bytes + 16 pad
+constexpr int kResRowBytes = 272;    // residual row in shared memory: 256 bytes + 16 pad
+constexpr int kResRoundTokens = 64;  // residual tokens staged per round (16 per warp)
 
 // ---------------------------------------------------------------- operand builders
 
-// Query-side operand of one k-step pair for the quantized planes:
-// hi = fp16(q*s) and lo = fp16(q*s - hi).  For fp16 data the product of two fp16
-// values is exact in 22 bits; hmul2 rounds it once and hfma2 returns the rest.
+// Query-side operand of one k-step pair: hi = fp16(q*s) and lo = fp16(q*s - hi).
+// For fp16 data the product of two fp16 values is exact in 22 bits; hmul2 rounds it
+// once and hfma2 returns the rest.
 __device__ __forceinline__ void fold_hilo(uint32_t q2, uint32_t s2, uint32_t& hi, uint32_t& lo, __half) {
   const __half2 q = u32_as_h2(q2), s = u32_as_h2(s2);
   const __half2 h = __hmul2(q, s);
@@ -53,6 +56,19 @@ __device__ __forceinline__ void fold_hilo(uint32_t q2, uint32_t s2, uint32_t& hi
   const float2 hf = __half22float2(h);
   hi = h2_as_u32(h);
   lo = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+}
+
+// For GQA <= 4 one column tile carries hi (columns 0..3) and lo (columns 4..7):
+// hfma2(q, s, -hi * m) with m = 0 or 1 per lane gives either part without a branch.
+__device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t negmask, __half) {
+  const __half2 q = u32_as_h2(q2), s = u32_as_h2(s2);
+  const __half2 h = __hmul2(q, s);
+  return h2_as_u32(__hfma2(q, s, __hmul2(h, u32_as_h2(negmask))));
+}
+__device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t negmask, __nv_bfloat16) {
+  uint32_t hi, lo;
+  fold_hilo(q2, s2, hi, lo, __nv_bfloat16());
+  return negmask ? lo : hi;
 }
 
 // fp16 hi/lo split of two fp32 values (probability-side operand of the code planes).
@@ -85,22 +101,38 @@ struct WarpState {
   float m[2], l[2], zv[2];
 };
 
-// Online-softmax update from the 2 x 4 logits of one 32-token group held by this
-// lane (rows g, g+8 of two 16-token tiles; heads hc0, hc1).  Logits are in log2 units.
-template <int GQA>
-__device__ __forceinline__ void softmax_step(WarpState<GQA>& st, const float (&L)[2][4], float (&alpha)[2]) {
-  float mx[2];
-  mx[0] = fmaxf(fmaxf(L[0][0], L[0][2]), fmaxf(L[1][0], L[1][2]));
-  mx[1] = fmaxf(fmaxf(L[0][1], L[0][3]), fmaxf(L[1][1], L[1][3]));
+// Per-lane constants of the query-side operand.
+struct LaneQ {
+  uint32_t qv[8][2];  // q pairs of this lane's B column for k-step s: channels 16s+2qd(+1), +8
+  uint32_t negmask;   // fp16x2 -1 for the lo-part columns (GQA <= 4), 0 otherwise
+  float zmul;         // weight of this lane's zero-point column in the logits
+};
+
+// Online-softmax update from the logits of MT 16-token tiles held by this lane
+// (rows g, g+8 of each tile; heads hc0, hc1).  Logits are in log2 units.  The running
+// maximum moves only when a logit exceeds it by more than 8, so probabilities stay
+// below 2^8 and most groups skip the rescale of the accumulators.
+template <int GQA, int MT>
+__device__ __forceinline__ void softmax_step(WarpState<GQA>& st, const float (&L)[MT][4]) {
+  float mx[2] = {L[0][0], L[0][1]};
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    mx[0] = fmaxf(mx[0], fmaxf(L[mt][0], L[mt][2]));
+    mx[1] = fmaxf(mx[1], fmaxf(L[mt][1], L[mt][3]));
+  }
+  float alpha[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(kFull, mx[j], off));
-    const float mn = fmaxf(st.m[j], mx[j]);
-    alpha[j] = (mn == -INFINITY) ? 1.0f : ex2(st.m[j] - mn);
-    st.m[j] = mn;
-    st.l[j] *= alpha[j];
-    st.zv[j] *= alpha[j];
+    if (mx[j] > st.m[j] + 8.0f) {
+      alpha[j] = ex2(st.m[j] - mx[j]);  // 0 on the first group (m = -inf)
+      st.m[j] = mx[j];
+      st.l[j] *= alpha[j];
+      st.zv[j] *= alpha[j];
+    } else {
+      alpha[j] = 1.0f;
+    }
   }
   if (!__all_sync(kFull, alpha[0] == 1.0f && alpha[1] == 1.0f)) {
 #pragma unroll
@@ -115,10 +147,11 @@ __device__ __forceinline__ void softmax_step(WarpState<GQA>& st, const float (&L
 // ---------------------------------------------------------------- one quantized group
 
 // Processes tokens [t0, t0+32) of the page record `rec` (in shared memory).
-template <typename T, int GQA>
-__device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t* rec, int t0,
-                                           const uint32_t (&qv)[8][2], const T* q_s, int hB, bool loB,
-                                           bool validB, WarpState<GQA>& st, int g, int qd) {
+// KB = boosted channels / 16.
+template <typename T, int GQA, int KB>
+__device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t* rec, int t0, const LaneQ& lq,
+                                           const uint16_t* q_s, int hB, bool validB, WarpState<GQA>& st, int g,
+                                           int qd) {
   constexpr int NT = WarpState<GQA>::NT;
   const int grp = t0 >> 5;
   float acc[2][NT][4];
@@ -129,90 +162,126 @@ __device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t*
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
 
-  // -- q . K^T over plane A (128 channels) --
+  // -- q . K^T over plane A: this lane's codes are words 2qd, 2qd+1 of each token row,
+  //    its scales positions 32qd .. 32qd+31 of the group's scale row --
   const uint8_t* kA = rec + p.L.k_codes;
-  const uint8_t* ksc = rec + p.L.k_scale + grp * kHeadDim * 2;
+  const uint4* psc = reinterpret_cast<const uint4*>(rec + p.L.k_scale + (grp * kHeadDim + 32 * qd) * 2);
+  uint2 w[2][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) w[mt][r] = lds64(kA + ((t0 + 16 * mt + g + 8 * r) * 8 + 2 * qd) * 4);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    uint4 w[2][2];
+    uint32_t sc[8];
+    {
+      const uint4 a = psc[2 * half], b = psc[2 * half + 1];
+      sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
+      sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
+    }
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      uint32_t c[2][2][4];  // [mt][row][byte]: byte 2j + r -> k-step 4*half + 2*pass + j, reg r
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t word = half ? w[mt][r].y : w[mt][r].x;
+          e2m1_pairs(code_pass(word, pass), c[mt][r][0], c[mt][r][1], c[mt][r][2], c[mt][r][3]);
+        }
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int s = 4 * half + 2 * pass + jj, sl = 2 * pass + jj;
+        uint32_t b[NT][2];
+        if constexpr (NT == 1) {
+          b[0][0] = fold_one(lq.qv[s][0], sc[2 * sl], lq.negmask, T());
+          b[0][1] = fold_one(lq.qv[s][1], sc[2 * sl + 1], lq.negmask, T());
+        } else {
+          fold_hilo(lq.qv[s][0], sc[2 * sl], b[0][0], b[1][0], T());
+          fold_hilo(lq.qv[s][1], sc[2 * sl + 1], b[0][1], b[1][1], T());
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const uint32_t a[4] = {c[mt][0][2 * jj], c[mt][1][2 * jj], c[mt][0][2 * jj + 1], c[mt][1][2 * jj + 1]};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+        }
+      }
+    }
+  }
+  // -- plane B: low bits of the boosted channels; rows 16s + 8r + 2qd + f of this lane
+  //    sit at positions 4*KB*qd + 4s + 2r + f of each token row --
+  if constexpr (KB > 0) {
+    const uint8_t* kB = rec + p.L.kb_codes;
+    const uint8_t* idx = rec + p.L.boost_idx;
+    const uint8_t* kbsc = rec + p.L.kb_scale + grp * (16 * KB) * 2;
+    const uint16_t* qh = q_s + hB * kHeadDim;
+    uint32_t cb[2][2][KB][2];  // [mt][row][s][r]
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int r = 0; r < 2; ++r) w[mt][r] = lds128(kA + ((t0 + 16 * mt + g + 8 * r) * 8 + 4 * half) * 4);
+      for (int rr = 0; rr < 2; ++rr) {
+        const uint8_t* row = kB + (t0 + 16 * mt + g + 8 * rr) * KB * 4;
+        if constexpr (KB == 1) {
+          // positions 4qd .. 4qd+3: word 0, pass qd >> 1, bytes 2(qd & 1), +1
+          const uint32_t x = code_pass(lds32(row), qd >> 1) >> (16 * (qd & 1));
+          cb[mt][rr][0][0] = e2m1_pair_lo(x);
+          cb[mt][rr][0][1] = e2m1_pair_lo(x >> 8);
+        } else {
+          // k-steps s, s+1 (s even) share a word and a pass: bytes 0..3
 #pragma unroll
-    for (int ss = 0; ss < 4; ++ss) {
-      const int s = 4 * half + ss;
-      const uint32_t sc0 = lds32(ksc + (16 * s + 2 * qd) * 2);
-      const uint32_t sc1 = lds32(ksc + (16 * s + 2 * qd + 8) * 2);
-      uint32_t h0, l0, h1, l1;
-      fold_hilo(qv[s][0], sc0, h0, l0, T());
-      fold_hilo(qv[s][1], sc1, h1, l1, T());
+          for (int s = 0; s < KB; s += 2) {
+            const int pos = 4 * KB * qd + 4 * s;
+            const uint32_t x = code_pass(lds32(row + (pos >> 4) * 4), (pos >> 3) & 1);
+            e2m1_pairs(x, cb[mt][rr][s][0], cb[mt][rr][s][1], cb[mt][rr][s + 1][0], cb[mt][rr][s + 1][1]);
+          }
+        }
+      }
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
+      uint32_t q0 = 0, q1 = 0;
+      if (validB) {
+        // indices are < 128 in any record the library wrote; the mask keeps a corrupt
+        // record from reading outside the query rows
+        q0 = uint32_t(qh[idx[j0] & 127]) | (uint32_t(qh[idx[j0 + 1] & 127]) << 16);
+        q1 = uint32_t(qh[idx[j1] & 127]) | (uint32_t(qh[idx[j1 + 1] & 127]) << 16);
+      }
+      const uint32_t s0 = lds32(kbsc + j0 * 2), s1 = lds32(kbsc + j1 * 2);
       uint32_t b[NT][2];
       if constexpr (NT == 1) {
-        b[0][0] = loB ? l0 : h0;
-        b[0][1] = loB ? l1 : h1;
+        b[0][0] = fold_one(q0, s0, lq.negmask, T());
+        b[0][1] = fold_one(q1, s1, lq.negmask, T());
       } else {
-        b[0][0] = h0; b[0][1] = h1;
-        b[1][0] = l0; b[1][1] = l1;
+        fold_hilo(q0, s0, b[0][0], b[1][0], T());
+        fold_hilo(q1, s1, b[0][1], b[1][1], T());
       }
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        const uint32_t wa = ss == 0 ? w[mt][0].x : ss == 1 ? w[mt][0].y : ss == 2 ? w[mt][0].z : w[mt][0].w;
-        const uint32_t wb = ss == 0 ? w[mt][1].x : ss == 1 ? w[mt][1].y : ss == 2 ? w[mt][1].z : w[mt][1].w;
-        const uint32_t a[4] = {code_pair(wa, qd), code_pair(wb, qd), code_pair(wa, qd + 4), code_pair(wb, qd + 4)};
+        const uint32_t a[4] = {cb[mt][0][s][0], cb[mt][1][s][0], cb[mt][0][s][1], cb[mt][1][s][1]};
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
       }
     }
   }
-  // -- plane B: low bits of the boosted channels (k rows) --
-  const uint8_t* kB = rec + p.L.kb_codes;
-  const uint8_t* idx = rec + p.L.boost_idx;
-  const uint8_t* kbsc = rec + p.L.kb_scale + grp * p.k * 2;
-  for (int s = 0; s < p.KB; ++s) {
-    const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
-    const uint16_t* qh = reinterpret_cast<const uint16_t*>(q_s) + hB * kHeadDim;
-    uint32_t q0 = 0, q1 = 0;
-    if (validB) {
-      // indices are < 128 in any record the library wrote; the mask keeps a corrupt
-      // record from reading outside the query rows
-      q0 = uint32_t(qh[idx[j0] & 127]) | (uint32_t(qh[idx[j0 + 1] & 127]) << 16);
-      q1 = uint32_t(qh[idx[j1] & 127]) | (uint32_t(qh[idx[j1 + 1] & 127]) << 16);
-    }
-    uint32_t h0, l0, h1, l1;
-    fold_hilo(q0, lds32(kbsc + j0 * 2), h0, l0, T());
-    fold_hilo(q1, lds32(kbsc + j1 * 2), h1, l1, T());
-    uint32_t b[NT][2];
-    if constexpr (NT == 1) {
-      b[0][0] = loB ? l0 : h0;
-      b[0][1] = loB ? l1 : h1;
-    } else {
-      b[0][0] = h0; b[0][1] = h1;
-      b[1][0] = l0; b[1][1] = l1;
-    }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const uint32_t wa = lds32(kB + ((t0 + 16 * mt + g) * p.KB + s) * 4);
-      const uint32_t wb = lds32(kB + ((t0 + 16 * mt + g + 8) * p.KB + s) * 4);
-      const uint32_t a[4] = {code_pair(wa, qd), code_pair(wb, qd), code_pair(wa, qd + 4), code_pair(wb, qd + 4)};
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
-    }
-  }
-  // -- zero-point term: Z[h] = sum_c q[h][c] * zA[g][c] (rows of A all equal) --
+  // -- zero-point term: Z[h] = sum_c q[h][c] * zA[g][c] (all rows of A equal) --
   float z[4] = {0.f, 0.f, 0.f, 0.f};
   {
-    const uint8_t* kzp = rec + p.L.k_zero + grp * kHeadDim * 2;
+    const uint4* pz = reinterpret_cast<const uint4*>(rec + p.L.k_zero + (grp * kHeadDim + 32 * qd) * 2);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t z0 = lds32(kzp + (16 * s + 2 * qd) * 2);
-      const uint32_t z1 = lds32(kzp + (16 * s + 2 * qd + 8) * 2);
-      const uint32_t a[4] = {z0, z0, z1, z1};
-      const bool useq = validB && !loB;
-      mma_16816(z, a, useq ? qv[s][0] : 0u, useq ? qv[s][1] : 0u, T());
+    for (int i = 0; i < 4; ++i) {
+      const uint4 zz = pz[i];
+      const uint32_t zr[4] = {zz.x, zz.y, zz.z, zz.w};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int s = 2 * i + u;
+        const uint32_t a[4] = {zr[2 * u], zr[2 * u], zr[2 * u + 1], zr[2 * u + 1]};
+        mma_16816(z, a, lq.qv[s][0], lq.qv[s][1], T());
+      }
     }
   }
-  // -- logits (log2 units) --
+  // -- logits (log2 units); code products carry a factor 0.5 --
+  const float ccode = p.c_log2 * kCodeScale;
   float L[2][4];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -220,15 +289,14 @@ __device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t*
     for (int i = 0; i < 4; ++i) {
       float v;
       if constexpr (NT == 1) {
-        v = (acc[mt][0][i] + z[i & 1]) * p.c_log2;
+        v = fmaf(acc[mt][0][i], ccode, z[i & 1] * lq.zmul);
         v += __shfl_xor_sync(kFull, v, 2);
       } else {
-        v = (acc[mt][0][i] + acc[mt][1][i] + z[i & 1]) * p.c_log2;
+        v = fmaf(acc[mt][0][i] + acc[mt][1][i], ccode, z[i & 1] * lq.zmul);
       }
       L[mt][i] = v;
     }
-  float alpha[2];
-  softmax_step<GQA>(st, L, alpha);
+  softmax_step<GQA, 2>(st, L);
 
   // -- probabilities, folded with the value scales, as the B operand of PV --
   const uint16_t* vs = reinterpret_cast<const uint16_t*>(rec + p.L.v_scale);
@@ -259,103 +327,93 @@ __device__ __forceinline__ void page_group(const DecodeParams& p, const uint8_t*
       pb[mt][1][1] = movmatrix_trans(bl);
     }
   }
-  // -- P V over the value codes (channel-major words of 16 tokens) --
-  const uint8_t* vq = rec + p.L.v_codes;
-  const int PW = p.P >> 4;
+  // -- P V: word 2*grp + qd/2 of each channel row holds this lane's 8 tokens (pass qd&1) --
+  const uint8_t* vq = rec + p.L.v_codes + (2 * grp + (qd >> 1)) * 4;
+  const int rowb = (p.P >> 4) * 4;  // bytes per channel row
+  const int vpass = qd & 1;
 #pragma unroll
   for (int mc = 0; mc < 8; ++mc) {
-    const uint2 w0 = lds64(vq + ((16 * mc + g) * PW + (t0 >> 4)) * 4);
-    const uint2 w1 = lds64(vq + ((16 * mc + g + 8) * PW + (t0 >> 4)) * 4);
+    uint32_t ca[4], cbv[4];
+    e2m1_pairs(code_pass(lds32(vq + (16 * mc + g) * rowb), vpass), ca[0], ca[1], ca[2], ca[3]);
+    e2m1_pairs(code_pass(lds32(vq + (16 * mc + g + 8) * rowb), vpass), cbv[0], cbv[1], cbv[2], cbv[3]);
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
-      const uint32_t wa = ks ? w0.y : w0.x, wb = ks ? w1.y : w1.x;
-      const uint32_t a[4] = {code_pair(wa, qd), code_pair(wb, qd), code_pair(wa, qd + 4), code_pair(wb, qd + 4)};
+      const uint32_t a[4] = {ca[2 * ks], cbv[2 * ks], ca[2 * ks + 1], cbv[2 * ks + 1]};
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[ks][nt][0], pb[ks][nt][1], __half());
     }
   }
 }
 
-// ---------------------------------------------------------------- residual group
+// ---------------------------------------------------------------- residual tokens
 
-// Tokens [tw, tw+32) of the residual window staged in shared memory (rows of 272 B);
-// rows at or beyond rl are zero and masked out of the softmax.
+// Tokens [tok0, tok0+16) of the residual window, staged in shared memory at rows
+// row0.. (rows of 272 B); rows at or beyond rl are zero and masked out of the softmax.
 template <typename T, int GQA>
-__device__ __forceinline__ void residual_group(const DecodeParams& p, const uint8_t* Kr, const uint8_t* Vr,
-                                               int tw, int rl, const uint32_t (&qv)[8][2], bool loB,
-                                               bool validB, WarpState<GQA>& st, int lane, int g, int qd) {
+__device__ __forceinline__ void residual_tile(const DecodeParams& p, const uint8_t* Kr, const uint8_t* Vr,
+                                              int row0, int tok0, int rl, const LaneQ& lq, bool loB, bool validB,
+                                              WarpState<GQA>& st, int lane, int g, int qd) {
   constexpr int NT = WarpState<GQA>::NT;
-  float acc[2][4];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const bool useq = validB && !loB;
   const int li = lane >> 3, lr = lane & 7;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t a[4];
-      const int row = tw + 16 * mt + lr + 8 * (li & 1);
-      const int col = 16 * s + 8 * (li >> 1);
-      ldmatrix_x4(a, smem_addr(Kr + row * kResRowBytes + col * 2));
-      mma_16816(acc[mt], a, useq ? qv[s][0] : 0u, useq ? qv[s][1] : 0u, T());
-    }
+    uint32_t a[4];
+    const int row = row0 + lr + 8 * (li & 1);
+    const int col = 16 * s + 8 * (li >> 1);
+    ldmatrix_x4(a, smem_addr(Kr + row * kResRowBytes + col * 2));
+    mma_16816(acc, a, useq ? lq.qv[s][0] : 0u, useq ? lq.qv[s][1] : 0u, T());
   }
-  float L[2][4];
+  float L[1][4];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float v = acc[mt][i] * p.c_log2;
-      if constexpr (NT == 1) v += __shfl_xor_sync(kFull, v, 2);
-      const int tok = tw + 16 * mt + g + 8 * (i >> 1);
-      L[mt][i] = tok < rl ? v : -INFINITY;
-    }
-  float alpha[2];
-  softmax_step<GQA>(st, L, alpha);
-  uint32_t pb[2][NT][2];
+  for (int i = 0; i < 4; ++i) {
+    float v = acc[i] * p.c_log2;
+    if constexpr (NT == 1) v += __shfl_xor_sync(kFull, v, 2);
+    const int tok = tok0 + g + 8 * (i >> 1);
+    L[0][i] = tok < rl ? v : -INFINITY;
+  }
+  softmax_step<GQA, 1>(st, L);
+  uint32_t pb[NT][2];
   const bool loC = qd >= 2;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-    const float p00 = ex2(L[mt][0] - st.m[0]), p01 = ex2(L[mt][1] - st.m[1]);
-    const float p10 = ex2(L[mt][2] - st.m[0]), p11 = ex2(L[mt][3] - st.m[1]);
+  {
+    const float p00 = ex2(L[0][0] - st.m[0]), p01 = ex2(L[0][1] - st.m[1]);
+    const float p10 = ex2(L[0][2] - st.m[0]), p11 = ex2(L[0][3] - st.m[1]);
     st.l[0] += p00 + p10;
     st.l[1] += p01 + p11;
     uint32_t th, tl, bh, bl;
     split_t(p00, p01, th, tl, T());
     split_t(p10, p11, bh, bl, T());
     if constexpr (NT == 1) {
-      pb[mt][0][0] = movmatrix_trans(loC ? tl : th);
-      pb[mt][0][1] = movmatrix_trans(loC ? bl : bh);
+      pb[0][0] = movmatrix_trans(loC ? tl : th);
+      pb[0][1] = movmatrix_trans(loC ? bl : bh);
     } else {
-      pb[mt][0][0] = movmatrix_trans(th);
-      pb[mt][0][1] = movmatrix_trans(bh);
-      pb[mt][1][0] = movmatrix_trans(tl);
-      pb[mt][1][1] = movmatrix_trans(bl);
+      pb[0][0] = movmatrix_trans(th);
+      pb[0][1] = movmatrix_trans(bh);
+      pb[1][0] = movmatrix_trans(tl);
+      pb[1][1] = movmatrix_trans(bl);
     }
   }
 #pragma unroll
-  for (int mc = 0; mc < 8; ++mc)
+  for (int mc = 0; mc < 8; ++mc) {
+    uint32_t a[4];
+    const int row = row0 + lr + 8 * (li >> 1);
+    const int col = 16 * mc + 8 * (li & 1);
+    ldmatrix_x4_trans(a, smem_addr(Vr + row * kResRowBytes + col * 2));
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t a[4];
-      const int row = tw + 16 * ks + lr + 8 * (li >> 1);
-      const int col = 16 * mc + 8 * (li & 1);
-      ldmatrix_x4_trans(a, smem_addr(Vr + row * kResRowBytes + col * 2));
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[ks][nt][0], pb[ks][nt][1], T());
-    }
+    for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[nt][0], pb[nt][1], T());
+  }
 }
 
 // ---------------------------------------------------------------- the kernel
 
-template <typename T, int GQA>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_constant__ DecodeParams p) {
+template <typename T, int GQA, int KB>
+__global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
+    decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NT = WarpState<GQA>::NT;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t bars[kStages];
+  __shared__ __align__(8) uint64_t full_bar[kStages];   // stage filled (bulk-copy bytes landed)
+  __shared__ __align__(8) uint64_t empty_bar[kStages];  // stage released by all 4 warps
   __shared__ __align__(16) uint16_t q_s[GQA * kHeadDim];
   __shared__ float s_m[4][GQA], s_l[4][GQA], s_zv[4][GQA];
   __shared__ int s_abort, s_last;
@@ -389,7 +447,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     for (int i = tid; i < GQA * kHeadDim / 8; i += kDecodeThreads) reinterpret_cast<uint4*>(q_s)[i] = qg[i];
   }
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 4);
+    }
     fence_mbar_init();
     s_abort = 0;
   }
@@ -400,27 +461,46 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
   const uint64_t policy = l2_evict_first_policy();
   auto issue = [&](int c) {
     const int st = c % kStages, first = c * ppc, nv = min(ppc, npg - first);
-    mbar_arrive_expect_tx(&bars[st], uint32_t(nv) * p.payload);
+    mbar_arrive_expect_tx(&full_bar[st], uint32_t(nv) * p.payload);
     for (int i = 0; i < nv; ++i) {
       const uint8_t* src = p.pool + (size_t(s_pages[first + i]) * p.Hkv + kvh) * p.rec_bytes;
-      bulk_g2s(main + st * p.stage_bytes + i * p.rec_bytes, src, p.payload, &bars[st], policy);
+      bulk_g2s(main + st * p.stage_bytes + i * p.rec_bytes, src, p.payload, &full_bar[st], policy);
     }
   };
+  // Thread 0 keeps the ring full: chunk x goes to stage x % kStages once the chunk
+  // x - kStages that used the stage before has been released by all four warps.
+  // It blocks only when a chunk up to `need` is not issued yet; further chunks up to
+  // `ahead` are issued if their stage is already free.
   int issued = 0;
-  if (tid == 0) {
-    for (; issued < min(kStages - 1, n_chunks); ++issued) issue(issued);
-  }
+  auto refill = [&](int need, int ahead) -> bool {
+    while (issued < n_chunks && issued <= ahead) {
+      if (issued >= kStages) {
+        const uint32_t par = uint32_t(issued / kStages - 1) & 1u;
+        uint64_t* eb = &empty_bar[issued % kStages];
+        if (issued <= need) {
+          if (!mbar_wait_bounded(eb, par)) return false;
+        } else if (!mbar_test_wait(eb, par)) {
+          break;
+        }
+      }
+      issue(issued++);
+    }
+    return true;
+  };
+  if (tid == 0) refill(-1, kStages - 1);
 
   // query fragments of this lane's B column (head hB; lo part for columns 4..7 when GQA <= 4)
   const int hB = GQA <= 4 ? (g & 3) : g;
   const bool loB = GQA <= 4 && g >= 4;
   const bool validB = hB < GQA;
-  uint32_t qv[8][2];
+  LaneQ lq;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
-    qv[s][0] = validB ? lds32(q_s + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
-    qv[s][1] = validB ? lds32(q_s + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+    lq.qv[s][0] = validB ? lds32(q_s + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
+    lq.qv[s][1] = validB ? lds32(q_s + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
   }
+  lq.negmask = loB ? 0xbc00bc00u : 0u;             // fp16x2 (-1, -1) or (0, 0)
+  lq.zmul = (NT == 2 || qd < 2) ? p.c_log2 : 0.0f;  // lo columns carry no zero-point term
 
   WarpState<GQA> st;
 #pragma unroll
@@ -434,47 +514,65 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
 
   // ---------------------------------------------------------------- page stream
   const int pi = (32 * warp) / p.P, t0 = (32 * warp) % p.P;
-  int consumed = 0;
   for (int c = 0; c < n_chunks; ++c) {
-    __syncthreads();  // every warp is done with chunk c-1; its stage may be refilled
-    if (s_abort) break;
-    if (tid == 0 && issued < n_chunks) issue(issued++);
-    const int stg = c % kStages;
-    if (!mbar_wait_bounded(&bars[stg], uint32_t(c / kStages) & 1u)) {
+    if (tid == 0 && !refill(c, c + kStages - 1)) {
       flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
       s_abort = 1;
-      continue;
+      break;
     }
-    consumed = c + 1;
+    const int stg = c % kStages;
+    if (!mbar_wait_bounded(&full_bar[stg], uint32_t(c / kStages) & 1u)) {
+      flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
+      s_abort = 1;
+      break;
+    }
     if (c * ppc + pi < npg)
-      page_group<T, GQA>(p, main + stg * p.stage_bytes + pi * p.rec_bytes, t0, qv,
-                         reinterpret_cast<const T*>(q_s), hB, loB, validB, st, g, qd);
+      page_group<T, GQA, KB>(p, main + stg * p.stage_bytes + pi * p.rec_bytes, t0, lq, q_s, hB, validB, st, g,
+                             qd);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[stg]);
   }
   __syncthreads();
   if (s_abort) {
-    // drain the copies still in flight (bounded), then leave; the output is undefined
+    // drain the copies that may still be in flight (bounded), then leave; the
+    // output is undefined and the error word says why
     if (tid == 0)
-      for (int c = consumed; c < issued; ++c) mbar_wait_bounded(&bars[c % kStages], uint32_t(c / kStages) & 1u);
+      for (int x = max(0, issued - kStages); x < issued; ++x)
+        mbar_wait_bounded(&full_bar[x % kStages], uint32_t(x / kStages) & 1u);
     __syncthreads();
     return;
   }
+  // page results carry the 0.5 of the code encoding; bring them to real units
+  if (npg > 0) {
+#pragma unroll
+    for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= kCodeScale;
+  }
+
   // ---------------------------------------------------------------- residual window
   if (own_res) {
-    const int rows = (rl + 31) & ~31;
     uint8_t* Kr = main;
-    uint8_t* Vr = main + p.P * kResRowBytes;
+    uint8_t* Vr = main + kResRoundTokens * kResRowBytes;
     const uint8_t* gk = reinterpret_cast<const uint8_t*>(p.res_k + (size_t(b) * p.Hkv + kvh) * p.P * kHeadDim);
     const uint8_t* gv = reinterpret_cast<const uint8_t*>(p.res_v + (size_t(b) * p.Hkv + kvh) * p.P * kHeadDim);
-    for (int i = tid; i < rows * 32; i += kDecodeThreads) {
-      const int which = i / (rows * 16), j = i % (rows * 16), t = j >> 4, c16 = j & 15;
-      const uint8_t* src = (which ? gv : gk) + t * 256 + c16 * 16;
-      uint8_t* dst = (which ? Vr : Kr) + t * kResRowBytes + c16 * 16;
-      cp_async16(dst, t < rl ? src : gk, t < rl ? 16u : 0u);
+    for (int base = 0; base < rl; base += kResRoundTokens) {
+      const int rows = min(kResRoundTokens, (rl - base + 15) & ~15);  // whole 16-row tiles
+      for (int i = tid; i < rows * 32; i += kDecodeThreads) {
+        const int which = i / (rows * 16), j = i % (rows * 16), t = j >> 4, c16 = j & 15;
+        const int tok = base + t;
+        const uint8_t* src = (which ? gv : gk) + tok * 256 + c16 * 16;
+        uint8_t* dst = (which ? Vr : Kr) + t * kResRowBytes + c16 * 16;
+        cp_async16(dst, tok < rl ? src : gk, tok < rl ? 16u : 0u);
+      }
+      cp_async_wait_all();
+      __syncthreads();
+      if (16 * warp < rows)
+        residual_tile<T, GQA>(p, Kr, Vr, 16 * warp, base + 16 * warp, rl, lq, loB, validB, st, lane, g, qd);
+      __syncthreads();
     }
-    cp_async_wait_all();
-    __syncthreads();
-    const int tw = 32 * warp;
-    if (tw < rl) residual_group<T, GQA>(p, Kr, Vr, tw, rl, qv, loB, validB, st, lane, g, qd);
   }
 
   // ---------------------------------------------------------------- merge the 4 warps
@@ -574,12 +672,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
 
 // ---------------------------------------------------------------- host side
 
-// Pages per split: minimises waves x (pages per CTA + startup), where a wave is
-// 2 resident CTAs per SM and the startup cost of a CTA is about 4 pages of streaming.
-SplitPlan plan_splits(int units, int max_pages, int sm_count) {
+// Pages per split.  Resident CTAs (SMs x CTAs per SM) form a wave; the plan
+// minimises waves x (pages per CTA + 2), the 2 standing for the startup of a CTA
+// (page-table read and first copy latency) in units of one page of streaming.
+SplitPlan plan_splits(int units, int max_pages, int slots) {
   SplitPlan best{max(max_pages, 1), 1};
   if (max_pages <= 1 || units <= 0) return best;
-  const long long slots = 2ll * sm_count;
   double best_cost = 1e300;
   const int min_splits = (max_pages + 2047) / 2048;  // page-id list fits in 8 KB of shared memory
   for (int s = max(1, min_splits); s <= min(max_pages, 64); ++s) {
@@ -587,7 +685,7 @@ SplitPlan plan_splits(int units, int max_pages, int sm_count) {
     const int se = (max_pages + pps - 1) / pps;
     const long long ctas = 1ll * units * se;
     const long long waves = (ctas + slots - 1) / slots;
-    const double cost = double(waves) * (pps + 4);
+    const double cost = double(waves) * (pps + 2);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = {pps, se};
@@ -596,43 +694,89 @@ SplitPlan plan_splits(int units, int max_pages, int sm_count) {
   return best;
 }
 
+// Calls f.template operator()<T, GQA, KB>() for the instantiation of a configuration.
+template <typename F>
+cudaError_t dispatch(int gqa, int dtype, int kb, F&& f) {
+#define KVQ_KB(T, G)                                 \
+  switch (kb) {                                      \
+    case 0: return f.template operator()<T, G, 0>(); \
+    case 1: return f.template operator()<T, G, 1>(); \
+    case 2: return f.template operator()<T, G, 2>(); \
+    case 4: return f.template operator()<T, G, 4>(); \
+    case 8: return f.template operator()<T, G, 8>(); \
+  }                                                  \
+  return cudaErrorInvalidValue;
+#define KVQ_GQA(T)           \
+  switch (gqa) {             \
+    case 1: { KVQ_KB(T, 1) } \
+    case 2: { KVQ_KB(T, 2) } \
+    case 4: { KVQ_KB(T, 4) } \
+    case 8: { KVQ_KB(T, 8) } \
+  }                          \
+  return cudaErrorInvalidValue;
+  if (dtype == KVQ_BF16) {
+    KVQ_GQA(__nv_bfloat16)
+  } else {
+    KVQ_GQA(__half)
+  }
+#undef KVQ_GQA
+#undef KVQ_KB
+}
+
+// Raises the dynamic shared-memory limit of one decode instantiation (once per size).
+template <typename T, int GQA, int KB>
+cudaError_t prepare_decode(size_t smem_bytes) {
+  static int seen[64];
+  return ensure_dynamic_smem(decode_kernel<T, GQA, KB>, int(smem_bytes), seen);
+}
+
+struct OccupancyQuery {
+  size_t smem;
+  int* n;
+  template <typename T, int GQA, int KB>
+  cudaError_t operator()() {
+    cudaError_t e = prepare_decode<T, GQA, KB>(smem);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, decode_kernel<T, GQA, KB>, kDecodeThreads, smem);
+  }
+};
+
+// Resident decode CTAs per SM for this configuration (2 when it cannot be queried,
+// e.g. without a device).
+int decode_ctas_per_sm(int gqa, int dtype, int kb, size_t smem_bytes) {
+  int n = 0;
+  if (dispatch(gqa, dtype, kb, OccupancyQuery{smem_bytes, &n}) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 2;
+  }
+  return n;
+}
+
 size_t decode_main_bytes(int P, int GQA, uint32_t rec_bytes) {
   const size_t stage = size_t(128 / P) * rec_bytes;
   size_t m = kStages * stage;
-  m = std::max(m, size_t(P) * 2 * kResRowBytes);
+  m = std::max(m, size_t(kResRoundTokens) * 2 * kResRowBytes);
   m = std::max(m, size_t(4) * GQA * kHeadDim * 4);
   return (m + 127) / 128 * 128;
 }
 
-template <typename T, int GQA>
-cudaError_t launch_decode_t(DecodeParams p, cudaStream_t stream) {
-  const size_t smem = size_t(p.main_bytes) + size_t(p.pps) * 4;
-  static int seen[64];
-  cudaError_t e = ensure_dynamic_smem(decode_kernel<T, GQA>, int(smem), seen);
-  if (e != cudaSuccess) return e;
-  const dim3 grid(p.max_splits, p.Hkv, p.batch);
-  decode_kernel<T, GQA><<<grid, kDecodeThreads, smem, stream>>>(p);
-  return cudaGetLastError();
-}
+struct DecodeLaunch {
+  const DecodeParams& p;
+  cudaStream_t stream;
+  template <typename T, int GQA, int KB>
+  cudaError_t operator()() {
+    const size_t smem = size_t(p.main_bytes) + size_t(p.pps) * 4;
+    cudaError_t e = prepare_decode<T, GQA, KB>(smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(p.max_splits, p.Hkv, p.batch);
+    decode_kernel<T, GQA, KB><<<grid, kDecodeThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  }
+};
 
 cudaError_t launch_decode(const DecodeParams& p, int gqa, int dtype, cudaStream_t stream) {
   if (p.batch <= 0) return cudaSuccess;
-  if (dtype == KVQ_BF16) {
-    switch (gqa) {
-      case 1: return launch_decode_t<__nv_bfloat16, 1>(p, stream);
-      case 2: return launch_decode_t<__nv_bfloat16, 2>(p, stream);
-      case 4: return launch_decode_t<__nv_bfloat16, 4>(p, stream);
-      case 8: return launch_decode_t<__nv_bfloat16, 8>(p, stream);
-    }
-  } else {
-    switch (gqa) {
-      case 1: return launch_decode_t<__half, 1>(p, stream);
-      case 2: return launch_decode_t<__half, 2>(p, stream);
-      case 4: return launch_decode_t<__half, 4>(p, stream);
-      case 8: return launch_decode_t<__half, 8>(p, stream);
-    }
-  }
-  return cudaErrorInvalidValue;
+  return dispatch(gqa, dtype, p.KB, DecodeLaunch{p, stream});
 }
 
 }  // namespace kvq

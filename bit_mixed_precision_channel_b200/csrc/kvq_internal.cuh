@@ -44,6 +44,24 @@ inline Layout make_layout(int P, int D, int k, int G) {
   return L;
 }
 
+// Storage order of the packed rows (see the page-record description in kvq.h).
+// Key channel c = 16s + 8r + 2q + f  <->  position 32q + 4s + 2r + f.
+__host__ __device__ __forceinline__ int key_pos(int c) {
+  return 32 * ((c >> 1) & 3) + 4 * (c >> 4) + 2 * ((c >> 3) & 1) + (c & 1);
+}
+// Boosted row j = 16s + 8r + 2q + f  <->  position 4*KB*q + 4s + 2r + f.
+__host__ __device__ __forceinline__ int boost_pos(int j, int KB) {
+  return 4 * KB * ((j >> 1) & 3) + 4 * (j >> 4) + 2 * ((j >> 3) & 1) + (j & 1);
+}
+// Value token at position p = 32g + 8q + 4s + 2r + f  <->  token 32g + 16s + 8r + 2q + f.
+__host__ __device__ __forceinline__ int value_token_at(int p) {
+  return (p & ~31) + 16 * ((p >> 2) & 1) + 8 * ((p >> 1) & 1) + 2 * ((p >> 3) & 3) + (p & 1);
+}
+// Bit of element e = 8a + 2b + f inside a code word: 8b + 4f + 2a.
+__host__ __device__ __forceinline__ int elem_bit(int e) {
+  return 8 * ((e >> 1) & 3) + 4 * (e & 1) + 2 * (e >> 3);
+}
+
 __device__ __forceinline__ void flag_error(int32_t* err, int bits) {
   if (err) atomicOr(err, bits);
 }
@@ -102,6 +120,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the same condition.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Arrives once on `bar` (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
 // Waits for the phase of `parity` to complete; gives up after ~2^32 SM cycles
 // (about two seconds) and returns false so the caller can flag an error and leave.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
@@ -143,7 +177,7 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // D += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
                                           __half) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -151,7 +185,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 }
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
                                           __nv_bfloat16) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -159,18 +193,20 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 }
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+               : "r"(addr)
+               : "memory");
 }
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+               : "r"(addr)
+               : "memory");
 }
 
 // 2^x (hardware approximation, relative error ~2^-22; -inf -> 0).
@@ -183,16 +219,35 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// Two 2-bit codes of a packed word as an exact fp16 pair for the tensor cores: pair j
-// holds elements 2j (low half) and 2j+1 (high half).  OR-ing a code into the mantissa
-// of 1024.0 (0x6400) gives the fp16 value 1024 + code exactly; subtracting 1024 leaves
-// the code.  (Feeding the masked bits directly as fp16 subnormals, code * 2^-24, saves
-// the subtraction but was measured to lose the small products of the low operand part
-// inside the tensor core, ~1e-3 output error; the integers keep every product exact.)
-__device__ __forceinline__ uint32_t code_pair(uint32_t w, int j) {
-  const uint32_t x = ((w >> (2 * j)) & 0x00030003u) | 0x64006400u;
-  return h2_as_u32(__hsub2(u32_as_h2(x), __half2(__half(1024.0f), __half(1024.0f))));
+// Four fp16 pairs from one masked pass of a code word.  After x = (w >> 2a) & 0x33333333
+// every nibble of x holds one 2-bit code in its low bits, which read as an FP4 (e2m1)
+// number is exactly 0.5 * code (0, 0.5, 1, 1.5).  The hardware conversion turns each
+// byte of x into an fp16 pair (low nibble -> low half): byte b gives elements
+// (8a + 2b, 8a + 2b + 1) of the word.  Products with the other operand stay exact;
+// the factor 0.5 is undone after the contraction.
+constexpr float kCodeScale = 2.0f;  // value of a code / value delivered to the tensor cores
+__device__ __forceinline__ void e2m1_pairs(uint32_t x, uint32_t& p0, uint32_t& p1, uint32_t& p2, uint32_t& p3) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(p0), "=r"(p1), "=r"(p2), "=r"(p3)
+      : "r"(x));
 }
+// The fp16 pair of byte 0 of x (x already masked).
+__device__ __forceinline__ uint32_t e2m1_pair_lo(uint32_t x) {
+  uint32_t d;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+      : "=r"(d)
+      : "r"(x));
+  return d;
+}
+__device__ __forceinline__ uint32_t code_pass(uint32_t w, int a) { return (w >> (2 * a)) & 0x33333333u; }
+
 __device__ __forceinline__ uint32_t bf2_as_u32(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
 // ------------------------------------------------------------------ launch parameters
@@ -252,7 +307,8 @@ cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, voi
 cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32_t* page_table, int max_pages,
                                 int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int gqa, int dtype, cudaStream_t stream);
-SplitPlan plan_splits(int units, int max_pages, int sm_count);
+SplitPlan plan_splits(int units, int max_pages, int slots);
+int decode_ctas_per_sm(int gqa, int dtype, int kb, size_t smem_bytes);
 
 // Raises a kernel's dynamic shared-memory limit once per device and size, so that
 // later calls (and calls made while a stream is being captured into a graph) issue

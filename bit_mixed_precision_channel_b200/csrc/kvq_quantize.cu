@@ -29,16 +29,18 @@ struct QSmem {
   }
 };
 
+// 16 codes given by element order (one byte each) -> one word, element e = 8a + 2b + f
+// at bit 8b + 4f + 2a.  Bytes 4i..4i+3 (element 4i + m) land at bit
+// 16*(i & 1) + 2*(i >> 1) + 4*m.
 __device__ __forceinline__ uint32_t pack16(const uint8_t* c) {
-  // 16 codes -> one word: element e at bit 16*(e & 1) + 2*(e >> 1).
   const uint4 v = lds128(c);
   const uint32_t q[4] = {v.x, v.y, v.z, v.w};
   uint32_t w = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t x = q[i];  // elements 4i .. 4i+3, one per byte
-    const uint32_t part = (x & 0x3u) | ((x >> 14) & 0xCu) | ((x << 8) & 0x30000u) | ((x >> 6) & 0xC0000u);
-    w |= part << (4 * i);
+    const uint32_t x = q[i];
+    const uint32_t nib = (x & 0x3u) | ((x >> 4) & 0x30u) | ((x >> 8) & 0x300u) | ((x >> 12) & 0x3000u);
+    w |= nib << (16 * (i & 1) + 2 * (i >> 1));
   }
   return w;
 }
@@ -89,8 +91,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
   uint16_t* Vs = Ks + P * kHeadDim;
-  uint8_t* cA = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);
-  uint8_t* cB = cA + P * kHeadDim;
+  uint8_t* cA = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);  // plane A codes [token][key position]
+  uint8_t* cB = cA + P * kHeadDim;                                // plane B codes [token][boost position]
   uint8_t* cV = cB + P * (k > 0 ? k : 16);
   float* score = reinterpret_cast<float*>(cV + P * kHeadDim);
   int* row_of = reinterpret_cast<int*>(score + kHeadDim);
@@ -172,6 +174,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       }
       const int j = row_of[c];
       const int qmax = j >= 0 ? 15 : 3;
+      const int pc = key_pos(c);
+      const int pj = j >= 0 ? boost_pos(j, k / 16) : 0;
       uint16_t sb, zb;
       float zero;
       const float scale = quant_params<T>(mn, mx, qmax, sb, zb, zero);
@@ -179,15 +183,15 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         const int tok = g * kKeyGroup + t;
         const int code = quant_code(bits_to_float(col[t * kHeadDim], T()), zero, scale, qmax);
         if (j >= 0) {
-          cA[tok * kHeadDim + c] = uint8_t(code >> 2);
-          cB[tok * k + j] = uint8_t(code & 3);
+          cA[tok * kHeadDim + pc] = uint8_t(code >> 2);
+          cB[tok * k + pj] = uint8_t(code & 3);
         } else {
-          cA[tok * kHeadDim + c] = uint8_t(code);
+          cA[tok * kHeadDim + pc] = uint8_t(code);
         }
       }
       // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
-      ks_out[g * kHeadDim + c] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
-      kz_out[g * kHeadDim + c] = zb;
+      ks_out[g * kHeadDim + pc] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
+      kz_out[g * kHeadDim + pc] = zb;
       if (j >= 0) kbs_out[g * k + j] = sb;
     }
   }
@@ -235,12 +239,12 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
     uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
     const int vw = P / 16;
     for (int i = tid; i < kHeadDim * vw; i += kQThreads) {
-      // word (channel c, w) holds tokens 16w .. 16w+15 of channel c
+      // word (channel c, w) holds the tokens stored at positions 16w .. 16w+15 of row c
       const int c = i / vw, w = i % vw;
       uint32_t word = 0;
 #pragma unroll
       for (int e = 0; e < 16; ++e)
-        word |= uint32_t(cV[(16 * w + e) * kHeadDim + c] & 3u) << (16 * (e & 1) + 2 * (e >> 1));
+        word |= uint32_t(cV[value_token_at(16 * w + e) * kHeadDim + c] & 3u) << elem_bit(e);
       vq[i] = word;
     }
   }

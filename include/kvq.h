@@ -53,20 +53,28 @@
  *   k_codes   uint32 [P][D/16]   plane A, token-major; word (t, w) = channels 16w..16w+15 of token t
  *   kb_codes  uint32 [P][k/16]   plane B, token-major; word (t, w) = boosted rows 16w..16w+15
  *   v_codes   uint32 [D][P/16]   values, channel-major; word (c, w) = tokens 16w..16w+15 of channel c
- *   k_scale   S [P/G][D]         plane-A scale per (group, channel)
- *   k_zero    S [P/G][D]         plane-A zero  per (group, channel)
+ *   k_scale   S [P/G][D]         plane-A scale per (group, key position)
+ *   k_zero    S [P/G][D]         plane-A zero  per (group, key position)
  *   kb_scale  S [P/G][k]         plane-B scale per (group, boosted row)
  *   v_scale   S [P]              value scale per token
  *   v_zero    S [P]              value zero  per token
  *   boost_idx uint8 [k]          boosted channels, ascending
  * The record stride (kvq_page_bytes) rounds the payload up to a multiple of 128 bytes;
  * the padding bytes are never read.
- * Inside a 32-bit code word the 16 two-bit elements e = 0..15 are interleaved:
- * element e sits at bit 16*(e & 1) + 2*(e >> 1), i.e. even elements fill the low
- * half-word and odd elements the high half-word, each half little-endian in 2-bit steps.
  * Keys are packed along channels and values along tokens — the contraction axis of
  * q.K^T and of p.V respectively — so that the decode kernel can feed codes straight
- * into its matrix products with the scales folded into the other operand.
+ * into its matrix products with the scales folded into the other operand.  Within a
+ * row, elements are stored in the order in which the decode kernel's matrix-fragment
+ * lanes consume them, and inside a 32-bit word so that one masked byte holds the two
+ * codes of one fragment register:
+ *   key channel c   = 16s + 8r + 2q + f        -> position 32q + 4s + 2r + f
+ *                     (plane-A codes of a token row, and the k_scale / k_zero rows)
+ *   boosted row j   = 16s + 8r + 2q + f        -> position 4*KB*q + 4s + 2r + f, KB = k/16
+ *   value token t   = 32g + 16s + 8r + 2q + f  -> position 32g + 8q + 4s + 2r + f
+ *   (s, r, f, q ranging over the values that keep each part in its range).  Position p
+ *   of a row is element p % 16 of word p / 16, and element e = 8a + 2b + f of a word
+ *   (a, f in {0,1}, b in 0..3) occupies bits 8b + 4f + 2a.  kb_scale, v_scale, v_zero
+ *   and boost_idx are in natural order.
  *
  * Pool: uint8 pool[pool_pages][num_kv_heads][kvq_page_bytes(cfg)], 256-byte aligned base.
  * Residual window: dtype res_k/res_v[batch][num_kv_heads][page_tokens][head_dim];
@@ -125,7 +133,8 @@ typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 /* Shape and precision of one attention layer's KV cache.
  * Supported: head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8};
  * page_tokens in {32, 64, 128}; key_group 32; key_bits 2, boost_bits 4, value_bits 2;
- * num_boost a multiple of 16 in [0, head_dim]; dtype KVQ_F16 or KVQ_BF16
+ * num_boost in {0, 16, 32, 64, 128} (0% .. 100% of the channels; 12.5% and 25% are the
+ * ratios the method is run with); dtype KVQ_F16 or KVQ_BF16
  * (keys, values, queries, residual, scales and zeros all use dtype). */
 typedef struct {
   int32_t head_dim;

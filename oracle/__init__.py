@@ -23,6 +23,8 @@ What it follows (web pages on the method, by title and section):
 
 Readings where the pages are silent (listed again in the design notes):
 scale = (max-min)/(2^b-1) in fp32, rounded up to the storage type; zero = min;
+a fixed storage order of channels and tokens inside the packed rows (see
+kvq_oracle.c: elem_shift, key_pos, boost_pos, value_pos);
 round half to even; clamp; scale 0 gives code 0; magnitude = max |x| over the page;
 ties to the lower channel index; boost set per (page, KV head); 4-bit code =
 4*hi + lo; key groups aligned to the page start; residual flushed when it holds a
@@ -81,6 +83,11 @@ def lib():
         L.kvqo_quant_group.restype = None
         L.kvqo_quant_group.argtypes = [u16p, ctypes.c_int, ctypes.c_long, ctypes.c_int,
                                        ctypes.c_int, u8p, u16p, u16p]
+        for name in ("kvqo_elem_shift", "kvqo_key_pos", "kvqo_value_pos"):
+            getattr(L, name).restype = ctypes.c_int
+            getattr(L, name).argtypes = [ctypes.c_int]
+        L.kvqo_boost_pos.restype = ctypes.c_int
+        L.kvqo_boost_pos.argtypes = [ctypes.c_int, ctypes.c_int]
         L.kvqo_layout.restype = None
         L.kvqo_layout.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(ctypes.c_long)]
         L.kvqo_select_boost.restype = None
@@ -140,6 +147,26 @@ def quant_group(x_bits: np.ndarray, bits: int, dtype: int):
 
 
 # ---------------------------------------------------------------------- page layout
+
+def elem_shift(e: int) -> int:
+    """Bit position of element e (0..15) of a 32-bit code word."""
+    return lib().kvqo_elem_shift(e)
+
+
+def key_pos(c: int) -> int:
+    """Storage position of key channel c in plane-A rows and plane-A scale/zero rows."""
+    return lib().kvqo_key_pos(c)
+
+
+def boost_pos(j: int, KB: int) -> int:
+    """Storage position of boosted row j in plane-B rows (KB = boosted channels / 16)."""
+    return lib().kvqo_boost_pos(j, KB)
+
+
+def value_pos(t: int) -> int:
+    """Storage position of token t in a value row."""
+    return lib().kvqo_value_pos(t)
+
 
 LAYOUT_KEYS = ("k_codes", "kb_codes", "v_codes", "k_scale", "k_zero", "kb_scale",
                "v_scale", "v_zero", "boost_idx", "payload_bytes", "record_bytes")

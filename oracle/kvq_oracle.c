@@ -200,16 +200,50 @@ void kvqo_layout(int P, int D, int k, int G, long* out /* 11 entries */) {
   memcpy(out, v, sizeof v);
 }
 
-/* Position of element e (0..15) inside a 32-bit code word: even elements in the low
- * half-word, odd elements in the high half-word, 2 bits apart. */
-static int elem_shift(int e) { return 16 * (e & 1) + 2 * (e >> 1); }
-
-static void put2(uint32_t* words, int word, int e, unsigned code) {
-  words[word] |= (uint32_t)(code & 3u) << elem_shift(e);
+/* Bit position of element e (0..15) inside a 32-bit code word.  Writing
+ * e = 8a + 2b + f (a, f in {0,1}, b in 0..3), element e occupies bits 8b + 4f + 2a:
+ * byte b holds elements 2b, 2b+1 (a = 0) in the low two bits of its two nibbles and
+ * elements 8+2b, 9+2b (a = 1) in the high two bits. */
+static int elem_shift(int e) {
+  const int a = e >> 3, b = (e >> 1) & 3, f = e & 1;
+  return 8 * b + 4 * f + 2 * a;
 }
 
-static unsigned get2(const uint32_t* words, int word, int e) {
-  return (words[word] >> elem_shift(e)) & 3u;
+/* Storage position of key channel c (0..127) inside a plane-A row and inside the
+ * plane-A scale and zero rows.  Writing c = 16s + 8r + 2q + f (s in 0..7, r, f in
+ * {0,1}, q in 0..3), the position is 32q + 4s + 2r + f. */
+static int key_pos(int c) {
+  const int s = c >> 4, r = (c >> 3) & 1, q = (c >> 1) & 3, f = c & 1;
+  return 32 * q + 4 * s + 2 * r + f;
+}
+
+/* Storage position of boosted row j (0..k-1) inside a plane-B row, KB = k/16:
+ * j = 16s + 8r + 2q + f -> 4*KB*q + 4s + 2r + f. */
+static int boost_pos(int j, int KB) {
+  const int s = j >> 4, r = (j >> 3) & 1, q = (j >> 1) & 3, f = j & 1;
+  return 4 * KB * q + 4 * s + 2 * r + f;
+}
+
+/* Storage position of token t (0..P-1) inside a value row (one channel):
+ * t = 32g + 16s + 8r + 2q + f (s, r, f in {0,1}, q in 0..3) -> 32g + 8q + 4s + 2r + f. */
+static int value_pos(int t) {
+  const int g = t >> 5, s = (t >> 4) & 1, r = (t >> 3) & 1, q = (t >> 1) & 3, f = t & 1;
+  return 32 * g + 8 * q + 4 * s + 2 * r + f;
+}
+
+int kvqo_elem_shift(int e) { return elem_shift(e); }
+int kvqo_key_pos(int c) { return key_pos(c); }
+int kvqo_boost_pos(int j, int KB) { return boost_pos(j, KB); }
+int kvqo_value_pos(int t) { return value_pos(t); }
+
+/* Writes / reads the 2-bit code at storage position pos of row `row` (words_per_row
+ * words of 16 elements each). */
+static void put2(uint32_t* words, int row, int words_per_row, int pos, unsigned code) {
+  words[row * words_per_row + pos / 16] |= (uint32_t)(code & 3u) << elem_shift(pos % 16);
+}
+
+static unsigned get2(const uint32_t* words, int row, int words_per_row, int pos) {
+  return (words[row * words_per_row + pos / 16] >> elem_shift(pos % 16)) & 3u;
 }
 
 /* -------------------------------------------------------------- boost selection (a1) */
@@ -278,21 +312,22 @@ void kvqo_quantize_page(const uint16_t* K, const uint16_t* V, long tok_stride, i
       const uint16_t* col = K + (long)g * G * tok_stride + c;
       uint16_t sb, zb;
       int j = row_of[c];
+      const int pc = key_pos(c);
       if (j < 0) {
         kvqo_quant_group(col, G, tok_stride, 2, dtype, codes, &sb, &zb);
-        for (int t = 0; t < G; ++t) put2(kA, (g * G + t) * kw + c / 16, c % 16, codes[t]);
-        ks[g * D + c] = sb;
+        for (int t = 0; t < G; ++t) put2(kA, g * G + t, kw, pc, codes[t]);
+        ks[g * D + pc] = sb;
       } else {
         kvqo_quant_group(col, G, tok_stride, 4, dtype, codes, &sb, &zb);
         for (int t = 0; t < G; ++t) {
-          put2(kA, (g * G + t) * kw + c / 16, c % 16, codes[t] >> 2);
-          put2(kB, (g * G + t) * kbw + j / 16, j % 16, codes[t] & 3);
+          put2(kA, g * G + t, kw, pc, codes[t] >> 2);
+          put2(kB, g * G + t, kbw, boost_pos(j, kbw), codes[t] & 3);
         }
         /* plane A carries the high bits with four times the 4-bit scale (exact) */
-        ks[g * D + c] = dt_round(4.0 * dt_value(sb, dtype), dtype, 0);
+        ks[g * D + pc] = dt_round(4.0 * dt_value(sb, dtype), dtype, 0);
         kbs[g * k + j] = sb;
       }
-      kz[g * D + c] = zb;
+      kz[g * D + pc] = zb;
     }
   }
 
@@ -301,7 +336,7 @@ void kvqo_quantize_page(const uint16_t* K, const uint16_t* V, long tok_stride, i
   for (int t = 0; t < P; ++t) {
     uint16_t sb, zb;
     kvqo_quant_group(V + (long)t * tok_stride, D, 1, 2, dtype, codes, &sb, &zb);
-    for (int c = 0; c < D; ++c) put2(vq, c * vw + t / 16, t % 16, codes[c]);
+    for (int c = 0; c < D; ++c) put2(vq, c, vw, value_pos(t), codes[c]);
     vs[t] = sb;
     vz[t] = zb;
   }
@@ -328,11 +363,12 @@ void kvqo_dequantize_page(const uint8_t* rec, int P, int D, int G, int k, int dt
     for (int t = 0; t < P; ++t) {
       int g = t / G;
       for (int c = 0; c < D; ++c) {
-        unsigned a = get2(kA, t * kw + c / 16, c % 16);
-        Khat[t * D + c] = a * dt_value(ks[g * D + c], dtype) + dt_value(kz[g * D + c], dtype);
+        const int pc = key_pos(c);
+        unsigned a = get2(kA, t, kw, pc);
+        Khat[t * D + c] = a * dt_value(ks[g * D + pc], dtype) + dt_value(kz[g * D + pc], dtype);
       }
       for (int j = 0; j < k; ++j) {
-        unsigned b = get2(kB, t * kbw + j / 16, j % 16);
+        unsigned b = get2(kB, t, kbw, boost_pos(j, kbw));
         Khat[t * D + bidx[j]] += b * dt_value(kbs[g * k + j], dtype);
       }
     }
@@ -340,7 +376,7 @@ void kvqo_dequantize_page(const uint8_t* rec, int P, int D, int G, int k, int dt
   if (Vhat) {
     for (int t = 0; t < P; ++t)
       for (int c = 0; c < D; ++c) {
-        unsigned v = get2(vq, c * vw + t / 16, t % 16);
+        unsigned v = get2(vq, c, vw, value_pos(t));
         Vhat[t * D + c] = v * dt_value(vs[t], dtype) + dt_value(vz[t], dtype);
       }
   }

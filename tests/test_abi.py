@@ -55,7 +55,7 @@ def test_layout_matches_hand_worked_sizes(lib):
 @pytest.mark.parametrize("over,status", [
     (dict(head_dim=64), 2), (dict(num_q_heads=12, num_kv_heads=8), 1), (dict(num_q_heads=48, num_kv_heads=4), 2),
     (dict(page_tokens=96), 2), (dict(page_tokens=100), 1), (dict(key_group=64), 2), (dict(num_boost=8), 1),
-    (dict(num_boost=144), 1), (dict(key_bits=3), 2), (dict(dtype=7), 2), (dict(), 0), (dict(num_boost=0), 0),
+    (dict(num_boost=144), 1), (dict(num_boost=48), 2), (dict(num_boost=64), 0), (dict(key_bits=3), 2), (dict(dtype=7), 2), (dict(), 0), (dict(num_boost=0), 0),
 ])
 def test_check_config(lib, over, status):
     assert kb.check_config(kb.Config(**over)) == status

@@ -70,10 +70,11 @@ SHAPES = [
     (8, kb.BF16, 128, 32, [2048 + 5, 130]),
     (8, kb.F16, 128, 32, [777, 256]),
     (1, kb.F16, 32, 16, [256, 250, 31]),
-    (2, kb.BF16, 64, 48, [64 * 9 + 63, 100]),
+    (2, kb.BF16, 64, 64, [64 * 9 + 63, 100]),
     (4, kb.F16, 64, 0, [64 * 20 + 3]),
     (1, kb.BF16, 32, 128, [32 * 13 + 17]),
-    (2, kb.F16, 128, 112, [128 * 3 + 127]),
+    (2, kb.F16, 128, 128, [128 * 3 + 127]),
+    (4, kb.F16, 128, 64, [128 * 9 + 3, 77]),
 ]
 
 

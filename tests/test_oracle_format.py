@@ -1,5 +1,10 @@
-"""Pins of the oracle's page record: layout sizes, bit packing, boost selection,
-the two-plane split of boosted channels and the KIVI (no boost) special case."""
+"""Pins of the oracle's page record: layout sizes, element and channel/token storage
+order (hand-worked golden values), boost selection, the two-plane split of boosted
+channels and the KIVI (no boost) special case.
+
+The decoder `_decode_record` below reads a record with numpy bit operations written
+from the rules stated in tests/golden/packing_examples.json, independently of the
+oracle's C code."""
 import json
 import os
 
@@ -18,6 +23,69 @@ def _golden():
         return json.load(f)
 
 
+# -------------------------------------------------------------- independent decoder
+
+def _shift(e):
+    """element e = 8a + 2b + f of a word sits at bit 8b + 4f + 2a"""
+    e = np.asarray(e)
+    return 8 * ((e >> 1) & 3) + 4 * (e & 1) + 2 * (e >> 3)
+
+
+def _key_channel(p):
+    """inverse of the key storage order: position 32q + 4s + 2r + f -> channel 16s + 8r + 2q + f"""
+    p = np.asarray(p)
+    q, s, r, f = p >> 5, (p >> 2) & 7, (p >> 1) & 1, p & 1
+    return 16 * s + 8 * r + 2 * q + f
+
+
+def _boost_row(p, KB):
+    p = np.asarray(p)
+    q, rem = p // (4 * KB), p % (4 * KB)
+    s, r, f = rem >> 2, (rem >> 1) & 1, rem & 1
+    return 16 * s + 8 * r + 2 * q + f
+
+
+def _value_token(p):
+    p = np.asarray(p)
+    g, rem = p >> 5, p & 31
+    q, s, r, f = rem >> 3, (rem >> 2) & 1, (rem >> 1) & 1, rem & 1
+    return 32 * g + 16 * s + 8 * r + 2 * q + f
+
+
+def _words_to_positions(words):
+    """[rows][n_words] uint32 -> [rows][16 * n_words] codes by storage position"""
+    w = np.asarray(words, np.uint32)
+    e = np.arange(16)
+    return ((w[..., None] >> _shift(e).astype(np.uint32)) & 3).reshape(w.shape[0], -1)
+
+
+def _decode_record(rec, P, k, dtype):
+    """-> dict of planes in natural order: kA [P][128], kB [P][k], v [P][128], scales..."""
+    L = oracle.layout(P, 128, k, 32)
+    KB = k // 16
+    u16 = lambda a, b: rec[a:b].view(np.uint16)
+    kA_pos = _words_to_positions(rec[L["k_codes"]:L["kb_codes"]].view(np.uint32).reshape(P, 8))
+    kA = np.zeros((P, 128), np.int64)
+    kA[:, _key_channel(np.arange(128))] = kA_pos
+    kB = np.zeros((P, k), np.int64)
+    if k:
+        kB_pos = _words_to_positions(rec[L["kb_codes"]:L["v_codes"]].view(np.uint32).reshape(P, KB))
+        kB[:, _boost_row(np.arange(k), KB)] = kB_pos
+    v_pos = _words_to_positions(rec[L["v_codes"]:L["k_scale"]].view(np.uint32).reshape(128, P // 16))
+    v = np.zeros((P, 128), np.int64)
+    v[_value_token(np.arange(P)), :] = v_pos.T
+    ks = np.zeros((P // 32, 128), np.uint16)
+    kz = np.zeros((P // 32, 128), np.uint16)
+    ks[:, _key_channel(np.arange(128))] = u16(L["k_scale"], L["k_zero"]).reshape(P // 32, 128)
+    kz[:, _key_channel(np.arange(128))] = u16(L["k_zero"], L["kb_scale"]).reshape(P // 32, 128)
+    return dict(kA=kA, kB=kB, v=v, ks=ks, kz=kz,
+                kbs=u16(L["kb_scale"], L["v_scale"]).reshape(P // 32, k),
+                vs=u16(L["v_scale"], L["v_zero"]), vz=u16(L["v_zero"], L["boost_idx"]),
+                idx=rec[L["boost_idx"]:L["boost_idx"] + k])
+
+
+# -------------------------------------------------------------------------- pins
+
 @pytest.mark.parametrize("row", _golden()["layout"], ids=lambda r: f"P{r['P']}k{r['k']}")
 def test_layout_sizes_hand_worked(row):
     L = oracle.layout(row["P"], row["D"], row["k"], row["G"])
@@ -30,41 +98,50 @@ def test_layout_sizes_hand_worked(row):
     assert all(o % 16 == 0 for o in offs[:-1])
 
 
-def _page_with_codes(word_codes, cfg):
-    """A page whose token 0 / channels 0..15 plane-A codes are word_codes and whose
-    other channels are constant, with no boost (k = 0) so codes are plain 2-bit."""
-    P, D = cfg.P, cfg.D
-    K = np.zeros((P, D), np.float32)
-    # channel c: token 0 carries code*1.0, the group spans [0, 3] (token 1 = 3, token 2 = 0)
-    for c in range(16):
-        K[0, c] = word_codes[c]
-        K[1, c] = 3.0
-        K[2, c] = 0.0
-    return syn.to_bits(K, cfg.dtype), syn.to_bits(np.zeros((P, D), np.float32), cfg.dtype)
+def test_storage_positions_hand_worked():
+    g = _golden()
+    for c, p in g["key_pos"]:
+        assert oracle.key_pos(c) == p
+    for KB, j, p in g["boost_pos"]:
+        assert oracle.boost_pos(j, KB) == p
+    for t, p in g["value_pos"]:
+        assert oracle.value_pos(t) == p
+    # each order is a permutation, and inverts the decoder's reading of the rule
+    assert sorted(oracle.key_pos(c) for c in range(128)) == list(range(128))
+    assert all(_key_channel(oracle.key_pos(c)) == c for c in range(128))
+    for KB in (1, 2, 4, 8):
+        assert sorted(oracle.boost_pos(j, KB) for j in range(16 * KB)) == list(range(16 * KB))
+        assert all(_boost_row(oracle.boost_pos(j, KB), KB) == j for j in range(16 * KB))
+    assert all(_value_token(oracle.value_pos(t)) == t for t in range(128))
+    assert [oracle.elem_shift(e) for e in range(16)] == list(_shift(np.arange(16)))
 
 
 @pytest.mark.parametrize("case", _golden()["words"], ids=lambda c: c["word"])
-def test_plane_a_word_packing_hand_worked(case):
-    cfg = oracle.Cfg(P=32, k=0, Hq=1, Hkv=1)
-    K, V = _page_with_codes(case["codes"], cfg)
-    rec = oracle.quantize_page(K, V, cfg)
+def test_key_word_packing_hand_worked(case):
+    """Word 0 of token row 0 holds the key channels stored at positions 0..15; give
+    element e the code case["codes"][e] through a real page and read the word back."""
+    cfg = oracle.Cfg(P=32, k=0)
+    K = np.zeros((cfg.P, cfg.D), np.float32)
+    for e, code in enumerate(case["codes"]):
+        c = int(_key_channel(e))
+        K[0, c] = code
+        K[1, c] = 3.0  # the group spans [0, 3]: scale 1, zero 0
+    rec = oracle.quantize_page(syn.to_bits(K, F16), syn.to_bits(np.zeros_like(K), F16), cfg)
     L = oracle.layout(cfg.P, cfg.D, cfg.k, cfg.G)
-    word = int(rec[L["k_codes"]:L["k_codes"] + 4].view(np.uint32)[0])
-    assert word == int(case["word"], 16)
+    assert int(rec[L["k_codes"]:L["k_codes"] + 4].view(np.uint32)[0]) == int(case["word"], 16)
 
 
 @pytest.mark.parametrize("case", _golden()["words"], ids=lambda c: c["word"])
 def test_value_word_packing_hand_worked(case):
-    """Values are packed along tokens: channel 0, tokens 0..15 form the first word."""
+    """Word 0 of channel row 0 holds the tokens stored at positions 0..15."""
     cfg = oracle.Cfg(P=32, k=0)
     V = np.zeros((cfg.P, cfg.D), np.float32)
-    V[:, 1] = 3.0                      # every token's range is [0, 3]: scale 1, zero 0
-    V[:16, 0] = case["codes"]
-    Vb = syn.to_bits(V, F16)
-    rec = oracle.quantize_page(np.zeros((cfg.P, cfg.D), np.uint16), Vb, cfg)
+    V[:, 1] = 3.0  # every token's range is [0, 3]: scale 1, zero 0
+    for e, code in enumerate(case["codes"]):
+        V[int(_value_token(e)), 0] = code
+    rec = oracle.quantize_page(np.zeros((cfg.P, cfg.D), np.uint16), syn.to_bits(V, F16), cfg)
     L = oracle.layout(cfg.P, cfg.D, cfg.k, cfg.G)
-    word = int(rec[L["v_codes"]:L["v_codes"] + 4].view(np.uint32)[0])
-    assert word == int(case["word"], 16)
+    assert int(rec[L["v_codes"]:L["v_codes"] + 4].view(np.uint32)[0]) == int(case["word"], 16)
 
 
 def test_select_boost_matches_full_sort():
@@ -83,51 +160,37 @@ def test_select_boost_matches_full_sort():
         assert idx.tolist() == want
 
 
-def _unpack(words, n_per_row):
-    """Reads 2-bit elements through numpy bit ops (independent of the oracle's helpers)."""
-    w = np.asarray(words, np.uint32)
-    e = np.arange(16)
-    shifts = (16 * (e & 1) + 2 * (e >> 1)).astype(np.uint32)
-    return ((w[..., None] >> shifts) & 3).reshape(*w.shape[:-1], -1)[..., :n_per_row]
-
-
 @pytest.mark.parametrize("dtype", [F16, BF16])
-@pytest.mark.parametrize("k", [0, 16, 32])
-def test_two_plane_split_reconstructs_4bit_codes(dtype, k):
-    """For boosted channels: hi*4 + lo equals the 4-bit code of that channel-group, plane A
-    scale is 4x the 4-bit scale, plane B scale is the 4-bit scale; for the other
-    channels plane A holds the 2-bit code.  Checked against quant_group directly."""
-    rng = np.random.default_rng(7 + k + dtype)
-    cfg = oracle.Cfg(P=128, k=k, dtype=dtype)
+@pytest.mark.parametrize("P,k", [(128, 0), (128, 16), (128, 32), (64, 64), (32, 128)])
+def test_two_plane_split_reconstructs_4bit_codes(dtype, P, k):
+    """Decoded independently: for boosted channels hi*4 + lo equals the 4-bit code of
+    that channel-group, plane A scale is 4x the 4-bit scale and plane B scale the 4-bit
+    scale; other channels hold their 2-bit code; values hold per-token 2-bit codes."""
+    rng = np.random.default_rng(7 + k + dtype + P)
+    cfg = oracle.Cfg(P=P, k=k, dtype=dtype)
     sig = np.exp(rng.standard_normal(cfg.D))
     K = syn.to_bits(rng.standard_normal((cfg.P, cfg.D)) * sig, dtype)
     V = syn.to_bits(rng.standard_normal((cfg.P, cfg.D)), dtype)
-    rec = oracle.quantize_page(K, V, cfg)
-    L = oracle.layout(cfg.P, cfg.D, k, cfg.G)
-    kA = _unpack(rec[L["k_codes"]:L["kb_codes"]].view(np.uint32).reshape(cfg.P, 8), 128)
-    kB = (_unpack(rec[L["kb_codes"]:L["v_codes"]].view(np.uint32).reshape(cfg.P, k // 16), k)
-          if k else np.zeros((cfg.P, 0), np.uint32))
-    ks = rec[L["k_scale"]:L["k_zero"]].view(np.uint16).reshape(4, 128)
-    kz = rec[L["k_zero"]:L["kb_scale"]].view(np.uint16).reshape(4, 128)
-    kbs = rec[L["kb_scale"]:L["v_scale"]].view(np.uint16).reshape(4, k)
-    idx = rec[L["boost_idx"]:L["boost_idx"] + k]
-    assert idx.tolist() == oracle.select_boost(K, k, dtype).tolist()
-    row = {int(c): j for j, c in enumerate(idx)}
-    for g in range(4):
+    d = _decode_record(oracle.quantize_page(K, V, cfg), P, k, dtype)
+    assert d["idx"].tolist() == oracle.select_boost(K, k, dtype).tolist()
+    row = {int(c): j for j, c in enumerate(d["idx"])}
+    for g in range(P // 32):
+        sl = slice(g * 32, (g + 1) * 32)
         for c in range(cfg.D):
-            grp = K[g * 32:(g + 1) * 32, c]
             if c in row:
                 j = row[c]
-                c4, s4, z4 = oracle.quant_group(grp, 4, dtype)
-                hi, lo = kA[g * 32:(g + 1) * 32, c], kB[g * 32:(g + 1) * 32, j]
-                assert np.array_equal(hi * 4 + lo, c4)
-                assert kbs[g, j] == s4
-                assert oracle.value(int(ks[g, c]), dtype) == 4 * oracle.value(s4, dtype)
-                assert kz[g, c] == z4
+                c4, s4, z4 = oracle.quant_group(K[sl, c], 4, dtype)
+                assert np.array_equal(d["kA"][sl, c] * 4 + d["kB"][sl, j], c4)
+                assert d["kbs"][g, j] == s4
+                assert oracle.value(int(d["ks"][g, c]), dtype) == 4 * oracle.value(s4, dtype)
+                assert d["kz"][g, c] == z4
             else:
-                c2, s2, z2 = oracle.quant_group(grp, 2, dtype)
-                assert np.array_equal(kA[g * 32:(g + 1) * 32, c], c2)
-                assert ks[g, c] == s2 and kz[g, c] == z2
+                c2, s2, z2 = oracle.quant_group(K[sl, c], 2, dtype)
+                assert np.array_equal(d["kA"][sl, c], c2)
+                assert d["ks"][g, c] == s2 and d["kz"][g, c] == z2
+    for t in range(P):
+        cv, sv, zv = oracle.quant_group(V[t], 2, dtype)
+        assert np.array_equal(d["v"][t], cv) and d["vs"][t] == sv and d["vz"][t] == zv
 
 
 def test_golden_4bit_split():
@@ -139,7 +202,7 @@ def test_golden_4bit_split():
 @pytest.mark.parametrize("dtype", [F16, BF16])
 def test_dequantize_page_matches_groupwise_dequant(dtype):
     """K^ from the two planes equals code4*s4 + mn (boosted) or code*s + mn (normal) and
-    V^ equals per-token code*s + mn, exactly in fp64; errors stay within scale/2."""
+    V^ equals per-token code*s + mn, exactly in fp64."""
     rng = np.random.default_rng(9 + dtype)
     cfg = oracle.Cfg(P=64, k=32, dtype=dtype)
     sig = np.exp(rng.standard_normal(cfg.D))
@@ -173,7 +236,7 @@ def test_k0_is_uniform_2bit_kivi():
             codes, sb, zb = oracle.quant_group(K[g * 32:(g + 1) * 32, c], 2, F16)
             assert np.array_equal(Kh[g * 32:(g + 1) * 32, c],
                                   codes * oracle.value(sb, F16) + oracle.value(zb, F16))
-    # boosting every channel (k = D) gives a strictly smaller key error than k = 0
+    # boosting every channel (k = D) gives a much smaller key error than k = 0
     cfgD = oracle.Cfg(P=128, k=128)
     KhD, _ = oracle.dequantize_page(oracle.quantize_page(K, V, cfgD), cfgD)
     Kv = syn.from_bits(K, F16).astype(np.float64)
