@@ -67,6 +67,22 @@ def peaks():
 
 # ------------------------------------------------------------------ workload bytes
 
+def max_over_ranks(times_ms, device, world):
+    """Per-rank times -> the maximum over all ranks (one all-reduce MAX; no-op at N = 1)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(times_ms, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_gbs(world, bytes_per_rank, ms):
+    """Whole-job throughput: every rank moves bytes_per_rank in the slowest rank's time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 def decode_bytes(w, payload, n_pages, res_len):
     """Algorithmic bytes of one decode-attention launch (one layer): packed pages
     (codes + scales + zeros + boost indices), the fp16 residual K and V, the query,
@@ -386,13 +402,10 @@ def run_gpu(args):
 
     bytes_step = L_layers * decode_bytes(w, payload, n_pages, res_avg)
     bytes_attn = decode_bytes(w, payload, n_pages, res_end)
-    t = torch.tensor([step_ms, e2e_ms, attn_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, e2e_ms, attn_ms = [float(x) for x in t.tolist()]
+    step_ms, e2e_ms, attn_ms = max_over_ranks([step_ms, e2e_ms, attn_ms], dev, world)
     peak, peak_kind = peaks()
-    value = world * bytes_step / (step_ms * 1e-3) / 1e9
-    e2e_value = world * bytes_step / (e2e_ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, bytes_step, step_ms)
+    e2e_value = whole_job_gbs(world, bytes_step, e2e_ms)
     achieved = bytes_attn / (attn_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
