@@ -9,6 +9,7 @@ process that already holds a CUDA context (PyTorch's primary context is shared).
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -43,14 +44,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    jobs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *FLAGS, "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
-        subprocess.check_call(cmd)
-        objs.append(obj)
+        jobs.append((cmd, obj))
+    # the translation units are independent: compile them in parallel
+    with concurrent.futures.ThreadPoolExecutor(max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
+        list(ex.map(lambda j: subprocess.check_call(j[0]), jobs))
+    objs = [obj for _, obj in jobs]
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                            "-o", tmp, *objs])

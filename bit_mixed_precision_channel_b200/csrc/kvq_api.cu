@@ -27,22 +27,21 @@ static int sm_count() {
   return n;
 }
 
+// Decode workspace: one partial slot per (CTA, unit) pair that can occur — CTA i and
+// unit u write slot i + u — then one arrival counter per unit.
 struct Plan {
-  SplitPlan split;
+  int ctas;
   size_t part_bytes, cnt_bytes;
 };
 
-static Plan decode_plan(const kvq_config* cfg, int batch, int max_pages) {
+static Plan decode_plan(const kvq_config* cfg, int batch) {
   const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
-  const int units = batch * cfg->num_kv_heads;
+  const size_t units = size_t(batch) * cfg->num_kv_heads;
   Plan pl;
-  // resident CTAs per SM, evaluated with a page-id list of 256 entries
-  const Layout L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
-  const size_t smem = decode_main_bytes(cfg->page_tokens, gqa, L.record) + 256 * 4;
-  pl.split = plan_splits(units, max_pages, sm_count() * decode_ctas_per_sm(gqa, cfg->dtype, cfg->num_boost / 16, smem));
-  pl.part_bytes = size_t(units) * pl.split.max_splits * gqa * (2 + kHeadDim) * sizeof(float);
+  pl.ctas = sm_count() * decode_ctas_per_sm(gqa, cfg->dtype, cfg->num_boost / 16, cfg->page_tokens);
+  pl.part_bytes = (size_t(pl.ctas) + units) * gqa * (kHeadDim + 4) * sizeof(float);
   pl.part_bytes = (pl.part_bytes + 255) / 256 * 256;
-  pl.cnt_bytes = size_t(units) * sizeof(uint32_t);
+  pl.cnt_bytes = units * sizeof(uint32_t);
   return pl;
 }
 
@@ -219,7 +218,7 @@ kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch, const void* 
 
 size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages) {
   if (kvq_check_config(cfg) != KVQ_OK || batch < 0 || max_pages < 0) return 0;
-  const Plan pl = decode_plan(cfg, batch, max_pages);
+  const Plan pl = decode_plan(cfg, batch);
   return pl.part_bytes + pl.cnt_bytes;
 }
 
@@ -237,7 +236,12 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(pool) || !aligned16(q) || !aligned16(res_k) || !aligned16(res_v) || !aligned16(workspace))
     return KVQ_ERR_INVALID_ARG;
-  const Plan pl = decode_plan(cfg, batch, max_pages);
+  // the kernel's work line (32-token groups and 16-token residual pieces of every
+  // (sequence, kv head)) is indexed with 32-bit integers
+  const long long line = (long long)batch * cfg->num_kv_heads *
+                         ((long long)max_pages * (cfg->page_tokens / 32) + (cfg->page_tokens + 15) / 16);
+  if (line >= (1ll << 31)) return KVQ_ERR_INVALID_ARG;
+  const Plan pl = decode_plan(cfg, batch);
   if (workspace_bytes < pl.part_bytes + pl.cnt_bytes) return KVQ_ERR_CAPACITY;
   const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
   DecodeParams p{};
@@ -248,10 +252,6 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   p.k = cfg->num_boost;
   p.KB = cfg->num_boost / 16;
   p.L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
-  p.rec_bytes = p.L.record;
-  p.payload = p.L.payload;
-  p.stage_bytes = uint32_t(128 / p.P) * p.L.record;
-  p.main_bytes = uint32_t(decode_main_bytes(p.P, gqa, p.L.record));
   p.q = static_cast<const uint16_t*>(q);
   p.batch = batch;
   p.Hq = cfg->num_q_heads;
@@ -265,8 +265,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   p.out = out;
   p.part = static_cast<float*>(workspace);
   p.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.part_bytes);
-  p.pps = pl.split.pps;
-  p.max_splits = pl.split.max_splits;
+  p.n_ctas = pl.ctas;
   p.err = err;
   return cuda_status(launch_decode(p, gqa, cfg->dtype, stream));
 }

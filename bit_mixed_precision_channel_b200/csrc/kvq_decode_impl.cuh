@@ -1,0 +1,1103 @@
+// kvq_decode_impl.cuh — decode attention over the paged 2-bit cache, sm_100a.
+// Kernel templates; kvq_decode_<dtype>_g<GQA>.cu instantiate them, kvq_decode.cu
+// holds the host side.
+//
+// Work decomposition (balanced streaming).  Every (sequence b, kv head h) is a unit;
+// its items are its pages, grouped into 128-token stages (1, 2 or 4 pages), followed by
+// its residual tokens in pieces of 16.  Item weights count 32-token groups (a full
+// stage weighs 4, a residual piece 1).  Units are laid end to end in (b, h) order and
+// the resulting weight line is cut into one equal range per CTA, one CTA per resident
+// slot of the GPU (SMs x CTAs per SM); a CTA processes the items that start inside its
+// range, so every SM receives the same amount of work whatever the sequence lengths.
+// A CTA that finishes a unit writes either the output (when it saw the whole unit) or a
+// partial (max, sum, unnormalised output); the last contributor of a unit merges the
+// partials (log-sum-exp), so there is no second launch.
+//
+// Data movement.  Warp 0 fills a 3-stage shared-memory ring with one cp.async.bulk per
+// page record (L2 evict-first hint), one bulk copy per residual row, and the unit's
+// query heads with the unit's first stage; completion is tracked with "full"
+// mbarriers, release with "empty" mbarriers, and every wait is bounded.  Each warp owns
+// one 32-token group of a page stage and runs its own online softmax; warps meet only
+// at the end of a unit.
+//
+// Arithmetic.  The 2-bit codes never become scaled values.  The scales are folded into
+// the other operand of each product, and the codes go to the tensor cores as they are
+// (Kitty abstract: page dequantization kernels; MiniKV proposed method: dequantization
+// fused into the attention matmul):
+//   q.k_t = sum_c codeA[t,c] (q_c sA_c) + sum_j codeB[t,j] (q_idx(j) sB_j) + sum_c q_c zA_c
+//   sum_t p_t v_t[c] = sum_t codeV[t,c] (p_t sV_t) + sum_t p_t zV_t
+// Codes reach the tensor cores exactly as 0.5 * code through the FP4 (e2m1) conversion;
+// the folded operands are carried as fp16 high and low parts (hi = fp16(x),
+// lo = fp16(x - hi)).  The eight columns of an m16n8k16 product hold four query heads,
+// each as an adjacent (hi, lo) column pair, so a lane's two accumulator columns are the
+// two parts of one head: the logits need no shuffle, and the (hi, lo) pair of
+// p * sV is one register that movmatrix turns into the B fragment of the PV product.
+#pragma once
+#include <algorithm>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+constexpr int kStages = 3;
+constexpr int kDecodeThreads = 128;
+constexpr int kResRowBytes = 272;  // residual row in shared memory: 256 bytes + 16 pad
+constexpr int kPieceTokens = 16;   // residual tokens per item
+
+// Compile-time offsets of one record (the same values as make_layout).
+template <int P, int KB>
+struct Rec {
+  static constexpr int k = 16 * KB;
+  static constexpr uint32_t k_codes = 0;
+  static constexpr uint32_t kb_codes = k_codes + P * 32;
+  static constexpr uint32_t v_codes = kb_codes + P * KB * 4;
+  static constexpr uint32_t k_scale = v_codes + P * 32;
+  static constexpr uint32_t k_zero = k_scale + (P / 32) * 256;
+  static constexpr uint32_t kb_scale = k_zero + (P / 32) * 256;
+  static constexpr uint32_t v_scale = kb_scale + (P / 32) * k * 2;
+  static constexpr uint32_t v_zero = v_scale + P * 2;
+  static constexpr uint32_t boost_idx = v_zero + P * 2;
+  static constexpr uint32_t payload = boost_idx + k;
+  static constexpr uint32_t record = (payload + 127u) / 128u * 128u;
+};
+
+// Dynamic shared memory of one CTA: kStages stages (page records, or the K and V rows
+// of a residual piece), then the merge buffer [4 warps][GQA][128] fp32.
+template <int GQA, int P, int KB>
+struct Smem {
+  static constexpr uint32_t body = std::max<uint32_t>((128 / P) * Rec<P, KB>::record, 2 * kPieceTokens * kResRowBytes);
+  static constexpr uint32_t stage = (body + 127u) / 128u * 128u;
+  static constexpr uint32_t merge = kStages * stage;
+  static constexpr uint32_t bytes = merge + 4u * GQA * 128u * 4u;
+};
+
+// ---------------------------------------------------------------- operand builders
+
+// One part of the folded query operand, chosen per lane without a branch:
+// hfma2(q, s, -fp16(q*s) * m) is fp16(q*s) for m = 0 (hi lanes) and the exact rest
+// q*s - fp16(q*s) for m = 1 (lo lanes); the product of two fp16 values is exact in fp32.
+__device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t negmask, __half) {
+  const __half2 q = u32_as_h2(q2), s = u32_as_h2(s2);
+  const __half2 h = __hmul2(q, s);
+  return h2_as_u32(__hfma2(q, s, __hmul2(h, u32_as_h2(negmask))));
+}
+// bf16 data: the product is exact in fp32; split it into fp16 parts there.
+__device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t negmask, __nv_bfloat16) {
+  const float x0 = __uint_as_float(q2 << 16) * __uint_as_float(s2 << 16);
+  const float x1 = __uint_as_float(q2 & 0xffff0000u) * __uint_as_float(s2 & 0xffff0000u);
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  const uint32_t lo = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+  return negmask ? lo : h2_as_u32(h);
+}
+
+// (hi, lo) of x as one register: low half = hi, high half = lo.
+__device__ __forceinline__ uint32_t hilo(float x, __half) {
+  const float hf = __half2float(__float2half_rn(x));
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x - hf), "f"(hf));
+  return d;
+}
+__device__ __forceinline__ uint32_t hilo(float x, __nv_bfloat16) {
+  const float hf = __bfloat162float(__float2bfloat16_rn(x));
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x - hf), "f"(hf));
+  return d;
+}
+
+// Two 16-bit values of a register as floats.
+__device__ __forceinline__ float2 t2_to_float2(uint32_t u, __half) { return __half22float2(u32_as_h2(u)); }
+__device__ __forceinline__ float2 t2_to_float2(uint32_t u, __nv_bfloat16) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// ---------------------------------------------------------------- per-warp state
+
+template <int NT>
+struct WarpState {
+  float o[8][NT][4];  // PV accumulator: rows = channels 16*mc + g (+8), cols (hi, lo) of head qd + 4*nt
+  float m[NT], l[NT], zv[NT];
+};
+
+// Query operand of this lane: B column g = (head g/2 (+4 nt), part g%2).
+template <int NT>
+struct LaneQ {
+  uint32_t qv[NT][8][2];  // q pairs: channels 16s + 2qd (+1), and +8
+  uint32_t negmask;       // fp16x2 -1 for lo-part lanes (odd g), 0 otherwise
+};
+
+template <int NT>
+__device__ __forceinline__ void reset_state(WarpState<NT>& st) {
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) st.o[mc][nt][i] = 0.0f;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    st.m[nt] = -INFINITY;
+    st.l[nt] = 0.0f;
+    st.zv[nt] = 0.0f;
+  }
+}
+
+// Online-softmax update from MT x 2 logits per head part of this lane (log2 units).  The
+// running maximum moves only when a logit exceeds it by more than 8, so probabilities
+// stay below 2^8 and most groups skip the rescale of the accumulators.
+template <int NT, int MT>
+__device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)[MT][NT][2]) {
+  bool moved = false;
+  float alpha[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float mx = L[0][nt][0];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(L[mt][nt][0], L[mt][nt][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+    alpha[nt] = 1.0f;
+    if (mx > st.m[nt] + 8.0f) {
+      alpha[nt] = ex2(st.m[nt] - mx);  // 0 on the first group (m = -inf)
+      st.m[nt] = mx;
+      st.l[nt] *= alpha[nt];
+      st.zv[nt] *= alpha[nt];
+      moved = true;
+    }
+  }
+  if (__any_sync(kFull, moved)) {
+#pragma unroll
+    for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= alpha[nt];
+  }
+}
+
+// ---------------------------------------------------------------- one quantized group
+
+// Tokens [32 grp, 32 grp + 32) of the page record `rec` (shared memory), for the lane
+// (g, qd): QK^T over planes A and B and the zero points, online softmax, then PV.
+template <typename T, int GQA, int KB, int P>
+__device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const LaneQ<(GQA > 4 ? 2 : 1)>& lq,
+                                           const uint16_t* qs, WarpState<(GQA > 4 ? 2 : 1)>& st, int lane,
+                                           float c_log2) {
+  constexpr int NT = GQA > 4 ? 2 : 1;
+  using R = Rec<P, KB>;
+  const int g = lane >> 2, qd = lane & 3;
+  float acc[2][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
+
+  // -- plane A: rows 32 grp + 16 mt + 8 r + g, words 2qd and 2qd+1 (channels of k-steps
+  //    0..3 and 4..7); scales of k-steps 2i, 2i+1 are 16 bytes at 64 i + 16 qd --
+  const uint8_t* kA = rec + R::k_codes + (32 * grp + g) * 32 + 8 * qd;
+  uint2 w[2][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) w[mt][r] = lds64(kA + (16 * mt + 8 * r) * 32);
+  const uint8_t* ksc = rec + R::k_scale + grp * 256 + 16 * qd;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 sc = lds128(ksc + 64 * i);
+    uint32_t c[2][2][4];  // [mt][row][byte]: byte 2jj + r -> k-step 2i + jj, A register (r ? 2 : 0) + row
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        e2m1_pairs(code_pass((i >> 1) ? w[mt][r].y : w[mt][r].x, i & 1), c[mt][r][0], c[mt][r][1], c[mt][r][2],
+                   c[mt][r][3]);
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int s = 2 * i + jj;
+      uint32_t b[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        b[nt][0] = fold_one(lq.qv[nt][s][0], jj ? sc.z : sc.x, lq.negmask, T());
+        b[nt][1] = fold_one(lq.qv[nt][s][1], jj ? sc.w : sc.y, lq.negmask, T());
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t a[4] = {c[mt][0][2 * jj], c[mt][1][2 * jj], c[mt][0][2 * jj + 1], c[mt][1][2 * jj + 1]};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+      }
+    }
+  }
+
+  // -- plane B: low bits of the boosted channels; rows 16s + 8r + 2qd + f of this lane sit
+  //    at positions 4 KB qd + 4s + 2r + f of each token row --
+  if constexpr (KB > 0) {
+    const uint8_t* kB = rec + R::kb_codes;
+    const uint8_t* idx = rec + R::boost_idx;
+    const uint8_t* kbsc = rec + R::kb_scale + grp * (32 * KB);
+    uint32_t cb[2][2][KB][2];  // [mt][row][s][r]
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const uint8_t* row = kB + (32 * grp + 16 * mt + g + 8 * rr) * KB * 4;
+        if constexpr (KB == 1) {
+          const uint32_t x = code_pass(lds32(row), qd >> 1) >> (16 * (qd & 1));
+          cb[mt][rr][0][0] = e2m1_pair_lo(x);
+          cb[mt][rr][0][1] = e2m1_pair_lo(x >> 8);
+        } else {
+#pragma unroll
+          for (int s = 0; s < KB; s += 2) {
+            const int pos = 4 * KB * qd + 4 * s;
+            const uint32_t x = code_pass(lds32(row + (pos >> 4) * 4), (pos >> 3) & 1);
+            e2m1_pairs(x, cb[mt][rr][s][0], cb[mt][rr][s][1], cb[mt][rr][s + 1][0], cb[mt][rr][s + 1][1]);
+          }
+        }
+      }
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
+      // indices are < 128 in any record the library wrote; the mask keeps a corrupt
+      // record from reading outside the query rows
+      const int i00 = idx[j0] & 127, i01 = idx[j0 + 1] & 127, i10 = idx[j1] & 127, i11 = idx[j1 + 1] & 127;
+      const uint32_t s0 = lds32(kbsc + j0 * 2), s1 = lds32(kbsc + j1 * 2);
+      uint32_t b[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hB = (g >> 1) + 4 * nt;
+        uint32_t q0 = 0u, q1 = 0u;
+        if (hB < GQA) {
+          const uint16_t* qh = qs + hB * kHeadDim;
+          q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
+          q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
+        }
+        b[nt][0] = fold_one(q0, s0, lq.negmask, T());
+        b[nt][1] = fold_one(q1, s1, lq.negmask, T());
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t a[4] = {cb[mt][0][s][0], cb[mt][1][s][0], cb[mt][0][s][1], cb[mt][1][s][1]};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+      }
+    }
+  }
+
+  // -- zero points: Z[h] = sum_c q[h][c] * zA[c] (every row of A is the zero row) --
+  float z[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) z[nt][i] = 0.0f;
+  {
+    const uint8_t* kz = rec + R::k_zero + grp * 256 + 16 * qd;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 zz = lds128(kz + 64 * i);
+      const uint32_t a0[4] = {zz.x, zz.x, zz.y, zz.y}, a1[4] = {zz.z, zz.z, zz.w, zz.w};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816(z[nt], a0, lq.qv[nt][2 * i][0], lq.qv[nt][2 * i][1], T());
+        mma_16816(z[nt], a1, lq.qv[nt][2 * i + 1][0], lq.qv[nt][2 * i + 1][1], T());
+      }
+    }
+  }
+
+  // -- logits (log2 units) of tokens 16 mt + 8 r + g for head qd + 4 nt; the code
+  //    products carry a factor 0.5 --
+  const float cc = c_log2 * kCodeScale;
+  float L[2][NT][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        L[mt][nt][r] = fmaf(acc[mt][nt][2 * r] + acc[mt][nt][2 * r + 1], cc, z[nt][0] * c_log2);
+  softmax_step<NT, 2>(st, L);
+
+  // -- probabilities times the value scales, as (hi, lo) pairs -> B operand of PV.
+  //    Value scale/zero positions 32 grp + 4 g + u hold tokens 8u + g --
+  const uint2 vsr = lds64(rec + R::v_scale + (32 * grp + 4 * g) * 2);
+  const uint2 vzr = lds64(rec + R::v_zero + (32 * grp + 4 * g) * 2);
+  const float2 s01 = t2_to_float2(vsr.x, T()), s23 = t2_to_float2(vsr.y, T());
+  const float2 z01 = t2_to_float2(vzr.x, T()), z23 = t2_to_float2(vzr.y, T());
+  const float sv[4] = {s01.x, s01.y, s23.x, s23.y}, zv[4] = {z01.x, z01.y, z23.x, z23.y};
+  uint32_t pb[2][NT][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int u = 2 * mt + r;
+        const float pr = ex2(L[mt][nt][r] - st.m[nt]);
+        st.l[nt] += pr;
+        st.zv[nt] = fmaf(pr, zv[u], st.zv[nt]);
+        pb[mt][nt][r] = movmatrix_trans(hilo(pr * sv[u], __half()));
+      }
+
+  // -- P V: words ((2 grp + n) * 32 + lane) * 4 + mm hold channel tile 4n + mm of this
+  //    lane; pass ks of a word is k-step ks, bytes in A-register order --
+  const uint8_t* vq = rec + R::v_codes + (64 * grp + lane) * 16;
+  const uint4 v0 = lds128(vq), v1 = lds128(vq + 512);
+  const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      e2m1_pairs(code_pass(vw[mc], ks), a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[ks][nt][0], pb[ks][nt][1], __half());
+    }
+}
+
+// ---------------------------------------------------------------- residual tokens
+
+// One piece of n <= 16 residual tokens staged in shared memory as K rows then V rows
+// (272-byte rows; V rows n..15 zeroed by the caller).  The PV operand carries 0.5 * p so
+// that the accumulator stays in the units of the code products.
+template <typename T, int GQA>
+__device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t* Vr, int n,
+                                               const LaneQ<(GQA > 4 ? 2 : 1)>& lq,
+                                               WarpState<(GQA > 4 ? 2 : 1)>& st, int lane, float c_log2) {
+  constexpr int NT = GQA > 4 ? 2 : 1;
+  const int g = lane >> 2, li = lane >> 3, lr = lane & 7;
+  const bool lo = g & 1;  // lo-part columns get no query: the raw query is exact
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    uint32_t a[4];
+    ldmatrix_x4(a, smem_addr(Kr + (lr + 8 * (li & 1)) * kResRowBytes + (16 * s + 8 * (li >> 1)) * 2));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      mma_16816(acc[nt], a, lo ? 0u : lq.qv[nt][s][0], lo ? 0u : lq.qv[nt][s][1], T());
+  }
+  float L[1][NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+      L[0][nt][r] = (g + 8 * r) < n ? (acc[nt][2 * r] + acc[nt][2 * r + 1]) * c_log2 : -INFINITY;
+  softmax_step<NT, 1>(st, L);
+  uint32_t pb[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float pr = ex2(L[0][nt][r] - st.m[nt]);
+      st.l[nt] += pr;
+      pb[nt][r] = movmatrix_trans(hilo(0.5f * pr, T()));
+    }
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc) {
+    uint32_t a[4];
+    ldmatrix_x4_trans(a, smem_addr(Vr + (lr + 8 * (li >> 1)) * kResRowBytes + (16 * mc + 8 * (li & 1)) * 2));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[nt][0], pb[nt][1], T());
+  }
+}
+
+// ---------------------------------------------------------------- work items
+
+// Position on the weight line: unit (b, h), item k of the unit, start weight s.  Every
+// warp walks the same sequence of items, so the loop structure (and every barrier in
+// it) is identical in all warps even when a copy fails.  Weights are 32-bit: the host
+// rejects shapes whose line could reach 2^31.
+struct Cursor {
+  int b, h, k;
+  int np, rl, nst, nres;  // pages, residual tokens, page stages, residual pieces of b
+  int s, ubase;           // start weight of item k and of the unit
+};
+
+// Unit weight of sequence b (-1 when its lengths are invalid), with its pages and
+// residual tokens (0 when invalid).
+template <int P>
+__device__ __forceinline__ int seq_weight(const DecodeParams& p, int b, int& np, int& rl) {
+  np = __ldcg(p.num_pages + b);
+  rl = __ldcg(p.res_len + b);
+  if (np < 0 || np > p.max_pages || rl < 0 || rl > P) {
+    np = 0;
+    rl = 0;
+    return -1;
+  }
+  return np * (P / 32) + (rl + kPieceTokens - 1) / kPieceTokens;
+}
+
+template <int P>
+__device__ __forceinline__ void cursor_load_seq(const DecodeParams& p, Cursor& c) {
+  // skip sequences without items; c.b == batch marks the end of the line
+  while (c.b < p.batch) {
+    if (seq_weight<P>(p, c.b, c.np, c.rl) > 0) break;
+    ++c.b;
+  }
+  if (c.b >= p.batch) c.np = c.rl = 0;
+  c.nst = (c.np * P + 127) / 128;
+  c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
+}
+
+// Weight of item k of the current unit: pages of the stage x groups per page, or 1.
+template <int P>
+__device__ __forceinline__ int item_weight(const Cursor& c) {
+  if (c.k < c.nst) return min(128 / P, c.np - c.k * (128 / P)) * (P / 32);
+  return 1;
+}
+template <int P>
+__device__ __forceinline__ int unit_weight(const Cursor& c) {
+  return c.np * (P / 32) + c.nres;
+}
+
+template <int P>
+__device__ __forceinline__ void cursor_next(const DecodeParams& p, Cursor& c) {
+  c.s += item_weight<P>(c);
+  if (++c.k < c.nst + c.nres) return;
+  c.k = 0;
+  c.ubase = c.s;
+  if (++c.h < p.Hkv) return;
+  c.h = 0;
+  ++c.b;
+  cursor_load_seq<P>(p, c);
+}
+
+// CTA that owns weight position s: the one whose range [ceil(W i / C), ceil(W (i+1) / C))
+// contains it.
+// Both are exact in double: the products stay below 2^53 and a quotient that is not an
+// integer is at least 1/(W C) away from one, far above the rounding error.
+__device__ __forceinline__ int owner_cta(int s, int W, int C) { return int(floor(double(s) * C / W)); }
+__device__ __forceinline__ int range_start(int i, int W, int C) { return int(ceil(double(W) * i / C)); }
+
+// Partial softmax state of one (CTA, unit) slot and head: unnormalised output [128],
+// then the maximum and the sum (floats 128, 129), padded to 16 bytes.
+constexpr int kPartStride = kHeadDim + 4;
+
+// Moves the cursor from offset `ou` of its unit to the first item that starts at or
+// after it, or to the first item of the next unit.
+template <int P>
+__device__ __forceinline__ void cursor_seek(const DecodeParams& p, Cursor& c, int ou) {
+  if (c.nst > 0 && ou <= 4 * (c.nst - 1)) {
+    c.k = (ou + 3) / 4;
+    c.s = c.ubase + 4 * c.k;
+    return;
+  }
+  const int j = max(0, ou - c.np * (P / 32));
+  if (j < c.nres) {
+    c.k = c.nst + j;
+    c.s = c.ubase + c.np * (P / 32) + j;
+    return;
+  }
+  c.s = c.ubase + unit_weight<P>(c);
+  c.ubase = c.s;
+  c.k = 0;
+  if (++c.h < p.Hkv) return;
+  c.h = 0;
+  ++c.b;
+  cursor_load_seq<P>(p, c);
+}
+
+// Total weight of the items of the unit at cursor c whose start lies in [a, e).
+template <int P>
+__device__ __forceinline__ int items_weight_in(const Cursor& c, int a, int e) {
+  int w = 0;
+  if (c.nst > 0) {
+    // stage k starts at ubase + 4k
+    const int ka = (max(0, a - c.ubase) + 3) / 4;
+    const int kb = min(c.nst, (max(0, e - c.ubase) + 3) / 4);
+    if (kb > ka) {
+      w += 4 * (kb - ka);
+      if (kb == c.nst) w -= 4 - (c.np - (c.nst - 1) * (128 / P)) * (P / 32);  // the last stage may be short
+    }
+  }
+  // residual piece j starts at ubase + np * P/32 + j
+  const int r0 = c.ubase + c.np * (P / 32);
+  const int ja = max(0, a - r0), jb = min(c.nres, max(0, e - r0));
+  if (jb > ja) w += jb - ja;
+  return w;
+}
+
+__device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void sts128_zero(void* p) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(smem_addr(p)), "r"(0u) : "memory");
+}
+
+// ---------------------------------------------------------------- item descriptors
+
+// A CTA walks its range in segments of up to kSegItems items.  Before a segment, the
+// CTA lists its items in shared memory (all threads, page ids loaded in parallel), so
+// that issuing the copies of an item and consuming it need no further bookkeeping.
+constexpr int kSegItems = 128;
+constexpr int kSeqCache = 128;  // (pages, residual) of the sequences from the first one on
+
+enum : uint32_t { kDescRes = 1u << 8, kDescFirst = 1u << 9, kDescLast = 1u << 10 };
+
+struct ItemDesc {
+  uint32_t w;   // bits 0-7: pages in the stage or residual tokens; kDescRes, kDescFirst,
+                // kDescLast; bits 11-12: query slot; bits 16-31: stage or piece index
+  int b, h;     // unit
+  uint32_t io;  // first and last contributing CTA of the unit (low, high 16 bits), kDescLast only
+};
+
+// Unit spans of one segment, found by one thread walking the line.
+struct UnitSpan {
+  int off;        // first item of the span within the segment
+  int b, h, k0;   // unit and its first item in the span
+  int n;          // items of the span
+  int np, rl;
+  int first, last;  // span starts / ends the unit's part in this CTA
+  int qslot;
+  uint32_t io;
+};
+
+// Pages and residual tokens of sequence b: from the cache filled during the scan, else
+// from global memory.  Returns the unit weight (0 for empty or invalid lengths).
+template <int P>
+__device__ __forceinline__ int seq_info(const DecodeParams& p, int b, int b0, const int2* s_seq, int& np, int& rl) {
+  if (b - b0 >= 0 && b - b0 < kSeqCache) {
+    const int2 v = s_seq[b - b0];
+    np = v.x;
+    rl = v.y;
+    return np * (P / 32) + (rl + kPieceTokens - 1) / kPieceTokens;
+  }
+  return max(0, seq_weight<P>(p, b, np, rl));
+}
+
+// ---------------------------------------------------------------- the kernel
+
+// Shared state of one CTA besides the stages.
+template <int GQA, int P>
+struct CtaShared {
+  uint64_t full_bar[kStages];  // stage filled (bulk-copy bytes landed)
+  int rel[kStages];            // warps that released the stage's current item
+  int red[4];
+  int b0, base0, abort_flag, issued;
+  int nseg, more, nspan, uord, qslot_cont;
+  Cursor cur;                  // first item of the next segment
+  float m[4][GQA], l[4][GQA], zv[4][GQA];
+  int2 seq[kSeqCache];
+  UnitSpan span[32];
+  ItemDesc desc[kSegItems];
+  int ids[kSegItems][128 / P];
+  __align__(16) uint16_t q[3][GQA * kHeadDim];  // query heads of the last 3 units
+};
+
+// Lists the next segment of this CTA's items (all threads).  One thread walks the units
+// from sh.cur; then every thread fills one descriptor and loads its page ids.
+template <int GQA, int P>
+__device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<GQA, P>& sh, int hi, int W, int C,
+                                              int tid) {
+  constexpr int PPC = 128 / P, GPP = P / 32;
+  if (tid == 0) {
+    Cursor c = sh.cur;
+    int n = 0, ns = 0, uord = sh.uord, qcont = sh.qslot_cont;
+    const bool cta_first = sh.issued == 0;
+    while (c.s < hi && n < kSegItems && ns < 32) {
+      const int nitems = c.nst + c.nres;
+      // items of the unit that start before hi
+      int kend = nitems;
+      const int kst = min(c.nst, max(0, hi - c.ubase + 3) / 4);
+      if (kst < c.nst) {
+        kend = kst;
+      } else {
+        const int r0 = c.ubase + c.np * GPP;
+        kend = c.nst + min(c.nres, max(0, hi - r0));
+      }
+      const int cnt = min(kend - c.k, kSegItems - n);
+      UnitSpan& sp = sh.span[ns];
+      sp.off = n;
+      sp.b = c.b;
+      sp.h = c.h;
+      sp.k0 = c.k;
+      sp.n = cnt;
+      sp.np = c.np;
+      sp.rl = c.rl;
+      sp.first = (c.k == 0) || (cta_first && n == 0);
+      sp.last = (c.k + cnt == kend);
+      if (sp.first) qcont = (++uord) % 3;
+      sp.qslot = qcont;
+      const int uw = unit_weight<P>(c);
+      const int last_start = c.ubase + uw - (c.nres > 0 ? 1 : (c.np - (c.nst - 1) * PPC) * GPP);
+      sp.io = uint32_t(owner_cta(c.ubase, W, C)) | (uint32_t(owner_cta(last_start, W, C)) << 16);
+      n += cnt;
+      ++ns;
+      c.k += cnt;
+      if (c.k == nitems) {
+        c.s = c.ubase + uw;
+        c.ubase = c.s;
+        c.k = 0;
+        if (++c.h == p.Hkv) {
+          c.h = 0;
+          ++c.b;
+          // next sequence with items
+          while (c.b < p.batch && seq_info<P>(p, c.b, sh.b0, sh.seq, c.np, c.rl) == 0) ++c.b;
+          if (c.b >= p.batch) c.np = c.rl = 0;
+          c.nst = (c.np * P + 127) / 128;
+          c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
+        }
+      } else if (c.k == kend) {
+        c.s = hi;  // the range ends inside this unit
+      } else {
+        c.s = c.ubase + (c.k < c.nst ? 4 * c.k : c.np * GPP + (c.k - c.nst));
+      }
+    }
+    sh.cur = c;
+    sh.nseg = n;
+    sh.nspan = ns;
+    sh.more = c.s < hi;
+    sh.uord = uord;
+    sh.qslot_cont = qcont;
+  }
+  __syncthreads();
+  const int n = sh.nseg, ns = sh.nspan;
+  for (int t = tid; t < n; t += kDecodeThreads) {
+    int si = 0;
+    while (si + 1 < ns && sh.span[si + 1].off <= t) ++si;
+    const UnitSpan& sp = sh.span[si];
+    const int k = sp.k0 + (t - sp.off);
+    const int nst = (sp.np * P + 127) / 128;
+    ItemDesc d;
+    d.b = sp.b;
+    d.h = sp.h;
+    d.io = sp.io;
+    uint32_t w = uint32_t(sp.qslot) << 11;
+    if (sp.first && t == sp.off) w |= kDescFirst;
+    if (sp.last && t == sp.off + sp.n - 1) w |= kDescLast;
+    if (k < nst) {
+      const int npg = min(PPC, sp.np - k * PPC);
+      w |= uint32_t(npg) | (uint32_t(k) << 16);
+      for (int i = 0; i < npg; ++i) {
+        int id = __ldcg(p.page_table + size_t(sp.b) * p.max_pages + k * PPC + i);
+        if (id < 0 || id >= p.pool_pages) {
+          flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
+          id = 0;
+        }
+        sh.ids[t][i] = id;
+      }
+    } else {
+      const int j = k - nst;
+      w |= uint32_t(min(kPieceTokens, sp.rl - kPieceTokens * j)) | kDescRes | (uint32_t(j) << 16);
+    }
+    sh.desc[t] = d;
+    sh.desc[t].w = w;
+  }
+  __syncthreads();
+}
+
+// Issues the copies of item x (descriptor slot t of the segment) into stage x % kStages:
+// the page records or residual rows, and the unit's query heads with its first item.
+// All lanes of the calling warp take part.
+template <int GQA, int KB, int P>
+__device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA, P>& sh, uint8_t* smem, int x, int t,
+                                           uint64_t policy, int lane) {
+  using R = Rec<P, KB>;
+  using S = Smem<GQA, P, KB>;
+  const ItemDesc d = sh.desc[t];
+  const int st = x % kStages, n = d.w & 0xff;
+  const bool res = d.w & kDescRes, first = d.w & kDescFirst;
+  uint8_t* sb = smem + st * S::stage;
+  const uint32_t bytes = (res ? uint32_t(n) * 512u : uint32_t(n) * R::payload) + (first ? GQA * 256u : 0u);
+  if (lane == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(&sh.full_bar[st], bytes);
+    atomicAdd(&sh.issued, 1);
+  }
+  __syncwarp();
+  if (!res) {
+    if (lane < n)
+      bulk_g2s(sb + lane * R::record, p.pool + (size_t(sh.ids[t][lane]) * p.Hkv + d.h) * R::record, R::payload,
+               &sh.full_bar[st], policy);
+  } else {
+    const int which = lane >> 4, r = lane & 15;
+    if (r < n) {
+      const int tok = kPieceTokens * int(d.w >> 16) + r;
+      const uint16_t* src = (which ? p.res_v : p.res_k) + ((size_t(d.b) * p.Hkv + d.h) * P + tok) * kHeadDim;
+      bulk_g2s(sb + (which * kPieceTokens + r) * kResRowBytes, src, 256u, &sh.full_bar[st], policy);
+    }
+  }
+  if (first && lane == 31) {
+    const uint16_t* src = p.q + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
+    bulk_g2s(sh.q[(d.w >> 11) & 3], src, GQA * 256u, &sh.full_bar[st], policy);
+  }
+}
+
+template <typename T, int GQA, int KB, int P>
+__global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
+    decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int NT = GQA > 4 ? 2 : 1;
+  using R = Rec<P, KB>;
+  using S = Smem<GQA, P, KB>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ CtaShared<GQA, P> sh;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
+  const int cta = blockIdx.x;
+
+  // ---------------------------------------------------------------- 1. the weight line
+  // Total weight W, then the sequence whose stretch holds this CTA's first position.  At
+  // most W/4 CTAs take part, so every CTA range is at least one full stage long and
+  // every CTA between a unit's first and last owner holds an item of it.
+  int W = 0, x0 = 0, np0 = 0, rl0 = 0;
+  const bool one_pass = p.batch <= kDecodeThreads;
+  for (int base = 0; base < p.batch; base += kDecodeThreads) {
+    const int b = base + tid;
+    int x = 0;
+    if (b < p.batch) {
+      int np, rl;
+      const int w = seq_weight<P>(p, b, np, rl);
+      if (w < 0 && cta == 0) flag_error(p.err, KVQ_DEV_ERR_LENGTH);
+      if (w <= 0 && b % p.n_ctas == cta) {  // nothing to attend to: the output is 0
+        float4* o = reinterpret_cast<float4*>(p.out + size_t(b) * p.Hq * kHeadDim);
+        for (int i = 0; i < p.Hq * kHeadDim / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      x = max(w, 0) * p.Hkv;
+      np0 = np;
+      rl0 = rl;
+    }
+    x0 = x;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(kFull, x, off);
+    if (lane == 0) sh.red[warp] = x;
+    __syncthreads();
+    W += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
+    __syncthreads();
+  }
+  if (W == 0) return;
+  const int C = min(p.n_ctas, max(1, W / 4));
+  if (cta >= C) return;
+  const int lo = range_start(cta, W, C), hi = range_start(cta + 1, W, C);
+  {
+    int run = 0;
+    for (int base = 0; base < p.batch; base += kDecodeThreads) {
+      const int b = base + tid;
+      int x = x0;
+      if (!one_pass) {
+        x = 0;
+        if (b < p.batch) x = max(seq_weight<P>(p, b, np0, rl0), 0) * p.Hkv;
+      }
+      int incl = x;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) sh.red[warp] = incl;
+      __syncthreads();
+      int before = run;
+      for (int w = 0; w < warp; ++w) before += sh.red[w];
+      const int end = before + incl, start = end - x;
+      if (x > 0 && start <= lo && lo < end) {
+        sh.b0 = b;
+        sh.base0 = start;
+      }
+      run += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
+      __syncthreads();
+    }
+  }
+  // sequence cache for the walk: the values this thread already holds (one pass only)
+  if (one_pass && tid < p.batch && tid >= sh.b0) sh.seq[tid - sh.b0] = make_int2(np0, rl0);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      sh.rel[s] = 0;
+    }
+    fence_mbar_init();
+    sh.abort_flag = 0;
+    sh.issued = 0;
+    sh.uord = -1;
+    sh.qslot_cont = 0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (!one_pass) {  // the cache is filled here instead (sequential, batch > 128 only)
+      for (int i = 0; i < kSeqCache && sh.b0 + i < p.batch; ++i) {
+        int np, rl;
+        seq_weight<P>(p, sh.b0 + i, np, rl);
+        sh.seq[i] = make_int2(np, rl);
+      }
+    }
+    Cursor c;
+    c.b = sh.b0;
+    c.np = sh.seq[0].x;
+    c.rl = sh.seq[0].y;
+    c.nst = (c.np * P + 127) / 128;
+    c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
+    c.k = 0;
+    const int wseq = unit_weight<P>(c);
+    const int off = lo - sh.base0;
+    c.h = off / wseq;
+    c.ubase = sh.base0 + c.h * wseq;
+    cursor_seek<P>(p, c, off - c.h * wseq);
+    sh.cur = c;
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- 2. items
+  LaneQ<NT> lq;
+  WarpState<NT> st;
+  float* sO = reinterpret_cast<float*>(smem + S::merge);  // [4][GQA][128]
+  const uint64_t policy = l2_evict_first_policy();
+  int x = 0;  // items of this CTA before the current segment
+  while (true) {
+    build_segment<GQA, P>(p, sh, hi, W, C, tid);
+    const int nseg = sh.nseg;
+    if (warp == 0)
+      for (int t = 0; t < min(kStages, nseg); ++t) issue_item<GQA, KB, P>(p, sh, smem, x + t, t, policy, lane);
+    for (int t = 0; t < nseg; ++t) {
+      const int xi = x + t, stg = xi % kStages;
+      const ItemDesc d = sh.desc[t];
+      bool ok = !*reinterpret_cast<volatile int*>(&sh.abort_flag);
+      if (ok && !mbar_wait_bounded(&sh.full_bar[stg], uint32_t(xi / kStages) & 1u)) {
+        if (lane == 0) flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
+        sh.abort_flag = 1;
+        ok = false;
+      }
+      ok = __all_sync(kFull, ok);
+      const uint8_t* sb = smem + stg * S::stage;
+      const uint16_t* qs = sh.q[(d.w >> 11) & 3];
+      const int n = d.w & 0xff;
+      if (d.w & kDescFirst) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hB = (g >> 1) + 4 * nt;
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            lq.qv[nt][s][0] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
+            lq.qv[nt][s][1] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+          }
+        }
+        lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
+        reset_state(st);
+      }
+      if (ok) {
+        if (!(d.w & kDescRes)) {
+          const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
+          if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
+        } else if (int(d.w >> 16) % 4 == warp) {
+          uint8_t* Vr = const_cast<uint8_t*>(sb) + kPieceTokens * kResRowBytes;
+          for (int i = lane; i < (kPieceTokens - n) * 16; i += 32)
+            sts128_zero(Vr + (n + (i >> 4)) * kResRowBytes + (i & 15) * 16);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          residual_piece<T, GQA>(sb, Vr, n, lq, st, lane, p.c_log2);
+        }
+      }
+      // release the stage; the last warp to release it refills it with item xi + kStages
+      __syncwarp();
+      int prev = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        prev = atomicAdd(&sh.rel[stg], 1);
+      }
+      prev = __shfl_sync(kFull, prev, 0);
+      if (prev == 3) {
+        if (lane == 0) sh.rel[stg] = 0;
+        if (t + kStages < nseg) issue_item<GQA, KB, P>(p, sh, smem, xi + kStages, t + kStages, policy, lane);
+      }
+
+      if (d.w & kDescLast) {
+        // ---- merge the four warps' states for this unit
+        named_sync();  // the previous merge no longer reads the merge buffer
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float l = st.l[nt], zv = st.zv[nt];
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            l += __shfl_xor_sync(kFull, l, off);
+            zv += __shfl_xor_sync(kFull, zv, off);
+          }
+          const int head = qd + 4 * nt;
+          if (g == 0 && head < GQA) {
+            sh.m[warp][head] = st.m[nt];
+            sh.l[warp][head] = l;
+            sh.zv[warp][head] = zv;
+          }
+          if (head < GQA) {
+#pragma unroll
+            for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+              for (int r = 0; r < 2; ++r)
+                sO[(warp * GQA + head) * kHeadDim + 16 * mc + g + 8 * r] =
+                    st.o[mc][nt][2 * r] + st.o[mc][nt][2 * r + 1];
+          }
+        }
+        named_sync();
+        const int u = d.b * p.Hkv + d.h;
+        const int i0 = int(d.io & 0xffffu), i1 = int(d.io >> 16);
+        const bool sole = i0 == i1;
+        float* outu = p.out + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
+        float* part_me = p.part + (size_t(cta) + u) * GQA * kPartStride;
+        for (int e = tid; e < GQA * kHeadDim; e += kDecodeThreads) {
+          const int h = e >> 7, ch = e & 127;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) M = fmaxf(M, sh.m[w][h]);
+          float Ls = 0.0f, O = 0.0f;
+          if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float f = ex2(sh.m[w][h] - M);
+              Ls += f * sh.l[w][h];
+              O += f * (kCodeScale * sO[(w * GQA + h) * kHeadDim + ch] + sh.zv[w][h]);
+            }
+          }
+          if (sole) {
+            outu[e] = Ls > 0.0f ? O / Ls : 0.0f;
+          } else {
+            float* pp = part_me + h * kPartStride;
+            pp[ch] = O;
+            if (ch == 0) {
+              pp[kHeadDim] = M;
+              pp[kHeadDim + 1] = Ls;
+            }
+          }
+        }
+        if (!sole) {
+          // ---- split merge: the last of the contributors i0..i1 merges their partials
+          __threadfence();
+          named_sync();
+          if (warp == 3) {
+            uint32_t arrived = 0;
+            if (lane == 0) arrived = atomicAdd(p.cnt + u, 1u);
+            arrived = __shfl_sync(kFull, arrived, 0);
+            const int nc = i1 - i0 + 1;
+            if (arrived == uint32_t(nc - 1)) {
+              __threadfence();
+              const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
+              const size_t slot = size_t(GQA) * kPartStride;  // floats per contributor
+              float Mh[GQA];
+#pragma unroll
+              for (int h = 0; h < GQA; ++h) Mh[h] = -INFINITY;
+              for (int i = lane; i < nc; i += 32)
+#pragma unroll
+                for (int h = 0; h < GQA; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + h * kPartStride + kHeadDim));
+              float Lh[GQA];
+              float4 Oh[GQA];
+#pragma unroll
+              for (int h = 0; h < GQA; ++h) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
+                Lh[h] = 0.0f;
+                Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll 2
+              for (int i = 0; i < nc; ++i) {
+                const float* pi = pu + i * slot;
+                float mi[GQA], li[GQA];
+                float4 oi[GQA];
+#pragma unroll
+                for (int h = 0; h < GQA; ++h) {
+                  mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
+                  li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
+                  oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
+                }
+#pragma unroll
+                for (int h = 0; h < GQA; ++h) {
+                  const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
+                  Lh[h] += f * li[h];
+                  Oh[h].x += f * oi[h].x;
+                  Oh[h].y += f * oi[h].y;
+                  Oh[h].z += f * oi[h].z;
+                  Oh[h].w += f * oi[h].w;
+                }
+              }
+#pragma unroll
+              for (int h = 0; h < GQA; ++h) {
+                const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
+                reinterpret_cast<float4*>(outu + h * kHeadDim)[lane] =
+                    make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
+              }
+              if (lane == 0) p.cnt[u] = 0u;  // ready for the next launch
+            }
+          }
+        }
+      }
+    }
+    x += nseg;
+    if (!sh.more) break;
+    __syncthreads();  // every item of the segment is consumed before its slots are reused
+  }
+
+  // ---------------------------------------------------------------- 3. leave
+  __syncthreads();
+  if (sh.abort_flag && warp == 0) {
+    // copies may still be in flight after a timeout: wait for them (bounded) before the
+    // shared memory is released; the output is undefined and the error word says why
+    const int issued = sh.issued;
+    for (int y = max(0, issued - kStages); y < issued; ++y) {
+      if (lane == 0) mbar_wait_bounded(&sh.full_bar[y % kStages], uint32_t(y / kStages) & 1u);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- per-instantiation host side
+
+template <typename T, int GQA, int KB, int P>
+cudaError_t prepare_decode() {
+  static int seen[64];
+  return ensure_dynamic_smem(decode_kernel<T, GQA, KB, P>, int(Smem<GQA, P, KB>::bytes), seen);
+}
+
+// Calls f.template operator()<KB, P>() for one (kb, P).
+template <typename F>
+cudaError_t dispatch_kb_p(int kb, int P, F&& f) {
+#define KVQ_P(K)                                     \
+  switch (P) {                                       \
+    case 32: return f.template operator()<K, 32>();   \
+    case 64: return f.template operator()<K, 64>();   \
+    case 128: return f.template operator()<K, 128>(); \
+  }                                                  \
+  return cudaErrorInvalidValue;
+  switch (kb) {
+    case 0: { KVQ_P(0) }
+    case 1: { KVQ_P(1) }
+    case 2: { KVQ_P(2) }
+    case 4: { KVQ_P(4) }
+    case 8: { KVQ_P(8) }
+  }
+  return cudaErrorInvalidValue;
+#undef KVQ_P
+}
+
+template <typename T, int GQA>
+struct DecodeOcc {
+  int* n;
+  template <int KB, int P>
+  cudaError_t operator()() {
+    cudaError_t e = prepare_decode<T, GQA, KB, P>();
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, decode_kernel<T, GQA, KB, P>, kDecodeThreads,
+                                                         Smem<GQA, P, KB>::bytes);
+  }
+};
+
+template <typename T, int GQA>
+struct DecodeRun {
+  const DecodeParams& p;
+  cudaStream_t stream;
+  template <int KB, int P>
+  cudaError_t operator()() {
+    if (p.L.record != Rec<P, KB>::record || p.L.payload != Rec<P, KB>::payload) return cudaErrorInvalidValue;
+    cudaError_t e = prepare_decode<T, GQA, KB, P>();
+    if (e != cudaSuccess) return e;
+    decode_kernel<T, GQA, KB, P><<<p.n_ctas, kDecodeThreads, Smem<GQA, P, KB>::bytes, stream>>>(p);
+    return cudaGetLastError();
+  }
+};
+
+// One translation unit per (dtype, GQA) defines these two entry points.
+#define KVQ_DECODE_INSTANCE(NAME, T, GQA)                                                       \
+  cudaError_t decode_occupancy_##NAME(int kb, int P, int* n) {                                 \
+    return dispatch_kb_p(kb, P, DecodeOcc<T, GQA>{n});                                          \
+  }                                                                                             \
+  cudaError_t decode_launch_##NAME(const DecodeParams& p, cudaStream_t stream) {               \
+    return dispatch_kb_p(p.KB, p.P, DecodeRun<T, GQA>{p, stream});                              \
+  }
+
+}  // namespace kvq

@@ -45,17 +45,31 @@ inline Layout make_layout(int P, int D, int k, int G) {
 }
 
 // Storage order of the packed rows (see the page-record description in kvq.h).
-// Key channel c = 16s + 8r + 2q + f  <->  position 32q + 4s + 2r + f.
+// Key channel c = 16s + 8r + 2q + f  <->  plane-A code position 32q + 4s + 2r + f.
 __host__ __device__ __forceinline__ int key_pos(int c) {
   return 32 * ((c >> 1) & 3) + 4 * (c >> 4) + 2 * ((c >> 3) & 1) + (c & 1);
+}
+// ... and k_scale / k_zero position 32*(s>>1) + 8q + 4*(s&1) + 2r + f.
+__host__ __device__ __forceinline__ int key_meta_pos(int c) {
+  const int s = c >> 4;
+  return 32 * (s >> 1) + 8 * ((c >> 1) & 3) + 4 * (s & 1) + 2 * ((c >> 3) & 1) + (c & 1);
 }
 // Boosted row j = 16s + 8r + 2q + f  <->  position 4*KB*q + 4s + 2r + f.
 __host__ __device__ __forceinline__ int boost_pos(int j, int KB) {
   return 4 * KB * ((j >> 1) & 3) + 4 * (j >> 4) + 2 * ((j >> 3) & 1) + (j & 1);
 }
-// Value token at position p = 32g + 8q + 4s + 2r + f  <->  token 32g + 16s + 8r + 2q + f.
-__host__ __device__ __forceinline__ int value_token_at(int p) {
-  return (p & ~31) + 16 * ((p >> 2) & 1) + 8 * ((p >> 1) & 1) + 2 * ((p >> 3) & 3) + (p & 1);
+// Value code slot (16 * word + element) -> token (32g + 16a + 8u + 2q + f) and channel
+// (16m + 8v + w): word = ((2g + (m>>2))*32 + 4w + q)*4 + (m&3), element 8a + 2(2u+v) + f.
+__host__ __device__ __forceinline__ void value_at_slot(int slot, int& t, int& c) {
+  const int word = slot >> 4, e = slot & 15;
+  const int mm = word & 3, lane = (word >> 2) & 31, blk = word >> 7;
+  const int a = e >> 3, b = (e >> 1) & 3, f = e & 1;
+  t = 32 * (blk >> 1) + 16 * a + 8 * (b >> 1) + 2 * (lane & 3) + f;
+  c = 16 * (4 * (blk & 1) + mm) + 8 * (b & 1) + (lane >> 2);
+}
+// Value scale / zero position of token t = 32g + 8u + w: 32g + 4w + u.
+__host__ __device__ __forceinline__ int value_meta_pos(int t) {
+  return (t & ~31) + 4 * (t & 7) + ((t >> 3) & 3);
 }
 // Bit of element e = 8a + 2b + f inside a code word: 8b + 4f + 2a.
 __host__ __device__ __forceinline__ int elem_bit(int e) {
@@ -279,7 +293,6 @@ struct DecodeParams {
   const uint8_t* pool;
   long long pool_pages;
   int Hkv, P, k, KB;  // KB = k / 16
-  uint32_t rec_bytes, payload, stage_bytes, main_bytes;
   Layout L;
   const uint16_t* q;
   int batch, Hq;
@@ -289,16 +302,12 @@ struct DecodeParams {
   const uint16_t* res_k;
   const uint16_t* res_v;
   const int32_t* res_len;
-  float c_log2;   // sm_scale * log2(e)
+  float c_log2;  // sm_scale * log2(e)
   float* out;
-  float* part;    // [B][Hkv][max_splits][GQA][2 + 128]: max, sum, unnormalised output
-  uint32_t* cnt;  // [B][Hkv] arrival counters
-  int pps, max_splits;
+  float* part;    // [n_ctas + batch * Hkv][GQA][128 + 4]: unnormalised output, max, sum
+  uint32_t* cnt;  // [batch * Hkv] arrival counters
+  int n_ctas;     // grid size: SMs x resident CTAs per SM
   int32_t* err;
-};
-
-struct SplitPlan {
-  int pps, max_splits;
 };
 
 cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream);
@@ -307,8 +316,7 @@ cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, voi
 cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32_t* page_table, int max_pages,
                                 int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int gqa, int dtype, cudaStream_t stream);
-SplitPlan plan_splits(int units, int max_pages, int slots);
-int decode_ctas_per_sm(int gqa, int dtype, int kb, size_t smem_bytes);
+int decode_ctas_per_sm(int gqa, int dtype, int kb, int P);
 
 // Raises a kernel's dynamic shared-memory limit once per device and size, so that
 // later calls (and calls made while a stream is being captured into a graph) issue

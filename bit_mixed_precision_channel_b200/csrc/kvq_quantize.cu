@@ -190,8 +190,9 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         }
       }
       // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
-      ks_out[g * kHeadDim + pc] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
-      kz_out[g * kHeadDim + pc] = zb;
+      const int pm = key_meta_pos(c);
+      ks_out[g * kHeadDim + pm] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
+      kz_out[g * kHeadDim + pm] = zb;
       if (j >= 0) kbs_out[g * k + j] = sb;
     }
   }
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       for (int i = 0; i < 4; ++i) four |= uint32_t(quant_code(x[i], zero, scale, 3)) << (8 * i);
       *reinterpret_cast<uint32_t*>(cV + t * kHeadDim + 4 * lane) = four;
       if (lane == 0) {
-        vs_out[t] = sb;
-        vz_out[t] = zb;
+        vs_out[value_meta_pos(t)] = sb;
+        vz_out[value_meta_pos(t)] = zb;
       }
     }
   }
@@ -237,14 +238,14 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   }
   if (need_v) {
     uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
-    const int vw = P / 16;
-    for (int i = tid; i < kHeadDim * vw; i += kQThreads) {
-      // word (channel c, w) holds the tokens stored at positions 16w .. 16w+15 of row c
-      const int c = i / vw, w = i % vw;
+    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) {
       uint32_t word = 0;
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        word |= uint32_t(cV[value_token_at(16 * w + e) * kHeadDim + c] & 3u) << elem_bit(e);
+      for (int e = 0; e < 16; ++e) {
+        int t, c;
+        value_at_slot(16 * i + e, t, c);
+        word |= uint32_t(cV[t * kHeadDim + c] & 3u) << elem_bit(e);
+      }
       vq[i] = word;
     }
   }

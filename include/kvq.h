@@ -52,29 +52,31 @@
  * without gaps, in this order:
  *   k_codes   uint32 [P][D/16]   plane A, token-major; word (t, w) = channels 16w..16w+15 of token t
  *   kb_codes  uint32 [P][k/16]   plane B, token-major; word (t, w) = boosted rows 16w..16w+15
- *   v_codes   uint32 [D][P/16]   values, channel-major; word (c, w) = tokens 16w..16w+15 of channel c
- *   k_scale   S [P/G][D]         plane-A scale per (group, key position)
- *   k_zero    S [P/G][D]         plane-A zero  per (group, key position)
+ *   v_codes   uint32 [P*D/16]    values, in the fragment order described below
+ *   k_scale   S [P/G][D]         plane-A scale per (group, key scale position)
+ *   k_zero    S [P/G][D]         plane-A zero  per (group, key scale position)
  *   kb_scale  S [P/G][k]         plane-B scale per (group, boosted row)
- *   v_scale   S [P]              value scale per token
- *   v_zero    S [P]              value zero  per token
+ *   v_scale   S [P]              value scale per value scale position
+ *   v_zero    S [P]              value zero  per value scale position
  *   boost_idx uint8 [k]          boosted channels, ascending
  * The record stride (kvq_page_bytes) rounds the payload up to a multiple of 128 bytes;
  * the padding bytes are never read.
  * Keys are packed along channels and values along tokens — the contraction axis of
  * q.K^T and of p.V respectively — so that the decode kernel can feed codes straight
- * into its matrix products with the scales folded into the other operand.  Within a
- * row, elements are stored in the order in which the decode kernel's matrix-fragment
- * lanes consume them, and inside a 32-bit word so that one masked byte holds the two
- * codes of one fragment register:
- *   key channel c   = 16s + 8r + 2q + f        -> position 32q + 4s + 2r + f
- *                     (plane-A codes of a token row, and the k_scale / k_zero rows)
- *   boosted row j   = 16s + 8r + 2q + f        -> position 4*KB*q + 4s + 2r + f, KB = k/16
- *   value token t   = 32g + 16s + 8r + 2q + f  -> position 32g + 8q + 4s + 2r + f
- *   (s, r, f, q ranging over the values that keep each part in its range).  Position p
- *   of a row is element p % 16 of word p / 16, and element e = 8a + 2b + f of a word
- *   (a, f in {0,1}, b in 0..3) occupies bits 8b + 4f + 2a.  kb_scale, v_scale, v_zero
- *   and boost_idx are in natural order.
+ * into its matrix products with the scales folded into the other operand.  Elements
+ * are stored in the order in which the decode kernel's matrix-fragment lanes consume
+ * them, and inside a 32-bit word so that one masked byte holds the two codes of one
+ * fragment register.  Element e = 8a + 2b + f of a word (a, f in {0,1}, b in 0..3)
+ * occupies bits 8b + 4f + 2a; position p of a row is element p % 16 of word p / 16.
+ *   key channel c = 16s + 8r + 2q + f  (s 0..7, r, f 0..1, q 0..3)
+ *       plane-A code row:      position 32q + 4s + 2r + f
+ *       k_scale / k_zero rows: position 32*(s>>1) + 8q + 4*(s&1) + 2r + f
+ *   boosted row j = 16s + 8r + 2q + f -> plane-B row position 4*KB*q + 4s + 2r + f, KB = k/16
+ *   value code of token t = 32g + 16a + 8u + 2q + f and channel c = 16m + 8v + w
+ *       (a, u, v, f 0..1, q 0..3, w 0..7, m 0..7): element 8a + 2(2u + v) + f of word
+ *       ((2g + (m>>2))*32 + 4w + q)*4 + (m&3)
+ *   v_scale / v_zero of token t = 32g + 8u + w (u 0..3, w 0..7): position 32g + 4w + u
+ *   kb_scale and boost_idx are in natural order.
  *
  * Pool: uint8 pool[pool_pages][num_kv_heads][kvq_page_bytes(cfg)], 256-byte aligned base.
  * Residual window: dtype res_k/res_v[batch][num_kv_heads][page_tokens][head_dim];
@@ -237,10 +239,13 @@ KVQ_API kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
                               void* pool, int64_t pool_pages, int32_t* err,
                               cudaStream_t stream);
 
-/* Scratch bytes kvq_decode_attention needs for (cfg, batch, max_pages).  The
- * workspace holds split-K partial results and one arrival counter per
- * (sequence, KV head).  The counters must be zero before the first call (clear the
- * whole workspace once after allocating it); every call leaves them zero again. */
+/* Scratch bytes kvq_decode_attention needs for (cfg, batch, max_pages) on the current
+ * device (max_pages does not change it).  The workspace holds the partial softmax
+ * states of sequences split across CTAs (one slot per pair of CTA and (sequence, KV
+ * head) that can meet) and one 32-bit counter per (sequence, KV head).  The counters
+ * must be zero before the first call (clear the whole workspace once after
+ * allocating it); every call leaves them zero again.  Without a visible device the
+ * size assumes the largest possible grid. */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages);
 
 /* a6 + a7 — decode attention over the paged, packed cache plus the residual window
@@ -249,9 +254,10 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, 
  * sequence b and query head h (KV head h / (Hq/Hkv)):
  *   out[b][h] = softmax(sm_scale * q[b][h] . K^T) V
  * over the num_pages[b] quantized pages of page_table[b] (dequantized inside the
- * kernel) followed by the res_len[b] residual tokens.  The token range of a sequence
- * is split across CTAs and the partial softmax states are merged by log-sum-exp in
- * the same launch (no second kernel).
+ * kernel) followed by the res_len[b] residual tokens.  All (sequence, KV head) token
+ * ranges are laid end to end and cut into equal shares, one per resident CTA, so the
+ * work per SM is the same whatever the sequence lengths; a range split across CTAs is
+ * merged by log-sum-exp in the same launch (no second kernel).
  * q: dtype [batch][Hq][D]; out: fp32 [batch][Hq][D]; sm_scale normally 1/sqrt(D).
  * workspace: device, >= kvq_decode_workspace_bytes(cfg, batch, max_pages) bytes,
  * see kvq_decode_workspace_bytes for its zero-counter contract.

@@ -87,9 +87,9 @@ def test_decode_matches_oracle(gqa, dtype, P, k, lens):
 
 
 def test_split_count_does_not_change_result():
-    """One sequence of 40 pages: with a 40-entry page table the launch splits it into
-    single-page CTAs merged by log-sum-exp; with a 4000-entry table it runs as one split.
-    Both agree with the oracle, and the arrival counters are left at zero."""
+    """One sequence of 40 pages is cut across many CTAs (one or a few pages each) and
+    merged by log-sum-exp; the weight counters are left at zero.  The same cache read
+    through a 4000-entry page table and a fresh workspace gives the same answer."""
     cfg = kb.Config(num_q_heads=4, num_kv_heads=1, page_tokens=128, num_boost=32)
     got1, want, cache = _run(cfg, [128 * 40 + 9], seed=5)
     assert_attention_close(got1, want, "many splits")

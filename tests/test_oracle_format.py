@@ -45,11 +45,32 @@ def _boost_row(p, KB):
     return 16 * s + 8 * r + 2 * q + f
 
 
-def _value_token(p):
+def _key_meta_channel(p):
+    """inverse of the scale/zero order: position 32i + 8q + 4j + 2r + f -> channel 16(2i + j) + 8r + 2q + f"""
     p = np.asarray(p)
-    g, rem = p >> 5, p & 31
-    q, s, r, f = rem >> 3, (rem >> 2) & 1, (rem >> 1) & 1, rem & 1
-    return 32 * g + 16 * s + 8 * r + 2 * q + f
+    i, q, j, r, f = p >> 5, (p >> 3) & 3, (p >> 2) & 1, (p >> 1) & 1, p & 1
+    return 16 * (2 * i + j) + 8 * r + 2 * q + f
+
+
+def _value_token_channel(slot):
+    """inverse of the value-code order: slot 16*word + element -> (token, channel), with
+    word = ((2g + n) * 32 + 4w + q) * 4 + mm, element = 8a + 2(2u + v) + f,
+    token 32g + 16a + 8u + 2q + f, channel 16(4n + mm) + 8v + w"""
+    slot = np.asarray(slot)
+    word, e = slot >> 4, slot & 15
+    mm, lane, blk = word & 3, (word >> 2) & 31, word >> 7
+    g, n = blk >> 1, blk & 1
+    w, q = lane >> 2, lane & 3
+    a, b, f = e >> 3, (e >> 1) & 3, e & 1
+    u, v = b >> 1, b & 1
+    return 32 * g + 16 * a + 8 * u + 2 * q + f, 16 * (4 * n + mm) + 8 * v + w
+
+
+def _value_meta_token(p):
+    """inverse of the value scale/zero order: position 32g + 4w + u -> token 32g + 8u + w"""
+    p = np.asarray(p)
+    g, w, u = p >> 5, (p >> 2) & 7, p & 3
+    return 32 * g + 8 * u + w
 
 
 def _words_to_positions(words):
@@ -71,17 +92,21 @@ def _decode_record(rec, P, k, dtype):
     if k:
         kB_pos = _words_to_positions(rec[L["kb_codes"]:L["v_codes"]].view(np.uint32).reshape(P, KB))
         kB[:, _boost_row(np.arange(k), KB)] = kB_pos
-    v_pos = _words_to_positions(rec[L["v_codes"]:L["k_scale"]].view(np.uint32).reshape(128, P // 16))
+    v_slots = _words_to_positions(rec[L["v_codes"]:L["k_scale"]].view(np.uint32)[None, :])[0]
     v = np.zeros((P, 128), np.int64)
-    v[_value_token(np.arange(P)), :] = v_pos.T
+    tok, ch = _value_token_channel(np.arange(P * 128))
+    v[tok, ch] = v_slots
     ks = np.zeros((P // 32, 128), np.uint16)
     kz = np.zeros((P // 32, 128), np.uint16)
-    ks[:, _key_channel(np.arange(128))] = u16(L["k_scale"], L["k_zero"]).reshape(P // 32, 128)
-    kz[:, _key_channel(np.arange(128))] = u16(L["k_zero"], L["kb_scale"]).reshape(P // 32, 128)
+    ks[:, _key_meta_channel(np.arange(128))] = u16(L["k_scale"], L["k_zero"]).reshape(P // 32, 128)
+    kz[:, _key_meta_channel(np.arange(128))] = u16(L["k_zero"], L["kb_scale"]).reshape(P // 32, 128)
+    vs = np.zeros(P, np.uint16)
+    vz = np.zeros(P, np.uint16)
+    vs[_value_meta_token(np.arange(P))] = u16(L["v_scale"], L["v_zero"])
+    vz[_value_meta_token(np.arange(P))] = u16(L["v_zero"], L["boost_idx"])
     return dict(kA=kA, kB=kB, v=v, ks=ks, kz=kz,
                 kbs=u16(L["kb_scale"], L["v_scale"]).reshape(P // 32, k),
-                vs=u16(L["v_scale"], L["v_zero"]), vz=u16(L["v_zero"], L["boost_idx"]),
-                idx=rec[L["boost_idx"]:L["boost_idx"] + k])
+                vs=vs, vz=vz, idx=rec[L["boost_idx"]:L["boost_idx"] + k])
 
 
 # -------------------------------------------------------------------------- pins
@@ -104,15 +129,26 @@ def test_storage_positions_hand_worked():
         assert oracle.key_pos(c) == p
     for KB, j, p in g["boost_pos"]:
         assert oracle.boost_pos(j, KB) == p
-    for t, p in g["value_pos"]:
-        assert oracle.value_pos(t) == p
+    for c, p in g["key_meta_pos"]:
+        assert oracle.key_meta_pos(c) == p
+    for t, c, word, elem in g["value_slot"]:
+        assert oracle.value_slot(t, c) == 16 * word + elem
+    for t, p in g["value_meta_pos"]:
+        assert oracle.value_meta_pos(t) == p
     # each order is a permutation, and inverts the decoder's reading of the rule
     assert sorted(oracle.key_pos(c) for c in range(128)) == list(range(128))
     assert all(_key_channel(oracle.key_pos(c)) == c for c in range(128))
     for KB in (1, 2, 4, 8):
         assert sorted(oracle.boost_pos(j, KB) for j in range(16 * KB)) == list(range(16 * KB))
         assert all(_boost_row(oracle.boost_pos(j, KB), KB) == j for j in range(16 * KB))
-    assert all(_value_token(oracle.value_pos(t)) == t for t in range(128))
+    assert sorted(oracle.key_meta_pos(c) for c in range(128)) == list(range(128))
+    assert all(_key_meta_channel(oracle.key_meta_pos(c)) == c for c in range(128))
+    slots = [oracle.value_slot(t, c) for t in range(128) for c in range(128)]
+    assert sorted(slots) == list(range(128 * 128))
+    tok, ch = _value_token_channel(np.array(slots))
+    assert (tok == np.repeat(np.arange(128), 128)).all() and (ch == np.tile(np.arange(128), 128)).all()
+    assert sorted(oracle.value_meta_pos(t) for t in range(128)) == list(range(128))
+    assert all(_value_meta_token(oracle.value_meta_pos(t)) == t for t in range(128))
     assert [oracle.elem_shift(e) for e in range(16)] == list(_shift(np.arange(16)))
 
 
@@ -133,12 +169,14 @@ def test_key_word_packing_hand_worked(case):
 
 @pytest.mark.parametrize("case", _golden()["words"], ids=lambda c: c["word"])
 def test_value_word_packing_hand_worked(case):
-    """Word 0 of channel row 0 holds the tokens stored at positions 0..15."""
+    """Word 0 of the value codes holds element e = 8a + 2(2u + v) + f <-> token 16a + 8u + f,
+    channel 8v."""
     cfg = oracle.Cfg(P=32, k=0)
     V = np.zeros((cfg.P, cfg.D), np.float32)
     V[:, 1] = 3.0  # every token's range is [0, 3]: scale 1, zero 0
     for e, code in enumerate(case["codes"]):
-        V[int(_value_token(e)), 0] = code
+        a, b, f = e >> 3, (e >> 1) & 3, e & 1
+        V[16 * a + 8 * (b >> 1) + f, 8 * (b & 1)] = code
     rec = oracle.quantize_page(np.zeros((cfg.P, cfg.D), np.uint16), syn.to_bits(V, F16), cfg)
     L = oracle.layout(cfg.P, cfg.D, cfg.k, cfg.G)
     assert int(rec[L["v_codes"]:L["v_codes"] + 4].view(np.uint32)[0]) == int(case["word"], 16)
