@@ -286,23 +286,21 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
     }
   }
 
-  // -- zero points: Z[h] = sum_c q[h][c] * zA[c] (every row of A is the zero row) --
+  // -- zero points: Z[h] = sum_c q[h][c] * zA[c] --
   float z[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) z[nt][i] = 0.0f;
   {
+    // only rows g of the product are used: rows g + 8 of A are zero, so each A fragment
+    // is two loaded registers and two zeros (no register copies)
     const uint8_t* kz = rec + R::k_zero + grp * 256 + 16 * qd;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 zz = lds128(kz + 64 * i);
-      const uint32_t a0[4] = {zz.x, zz.x, zz.y, zz.y}, a1[4] = {zz.z, zz.z, zz.w, zz.w};
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t a[4] = {lds32(kz + 64 * (s >> 1) + 8 * (s & 1)), 0u, lds32(kz + 64 * (s >> 1) + 8 * (s & 1) + 4), 0u};
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_16816(z[nt], a0, lq.qv[nt][2 * i][0], lq.qv[nt][2 * i][1], T());
-        mma_16816(z[nt], a1, lq.qv[nt][2 * i + 1][0], lq.qv[nt][2 * i + 1][1], T());
-      }
+      for (int nt = 0; nt < NT; ++nt) mma_16816(z[nt], a, lq.qv[nt][s][0], lq.qv[nt][s][1], T());
     }
   }
 
@@ -456,6 +454,11 @@ __device__ __forceinline__ int unit_weight(const Cursor& c) {
 }
 
 template <int P>
+__device__ __forceinline__ int unit_weight_of(int2 v) {
+  return v.x * (P / 32) + (v.y + kPieceTokens - 1) / kPieceTokens;
+}
+
+template <int P>
 __device__ __forceinline__ void cursor_next(const DecodeParams& p, Cursor& c) {
   c.s += item_weight<P>(c);
   if (++c.k < c.nst + c.nres) return;
@@ -473,6 +476,14 @@ __device__ __forceinline__ void cursor_next(const DecodeParams& p, Cursor& c) {
 // integer is at least 1/(W C) away from one, far above the rounding error.
 __device__ __forceinline__ int owner_cta(int s, int W, int C) { return int(floor(double(s) * C / W)); }
 __device__ __forceinline__ int range_start(int i, int W, int C) { return int(ceil(double(W) * i / C)); }
+
+// Owners of positions on the weight line: the line is cut into Cs equal ranges and CTA
+// i owns range i.  Every range is at least 4 long, so every owner between a unit's
+// first and last owner holds an item of the unit.
+struct Owners {
+  int W, Cs;
+  __device__ __forceinline__ int of(int s) const { return owner_cta(s, W, Cs); }
+};
 
 // Partial softmax state of one (CTA, unit) slot and head: unnormalised output [128],
 // then the maximum and the sum (floats 128, 129), padded to 16 bytes.
@@ -524,6 +535,20 @@ __device__ __forceinline__ int items_weight_in(const Cursor& c, int a, int e) {
 
 __device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Shared-memory atomic add with acquire-release semantics at CTA scope.
+__device__ __forceinline__ int atomic_add_acq_rel_cta(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], %2;" : "=r"(old) : "r"(smem_addr(p)), "r"(v) : "memory");
+  return old;
+}
+
+// Device-scope atomic add with acquire-release semantics.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void sts128_zero(void* p) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(smem_addr(p)), "r"(0u) : "memory");
 }
@@ -560,7 +585,7 @@ struct UnitSpan {
 // from global memory.  Returns the unit weight (0 for empty or invalid lengths).
 template <int P>
 __device__ __forceinline__ int seq_info(const DecodeParams& p, int b, int b0, const int2* s_seq, int& np, int& rl) {
-  if (b - b0 >= 0 && b - b0 < kSeqCache) {
+  if (b0 >= 0 && b - b0 >= 0 && b - b0 < kSeqCache) {
     const int2 v = s_seq[b - b0];
     np = v.x;
     rl = v.y;
@@ -578,6 +603,7 @@ struct CtaShared {
   int rel[kStages];            // warps that released the stage's current item
   int red[4];
   int b0, base0, abort_flag, issued;
+  int pref[kSeqCache];         // exclusive prefix of the weights (x kv heads), one-pass case
   int nseg, more, nspan, uord, qslot_cont;
   Cursor cur;                  // first item of the next segment
   float m[4][GQA], l[4][GQA], zv[4][GQA];
@@ -590,14 +616,14 @@ struct CtaShared {
 
 // Lists the next segment of this CTA's items (all threads).  One thread walks the units
 // from sh.cur; then every thread fills one descriptor and loads its page ids.
-template <int GQA, int P>
-__device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<GQA, P>& sh, int hi, int W, int C,
-                                              int tid) {
+template <int GQA, int KB, int P>
+__device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<GQA, P>& sh, int hi, const Owners& ow,
+                                              int tid, bool one_pass) {
   constexpr int PPC = 128 / P, GPP = P / 32;
   if (tid == 0) {
     Cursor c = sh.cur;
     int n = 0, ns = 0, uord = sh.uord, qcont = sh.qslot_cont;
-    const bool cta_first = sh.issued == 0;
+    const bool cta_first = sh.uord < 0;  // no unit started yet: the range's first segment
     while (c.s < hi && n < kSegItems && ns < 32) {
       const int nitems = c.nst + c.nres;
       // items of the unit that start before hi
@@ -624,7 +650,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
       sp.qslot = qcont;
       const int uw = unit_weight<P>(c);
       const int last_start = c.ubase + uw - (c.nres > 0 ? 1 : (c.np - (c.nst - 1) * PPC) * GPP);
-      sp.io = uint32_t(owner_cta(c.ubase, W, C)) | (uint32_t(owner_cta(last_start, W, C)) << 16);
+      sp.io = uint32_t(ow.of(c.ubase)) | (uint32_t(ow.of(last_start)) << 16);
       n += cnt;
       ++ns;
       c.k += cnt;
@@ -636,7 +662,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
           c.h = 0;
           ++c.b;
           // next sequence with items
-          while (c.b < p.batch && seq_info<P>(p, c.b, sh.b0, sh.seq, c.np, c.rl) == 0) ++c.b;
+          while (c.b < p.batch && seq_info<P>(p, c.b, one_pass ? 0 : sh.b0, sh.seq, c.np, c.rl) == 0) ++c.b;
           if (c.b >= p.batch) c.np = c.rl = 0;
           c.nst = (c.np * P + 127) / 128;
           c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
@@ -727,6 +753,62 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA,
   }
 }
 
+// One warp: counts this contributor in for unit u and, if it is the last of the
+// contributors i0..i1, merges their partial states (log-sum-exp) into the output.
+template <int GQA>
+__device__ __forceinline__ void merge_partials(const DecodeParams& p, int u, int i0, int i1, float* outu, int lane) {
+  uint32_t arrived = 0;
+  if (lane == 0) arrived = atomic_add_acq_rel_gpu(p.cnt + u, 1u);
+  arrived = __shfl_sync(kFull, arrived, 0);
+  const int nc = i1 - i0 + 1;
+  if (arrived != uint32_t(nc - 1)) return;
+  const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
+  const size_t slot = size_t(GQA) * kPartStride;  // floats per contributor
+  float Mh[GQA];
+#pragma unroll
+  for (int h = 0; h < GQA; ++h) Mh[h] = -INFINITY;
+  for (int i = lane; i < nc; i += 32)
+#pragma unroll
+    for (int h = 0; h < GQA; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + h * kPartStride + kHeadDim));
+  float Lh[GQA];
+  float4 Oh[GQA];
+#pragma unroll
+  for (int h = 0; h < GQA; ++h) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
+    Lh[h] = 0.0f;
+    Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll 4
+  for (int i = 0; i < nc; ++i) {
+    const float* pi = pu + i * slot;
+    float mi[GQA], li[GQA];
+    float4 oi[GQA];
+#pragma unroll
+    for (int h = 0; h < GQA; ++h) {
+      mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
+      li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
+      oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
+    }
+#pragma unroll
+    for (int h = 0; h < GQA; ++h) {
+      const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
+      Lh[h] += f * li[h];
+      Oh[h].x += f * oi[h].x;
+      Oh[h].y += f * oi[h].y;
+      Oh[h].z += f * oi[h].z;
+      Oh[h].w += f * oi[h].w;
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GQA; ++h) {
+    const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
+    reinterpret_cast<float4*>(outu + h * kHeadDim)[lane] =
+        make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
+  }
+  if (lane == 0) p.cnt[u] = 0u;  // ready for the next launch
+}
+
 template <typename T, int GQA, int KB, int P>
 __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
     decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -740,9 +822,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
   const int cta = blockIdx.x;
 
   // ---------------------------------------------------------------- 1. the weight line
-  // Total weight W, then the sequence whose stretch holds this CTA's first position.  At
-  // most W/4 CTAs take part, so every CTA range is at least one full stage long and
-  // every CTA between a unit's first and last owner holds an item of it.
+  // Total weight W; with one sequence per thread (batch <= 128) the per-sequence prefix
+  // and lengths stay in shared memory for locating any position later.
   int W = 0, x0 = 0, np0 = 0, rl0 = 0;
   const bool one_pass = p.batch <= kDecodeThreads;
   for (int base = 0; base < p.batch; base += kDecodeThreads) {
@@ -761,47 +842,32 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
       rl0 = rl;
     }
     x0 = x;
+    int incl = x;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(kFull, x, off);
-    if (lane == 0) sh.red[warp] = x;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) sh.red[warp] = incl;
     __syncthreads();
+    if (one_pass) {
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += sh.red[w];
+      if (b < p.batch) {
+        sh.pref[b] = before + incl - x;
+        sh.seq[b] = make_int2(np0, rl0);
+      }
+    }
     W += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
     __syncthreads();
   }
   if (W == 0) return;
-  const int C = min(p.n_ctas, max(1, W / 4));
-  if (cta >= C) return;
-  const int lo = range_start(cta, W, C), hi = range_start(cta + 1, W, C);
-  {
-    int run = 0;
-    for (int base = 0; base < p.batch; base += kDecodeThreads) {
-      const int b = base + tid;
-      int x = x0;
-      if (!one_pass) {
-        x = 0;
-        if (b < p.batch) x = max(seq_weight<P>(p, b, np0, rl0), 0) * p.Hkv;
-      }
-      int incl = x;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, off);
-        if (lane >= off) incl += y;
-      }
-      if (lane == 31) sh.red[warp] = incl;
-      __syncthreads();
-      int before = run;
-      for (int w = 0; w < warp; ++w) before += sh.red[w];
-      const int end = before + incl, start = end - x;
-      if (x > 0 && start <= lo && lo < end) {
-        sh.b0 = b;
-        sh.base0 = start;
-      }
-      run += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
-      __syncthreads();
-    }
-  }
-  // sequence cache for the walk: the values this thread already holds (one pass only)
-  if (one_pass && tid < p.batch && tid >= sh.b0) sh.seq[tid - sh.b0] = make_int2(np0, rl0);
+
+  // At most W/4 CTAs take part, so that every range is at least one full stage long.
+  Owners ow;
+  ow.W = W;
+  ow.Cs = min(p.n_ctas, max(1, W / 4));
+  if (cta >= ow.Cs) return;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh.full_bar[s], 1);
@@ -810,218 +876,212 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
     fence_mbar_init();
     sh.abort_flag = 0;
     sh.issued = 0;
-    sh.uord = -1;
-    sh.qslot_cont = 0;
   }
-  __syncthreads();
-  if (tid == 0) {
-    if (!one_pass) {  // the cache is filled here instead (sequential, batch > 128 only)
-      for (int i = 0; i < kSeqCache && sh.b0 + i < p.batch; ++i) {
+
+  // Moves sh.cur to the first item at or after position pos (all threads).
+  auto locate = [&](int pos) {
+    if (one_pass) {
+      __syncthreads();
+      if (tid < p.batch) {
+        const int st0 = sh.pref[tid], w = unit_weight_of<P>(sh.seq[tid]) * p.Hkv;
+        if (w > 0 && st0 <= pos && pos < st0 + w) {
+          sh.b0 = tid;
+          sh.base0 = st0;
+        }
+      }
+    } else {
+      int run = 0;
+      for (int base = 0; base < p.batch; base += kDecodeThreads) {
+        const int b = base + tid;
+        int x = 0;
+        if (b < p.batch) x = max(seq_weight<P>(p, b, np0, rl0), 0) * p.Hkv;
+        int incl = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(kFull, incl, off);
+          if (lane >= off) incl += y;
+        }
+        if (lane == 31) sh.red[warp] = incl;
+        __syncthreads();
+        int before = run;
+        for (int w = 0; w < warp; ++w) before += sh.red[w];
+        const int end = before + incl, start = end - x;
+        if (x > 0 && start <= pos && pos < end) {
+          sh.b0 = b;
+          sh.base0 = start;
+        }
+        run += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
+        __syncthreads();
+      }
+      // lengths of the sequences from the located one on
+      for (int i = tid; i < kSeqCache && sh.b0 + i < p.batch; i += kDecodeThreads) {
         int np, rl;
         seq_weight<P>(p, sh.b0 + i, np, rl);
         sh.seq[i] = make_int2(np, rl);
       }
     }
-    Cursor c;
-    c.b = sh.b0;
-    c.np = sh.seq[0].x;
-    c.rl = sh.seq[0].y;
-    c.nst = (c.np * P + 127) / 128;
-    c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
-    c.k = 0;
-    const int wseq = unit_weight<P>(c);
-    const int off = lo - sh.base0;
-    c.h = off / wseq;
-    c.ubase = sh.base0 + c.h * wseq;
-    cursor_seek<P>(p, c, off - c.h * wseq);
-    sh.cur = c;
-  }
-  __syncthreads();
+    __syncthreads();
+    if (tid == 0) {
+      Cursor c;
+      c.b = sh.b0;
+      const int2 v = sh.seq[one_pass ? sh.b0 : 0];
+      c.np = v.x;
+      c.rl = v.y;
+      c.nst = (c.np * P + 127) / 128;
+      c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
+      c.k = 0;
+      const int wseq = unit_weight<P>(c);
+      const int off = pos - sh.base0;
+      c.h = off / wseq;
+      c.ubase = sh.base0 + c.h * wseq;
+      cursor_seek<P>(p, c, off - c.h * wseq);
+      sh.cur = c;
+      sh.uord = -1;
+      sh.qslot_cont = 0;
+    }
+    __syncthreads();
+  };
 
   // ---------------------------------------------------------------- 2. items
   LaneQ<NT> lq;
   WarpState<NT> st;
   float* sO = reinterpret_cast<float*>(smem + S::merge);  // [4][GQA][128]
   const uint64_t policy = l2_evict_first_policy();
-  int x = 0;  // items of this CTA before the current segment
-  while (true) {
-    build_segment<GQA, P>(p, sh, hi, W, C, tid);
-    const int nseg = sh.nseg;
-    if (warp == 0)
-      for (int t = 0; t < min(kStages, nseg); ++t) issue_item<GQA, KB, P>(p, sh, smem, x + t, t, policy, lane);
-    for (int t = 0; t < nseg; ++t) {
-      const int xi = x + t, stg = xi % kStages;
-      const ItemDesc d = sh.desc[t];
-      bool ok = !*reinterpret_cast<volatile int*>(&sh.abort_flag);
-      if (ok && !mbar_wait_bounded(&sh.full_bar[stg], uint32_t(xi / kStages) & 1u)) {
-        if (lane == 0) flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
-        sh.abort_flag = 1;
-        ok = false;
-      }
-      ok = __all_sync(kFull, ok);
-      const uint8_t* sb = smem + stg * S::stage;
-      const uint16_t* qs = sh.q[(d.w >> 11) & 3];
-      const int n = d.w & 0xff;
-      if (d.w & kDescFirst) {
+  int x = 0;  // items of this CTA so far
+  const int owner = cta;
+  const int lo = range_start(cta, ow.W, ow.Cs), hi = range_start(cta + 1, ow.W, ow.Cs);
+  {
+    locate(lo);
+    while (true) {
+      build_segment<GQA, P>(p, sh, hi, ow, tid, one_pass);
+      const int nseg = sh.nseg;
+      if (warp == 0)
+        for (int t = 0; t < min(kStages, nseg); ++t) issue_item<GQA, KB, P>(p, sh, smem, x + t, t, policy, lane);
+      int stg = x % kStages;
+      uint32_t par = uint32_t(x / kStages) & 1u;
+      for (int t = 0; t < nseg; ++t) {
+        const int xi = x + t;
+        const ItemDesc d = sh.desc[t];
+        bool ok = !*reinterpret_cast<volatile int*>(&sh.abort_flag);
+        if (ok && !mbar_wait_bounded(&sh.full_bar[stg], par)) {
+          if (lane == 0) flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
+          sh.abort_flag = 1;
+          ok = false;
+        }
+        ok = __all_sync(kFull, ok);
+        const uint8_t* sb = smem + stg * S::stage;
+        const uint16_t* qs = sh.q[(d.w >> 11) & 3];
+        const int n = d.w & 0xff;
+        if (d.w & kDescFirst) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int hB = (g >> 1) + 4 * nt;
+          for (int nt = 0; nt < NT; ++nt) {
+            const int hB = (g >> 1) + 4 * nt;
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            lq.qv[nt][s][0] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
-            lq.qv[nt][s][1] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+            for (int s = 0; s < 8; ++s) {
+              lq.qv[nt][s][0] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
+              lq.qv[nt][s][1] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+            }
+          }
+          lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
+          reset_state(st);
+        }
+        if (ok) {
+          if (!(d.w & kDescRes)) {
+            const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
+            if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
+          } else if (int(d.w >> 16) % 4 == warp) {
+            uint8_t* Vr = const_cast<uint8_t*>(sb) + kPieceTokens * kResRowBytes;
+            for (int i = lane; i < (kPieceTokens - n) * 16; i += 32)
+              sts128_zero(Vr + (n + (i >> 4)) * kResRowBytes + (i & 15) * 16);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            residual_piece<T, GQA>(sb, Vr, n, lq, st, lane, p.c_log2);
           }
         }
-        lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
-        reset_state(st);
-      }
-      if (ok) {
-        if (!(d.w & kDescRes)) {
-          const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
-          if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
-        } else if (int(d.w >> 16) % 4 == warp) {
-          uint8_t* Vr = const_cast<uint8_t*>(sb) + kPieceTokens * kResRowBytes;
-          for (int i = lane; i < (kPieceTokens - n) * 16; i += 32)
-            sts128_zero(Vr + (n + (i >> 4)) * kResRowBytes + (i & 15) * 16);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          residual_piece<T, GQA>(sb, Vr, n, lq, st, lane, p.c_log2);
+        // release the stage; the last warp to release it refills it with item xi + kStages
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomic_add_acq_rel_cta(&sh.rel[stg], 1);
+        prev = __shfl_sync(kFull, prev, 0);
+        if (prev == 3) {
+          if (lane == 0) sh.rel[stg] = 0;
+          if (t + kStages < nseg) issue_item<GQA, KB, P>(p, sh, smem, xi + kStages, t + kStages, policy, lane);
         }
-      }
-      // release the stage; the last warp to release it refills it with item xi + kStages
-      __syncwarp();
-      int prev = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        prev = atomicAdd(&sh.rel[stg], 1);
-      }
-      prev = __shfl_sync(kFull, prev, 0);
-      if (prev == 3) {
-        if (lane == 0) sh.rel[stg] = 0;
-        if (t + kStages < nseg) issue_item<GQA, KB, P>(p, sh, smem, xi + kStages, t + kStages, policy, lane);
-      }
+        if (++stg == kStages) {
+          stg = 0;
+          par ^= 1u;
+        }
 
-      if (d.w & kDescLast) {
-        // ---- merge the four warps' states for this unit
-        named_sync();  // the previous merge no longer reads the merge buffer
+        if (d.w & kDescLast) {
+          // ---- merge the four warps' states for this unit
+          named_sync();  // the previous merge no longer reads the merge buffer
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float l = st.l[nt], zv = st.zv[nt];
+          for (int nt = 0; nt < NT; ++nt) {
+            float l = st.l[nt], zv = st.zv[nt];
 #pragma unroll
-          for (int off = 4; off < 32; off <<= 1) {
-            l += __shfl_xor_sync(kFull, l, off);
-            zv += __shfl_xor_sync(kFull, zv, off);
-          }
-          const int head = qd + 4 * nt;
-          if (g == 0 && head < GQA) {
-            sh.m[warp][head] = st.m[nt];
-            sh.l[warp][head] = l;
-            sh.zv[warp][head] = zv;
-          }
-          if (head < GQA) {
+            for (int off = 4; off < 32; off <<= 1) {
+              l += __shfl_xor_sync(kFull, l, off);
+              zv += __shfl_xor_sync(kFull, zv, off);
+            }
+            const int head = qd + 4 * nt;
+            if (g == 0 && head < GQA) {
+              sh.m[warp][head] = st.m[nt];
+              sh.l[warp][head] = l;
+              sh.zv[warp][head] = zv;
+            }
+            if (head < GQA) {
 #pragma unroll
-            for (int mc = 0; mc < 8; ++mc)
+              for (int mc = 0; mc < 8; ++mc)
 #pragma unroll
-              for (int r = 0; r < 2; ++r)
-                sO[(warp * GQA + head) * kHeadDim + 16 * mc + g + 8 * r] =
-                    st.o[mc][nt][2 * r] + st.o[mc][nt][2 * r + 1];
-          }
-        }
-        named_sync();
-        const int u = d.b * p.Hkv + d.h;
-        const int i0 = int(d.io & 0xffffu), i1 = int(d.io >> 16);
-        const bool sole = i0 == i1;
-        float* outu = p.out + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
-        float* part_me = p.part + (size_t(cta) + u) * GQA * kPartStride;
-        for (int e = tid; e < GQA * kHeadDim; e += kDecodeThreads) {
-          const int h = e >> 7, ch = e & 127;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) M = fmaxf(M, sh.m[w][h]);
-          float Ls = 0.0f, O = 0.0f;
-          if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const float f = ex2(sh.m[w][h] - M);
-              Ls += f * sh.l[w][h];
-              O += f * (kCodeScale * sO[(w * GQA + h) * kHeadDim + ch] + sh.zv[w][h]);
+                for (int r = 0; r < 2; ++r)
+                  sO[(warp * GQA + head) * kHeadDim + 16 * mc + g + 8 * r] =
+                      st.o[mc][nt][2 * r] + st.o[mc][nt][2 * r + 1];
             }
           }
-          if (sole) {
-            outu[e] = Ls > 0.0f ? O / Ls : 0.0f;
-          } else {
-            float* pp = part_me + h * kPartStride;
-            pp[ch] = O;
-            if (ch == 0) {
-              pp[kHeadDim] = M;
-              pp[kHeadDim + 1] = Ls;
-            }
-          }
-        }
-        if (!sole) {
-          // ---- split merge: the last of the contributors i0..i1 merges their partials
-          __threadfence();
           named_sync();
-          if (warp == 3) {
-            uint32_t arrived = 0;
-            if (lane == 0) arrived = atomicAdd(p.cnt + u, 1u);
-            arrived = __shfl_sync(kFull, arrived, 0);
-            const int nc = i1 - i0 + 1;
-            if (arrived == uint32_t(nc - 1)) {
-              __threadfence();
-              const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
-              const size_t slot = size_t(GQA) * kPartStride;  // floats per contributor
-              float Mh[GQA];
+          const int u = d.b * p.Hkv + d.h;
+          const int i0 = int(d.io & 0xffffu), i1 = int(d.io >> 16);
+          const bool sole = i0 == i1;
+          float* outu = p.out + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
+          float* part_me = p.part + (size_t(owner) + u) * GQA * kPartStride;
+          for (int e = tid; e < GQA * kHeadDim; e += kDecodeThreads) {
+            const int h = e >> 7, ch = e & 127;
+            float M = -INFINITY;
 #pragma unroll
-              for (int h = 0; h < GQA; ++h) Mh[h] = -INFINITY;
-              for (int i = lane; i < nc; i += 32)
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, sh.m[w][h]);
+            float Ls = 0.0f, O = 0.0f;
+            if (M != -INFINITY) {
 #pragma unroll
-                for (int h = 0; h < GQA; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + h * kPartStride + kHeadDim));
-              float Lh[GQA];
-              float4 Oh[GQA];
-#pragma unroll
-              for (int h = 0; h < GQA; ++h) {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
-                Lh[h] = 0.0f;
-                Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int w = 0; w < 4; ++w) {
+                const float f = ex2(sh.m[w][h] - M);
+                Ls += f * sh.l[w][h];
+                O += f * (kCodeScale * sO[(w * GQA + h) * kHeadDim + ch] + sh.zv[w][h]);
               }
-#pragma unroll 2
-              for (int i = 0; i < nc; ++i) {
-                const float* pi = pu + i * slot;
-                float mi[GQA], li[GQA];
-                float4 oi[GQA];
-#pragma unroll
-                for (int h = 0; h < GQA; ++h) {
-                  mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
-                  li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
-                  oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
-                }
-#pragma unroll
-                for (int h = 0; h < GQA; ++h) {
-                  const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
-                  Lh[h] += f * li[h];
-                  Oh[h].x += f * oi[h].x;
-                  Oh[h].y += f * oi[h].y;
-                  Oh[h].z += f * oi[h].z;
-                  Oh[h].w += f * oi[h].w;
-                }
-              }
-#pragma unroll
-              for (int h = 0; h < GQA; ++h) {
-                const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
-                reinterpret_cast<float4*>(outu + h * kHeadDim)[lane] =
-                    make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
-              }
-              if (lane == 0) p.cnt[u] = 0u;  // ready for the next launch
             }
+            if (sole) {
+              outu[e] = Ls > 0.0f ? O / Ls : 0.0f;
+            } else {
+              float* pp = part_me + h * kPartStride;
+              pp[ch] = O;
+              if (ch == 0) {
+                pp[kHeadDim] = M;
+                pp[kHeadDim + 1] = Ls;
+              }
+            }
+          }
+          if (!sole) {
+            // ---- split merge: the last of the contributors i0..i1 merges their partials.
+            // The barrier orders every thread's partial writes before the counter update,
+            // which is a release at device scope; the merging CTA acquires it.
+            named_sync();
+            if (warp == 3) merge_partials<GQA>(p, u, i0, i1, outu, lane);
           }
         }
       }
+      x += nseg;
+      if (!sh.more) break;
+      __syncthreads();  // every item of the segment is consumed before its slots are reused
     }
-    x += nseg;
-    if (!sh.more) break;
-    __syncthreads();  // every item of the segment is consumed before its slots are reused
   }
 
   // ---------------------------------------------------------------- 3. leave

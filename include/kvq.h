@@ -243,9 +243,9 @@ KVQ_API kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
  * device (max_pages does not change it).  The workspace holds the partial softmax
  * states of sequences split across CTAs (one slot per pair of CTA and (sequence, KV
  * head) that can meet) and one 32-bit counter per (sequence, KV head).  The counters
- * must be zero before the first call (clear the whole workspace once after
- * allocating it); every call leaves them zero again.  Without a visible device the
- * size assumes the largest possible grid. */
+ * must be zero before the first call (clear the whole workspace once after allocating
+ * it); every call leaves them zero again.  Without a visible device the size assumes
+ * the largest possible grid. */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, int32_t max_pages);
 
 /* a6 + a7 — decode attention over the paged, packed cache plus the residual window
