@@ -43,6 +43,10 @@ constexpr int kStages = 3;
 constexpr int kDecodeThreads = 128;
 constexpr int kResRowBytes = 272;  // residual row in shared memory: 256 bytes + 16 pad
 constexpr int kPieceTokens = 16;   // residual tokens per item
+// Extra weight at the end of every unit for the cost of merging its state (about one
+// 32-token group of work); no item starts there.  It keeps a CTA whose range holds a
+// unit end from carrying more work than the others.
+constexpr int kMergeWeight = 3;
 
 // Compile-time offsets of one record (the same values as make_layout).
 template <int P, int KB>
@@ -357,7 +361,7 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
 // ---------------------------------------------------------------- residual tokens
 
 // One piece of n <= 16 residual tokens staged in shared memory as K rows then V rows
-// (272-byte rows; V rows n..15 zeroed by the caller).  The PV operand carries 0.5 * p so
+// (272-byte rows; rows n..15 hold zeros).  The PV operand carries 0.5 * p so
 // that the accumulator stays in the units of the code products.
 template <typename T, int GQA>
 __device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t* Vr, int n,
@@ -427,7 +431,8 @@ __device__ __forceinline__ int seq_weight(const DecodeParams& p, int b, int& np,
     rl = 0;
     return -1;
   }
-  return np * (P / 32) + (rl + kPieceTokens - 1) / kPieceTokens;
+  const int items = np * (P / 32) + (rl + kPieceTokens - 1) / kPieceTokens;
+  return items > 0 ? items + kMergeWeight : 0;
 }
 
 template <int P>
@@ -448,14 +453,17 @@ __device__ __forceinline__ int item_weight(const Cursor& c) {
   if (c.k < c.nst) return min(128 / P, c.np - c.k * (128 / P)) * (P / 32);
   return 1;
 }
+// Weight of a unit: its items, then the merge weight (0 for a unit without items).
 template <int P>
 __device__ __forceinline__ int unit_weight(const Cursor& c) {
-  return c.np * (P / 32) + c.nres;
+  const int items = c.np * (P / 32) + c.nres;
+  return items > 0 ? items + kMergeWeight : 0;
 }
 
 template <int P>
 __device__ __forceinline__ int unit_weight_of(int2 v) {
-  return v.x * (P / 32) + (v.y + kPieceTokens - 1) / kPieceTokens;
+  const int items = v.x * (P / 32) + (v.y + kPieceTokens - 1) / kPieceTokens;
+  return items > 0 ? items + kMergeWeight : 0;
 }
 
 template <int P>
@@ -463,6 +471,7 @@ __device__ __forceinline__ void cursor_next(const DecodeParams& p, Cursor& c) {
   c.s += item_weight<P>(c);
   if (++c.k < c.nst + c.nres) return;
   c.k = 0;
+  c.s += kMergeWeight;
   c.ubase = c.s;
   if (++c.h < p.Hkv) return;
   c.h = 0;
@@ -513,25 +522,6 @@ __device__ __forceinline__ void cursor_seek(const DecodeParams& p, Cursor& c, in
   cursor_load_seq<P>(p, c);
 }
 
-// Total weight of the items of the unit at cursor c whose start lies in [a, e).
-template <int P>
-__device__ __forceinline__ int items_weight_in(const Cursor& c, int a, int e) {
-  int w = 0;
-  if (c.nst > 0) {
-    // stage k starts at ubase + 4k
-    const int ka = (max(0, a - c.ubase) + 3) / 4;
-    const int kb = min(c.nst, (max(0, e - c.ubase) + 3) / 4);
-    if (kb > ka) {
-      w += 4 * (kb - ka);
-      if (kb == c.nst) w -= 4 - (c.np - (c.nst - 1) * (128 / P)) * (P / 32);  // the last stage may be short
-    }
-  }
-  // residual piece j starts at ubase + np * P/32 + j
-  const int r0 = c.ubase + c.np * (P / 32);
-  const int ja = max(0, a - r0), jb = min(c.nres, max(0, e - r0));
-  if (jb > ja) w += jb - ja;
-  return w;
-}
 
 __device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
@@ -549,9 +539,6 @@ __device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t
   return old;
 }
 
-__device__ __forceinline__ void sts128_zero(void* p) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(smem_addr(p)), "r"(0u) : "memory");
-}
 
 // ---------------------------------------------------------------- item descriptors
 
@@ -589,7 +576,7 @@ __device__ __forceinline__ int seq_info(const DecodeParams& p, int b, int b0, co
     const int2 v = s_seq[b - b0];
     np = v.x;
     rl = v.y;
-    return np * (P / 32) + (rl + kPieceTokens - 1) / kPieceTokens;
+    return unit_weight_of<P>(v);
   }
   return max(0, seq_weight<P>(p, b, np, rl));
 }
@@ -649,7 +636,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
       if (sp.first) qcont = (++uord) % 3;
       sp.qslot = qcont;
       const int uw = unit_weight<P>(c);
-      const int last_start = c.ubase + uw - (c.nres > 0 ? 1 : (c.np - (c.nst - 1) * PPC) * GPP);
+      const int last_start = c.ubase + uw - kMergeWeight - (c.nres > 0 ? 1 : (c.np - (c.nst - 1) * PPC) * GPP);
       sp.io = uint32_t(ow.of(c.ubase)) | (uint32_t(ow.of(last_start)) << 16);
       n += cnt;
       ++ns;
@@ -728,10 +715,10 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA,
   const int st = x % kStages, n = d.w & 0xff;
   const bool res = d.w & kDescRes, first = d.w & kDescFirst;
   uint8_t* sb = smem + st * S::stage;
-  const uint32_t bytes = (res ? uint32_t(n) * 512u : uint32_t(n) * R::payload) + (first ? GQA * 256u : 0u);
+  const uint32_t bytes = (res ? 0u : uint32_t(n) * R::payload) + (first ? GQA * 256u : 0u);
   if (lane == 0) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(&sh.full_bar[st], bytes);
+    if (!res) mbar_arrive_expect_tx(&sh.full_bar[st], bytes);
     atomicAdd(&sh.issued, 1);
   }
   __syncwarp();
@@ -740,12 +727,24 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA,
       bulk_g2s(sb + lane * R::record, p.pool + (size_t(sh.ids[t][lane]) * p.Hkv + d.h) * R::record, R::payload,
                &sh.full_bar[st], policy);
   } else {
-    const int which = lane >> 4, r = lane & 15;
-    if (r < n) {
-      const int tok = kPieceTokens * int(d.w >> 16) + r;
-      const uint16_t* src = (which ? p.res_v : p.res_k) + ((size_t(d.b) * p.Hkv + d.h) * P + tok) * kHeadDim;
-      bulk_g2s(sb + (which * kPieceTokens + r) * kResRowBytes, src, 256u, &sh.full_bar[st], policy);
+    // residual rows: 16-byte asynchronous copies into the padded rows, zero-filled past
+    // the last token; each lane's copies arrive on the stage's barrier when they land
+    const int t0 = kPieceTokens * int(d.w >> 16);
+    const uint16_t* kr = p.res_k + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+    const uint16_t* vr = p.res_v + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+#pragma unroll 4
+    for (int i = lane; i < 2 * kPieceTokens * 16; i += 32) {
+      const int which = i >> 8, row = (i >> 4) & 15, chunk = i & 15;
+      const uint16_t* src = (which ? vr : kr) + (row < n ? row : 0) * kHeadDim + chunk * 8;
+      cp_async16(sb + (which * kPieceTokens + row) * kResRowBytes + chunk * 16, src, row < n ? 16u : 0u);
     }
+    cp_async_arrive(&sh.full_bar[st]);
+  }
+  if (res) {
+    // every lane's asynchronous arrival is registered: now the one expected arrival
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(&sh.full_bar[st], bytes);
+    __syncwarp();
   }
   if (first && lane == 31) {
     const uint16_t* src = p.q + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
@@ -990,12 +989,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
             const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
             if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
           } else if (int(d.w >> 16) % 4 == warp) {
-            uint8_t* Vr = const_cast<uint8_t*>(sb) + kPieceTokens * kResRowBytes;
-            for (int i = lane; i < (kPieceTokens - n) * 16; i += 32)
-              sts128_zero(Vr + (n + (i >> 4)) * kResRowBytes + (i & 15) * 16);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            residual_piece<T, GQA>(sb, Vr, n, lq, st, lane, p.c_log2);
+            residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, lq, st, lane, p.c_log2);
           }
         }
         // release the stage; the last warp to release it refills it with item xi + kStages
