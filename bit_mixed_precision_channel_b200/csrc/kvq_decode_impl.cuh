@@ -43,10 +43,10 @@ constexpr int kStages = 3;
 constexpr int kDecodeThreads = 128;
 constexpr int kResRowBytes = 272;  // residual row in shared memory: 256 bytes + 16 pad
 constexpr int kPieceTokens = 16;   // residual tokens per item
-// Extra weight at the end of every unit for the cost of merging its state (about one
-// 32-token group of work); no item starts there.  It keeps a CTA whose range holds a
-// unit end from carrying more work than the others.
-constexpr int kMergeWeight = 3;
+// Extra weight at the end of every unit for the cost of merging its state (measured on
+// B200 to be worth about three stages of streaming work); no item starts there.  It
+// keeps a CTA whose range holds a unit end from carrying more work than the others.
+constexpr int kMergeWeight = 12;
 
 // Compile-time offsets of one record (the same values as make_layout).
 template <int P, int KB>
