@@ -819,6 +819,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
   const int cta = blockIdx.x;
+  // the grid fills every resident slot at once, so the next kernel in the stream may be
+  // scheduled right away: its CTAs take the slots this grid releases
+  pdl_wait();
+  pdl_trigger();
 
   // ---------------------------------------------------------------- 1. the weight line
   // Total weight W; with one sequence per thread (batch <= 128) the per-sequence prefix
@@ -1140,8 +1144,8 @@ struct DecodeRun {
     if (p.L.record != Rec<P, KB>::record || p.L.payload != Rec<P, KB>::payload) return cudaErrorInvalidValue;
     cudaError_t e = prepare_decode<T, GQA, KB, P>();
     if (e != cudaSuccess) return e;
-    decode_kernel<T, GQA, KB, P><<<p.n_ctas, kDecodeThreads, Smem<GQA, P, KB>::bytes, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(decode_kernel<T, GQA, KB, P>, dim3(p.n_ctas), dim3(kDecodeThreads), Smem<GQA, P, KB>::bytes,
+                      stream, p);
   }
 };
 

@@ -3,6 +3,7 @@
 // Record layout, launch helpers and thin inline-PTX wrappers used by the quantize
 // and decode kernels.  Nothing here is exported; the C ABI lives in include/kvq.h.
 #pragma once
+#include <utility>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -281,6 +282,31 @@ __device__ __forceinline__ uint32_t e2m1_pair_lo(uint32_t x) {
 __device__ __forceinline__ uint32_t code_pass(uint32_t w, int a) { return (w >> (2 * a)) & 0x33333333u; }
 
 __device__ __forceinline__ uint32_t bf2_as_u32(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// ------------------------------------------------------------------ dependent launches
+
+// Every kernel of the library is launched with programmatic stream serialization: it
+// may be scheduled while the kernel before it in the stream is still finishing, and it
+// waits for that kernel's completion (griddepcontrol.wait) before it reads anything.
+// A kernel signals with pdl_trigger() when the next one may be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ launch parameters
 

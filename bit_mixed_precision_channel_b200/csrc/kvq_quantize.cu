@@ -68,6 +68,7 @@ __device__ __forceinline__ int quant_code(float x, float zero, float scale, int 
 
 template <typename T>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p) {
+  pdl_wait();
   const int item = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int P = p.P, k = p.k;
   int dst;
@@ -249,6 +250,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       vq[i] = word;
     }
   }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ residual window
@@ -258,6 +260,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
 __global__ void __launch_bounds__(256) append_kernel(const uint4* k_new, const uint4* v_new, uint4* res_k,
                                                      uint4* res_v, int32_t* res_len, int Hkv, int P,
                                                      int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   __shared__ int s_r;
   if (threadIdx.x == 0) s_r = res_len[b];
@@ -284,6 +288,8 @@ __global__ void __launch_bounds__(256) append_kernel(const uint4* k_new, const u
 __global__ void flush_commit_kernel(int32_t* res_len, const int32_t* new_page, int32_t* page_table,
                                     int max_pages, int32_t* num_pages, long long pool_pages, int batch,
                                     int P) {
+  pdl_wait();
+  pdl_trigger();
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
     if (res_len[b] != P) continue;
     const int dst = new_page[b], np = num_pages[b];
@@ -304,31 +310,28 @@ cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaSt
   if (dtype == KVQ_BF16) {
     const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__nv_bfloat16>, int(smem), seen_bf16);
     if (e != cudaSuccess) return e;
-    quantize_kernel<__nv_bfloat16><<<grid, kQThreads, smem, stream>>>(p);
+    return launch_pdl(quantize_kernel<__nv_bfloat16>, grid, dim3(kQThreads), smem, stream, p);
   } else {
     const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__half>, int(smem), seen_f16);
     if (e != cudaSuccess) return e;
-    quantize_kernel<__half><<<grid, kQThreads, smem, stream>>>(p);
+    return launch_pdl(quantize_kernel<__half>, grid, dim3(kQThreads), smem, stream, p);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, void* res_v, int32_t* res_len,
                           int batch, int Hkv, int P, int32_t* err, cudaStream_t stream) {
   if (batch <= 0) return cudaSuccess;
-  append_kernel<<<batch, 256, 0, stream>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-                                           static_cast<uint4*>(res_k), static_cast<uint4*>(res_v), res_len, Hkv,
-                                           P, err);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel, dim3(batch), dim3(256), 0, stream, static_cast<const uint4*>(k_new),
+                    static_cast<const uint4*>(v_new), static_cast<uint4*>(res_k), static_cast<uint4*>(res_v), res_len,
+                    Hkv, P, err);
 }
 
 cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32_t* page_table, int max_pages,
                                 int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream) {
   if (batch <= 0) return cudaSuccess;
   const int threads = 256, blocks = (batch + threads - 1) / threads;
-  flush_commit_kernel<<<blocks, threads, 0, stream>>>(res_len, new_page, page_table, max_pages, num_pages,
-                                                      pool_pages, batch, P);
-  return cudaGetLastError();
+  return launch_pdl(flush_commit_kernel, dim3(blocks), dim3(threads), 0, stream, res_len, new_page, page_table,
+                    max_pages, num_pages, pool_pages, batch, P);
 }
 
 }  // namespace kvq
