@@ -41,6 +41,12 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 WORKLOAD = "llama3_8b"
+# DRAM traffic of one decode launch of this workload (dram__bytes_read.sum +
+# dram__bytes_write.sum from the ncu capture summarised in
+# profiles/decode_kernel_llama3_8b_layer.md), valid only for the kernel source it was taken
+# on: the bench reports it when the decode kernel source still hashes to this value.
+DECODE_TRAFFIC = {"source_sha256": "662fbf98dc0fca0e0d36808ad9e30cec455b87c14ba3c26d58dbd35d4a6bf4f6",
+                  "bytes": 50285824 + 9216}
 LAYERS = 32
 METRIC = "2-bit KV decode-attn GB/s & % of HBM peak; quantize tokens/s"
 
@@ -66,6 +72,15 @@ def peaks():
 
 
 # ------------------------------------------------------------------ workload bytes
+
+def decode_traffic():
+    """ncu DRAM bytes per decode launch, or None once the kernel source has changed."""
+    import hashlib
+    src = os.path.join(ROOT, "bit_mixed_precision_channel_b200", "csrc", "kvq_decode_impl.cuh")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    return DECODE_TRAFFIC["bytes"] if digest == DECODE_TRAFFIC["source_sha256"] else None
+
 
 def max_over_ranks(times_ms, device, world):
     """Per-rank times -> the maximum over all ranks (one all-reduce MAX; no-op at N = 1)."""
@@ -423,7 +438,7 @@ def run_gpu(args):
                      "gbs": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
                      "what": f"prefill of {B} x {w.context} tokens into pages (select + keys + values), per layer"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": decode_traffic(),
                      "kernel": "decode_kernel<__half,4>", "peak_source": peak_kind,
                      "per_launch_bytes": bytes_attn, "ms_per_launch": round(attn_ms, 5)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
