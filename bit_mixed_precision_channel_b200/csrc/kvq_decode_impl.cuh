@@ -186,7 +186,7 @@ __device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)
 // (g, qd): QK^T over planes A and B and the zero points, online softmax, then PV.
 template <typename T, int GQA, int KB, int P>
 __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const LaneQ<(GQA > 4 ? 2 : 1)>& lq,
-                                           const uint16_t* qb, WarpState<(GQA > 4 ? 2 : 1)>& st, int lane,
+                                           const uint16_t* qs, WarpState<(GQA > 4 ? 2 : 1)>& st, int lane,
                                            float c_log2) {
   constexpr int NT = GQA > 4 ? 2 : 1;
   using R = Rec<P, KB>;
@@ -237,11 +237,10 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
   }
 
   // -- plane B: low bits of the boosted channels; rows 16s + 8r + 2qd + f of this lane sit
-  //    at positions 4 KB qd + 4s + 2r + f of each token row.  qb holds the query values
-  //    of the page's boosted channels, [head][row], gathered once per page by the CTA --
+  //    at positions 4 KB qd + 4s + 2r + f of each token row --
   if constexpr (KB > 0) {
-    constexpr int k = 16 * KB;
     const uint8_t* kB = rec + R::kb_codes;
+    const uint8_t* idx = rec + R::boost_idx;
     const uint8_t* kbsc = rec + R::kb_scale + grp * (32 * KB);
     uint32_t cb[2][2][KB][2];  // [mt][row][s][r]
 #pragma unroll
@@ -265,13 +264,20 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
 #pragma unroll
     for (int s = 0; s < KB; ++s) {
       const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
+      // indices are < 128 in any record the library wrote; the mask keeps a corrupt
+      // record from reading outside the query rows
+      const int i00 = idx[j0] & 127, i01 = idx[j0 + 1] & 127, i10 = idx[j1] & 127, i11 = idx[j1 + 1] & 127;
       const uint32_t s0 = lds32(kbsc + j0 * 2), s1 = lds32(kbsc + j1 * 2);
       uint32_t b[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int hB = (g >> 1) + 4 * nt;
-        const uint32_t q0 = hB < GQA ? lds32(qb + hB * k + j0) : 0u;
-        const uint32_t q1 = hB < GQA ? lds32(qb + hB * k + j1) : 0u;
+        uint32_t q0 = 0u, q1 = 0u;
+        if (hB < GQA) {
+          const uint16_t* qh = qs + hB * kHeadDim;
+          q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
+          q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
+        }
         b[nt][0] = fold_one(q0, s0, lq.negmask, T());
         b[nt][1] = fold_one(q1, s1, lq.negmask, T());
       }
@@ -578,10 +584,8 @@ __device__ __forceinline__ int seq_info(const DecodeParams& p, int b, int b0, co
 // ---------------------------------------------------------------- the kernel
 
 // Shared state of one CTA besides the stages.
-template <int GQA, int KB, int P>
+template <int GQA, int P>
 struct CtaShared {
-  // query values of each stage's boosted channels, [page][head][row], gathered by the CTA
-  uint16_t qb[kStages][128 / P][GQA][KB > 0 ? 16 * KB : 2];
   uint64_t full_bar[kStages];  // stage filled (bulk-copy bytes landed)
   int rel[kStages];            // warps that released the stage's current item
   int red[4];
@@ -600,7 +604,7 @@ struct CtaShared {
 // Lists the next segment of this CTA's items (all threads).  One thread walks the units
 // from sh.cur; then every thread fills one descriptor and loads its page ids.
 template <int GQA, int KB, int P>
-__device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<GQA, KB, P>& sh, int hi, const Owners& ow,
+__device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<GQA, P>& sh, int hi, const Owners& ow,
                                               int tid, bool one_pass) {
   constexpr int PPC = 128 / P, GPP = P / 32;
   if (tid == 0) {
@@ -703,7 +707,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
 // the page records or residual rows, and the unit's query heads with its first item.
 // All lanes of the calling warp take part.
 template <int GQA, int KB, int P>
-__device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA, KB, P>& sh, uint8_t* smem, int x, int t,
+__device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA, P>& sh, uint8_t* smem, int x, int t,
                                            uint64_t policy, int lane) {
   using R = Rec<P, KB>;
   using S = Smem<GQA, P, KB>;
@@ -811,7 +815,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
   using R = Rec<P, KB>;
   using S = Smem<GQA, P, KB>;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ CtaShared<GQA, KB, P> sh;
+  __shared__ CtaShared<GQA, P> sh;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
   const int cta = blockIdx.x;
@@ -952,7 +956,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
   {
     locate(lo);
     while (true) {
-      build_segment<GQA, KB, P>(p, sh, hi, ow, tid, one_pass);
+      build_segment<GQA, P>(p, sh, hi, ow, tid, one_pass);
       const int nseg = sh.nseg;
       if (warp == 0)
         for (int t = 0; t < min(kStages, nseg); ++t) issue_item<GQA, KB, P>(p, sh, smem, x + t, t, policy, lane);
@@ -984,25 +988,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
           lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
           reset_state(st);
         }
-        if constexpr (KB > 0) {
-          if (!(d.w & kDescRes)) {
-            // gather the query values of the stage's boosted channels once for all warps
-            // (indices are < 128 in any record the library wrote; the mask keeps a corrupt
-            // record from reading outside the query rows)
-            constexpr int kq = GQA * 16 * KB;
-            uint16_t* qbs = &sh.qb[stg][0][0][0];
-            for (int e = tid; e < n * kq; e += kDecodeThreads) {
-              const int pi = e / kq, h = (e % kq) / (16 * KB), j = e % (16 * KB);
-              qbs[e] = ok ? qs[h * kHeadDim + (sb[pi * R::record + R::boost_idx + j] & 127)] : 0;
-            }
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-          }
-        }
         if (ok) {
           if (!(d.w & kDescRes)) {
             const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
-            if (pw < n)
-              page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, &sh.qb[stg][pw][0][0], st, lane, p.c_log2);
+            if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
           } else if (int(d.w >> 16) % 4 == warp) {
             residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, lq, st, lane, p.c_log2);
           }
