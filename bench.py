@@ -329,16 +329,39 @@ def run_gpu(args):
     kn_pin = [torch.from_numpy(kn.view(np.int16)).view(tdt).pin_memory() for _ in range(L_layers)]
     vn_pin = [torch.from_numpy(vn.view(np.int16)).view(tdt).pin_memory() for _ in range(L_layers)]
     out_pin = [torch.empty(B, w.Hq, D).pin_memory() for _ in range(L_layers)]
+    # The copies run on two copy streams forked inside the graph: every layer's inputs go
+    # up in layer order while earlier layers compute, and every layer's output comes back
+    # while later layers compute.  Each step still moves all inputs and all outputs.
     g_e2e = torch.cuda.CUDAGraph()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     with torch.cuda.graph(g_e2e, stream=stream):
+        start = torch.cuda.Event()
+        start.record(stream)
+        up.wait_event(start)
+        down.wait_event(start)
+        landed, done = [], []
+        with torch.cuda.stream(up):
+            for i in range(L_layers):
+                qs[i].copy_(q_pin[i], non_blocking=True)
+                kns[i].copy_(kn_pin[i], non_blocking=True)
+                vns[i].copy_(vn_pin[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(up)
+                landed.append(ev)
         for i, c in enumerate(caches):
-            qs[i].copy_(q_pin[i], non_blocking=True)
-            kns[i].copy_(kn_pin[i], non_blocking=True)
-            vns[i].copy_(vn_pin[i], non_blocking=True)
+            stream.wait_event(landed[i])
             c.append(kns[i], vns[i])
             c.flush()
             c.attend(qs[i], outs[i])
-            out_pin[i].copy_(outs[i], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            done.append(ev)
+        with torch.cuda.stream(down):
+            for i in range(L_layers):
+                down.wait_event(done[i])
+                out_pin[i].copy_(outs[i], non_blocking=True)
+        stream.wait_stream(down)
+        stream.wait_stream(up)
     h2d_bytes = L_layers * (qh.nbytes + kn.nbytes + vn.nbytes)
     d2h_bytes = L_layers * B * w.Hq * D * 4
 
