@@ -85,14 +85,14 @@ __device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t 
   const __half2 h = __hmul2(q, s);
   return h2_as_u32(__hfma2(q, s, __hmul2(h, u32_as_h2(negmask))));
 }
-// bf16 data: the product is exact in fp32; split it into fp16 parts there.
-__device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t negmask, __nv_bfloat16) {
-  const float x0 = __uint_as_float(q2 << 16) * __uint_as_float(s2 << 16);
-  const float x1 = __uint_as_float(q2 & 0xffff0000u) * __uint_as_float(s2 & 0xffff0000u);
-  const __half2 h = __floats2half2_rn(x0, x1);
-  const float2 hf = __half22float2(h);
-  const uint32_t lo = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
-  return negmask ? lo : h2_as_u32(h);
+// Two cache-dtype values as an fp16 pair.  bf16 values are exact in fp16 inside its
+// normal range (8 significant bits fit in 11), which is where the kernel carries bf16
+// queries, scales and zero points: the folded products then use the fp16 path above.
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t x, __half) { return x; }
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t x, __nv_bfloat16) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(__uint_as_float(x & 0xffff0000u)), "f"(__uint_as_float(x << 16)));
+  return d;
 }
 
 // (hi, lo) of x as one register: low half = hi, high half = lo.
@@ -126,7 +126,7 @@ struct WarpState {
 // Query operand of this lane: B column g = (head g/2 (+4 nt), part g%2).
 template <int NT>
 struct LaneQ {
-  uint32_t qv[NT][8][2];  // q pairs: channels 16s + 2qd (+1), and +8
+  uint32_t qv[NT][8][2];  // q pairs in fp16: channels 16s + 2qd (+1), and +8
   uint32_t negmask;       // fp16x2 -1 for lo-part lanes (odd g), 0 otherwise
 };
 
@@ -224,8 +224,8 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
       uint32_t b[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        b[nt][0] = fold_one(lq.qv[nt][s][0], jj ? sc.z : sc.x, lq.negmask, T());
-        b[nt][1] = fold_one(lq.qv[nt][s][1], jj ? sc.w : sc.y, lq.negmask, T());
+        b[nt][0] = fold_one(lq.qv[nt][s][0], to_f16x2(jj ? sc.z : sc.x, T()), lq.negmask, __half());
+        b[nt][1] = fold_one(lq.qv[nt][s][1], to_f16x2(jj ? sc.w : sc.y, T()), lq.negmask, __half());
       }
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
@@ -267,7 +267,7 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
       // indices are < 128 in any record the library wrote; the mask keeps a corrupt
       // record from reading outside the query rows
       const int i00 = idx[j0] & 127, i01 = idx[j0 + 1] & 127, i10 = idx[j1] & 127, i11 = idx[j1 + 1] & 127;
-      const uint32_t s0 = lds32(kbsc + j0 * 2), s1 = lds32(kbsc + j1 * 2);
+      const uint32_t s0 = to_f16x2(lds32(kbsc + j0 * 2), T()), s1 = to_f16x2(lds32(kbsc + j1 * 2), T());
       uint32_t b[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -278,8 +278,8 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
           q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
           q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
         }
-        b[nt][0] = fold_one(q0, s0, lq.negmask, T());
-        b[nt][1] = fold_one(q1, s1, lq.negmask, T());
+        b[nt][0] = fold_one(to_f16x2(q0, T()), s0, lq.negmask, __half());
+        b[nt][1] = fold_one(to_f16x2(q1, T()), s1, lq.negmask, __half());
       }
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
@@ -302,9 +302,10 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
     const uint8_t* kz = rec + R::k_zero + grp * 256 + 16 * qd;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const uint32_t a[4] = {lds32(kz + 64 * (s >> 1) + 8 * (s & 1)), 0u, lds32(kz + 64 * (s >> 1) + 8 * (s & 1) + 4), 0u};
+      const uint32_t a[4] = {to_f16x2(lds32(kz + 64 * (s >> 1) + 8 * (s & 1)), T()), 0u,
+                             to_f16x2(lds32(kz + 64 * (s >> 1) + 8 * (s & 1) + 4), T()), 0u};
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816(z[nt], a, lq.qv[nt][s][0], lq.qv[nt][s][1], T());
+      for (int nt = 0; nt < NT; ++nt) mma_16816(z[nt], a, lq.qv[nt][s][0], lq.qv[nt][s][1], __half());
     }
   }
 
@@ -364,8 +365,7 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
 // (272-byte rows; rows n..15 hold zeros).  The PV operand carries 0.5 * p so
 // that the accumulator stays in the units of the code products.
 template <typename T, int GQA>
-__device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t* Vr, int n,
-                                               const LaneQ<(GQA > 4 ? 2 : 1)>& lq,
+__device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t* Vr, int n, const uint16_t* qs,
                                                WarpState<(GQA > 4 ? 2 : 1)>& st, int lane, float c_log2) {
   constexpr int NT = GQA > 4 ? 2 : 1;
   const int g = lane >> 2, li = lane >> 3, lr = lane & 7;
@@ -380,8 +380,14 @@ __device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t*
     uint32_t a[4];
     ldmatrix_x4(a, smem_addr(Kr + (lr + 8 * (li & 1)) * kResRowBytes + (16 * s + 8 * (li >> 1)) * 2));
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      mma_16816(acc[nt], a, lo ? 0u : lq.qv[nt][s][0], lo ? 0u : lq.qv[nt][s][1], T());
+    for (int nt = 0; nt < NT; ++nt) {
+      // the raw query in the cache dtype (exact); lo-part columns get none
+      const int hB = (g >> 1) + 4 * nt, qd = lane & 3;
+      const bool use = !lo && hB < GQA;
+      const uint32_t b0 = use ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
+      const uint32_t b1 = use ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+      mma_16816(acc[nt], a, b0, b1, T());
+    }
   }
   float L[1][NT][2];
 #pragma unroll
@@ -763,47 +769,51 @@ __device__ __forceinline__ void merge_partials(const DecodeParams& p, int u, int
   if (arrived != uint32_t(nc - 1)) return;
   const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
   const size_t slot = size_t(GQA) * kPartStride;  // floats per contributor
-  float Mh[GQA];
+  // up to four heads at a time, so that every contributor's loads are in flight together
+  constexpr int HC = GQA < 4 ? GQA : 4;
 #pragma unroll
-  for (int h = 0; h < GQA; ++h) Mh[h] = -INFINITY;
-  for (int i = lane; i < nc; i += 32)
+  for (int h0 = 0; h0 < GQA; h0 += HC) {
+    float Mh[HC], Lh[HC];
+    float4 Oh[HC];
 #pragma unroll
-    for (int h = 0; h < GQA; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + h * kPartStride + kHeadDim));
-  float Lh[GQA];
-  float4 Oh[GQA];
+    for (int h = 0; h < HC; ++h) Mh[h] = -INFINITY;
+    for (int i = lane; i < nc; i += 32)
 #pragma unroll
-  for (int h = 0; h < GQA; ++h) {
+      for (int h = 0; h < HC; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + (h0 + h) * kPartStride + kHeadDim));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
-    Lh[h] = 0.0f;
-    Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+    for (int h = 0; h < HC; ++h) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
+      Lh[h] = 0.0f;
+      Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll 4
-  for (int i = 0; i < nc; ++i) {
-    const float* pi = pu + i * slot;
-    float mi[GQA], li[GQA];
-    float4 oi[GQA];
+    for (int i = 0; i < nc; ++i) {
+      const float* pi = pu + i * slot + h0 * kPartStride;
+      float mi[HC], li[HC];
+      float4 oi[HC];
 #pragma unroll
-    for (int h = 0; h < GQA; ++h) {
-      mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
-      li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
-      oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
+      for (int h = 0; h < HC; ++h) {
+        mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
+        li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
+        oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
+      }
+#pragma unroll
+      for (int h = 0; h < HC; ++h) {
+        const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
+        Lh[h] += f * li[h];
+        Oh[h].x += f * oi[h].x;
+        Oh[h].y += f * oi[h].y;
+        Oh[h].z += f * oi[h].z;
+        Oh[h].w += f * oi[h].w;
+      }
     }
 #pragma unroll
-    for (int h = 0; h < GQA; ++h) {
-      const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
-      Lh[h] += f * li[h];
-      Oh[h].x += f * oi[h].x;
-      Oh[h].y += f * oi[h].y;
-      Oh[h].z += f * oi[h].z;
-      Oh[h].w += f * oi[h].w;
+    for (int h = 0; h < HC; ++h) {
+      const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
+      reinterpret_cast<float4*>(outu + (h0 + h) * kHeadDim)[lane] =
+          make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
     }
-  }
-#pragma unroll
-  for (int h = 0; h < GQA; ++h) {
-    const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
-    reinterpret_cast<float4*>(outu + h * kHeadDim)[lane] =
-        make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
   }
   if (lane == 0) p.cnt[u] = 0u;  // ready for the next launch
 }
@@ -981,8 +991,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
             const int hB = (g >> 1) + 4 * nt;
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-              lq.qv[nt][s][0] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
-              lq.qv[nt][s][1] = hB < GQA ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+              lq.qv[nt][s][0] = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd), T()) : 0u;
+              lq.qv[nt][s][1] = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8), T()) : 0u;
             }
           }
           lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
@@ -993,7 +1003,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
             const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
             if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
           } else if (int(d.w >> 16) % 4 == warp) {
-            residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, lq, st, lane, p.c_log2);
+            residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, qs, st, lane, p.c_log2);
           }
         }
         // release the stage; the last warp to release it refills it with item xi + kStages
