@@ -123,11 +123,24 @@ struct WarpState {
   float m[NT], l[NT], zv[NT];
 };
 
-// Query operand of this lane: B column g = (head g/2 (+4 nt), part g%2).
+// Query pairs of this lane in fp16: head (g/2) + 4 nt, channels 16 s + 2 qd (+1) for
+// j = 0 and 8 more for j = 1.  They are the B column g of the code products (with the
+// part g % 2 chosen by negmask) and, stored as register quads, the A operand of the
+// zero-point product, whose rows are heads:
+//   NT = 2: quad s = {q(0,s,0), q(1,s,0), q(0,s,1), q(1,s,1)}: rows g / g+8 = heads
+//           g/2 and g/2 + 4 at k-step s;
+//   NT = 1: quad i = {q(0,i,0), q(0,i+4,0), q(0,i,1), q(0,i+4,1)}: rows g / g+8 = head
+//           g/2 at k-steps i and i + 4.
 template <int NT>
 struct LaneQ {
-  uint32_t qv[NT][8][2];  // q pairs in fp16: channels 16s + 2qd (+1), and +8
-  uint32_t negmask;       // fp16x2 -1 for lo-part lanes (odd g), 0 otherwise
+  uint32_t qa[NT == 2 ? 8 : 4][4];
+  uint32_t negmask;  // fp16x2 -1 for lo-part lanes (odd g), 0 otherwise
+  __device__ __forceinline__ uint32_t& qv(int nt, int s, int j) {
+    return NT == 2 ? qa[s][2 * j + nt] : qa[s & 3][2 * j + (s >> 2)];
+  }
+  __device__ __forceinline__ uint32_t qv(int nt, int s, int j) const {
+    return NT == 2 ? qa[s][2 * j + nt] : qa[s & 3][2 * j + (s >> 2)];
+  }
 };
 
 template <int NT>
@@ -224,8 +237,8 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
       uint32_t b[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        b[nt][0] = fold_one(lq.qv[nt][s][0], to_f16x2(jj ? sc.z : sc.x, T()), lq.negmask, __half());
-        b[nt][1] = fold_one(lq.qv[nt][s][1], to_f16x2(jj ? sc.w : sc.y, T()), lq.negmask, __half());
+        b[nt][0] = fold_one(lq.qv(nt, s, 0), to_f16x2(jj ? sc.z : sc.x, T()), lq.negmask, __half());
+        b[nt][1] = fold_one(lq.qv(nt, s, 1), to_f16x2(jj ? sc.w : sc.y, T()), lq.negmask, __half());
       }
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
@@ -290,22 +303,36 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
     }
   }
 
-  // -- zero points: Z[h] = sum_c q[h][c] * zA[c] --
-  float z[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) z[nt][i] = 0.0f;
+  // -- zero points: Z[h] = sum_c q[h][c] * zA[c], with the query quads as A (rows are
+  //    heads) and the zero points as B (every column the same); the 16 bytes at
+  //    64 i + 16 qd are the B pairs of k-steps 2i and 2i+1 --
+  float zh[NT];
   {
-    // only rows g of the product are used: rows g + 8 of A are zero, so each A fragment
-    // is two loaded registers and two zeros (no register copies)
     const uint8_t* kz = rec + R::k_zero + grp * 256 + 16 * qd;
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t a[4] = {to_f16x2(lds32(kz + 64 * (s >> 1) + 8 * (s & 1)), T()), 0u,
-                             to_f16x2(lds32(kz + 64 * (s >> 1) + 8 * (s & 1) + 4), T()), 0u};
+    for (int i = 0; i < 4; ++i) {
+      const uint4 zz = lds128(kz + 64 * i);
+      const uint32_t b0[2] = {to_f16x2(zz.x, T()), to_f16x2(zz.z, T())};
+      const uint32_t b1[2] = {to_f16x2(zz.y, T()), to_f16x2(zz.w, T())};
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816(z[nt], a, lq.qv[nt][s][0], lq.qv[nt][s][1], __half());
+      for (int jj = 0; jj < 2; ++jj) {
+        const int s = 2 * i + jj;
+        if constexpr (NT == 2) {
+          mma_16816(z0, lq.qa[s], b0[jj], b1[jj], __half());  // rows g: head g/2, g+8: head g/2 + 4
+        } else if (s < 4) {
+          mma_16816(z0, lq.qa[s], b0[jj], b1[jj], __half());  // rows g: k-step s
+        } else {
+          mma_16816(z1, lq.qa[s - 4], b0[jj], b1[jj], __half());  // rows g+8: k-step s
+        }
+      }
+    }
+    // this lane holds Z of head g/2 (+4); head qd (+4) sits in lane 8 qd
+    if constexpr (NT == 2) {
+      zh[0] = __shfl_sync(kFull, z0[0], 8 * qd);
+      zh[1] = __shfl_sync(kFull, z0[2], 8 * qd);
+    } else {
+      zh[0] = __shfl_sync(kFull, z0[0] + z1[2], 8 * qd);
     }
   }
 
@@ -319,7 +346,7 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int r = 0; r < 2; ++r)
-        L[mt][nt][r] = fmaf(acc[mt][nt][2 * r] + acc[mt][nt][2 * r + 1], cc, z[nt][0] * c_log2);
+        L[mt][nt][r] = fmaf(acc[mt][nt][2 * r] + acc[mt][nt][2 * r + 1], cc, zh[nt] * c_log2);
   softmax_step<NT, 2>(st, L);
 
   // -- probabilities times the value scales, as (hi, lo) pairs -> B operand of PV.
@@ -991,8 +1018,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
             const int hB = (g >> 1) + 4 * nt;
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-              lq.qv[nt][s][0] = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd), T()) : 0u;
-              lq.qv[nt][s][1] = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8), T()) : 0u;
+              lq.qv(nt, s, 0) = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd), T()) : 0u;
+              lq.qv(nt, s, 1) = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8), T()) : 0u;
             }
           }
           lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
