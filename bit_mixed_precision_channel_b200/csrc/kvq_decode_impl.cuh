@@ -164,33 +164,37 @@ __device__ __forceinline__ void reset_state(WarpState<NT>& st) {
 // stay below 2^8 and most groups skip the rescale of the accumulators.
 template <int NT, int MT>
 __device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)[MT][NT][2]) {
-  bool moved = false;
+  // the lanes' own maxima decide whether any head can move; only then are they reduced
+  float mx[NT];
+  bool big = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    mx[nt] = L[0][nt][0];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) mx[nt] = fmaxf(mx[nt], fmaxf(L[mt][nt][0], L[mt][nt][1]));
+    big |= mx[nt] > st.m[nt] + 8.0f;
+  }
+  if (!__any_sync(kFull, big)) return;
   float alpha[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    float mx = L[0][nt][0];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(L[mt][nt][0], L[mt][nt][1]));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+    mx[nt] = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 4));
+    mx[nt] = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 8));
+    mx[nt] = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 16));
     alpha[nt] = 1.0f;
-    if (mx > st.m[nt] + 8.0f) {
-      alpha[nt] = ex2(st.m[nt] - mx);  // 0 on the first group (m = -inf)
-      st.m[nt] = mx;
+    if (mx[nt] > st.m[nt] + 8.0f) {
+      alpha[nt] = ex2(st.m[nt] - mx[nt]);  // 0 on the first group (m = -inf)
+      st.m[nt] = mx[nt];
       st.l[nt] *= alpha[nt];
       st.zv[nt] *= alpha[nt];
-      moved = true;
     }
   }
-  if (__any_sync(kFull, moved)) {
 #pragma unroll
-    for (int mc = 0; mc < 8; ++mc)
+  for (int mc = 0; mc < 8; ++mc)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= alpha[nt];
-  }
+      for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= alpha[nt];
 }
 
 // ---------------------------------------------------------------- one quantized group
@@ -622,7 +626,9 @@ struct CtaShared {
   uint64_t full_bar[kStages];  // stage filled (bulk-copy bytes landed)
   int rel[kStages];            // warps that released the stage's current item
   int red[4];
-  int b0, base0, abort_flag, issued;
+  int b0, base0, abort_flag, issued, arrived;
+  int tail_u;         // unit whose split merge waits for the end of the range, or -1
+  uint32_t tail_io;   // its first and last contributors
   int pref[kSeqCache];         // exclusive prefix of the weights (x kv heads), one-pass case
   int nseg, more, nspan, uord, qslot_cont;
   Cursor cur;                  // first item of the next segment
@@ -785,6 +791,54 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA,
   }
 }
 
+// Merges heads h0 .. h0 + HC - 1 of the nc partial states at pu (log-sum-exp) into outu.
+// One warp; lane i holds channels 4i .. 4i + 3.
+template <int HC, int UNROLL>
+__device__ __forceinline__ void merge_heads(const float* pu, size_t slot, int nc, int h0, float* outu, int lane) {
+  float Mh[HC], Lh[HC];
+  float4 Oh[HC];
+#pragma unroll
+  for (int h = 0; h < HC; ++h) Mh[h] = -INFINITY;
+  for (int i = lane; i < nc; i += 32)
+#pragma unroll
+    for (int h = 0; h < HC; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + (h0 + h) * kPartStride + kHeadDim));
+#pragma unroll
+  for (int h = 0; h < HC; ++h) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
+    Lh[h] = 0.0f;
+    Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // every contributor's loads of a batch are in flight together
+#pragma unroll UNROLL
+  for (int i = 0; i < nc; ++i) {
+    const float* pi = pu + i * slot + h0 * kPartStride;
+    float mi[HC], li[HC];
+    float4 oi[HC];
+#pragma unroll
+    for (int h = 0; h < HC; ++h) {
+      mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
+      li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
+      oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
+    }
+#pragma unroll
+    for (int h = 0; h < HC; ++h) {
+      const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
+      Lh[h] += f * li[h];
+      Oh[h].x += f * oi[h].x;
+      Oh[h].y += f * oi[h].y;
+      Oh[h].z += f * oi[h].z;
+      Oh[h].w += f * oi[h].w;
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < HC; ++h) {
+    const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
+    reinterpret_cast<float4*>(outu + (h0 + h) * kHeadDim)[lane] =
+        make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
+  }
+}
+
 // One warp: counts this contributor in for unit u and, if it is the last of the
 // contributors i0..i1, merges their partial states (log-sum-exp) into the output.
 template <int GQA>
@@ -843,6 +897,21 @@ __device__ __forceinline__ void merge_partials(const DecodeParams& p, int u, int
     }
   }
   if (lane == 0) p.cnt[u] = 0u;  // ready for the next launch
+}
+
+// The same with the whole CTA, for a unit end that is the CTA's last item (all four
+// warps are free): thread 96 counts in; if the CTA is the last contributor, warp w
+// merges heads w, w + 4, ...
+template <int GQA>
+__device__ __noinline__ void merge_partials_cta(const DecodeParams& p, int* flag, int u, int i0, int i1, float* outu,
+                                                   int warp, int lane) {
+  const int nc = i1 - i0 + 1;
+  if (warp == 3 && lane == 0) *flag = int(atomic_add_acq_rel_gpu(p.cnt + u, 1u));
+  named_sync();  // the count (and, through it, the other contributors' partials) is seen by all
+  if (*flag != nc - 1) return;
+  const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
+  for (int h = warp; h < GQA; h += 4) merge_heads<1, 8>(pu, size_t(GQA) * kPartStride, nc, h, outu, lane);
+  if (warp == 3 && lane == 0) p.cnt[u] = 0u;  // ready for the next launch
 }
 
 template <typename T, int GQA, int KB, int P>
@@ -916,6 +985,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
     fence_mbar_init();
     sh.abort_flag = 0;
     sh.issued = 0;
+    sh.tail_u = -1;
   }
 
   // Moves sh.cur to the first item at or after position pos (all threads).
@@ -1109,7 +1179,15 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
             // The barrier orders every thread's partial writes before the counter update,
             // which is a release at device scope; the merging CTA acquires it.
             named_sync();
-            if (warp == 3) merge_partials<GQA>(p, u, i0, i1, outu, lane);
+            if (t == nseg - 1 && !sh.more) {
+              // the CTA's last item: all warps merge, after the loop
+              if (tid == 0) {
+                sh.tail_u = u;
+                sh.tail_io = d.io;
+              }
+            } else if (warp == 3) {
+              merge_partials<GQA>(p, u, i0, i1, outu, lane);
+            }
           }
         }
       }
@@ -1117,6 +1195,14 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
       if (!sh.more) break;
       __syncthreads();  // every item of the segment is consumed before its slots are reused
     }
+  }
+
+  named_sync();
+  if (sh.tail_u >= 0) {
+    const int u = sh.tail_u, b = u / p.Hkv, h = u - b * p.Hkv;
+    const uint32_t io = sh.tail_io;
+    merge_partials_cta<GQA>(p, &sh.arrived, u, int(io & 0xffffu), int(io >> 16),
+                            p.out + (size_t(b) * p.Hq + size_t(h) * GQA) * kHeadDim, warp, lane);
   }
 
   // ---------------------------------------------------------------- 3. leave
