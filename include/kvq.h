@@ -265,7 +265,10 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, 
  * all-zero output row.
  * Precision: inside the kernel q*scale (keys) and p*scale (values) are carried as an
  * fp16 high part plus an fp16 low part, so |q| * key scale must stay below the fp16
- * maximum (65504); codes are exact.  Accumulation is fp32. */
+ * maximum (65504); codes are exact.  Accumulation is fp32.  For bf16 caches the query,
+ * the key scales and the key zero points enter the tensor cores as fp16: they must lie
+ * within fp16's range (|x| <= 65504), where bf16 values are exact in fp16 down to 2^-14
+ * and keep fewer bits below it (fp16 subnormals). */
 KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t pool_pages,
                                 const void* q, int32_t batch,
                                 const int32_t* page_table, int32_t max_pages,
