@@ -236,10 +236,11 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(pool) || !aligned16(q) || !aligned16(res_k) || !aligned16(res_v) || !aligned16(workspace))
     return KVQ_ERR_INVALID_ARG;
-  // the kernel's work line (32-token groups, 16-token residual pieces and a merge
-  // weight of 12 per (sequence, kv head)) is indexed with 32-bit integers
+  // the kernel's work line (32-token groups, weighted 16-token residual pieces and a
+  // merge weight per (sequence, kv head)) is indexed with 32-bit integers
   const long long line = (long long)batch * cfg->num_kv_heads *
-                         ((long long)max_pages * (cfg->page_tokens / 32) + (cfg->page_tokens + 15) / 16 + 12);
+                         ((long long)max_pages * (cfg->page_tokens / 32) +
+                          (long long)kDecodePieceWeight * ((cfg->page_tokens + 15) / 16) + kDecodeMergeWeight);
   if (line >= (1ll << 31)) return KVQ_ERR_INVALID_ARG;
   const Plan pl = decode_plan(cfg, batch);
   if (workspace_bytes < pl.part_bytes + pl.cnt_bytes) return KVQ_ERR_CAPACITY;

@@ -43,10 +43,8 @@ constexpr int kStages = 3;
 constexpr int kDecodeThreads = 128;
 constexpr int kResRowBytes = 272;  // residual row in shared memory: 256 bytes + 16 pad
 constexpr int kPieceTokens = 16;   // residual tokens per item
-// Extra weight at the end of every unit for the cost of merging its state (measured on
-// B200 to be worth about three stages of streaming work); no item starts there.  It
-// keeps a CTA whose range holds a unit end from carrying more work than the others.
-constexpr int kMergeWeight = 12;
+constexpr int kPieceWeight = kDecodePieceWeight;
+constexpr int kMergeWeight = kDecodeMergeWeight;
 
 // Compile-time offsets of one record (the same values as make_layout).
 template <int P, int KB>
@@ -468,7 +466,7 @@ __device__ __forceinline__ int seq_weight(const DecodeParams& p, int b, int& np,
     rl = 0;
     return -1;
   }
-  const int items = np * (P / 32) + (rl + kPieceTokens - 1) / kPieceTokens;
+  const int items = np * (P / 32) + kPieceWeight * ((rl + kPieceTokens - 1) / kPieceTokens);
   return items > 0 ? items + kMergeWeight : 0;
 }
 
@@ -488,18 +486,18 @@ __device__ __forceinline__ void cursor_load_seq(const DecodeParams& p, Cursor& c
 template <int P>
 __device__ __forceinline__ int item_weight(const Cursor& c) {
   if (c.k < c.nst) return min(128 / P, c.np - c.k * (128 / P)) * (P / 32);
-  return 1;
+  return kPieceWeight;
 }
 // Weight of a unit: its items, then the merge weight (0 for a unit without items).
 template <int P>
 __device__ __forceinline__ int unit_weight(const Cursor& c) {
-  const int items = c.np * (P / 32) + c.nres;
+  const int items = c.np * (P / 32) + kPieceWeight * c.nres;
   return items > 0 ? items + kMergeWeight : 0;
 }
 
 template <int P>
 __device__ __forceinline__ int unit_weight_of(int2 v) {
-  const int items = v.x * (P / 32) + (v.y + kPieceTokens - 1) / kPieceTokens;
+  const int items = v.x * (P / 32) + kPieceWeight * ((v.y + kPieceTokens - 1) / kPieceTokens);
   return items > 0 ? items + kMergeWeight : 0;
 }
 
@@ -544,10 +542,10 @@ __device__ __forceinline__ void cursor_seek(const DecodeParams& p, Cursor& c, in
     c.s = c.ubase + 4 * c.k;
     return;
   }
-  const int j = max(0, ou - c.np * (P / 32));
+  const int j = max(0, (ou - c.np * (P / 32) + kPieceWeight - 1) / kPieceWeight);
   if (j < c.nres) {
     c.k = c.nst + j;
-    c.s = c.ubase + c.np * (P / 32) + j;
+    c.s = c.ubase + c.np * (P / 32) + kPieceWeight * j;
     return;
   }
   c.s = c.ubase + unit_weight<P>(c);
@@ -659,7 +657,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
         kend = kst;
       } else {
         const int r0 = c.ubase + c.np * GPP;
-        kend = c.nst + min(c.nres, max(0, hi - r0));
+        kend = c.nst + min(c.nres, max(0, (hi - r0 + kPieceWeight - 1) / kPieceWeight));
       }
       const int cnt = min(kend - c.k, kSegItems - n);
       UnitSpan& sp = sh.span[ns];
@@ -675,7 +673,8 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
       if (sp.first) qcont = (++uord) % 3;
       sp.qslot = qcont;
       const int uw = unit_weight<P>(c);
-      const int last_start = c.ubase + uw - kMergeWeight - (c.nres > 0 ? 1 : (c.np - (c.nst - 1) * PPC) * GPP);
+      const int last_start =
+          c.ubase + uw - kMergeWeight - (c.nres > 0 ? kPieceWeight : (c.np - (c.nst - 1) * PPC) * GPP);
       sp.io = uint32_t(ow.of(c.ubase)) | (uint32_t(ow.of(last_start)) << 16);
       n += cnt;
       ++ns;
@@ -696,7 +695,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<G
       } else if (c.k == kend) {
         c.s = hi;  // the range ends inside this unit
       } else {
-        c.s = c.ubase + (c.k < c.nst ? 4 * c.k : c.np * GPP + (c.k - c.nst));
+        c.s = c.ubase + (c.k < c.nst ? 4 * c.k : c.np * GPP + kPieceWeight * (c.k - c.nst));
       }
     }
     sh.cur = c;

@@ -14,6 +14,14 @@
 
 namespace kvq {
 
+// Weights of the decode kernel's work line, in units of one 32-token page group (a page
+// stage of 128 tokens weighs 4).  Measured on B200 (per-CTA traces regressed on the
+// items each CTA held): a 16-token residual piece, which one warp processes while the
+// stage waits for it, costs about as much time as three page groups; the merge at the
+// end of a (sequence, KV head) is given extra weight where no item starts.
+constexpr int kDecodePieceWeight = 3;
+constexpr int kDecodeMergeWeight = 6;
+
 constexpr int kHeadDim = 128;
 constexpr int kKeyGroup = 32;
 constexpr unsigned kFull = 0xffffffffu;
