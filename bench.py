@@ -268,14 +268,20 @@ def run_gpu(args):
     Kd, Vd = dev_bits(Kh), dev_bits(Vh)
     caches = [PagedKVCache(cfg, B, max_pages, pool_pages, device=dev) for _ in range(L_layers)]
 
-    # quantize leg: prefill of every layer, one launch per layer, timed
-    caches[0].prefill_batch(Kd, Vd)  # warm-up launch (first-call attribute setup)
-    caches[0] = PagedKVCache(cfg, B, max_pages, pool_pages, device=dev)
+    # quantize leg: prefill of every layer (page allocation and tables untimed), then the
+    # quantize launches of all layers timed: one launch per layer quantizes its 16 x 4096
+    # tokens into the pages the prefill assigned (the same records again)
+    for c in caches:
+        c.prefill_batch(Kd, Vd)
+    n_seq_pages = w.context // P
+    srcK = kb.Source.token_major(Kd.view(B * w.context, w.Hkv, D), cfg)
+    srcV = kb.Source.token_major(Vd.view(B * w.context, w.Hkv, D), cfg)
+    dsts = [c.page_table[:, :n_seq_pages].contiguous().view(-1) for c in caches]
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for c in caches:
-        c.prefill_batch(Kd, Vd)
+    for c, dst in zip(caches, dsts):
+        kb.quantize_pages(cfg, srcK, srcV, dst, c.pool, c.err)
     e1.record()
     torch.cuda.synchronize()
     q_ms = e0.elapsed_time(e1) / L_layers

@@ -66,6 +66,31 @@ __device__ __forceinline__ int quant_code(float x, float zero, float scale, int 
   return int(r);
 }
 
+// Reciprocal of a group's scale for quant_code_fast, or 0 when the fast path may not be
+// used (scale 0, or below the smallest normal float, where the approximate reciprocal
+// flushes).
+__device__ __forceinline__ float quant_rcp(float scale) {
+  if (!(scale >= 1.17549435e-38f)) return 0.0f;
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(scale));
+  return r;
+}
+
+// The same code as quant_code, bit for bit, with one multiply instead of the IEEE divide
+// in almost every case.  x - zero >= 0 and the quotient that matters is at most
+// qmax + 1/2 <= 15.5 (above it the clamp decides), so d * rcp is within 2^-17 of the
+// correctly rounded quotient (rcp.approx: relative error below 2^-22; the divide: half
+// an ulp, at most 2^-20).  rint of the two agrees unless the quotient lies within that
+// distance of a rounding boundary k + 1/2; inside 2^-14 of one, the IEEE divide decides.
+__device__ __forceinline__ int quant_code_fast(float x, float zero, float scale, float rcp, int qmax) {
+  if (rcp == 0.0f) return quant_code(x, zero, scale, qmax);
+  const float d = __fsub_rn(x, zero);
+  float q = __fmul_rn(d, rcp);
+  if (fabsf(__fsub_rn(q, floorf(q)) - 0.5f) < 1.0f / 16384.0f) q = __fdiv_rn(d, scale);
+  const float r = fminf(fmaxf(rintf(q), 0.0f), float(qmax));
+  return int(r);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p) {
   pdl_wait();
@@ -180,9 +205,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       uint16_t sb, zb;
       float zero;
       const float scale = quant_params<T>(mn, mx, qmax, sb, zb, zero);
+      const float rcp = quant_rcp(scale);
       for (int t = 0; t < kKeyGroup; ++t) {
         const int tok = g * kKeyGroup + t;
-        const int code = quant_code(bits_to_float(col[t * kHeadDim], T()), zero, scale, qmax);
+        const int code = quant_code_fast(bits_to_float(col[t * kHeadDim], T()), zero, scale, rcp, qmax);
         if (j >= 0) {
           cA[tok * kHeadDim + pc] = uint8_t(code >> 2);
           cB[tok * k + pj] = uint8_t(code & 3);
@@ -217,9 +243,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       uint16_t sb, zb;
       float zero;
       const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
+      const float rcp = quant_rcp(scale);
       uint32_t four = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) four |= uint32_t(quant_code(x[i], zero, scale, 3)) << (8 * i);
+      for (int i = 0; i < 4; ++i) four |= uint32_t(quant_code_fast(x[i], zero, scale, rcp, 3)) << (8 * i);
       *reinterpret_cast<uint32_t*>(cV + t * kHeadDim + 4 * lane) = four;
       if (lane == 0) {
         vs_out[value_meta_pos(t)] = sb;
@@ -240,12 +267,15 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   if (need_v) {
     uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
     for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) {
+      // element e = 8a + 2b + f of word i holds token t0 + 16a + 8(b >> 1) + f and
+      // channel c0 + 8(b & 1) (the inverse of value_at_slot), at bit elem_bit(e)
+      const int mm = i & 3, ln = (i >> 2) & 31, blk = i >> 7;
+      const uint8_t* base = cV + (32 * (blk >> 1) + 2 * (ln & 3)) * kHeadDim + 16 * (4 * (blk & 1) + mm) + (ln >> 2);
       uint32_t word = 0;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        int t, c;
-        value_at_slot(16 * i + e, t, c);
-        word |= uint32_t(cV[t * kHeadDim + c] & 3u) << elem_bit(e);
+        const int a = e >> 3, b = (e >> 1) & 3, f = e & 1;
+        word |= uint32_t(base[(16 * a + 8 * (b >> 1) + f) * kHeadDim + 8 * (b & 1)] & 3u) << elem_bit(e);
       }
       vq[i] = word;
     }
