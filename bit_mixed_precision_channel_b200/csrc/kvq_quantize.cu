@@ -18,14 +18,24 @@ namespace kvq {
 
 constexpr int kQThreads = 256;
 
-// Shared memory of one quantize CTA.
+// Shared memory of one quantize CTA.  A CTA quantizes either the keys of a (page, kv
+// head) (selection and both planes) or its values, so that four CTAs fit on an SM.
 struct QSmem {
-  static size_t bytes(int P, int k) {
-    return size_t(P) * kHeadDim * 2 * 2    // K and V tiles
+  static size_t key_bytes(int P, int k) {
+    return size_t(P) * kHeadDim * 2        // K tile
            + size_t(P) * kHeadDim          // plane-A codes [P][128]
            + size_t(P) * (k > 0 ? k : 16)  // plane-B codes [P][k]
-           + size_t(P) * kHeadDim          // value codes [P][128]
            + kHeadDim * 4 * 2 + 16 * 4;    // scores, plane-B row of each channel, warp counts
+  }
+  static size_t value_bytes(int P) {
+    return size_t(P) * kHeadDim * 2  // V tile
+           + size_t(P) * kHeadDim;   // value codes [P][128]
+  }
+  static size_t bytes(int P, int k, int mode) {
+    size_t b = 0;
+    if (mode & (kModeSelect | kModeKeys)) b = key_bytes(P, k);
+    if (mode & kModeValues) b = b > value_bytes(P) ? b : value_bytes(P);
+    return b;
   }
 };
 
@@ -114,18 +124,23 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   }
   uint8_t* rec = p.pool + (size_t(dst) * p.Hkv + h) * p.L.record;
 
+  // z = 0: the key part of the requested modes, z = gridDim.z - 1: the value part
+  const int kmodes = blockIdx.z == 0 ? p.mode & (kModeSelect | kModeKeys) : 0;
+  const int mode = kmodes | (blockIdx.z == gridDim.z - 1 ? p.mode & kModeValues : 0);
+  const bool need_k = kmodes != 0;
+  const bool need_v = mode & kModeValues;
+
   extern __shared__ __align__(16) uint8_t smem[];
+  // key part: K tile, plane A codes [token][key position], plane B codes [token][boost
+  // position], scores; value part: V tile, value codes [token][channel]
   uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* Vs = Ks + P * kHeadDim;
-  uint8_t* cA = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);  // plane A codes [token][key position]
-  uint8_t* cB = cA + P * kHeadDim;                                // plane B codes [token][boost position]
-  uint8_t* cV = cB + P * (k > 0 ? k : 16);
-  float* score = reinterpret_cast<float*>(cV + P * kHeadDim);
+  uint8_t* cA = reinterpret_cast<uint8_t*>(Ks + P * kHeadDim);
+  uint8_t* cB = cA + P * kHeadDim;
+  float* score = reinterpret_cast<float*>(cB + P * (k > 0 ? k : 16));
   int* row_of = reinterpret_cast<int*>(score + kHeadDim);
   int* warp_cnt = row_of + kHeadDim;
-
-  const bool need_k = p.mode & (kModeSelect | kModeKeys);
-  const bool need_v = p.mode & kModeValues;
+  uint16_t* Vs = reinterpret_cast<uint16_t*>(smem);
+  uint8_t* cV = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);
 
   // ---- stage the page tiles (rows of 128 x 16-bit = 16 x 16 bytes)
   if (need_k) {
@@ -145,7 +160,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   __syncthreads();
 
   // ---- a1: boosted channels (or read them back from the record)
-  if (p.mode & kModeSelect) {
+  if (mode & kModeSelect) {
     if (tid < kHeadDim) {
       float m = 0.0f;
       for (int t = 0; t < P; ++t) m = fmaxf(m, fabsf(bits_to_float(Ks[t * kHeadDim + tid], T())));
@@ -173,7 +188,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       rec[p.L.boost_idx + row_of[tid]] = uint8_t(tid);
     }
     __syncthreads();
-  } else if (p.mode & kModeKeys) {
+  } else if (mode & kModeKeys) {
     if (tid < kHeadDim) row_of[tid] = -1;
     __syncthreads();
     if (tid < k) {
@@ -184,7 +199,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   }
 
   // ---- a2: keys, one task per (group, channel)
-  if (p.mode & kModeKeys) {
+  if (mode & kModeKeys) {
     const int n_groups = P / kKeyGroup;
     uint16_t* ks_out = reinterpret_cast<uint16_t*>(rec + p.L.k_scale);
     uint16_t* kz_out = reinterpret_cast<uint16_t*>(rec + p.L.k_zero);
@@ -257,7 +272,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   __syncthreads();
 
   // ---- pack the code planes into the record
-  if (p.mode & kModeKeys) {
+  if (mode & kModeKeys) {
     uint32_t* kA = reinterpret_cast<uint32_t*>(rec + p.L.k_codes);
     for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) kA[i] = pack16(cA + 16 * i);
     const int kbw = k / 16;
@@ -334,8 +349,10 @@ __global__ void flush_commit_kernel(int32_t* res_len, const int32_t* new_page, i
 
 cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream) {
   if (n_items <= 0) return cudaSuccess;
-  const size_t smem = QSmem::bytes(p.P, p.k);
-  const dim3 grid(n_items, p.Hkv);
+  const size_t smem = QSmem::bytes(p.P, p.k, p.mode);
+  // keys and values of a page in separate CTAs when both are requested
+  const bool both = (p.mode & (kModeSelect | kModeKeys)) && (p.mode & kModeValues);
+  const dim3 grid(n_items, p.Hkv, both ? 2 : 1);
   static int seen_bf16[64], seen_f16[64];
   if (dtype == KVQ_BF16) {
     const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__nv_bfloat16>, int(smem), seen_bf16);
