@@ -290,6 +290,13 @@ __device__ __forceinline__ uint32_t e2m1_pair_lo(uint32_t x) {
 __device__ __forceinline__ uint32_t code_pass(uint32_t w, int a) { return (w >> (2 * a)) & 0x33333333u; }
 
 __device__ __forceinline__ uint32_t bf2_as_u32(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
+// A register of two cache-dtype values as the dtype's pair type, and back.
+__device__ __forceinline__ __half2 u32_as_pair(uint32_t x, __half) { return u32_as_h2(x); }
+__device__ __forceinline__ __nv_bfloat162 u32_as_pair(uint32_t x, __nv_bfloat16) {
+  return *reinterpret_cast<__nv_bfloat162*>(&x);
+}
+__device__ __forceinline__ uint32_t pair_as_u32(__half2 h) { return h2_as_u32(h); }
+__device__ __forceinline__ uint32_t pair_as_u32(__nv_bfloat162 h) { return bf2_as_u32(h); }
 
 // ------------------------------------------------------------------ dependent launches
 

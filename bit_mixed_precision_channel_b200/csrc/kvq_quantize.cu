@@ -60,7 +60,8 @@ __device__ __forceinline__ uint32_t pack16(const uint8_t* c) {
 template <typename T>
 __device__ __forceinline__ float quant_params(float mn, float mx, int qmax, uint16_t& sbits, uint16_t& zbits,
                                               float& zero) {
-  const float range = __fsub_rn(mx, mn);
+  // +0 for a group of zeros whatever the signs the min/max kept (x - x is +0 too)
+  const float range = __fsub_rn(__fadd_rn(mx, 0.0f), __fadd_rn(mn, 0.0f));
   const float s32 = __fdiv_rn(range, float(qmax));
   sbits = round_up_bits(s32, T());
   zero = __fadd_rn(mn, 0.0f);  // -0 -> +0
@@ -86,19 +87,21 @@ __device__ __forceinline__ float quant_rcp(float scale) {
   return r;
 }
 
-// The same code as quant_code, bit for bit, with one multiply instead of the IEEE divide
-// in almost every case.  x - zero >= 0 and the quotient that matters is at most
-// qmax + 1/2 <= 15.5 (above it the clamp decides), so d * rcp is within 2^-17 of the
-// correctly rounded quotient (rcp.approx: relative error below 2^-22; the divide: half
-// an ulp, at most 2^-20).  rint of the two agrees unless the quotient lies within that
-// distance of a rounding boundary k + 1/2; inside 2^-14 of one, the IEEE divide decides.
-__device__ __forceinline__ int quant_code_fast(float x, float zero, float scale, float rcp, int qmax) {
-  if (rcp == 0.0f) return quant_code(x, zero, scale, qmax);
-  const float d = __fsub_rn(x, zero);
-  float q = __fmul_rn(d, rcp);
-  if (fabsf(__fsub_rn(q, floorf(q)) - 0.5f) < 1.0f / 16384.0f) q = __fdiv_rn(d, scale);
-  const float r = fminf(fmaxf(rintf(q), 0.0f), float(qmax));
-  return int(r);
+// The same code as quant_code, bit for bit, without a divide in almost every case.
+// x - zero >= 0 and the quotient that matters is at most qmax + 1/2 <= 15.5 (above it
+// the clamp decides).  fma(d, rcp, 1.5 * 2^23) rounds the exact product d * rcp to an
+// integer n held in the low mantissa bits; d * rcp is within 2^-17 of the correctly
+// rounded quotient (rcp.approx: relative error below 2^-22; the divide: half an ulp,
+// at most 2^-20), so n is the code unless d * rcp lies within 2^-14 of a rounding
+// boundary n +- 1/2, where the IEEE divide decides.
+__device__ __forceinline__ uint32_t quant_code_fast(float x, float zero, float scale, float rcp, int qmax) {
+  if (rcp != 0.0f) {
+    const float d = __fsub_rn(x, zero);
+    const float t = __fmaf_rn(d, rcp, 12582912.0f);
+    const float res = __fmaf_rn(d, rcp, -__fsub_rn(t, 12582912.0f));  // d * rcp - n
+    if (fabsf(res) < 0.5f - 1.0f / 16384.0f) return min(__float_as_uint(t) & 0xffu, uint32_t(qmax));
+  }
+  return uint32_t(quant_code(x, zero, scale, qmax));
 }
 
 template <typename T>
@@ -198,60 +201,82 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
     __syncthreads();
   }
 
-  // ---- a2: keys, one task per (group, channel)
+  // ---- a2: keys, one task per (group, pair of adjacent channels): 32-bit loads and
+  //      packed min/max (exact) over the group's tokens
   if (mode & kModeKeys) {
+    using T2 = typename Pair<T>::type;
     const int n_groups = P / kKeyGroup;
     uint16_t* ks_out = reinterpret_cast<uint16_t*>(rec + p.L.k_scale);
     uint16_t* kz_out = reinterpret_cast<uint16_t*>(rec + p.L.k_zero);
     uint16_t* kbs_out = reinterpret_cast<uint16_t*>(rec + p.L.kb_scale);
-    for (int task = tid; task < n_groups * kHeadDim; task += kQThreads) {
-      const int g = task / kHeadDim, c = task % kHeadDim;
-      const uint16_t* col = Ks + g * kKeyGroup * kHeadDim + c;
-      float mn = bits_to_float(col[0], T()), mx = mn;
+    for (int task = tid; task < n_groups * (kHeadDim / 2); task += kQThreads) {
+      const int g = task / (kHeadDim / 2), c0 = 2 * (task % (kHeadDim / 2));
+      const uint32_t* col = reinterpret_cast<const uint32_t*>(Ks + g * kKeyGroup * kHeadDim + c0);
+      T2 lo = u32_as_pair(col[0], T()), hi = lo;
+#pragma unroll 8
       for (int t = 1; t < kKeyGroup; ++t) {
-        const float v = bits_to_float(col[t * kHeadDim], T());
-        mn = fminf(mn, v);
-        mx = fmaxf(mx, v);
+        const T2 v = u32_as_pair(col[t * (kHeadDim / 2)], T());
+        lo = __hmin2(lo, v);
+        hi = __hmax2(hi, v);
       }
-      const int j = row_of[c];
-      const int qmax = j >= 0 ? 15 : 3;
-      const int pc = key_pos(c);
-      const int pj = j >= 0 ? boost_pos(j, k / 16) : 0;
-      uint16_t sb, zb;
-      float zero;
-      const float scale = quant_params<T>(mn, mx, qmax, sb, zb, zero);
-      const float rcp = quant_rcp(scale);
+      const uint32_t lob = pair_as_u32(lo), hib = pair_as_u32(hi);
+      float scale[2], rcp[2], zero[2];
+      int qmax[2], j[2], pc[2], pj[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = c0 + e;
+        j[e] = row_of[c];
+        qmax[e] = j[e] >= 0 ? 15 : 3;
+        pc[e] = key_pos(c);
+        pj[e] = j[e] >= 0 ? boost_pos(j[e], k / 16) : 0;
+        uint16_t sb, zb;
+        scale[e] = quant_params<T>(bits_to_float(uint16_t(lob >> (16 * e)), T()),
+                                   bits_to_float(uint16_t(hib >> (16 * e)), T()), qmax[e], sb, zb, zero[e]);
+        rcp[e] = quant_rcp(scale[e]);
+        // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
+        const int pm = key_meta_pos(c);
+        ks_out[g * kHeadDim + pm] = j[e] >= 0 ? exact_bits(4.0f * scale[e], T()) : sb;
+        kz_out[g * kHeadDim + pm] = zb;
+        if (j[e] >= 0) kbs_out[g * k + j[e]] = sb;
+      }
       for (int t = 0; t < kKeyGroup; ++t) {
         const int tok = g * kKeyGroup + t;
-        const int code = quant_code_fast(bits_to_float(col[t * kHeadDim], T()), zero, scale, rcp, qmax);
-        if (j >= 0) {
-          cA[tok * kHeadDim + pc] = uint8_t(code >> 2);
-          cB[tok * k + pj] = uint8_t(code & 3);
-        } else {
-          cA[tok * kHeadDim + pc] = uint8_t(code);
+        const uint32_t w = col[t * (kHeadDim / 2)];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t code = quant_code_fast(bits_to_float(uint16_t(w >> (16 * e)), T()), zero[e], scale[e],
+                                                rcp[e], qmax[e]);
+          if (j[e] >= 0) {
+            cA[tok * kHeadDim + pc[e]] = uint8_t(code >> 2);
+            cB[tok * k + pj[e]] = uint8_t(code & 3);
+          } else {
+            cA[tok * kHeadDim + pc[e]] = uint8_t(code);
+          }
         }
       }
-      // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
-      const int pm = key_meta_pos(c);
-      ks_out[g * kHeadDim + pm] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
-      kz_out[g * kHeadDim + pm] = zb;
-      if (j >= 0) kbs_out[g * k + j] = sb;
     }
   }
 
-  // ---- a3: values, one warp per token
+  // ---- a3: values, two tokens per warp (a half-warp each, 8 channels per lane)
   if (need_v) {
-    const int warp = tid >> 5, lane = tid & 31;
+    using T2 = typename Pair<T>::type;
+    const int warp = tid >> 5, lane = tid & 31, hl = lane & 15;
     uint16_t* vs_out = reinterpret_cast<uint16_t*>(rec + p.L.v_scale);
     uint16_t* vz_out = reinterpret_cast<uint16_t*>(rec + p.L.v_zero);
-    for (int t = warp; t < P; t += kQThreads / 32) {
-      const uint2 raw = lds64(Vs + t * kHeadDim + 4 * lane);
-      float x[4] = {bits_to_float(uint16_t(raw.x & 0xffff), T()), bits_to_float(uint16_t(raw.x >> 16), T()),
-                    bits_to_float(uint16_t(raw.y & 0xffff), T()), bits_to_float(uint16_t(raw.y >> 16), T())};
-      float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
-      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    for (int t0 = 2 * warp; t0 < P; t0 += 2 * (kQThreads / 32)) {
+      const int t = t0 + (lane >> 4);
+      const uint4 raw = lds128(Vs + t * kHeadDim + 8 * hl);
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+      T2 lo = u32_as_pair(wv[0], T()), hi = lo;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
+      for (int i = 1; i < 4; ++i) {
+        lo = __hmin2(lo, u32_as_pair(wv[i], T()));
+        hi = __hmax2(hi, u32_as_pair(wv[i], T()));
+      }
+      float mn = fminf(bits_to_float(uint16_t(pair_as_u32(lo)), T()), bits_to_float(uint16_t(pair_as_u32(lo) >> 16), T()));
+      float mx = fmaxf(bits_to_float(uint16_t(pair_as_u32(hi)), T()), bits_to_float(uint16_t(pair_as_u32(hi) >> 16), T()));
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(kFull, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
       }
@@ -259,11 +284,14 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       float zero;
       const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
       const float rcp = quant_rcp(scale);
-      uint32_t four = 0;
+      uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) four |= uint32_t(quant_code_fast(x[i], zero, scale, rcp, 3)) << (8 * i);
-      *reinterpret_cast<uint32_t*>(cV + t * kHeadDim + 4 * lane) = four;
-      if (lane == 0) {
+      for (int i = 0; i < 8; ++i) {
+        const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
+        packed[i >> 2] |= quant_code_fast(x, zero, scale, rcp, 3) << (8 * (i & 3));
+      }
+      *reinterpret_cast<uint2*>(cV + t * kHeadDim + 8 * hl) = make_uint2(packed[0], packed[1]);
+      if (hl == 0) {
         vs_out[value_meta_pos(t)] = sb;
         vz_out[value_meta_pos(t)] = zb;
       }
