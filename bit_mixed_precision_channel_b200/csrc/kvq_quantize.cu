@@ -25,6 +25,7 @@ struct QSmem {
     return size_t(P) * kHeadDim * 2        // K tile
            + size_t(P) * kHeadDim          // plane-A codes [P][128]
            + size_t(P) * (k > 0 ? k : 16)  // plane-B codes [P][k]
+           + 16                            // scratch byte of channels that are not boosted
            + kHeadDim * 4 * 2 + 16 * 4;    // scores, plane-B row of each channel, warp counts
   }
   static size_t value_bytes(int P) {
@@ -77,7 +78,7 @@ __device__ __forceinline__ int quant_code(float x, float zero, float scale, int 
   return int(r);
 }
 
-// Reciprocal of a group's scale for quant_code_fast, or 0 when the fast path may not be
+// Reciprocal of a group's scale for quant_code_fma, or 0 when the fast path may not be
 // used (scale 0, or below the smallest normal float, where the approximate reciprocal
 // flushes).
 __device__ __forceinline__ float quant_rcp(float scale) {
@@ -87,21 +88,20 @@ __device__ __forceinline__ float quant_rcp(float scale) {
   return r;
 }
 
-// The same code as quant_code, bit for bit, without a divide in almost every case.
+// The code quant_code gives, bit for bit, without a divide in almost every case.
 // x - zero >= 0 and the quotient that matters is at most qmax + 1/2 <= 15.5 (above it
 // the clamp decides).  fma(d, rcp, 1.5 * 2^23) rounds the exact product d * rcp to an
 // integer n held in the low mantissa bits; d * rcp is within 2^-17 of the correctly
 // rounded quotient (rcp.approx: relative error below 2^-22; the divide: half an ulp,
 // at most 2^-20), so n is the code unless d * rcp lies within 2^-14 of a rounding
-// boundary n +- 1/2, where the IEEE divide decides.
-__device__ __forceinline__ uint32_t quant_code_fast(float x, float zero, float scale, float rcp, int qmax) {
-  if (rcp != 0.0f) {
-    const float d = __fsub_rn(x, zero);
-    const float t = __fmaf_rn(d, rcp, 12582912.0f);
-    const float res = __fmaf_rn(d, rcp, -__fsub_rn(t, 12582912.0f));  // d * rcp - n
-    if (fabsf(res) < 0.5f - 1.0f / 16384.0f) return min(__float_as_uint(t) & 0xffu, uint32_t(qmax));
-  }
-  return uint32_t(quant_code(x, zero, scale, qmax));
+// boundary n +- 1/2.  There `near` is set and the caller redoes the element with
+// quant_code.  With rcp = 0 (scale 0) the code is 0, as quant_code gives.
+__device__ __forceinline__ uint32_t quant_code_fma(float x, float zero, float rcp, uint32_t qmax, bool& near) {
+  const float d = __fsub_rn(x, zero);
+  const float t = __fmaf_rn(d, rcp, 12582912.0f);
+  const float res = __fmaf_rn(d, rcp, -__fsub_rn(t, 12582912.0f));
+  near = !(fabsf(res) < 0.5f - 1.0f / 16384.0f);
+  return min(__float_as_uint(t) & 0xffu, qmax);
 }
 
 template <typename T>
@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
   uint8_t* cA = reinterpret_cast<uint8_t*>(Ks + P * kHeadDim);
   uint8_t* cB = cA + P * kHeadDim;
-  float* score = reinterpret_cast<float*>(cB + P * (k > 0 ? k : 16));
+  uint8_t* cScratch = cB + P * (k > 0 ? k : 16);  // plane-B bytes of channels that are not boosted
+  float* score = reinterpret_cast<float*>(cScratch + 16);
   int* row_of = reinterpret_cast<int*>(score + kHeadDim);
   int* warp_cnt = row_of + kHeadDim;
   uint16_t* Vs = reinterpret_cast<uint16_t*>(smem);
@@ -164,31 +165,51 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
 
   // ---- a1: boosted channels (or read them back from the record)
   if (mode & kModeSelect) {
-    if (tid < kHeadDim) {
-      float m = 0.0f;
-      for (int t = 0; t < P; ++t) m = fmaxf(m, fabsf(bits_to_float(Ks[t * kHeadDim + tid], T())));
-      score[tid] = m;
-    }
-    __syncthreads();
-    if (tid < kHeadDim) {
-      const float s = score[tid];
-      int rank = 0;
-      for (int c = 0; c < kHeadDim; ++c) {
-        const float o = score[c];
-        rank += (o > s) || (o == s && c < tid);
+    using T2 = typename Pair<T>::type;
+    // score_c = max |K[t][c]|: thread = (channel pair tid / 4, token quarter tid % 4),
+    // packed abs/max (exact), then the four quarters by shuffles
+    {
+      const int pr = tid >> 2, qt = tid & 3;
+      const uint32_t* col = reinterpret_cast<const uint32_t*>(Ks) + pr;
+      const int tq = P / 4;
+      T2 m = __habs2(u32_as_pair(col[qt * tq * (kHeadDim / 2)], T()));
+#pragma unroll 8
+      for (int t = 1; t < tq; ++t) m = __hmax2(m, __habs2(u32_as_pair(col[(qt * tq + t) * (kHeadDim / 2)], T())));
+      uint32_t mb = pair_as_u32(m);
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1)
+        mb = pair_as_u32(__hmax2(u32_as_pair(mb, T()), u32_as_pair(__shfl_xor_sync(kFull, mb, off), T())));
+      if (qt == 0) {
+        score[2 * pr] = bits_to_float(uint16_t(mb), T());
+        score[2 * pr + 1] = bits_to_float(uint16_t(mb >> 16), T());
       }
-      const bool boosted = rank < k;
-      const unsigned ballot = __ballot_sync(kFull, boosted);
-      if ((tid & 31) == 0) warp_cnt[tid >> 5] = __popc(ballot);
-      __syncwarp();
-      row_of[tid] = boosted ? int(__popc(ballot & ((1u << (tid & 31)) - 1u))) : -1;
     }
     __syncthreads();
-    if (tid < kHeadDim && row_of[tid] >= 0) {
-      int before = 0;
-      for (int w = 0; w < (tid >> 5); ++w) before += warp_cnt[w];
-      row_of[tid] += before;
-      rec[p.L.boost_idx + row_of[tid]] = uint8_t(tid);
+    // rank of channel c: channels with a higher score, or an equal score and a lower
+    // index; two threads per channel (channels c' < 64 and >= 64), summed by a shuffle
+    {
+      const int c = tid >> 1, half = tid & 1;
+      const float sc = score[c];
+      int rank = 0;
+#pragma unroll 8
+      for (int i = 0; i < kHeadDim / 2; ++i) {
+        const int o = half * (kHeadDim / 2) + i;
+        const float so = score[o];
+        rank += (so > sc) || (so == sc && o < c);
+      }
+      rank += __shfl_xor_sync(kFull, rank, 1);
+      const bool boosted = rank < k;
+      // plane-B row of a boosted channel: boosted channels with a lower index before it
+      const unsigned ballot = __ballot_sync(kFull, boosted && half == 0);
+      if ((tid & 31) == 0) warp_cnt[tid >> 5] = __popc(ballot);
+      __syncthreads();
+      if (half == 0) {
+        int before = 0;
+        for (int w = 0; w < (tid >> 5); ++w) before += warp_cnt[w];
+        const int row = boosted ? before + int(__popc(ballot & ((1u << (tid & 31)) - 1u))) : -1;
+        row_of[c] = row;
+        if (row >= 0) rec[p.L.boost_idx + row] = uint8_t(c);
+      }
     }
     __syncthreads();
   } else if (mode & kModeKeys) {
@@ -239,20 +260,44 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         kz_out[g * kHeadDim + pm] = zb;
         if (j[e] >= 0) kbs_out[g * k + j[e]] = sb;
       }
+      // codes of the group's 32 tokens; plane A gets code >> 2 for a boosted channel (its
+      // low bits go to plane B) and the code itself otherwise; a channel that is not
+      // boosted writes its "plane B" byte to a scratch row.  Elements within 2^-14 of a
+      // rounding boundary (or of a group whose scale has no fast reciprocal) are redone
+      // with the IEEE divide afterwards.
+      uint8_t* a_base[2];
+      uint8_t* b_base[2];
+      int shift[2];
+      bool all_exact[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        a_base[e] = cA + g * kKeyGroup * kHeadDim + pc[e];
+        b_base[e] = j[e] >= 0 ? cB + g * kKeyGroup * k + pj[e] : cScratch;
+        shift[e] = j[e] >= 0 ? 2 : 0;
+        all_exact[e] = rcp[e] == 0.0f && scale[e] != 0.0f;
+      }
+      uint64_t redo = 0;
+#pragma unroll 8
       for (int t = 0; t < kKeyGroup; ++t) {
-        const int tok = g * kKeyGroup + t;
         const uint32_t w = col[t * (kHeadDim / 2)];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const uint32_t code = quant_code_fast(bits_to_float(uint16_t(w >> (16 * e)), T()), zero[e], scale[e],
-                                                rcp[e], qmax[e]);
-          if (j[e] >= 0) {
-            cA[tok * kHeadDim + pc[e]] = uint8_t(code >> 2);
-            cB[tok * k + pj[e]] = uint8_t(code & 3);
-          } else {
-            cA[tok * kHeadDim + pc[e]] = uint8_t(code);
-          }
+          bool near;
+          const uint32_t code = quant_code_fma(bits_to_float(uint16_t(w >> (16 * e)), T()), zero[e], rcp[e],
+                                               uint32_t(qmax[e]), near);
+          redo |= uint64_t(near || all_exact[e]) << (2 * t + e);
+          a_base[e][t * kHeadDim] = uint8_t(code >> shift[e]);
+          b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(code & 3u);
         }
+      }
+      while (redo) {
+        const int bit = __ffsll((long long)redo) - 1;
+        redo &= redo - 1;
+        const int t = bit >> 1, e = bit & 1;
+        const uint32_t code = uint32_t(quant_code(bits_to_float(uint16_t(col[t * (kHeadDim / 2)] >> (16 * e)), T()),
+                                                  zero[e], scale[e], qmax[e]));
+        a_base[e][t * kHeadDim] = uint8_t(code >> shift[e]);
+        b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(code & 3u);
       }
     }
   }
@@ -285,10 +330,21 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
       const float rcp = quant_rcp(scale);
       uint32_t packed[2] = {0u, 0u};
+      bool redo = rcp == 0.0f && scale != 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
-        packed[i >> 2] |= quant_code_fast(x, zero, scale, rcp, 3) << (8 * (i & 3));
+        bool near;
+        packed[i >> 2] |= quant_code_fma(x, zero, rcp, 3u, near) << (8 * (i & 3));
+        redo |= near;
+      }
+      if (redo) {  // near a rounding boundary: the IEEE divide decides
+        packed[0] = packed[1] = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
+          packed[i >> 2] |= uint32_t(quant_code(x, zero, scale, 3)) << (8 * (i & 3));
+        }
       }
       *reinterpret_cast<uint2*>(cV + t * kHeadDim + 8 * hl) = make_uint2(packed[0], packed[1]);
       if (hl == 0) {
