@@ -78,7 +78,7 @@ __device__ __forceinline__ int quant_code(float x, float zero, float scale, int 
   return int(r);
 }
 
-// Reciprocal of a group's scale for quant_code_fma, or 0 when the fast path may not be
+// Reciprocal of a group's scale for quant_bits_fma, or 0 when the fast path may not be
 // used (scale 0, or below the smallest normal float, where the approximate reciprocal
 // flushes).
 __device__ __forceinline__ float quant_rcp(float scale) {
@@ -89,19 +89,20 @@ __device__ __forceinline__ float quant_rcp(float scale) {
 }
 
 // The code quant_code gives, bit for bit, without a divide in almost every case.
-// x - zero >= 0 and the quotient that matters is at most qmax + 1/2 <= 15.5 (above it
-// the clamp decides).  fma(d, rcp, 1.5 * 2^23) rounds the exact product d * rcp to an
-// integer n held in the low mantissa bits; d * rcp is within 2^-17 of the correctly
-// rounded quotient (rcp.approx: relative error below 2^-22; the divide: half an ulp,
-// at most 2^-20), so n is the code unless d * rcp lies within 2^-14 of a rounding
-// boundary n +- 1/2.  There `near` is set and the caller redoes the element with
-// quant_code.  With rcp = 0 (scale 0) the code is 0, as quant_code gives.
-__device__ __forceinline__ uint32_t quant_code_fma(float x, float zero, float rcp, uint32_t qmax, bool& near) {
+// x - zero >= 0, and scale >= (max - min) / qmax (rounded up), so x - zero <= qmax * scale
+// and no code exceeds qmax: the clamp never acts.  fma(d, rcp, 1.5 * 2^23) rounds the
+// exact product d * rcp to an integer n held in the low byte of the result's bits
+// (0x4B400000 + n, returned).  d * rcp is within 2^-17 of the correctly rounded quotient
+// (rcp.approx: relative error below 2^-22; the divide: half an ulp, at most 2^-20), so n
+// is the code unless d * rcp lies within 2^-14 of a rounding boundary n +- 1/2.  There
+// `near` is set and the caller redoes the element with quant_code.  With rcp = 0
+// (scale 0) the code is 0, as quant_code gives.
+__device__ __forceinline__ uint32_t quant_bits_fma(float x, float zero, float rcp, bool& near) {
   const float d = __fsub_rn(x, zero);
   const float t = __fmaf_rn(d, rcp, 12582912.0f);
   const float res = __fmaf_rn(d, rcp, -__fsub_rn(t, 12582912.0f));
   near = !(fabsf(res) < 0.5f - 1.0f / 16384.0f);
-  return min(__float_as_uint(t) & 0xffu, qmax);
+  return __float_as_uint(t);
 }
 
 template <typename T>
@@ -282,12 +283,12 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         const uint32_t w = col[t * (kHeadDim / 2)];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
+          // the low byte of the bits is the code (the packing keeps two bits per byte)
           bool near;
-          const uint32_t code = quant_code_fma(bits_to_float(uint16_t(w >> (16 * e)), T()), zero[e], rcp[e],
-                                               uint32_t(qmax[e]), near);
+          const uint32_t bits = quant_bits_fma(bits_to_float(uint16_t(w >> (16 * e)), T()), zero[e], rcp[e], near);
           redo |= uint64_t(near || all_exact[e]) << (2 * t + e);
-          a_base[e][t * kHeadDim] = uint8_t(code >> shift[e]);
-          b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(code & 3u);
+          a_base[e][t * kHeadDim] = uint8_t(bits >> shift[e]);
+          b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(bits);
         }
       }
       while (redo) {
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         const uint32_t code = uint32_t(quant_code(bits_to_float(uint16_t(col[t * (kHeadDim / 2)] >> (16 * e)), T()),
                                                   zero[e], scale[e], qmax[e]));
         a_base[e][t * kHeadDim] = uint8_t(code >> shift[e]);
-        b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(code & 3u);
+        b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(code);
       }
     }
   }
@@ -335,7 +336,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       for (int i = 0; i < 8; ++i) {
         const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
         bool near;
-        packed[i >> 2] |= quant_code_fma(x, zero, rcp, 3u, near) << (8 * (i & 3));
+        packed[i >> 2] |= (quant_bits_fma(x, zero, rcp, near) & 0xffu) << (8 * (i & 3));
         redo |= near;
       }
       if (redo) {  // near a rounding boundary: the IEEE divide decides
