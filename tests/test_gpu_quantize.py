@@ -107,6 +107,30 @@ def test_constant_and_degenerate_pages():
     _check_records(_records(pool, cfg, 3), cfg, K, V, [0, 1, 2], kb.page_layout(cfg)["payload_bytes"])
 
 
+def test_rounding_ties_take_the_exact_path():
+    """Codes that land exactly on k + 1/2 (unit scales: groups spanning 0..3 and 0..15)
+    must round half to even like the IEEE divide followed by rint, for keys (2- and 4-bit)
+    and values; the kernel's multiply-by-reciprocal path hands such elements to the
+    divide."""
+    cfg = kb.Config(num_q_heads=1, num_kv_heads=1, page_tokens=32, num_boost=16, dtype=kb.F16)
+    P, D = 32, 128
+    t = np.arange(P)[:, None]
+    c = np.arange(D)[None, :]
+    hi = np.concatenate([[0.0, 15.0], np.arange(15) + 0.5, np.arange(15) + 0.25])  # 32 values, 0..15
+    lo = np.array([0.0, 3.0, 0.5, 1.5, 2.5, 1.0, 2.0, 0.25])                       # 8 values, 0..3
+    K = np.where(c < 16, hi[(t + c) % 32], lo[(t + c) % 8]).astype(np.float32)[:, None, :]
+    V = lo[(t + 3 * c) % 8].astype(np.float32)[:, None, :]
+    K, V = syn.to_bits(K, kb.F16), syn.to_bits(V, kb.F16)
+    pool = _pool(cfg, 1)
+    kb.quantize_pages(cfg, kb.Source.token_major(to_dev(K, kb.F16), cfg), kb.Source.token_major(to_dev(V, kb.F16), cfg),
+                      torch.tensor([0], dtype=torch.int32, device="cuda"), pool)
+    torch.cuda.synchronize()
+    _check_records(_records(pool, cfg, 1), cfg, K, V, [0], kb.page_layout(cfg)["payload_bytes"])
+    # the ties are really there: a unit-scale group rounds 0.5 / 1.5 / 2.5 to 0 / 2 / 2
+    codes, _, _ = oracle.quant_group(V[:8, 0, 0], 2, kb.F16)
+    assert list(codes) == [0, 3, 0, 2, 2, 1, 2, 0]
+
+
 def test_bad_destination_page_sets_error_and_writes_nothing():
     cfg = kb.Config(num_q_heads=1, num_kv_heads=1, page_tokens=32, num_boost=16)
     rng = np.random.default_rng(3)
