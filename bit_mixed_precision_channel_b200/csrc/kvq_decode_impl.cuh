@@ -257,50 +257,54 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
     const uint8_t* kB = rec + R::kb_codes;
     const uint8_t* idx = rec + R::boost_idx;
     const uint8_t* kbsc = rec + R::kb_scale + grp * (32 * KB);
-    uint32_t cb[2][2][KB][2];  // [mt][row][s][r]
+    // k-steps in pairs: the codes of two k-steps sit in one word of each token row, so at
+    // most 16 code registers are live whatever KB is
+    constexpr int SP = KB == 1 ? 1 : 2;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int sp = 0; sp < KB; sp += SP) {
+      uint32_t cb[2][2][SP][2];  // [mt][row][s - sp][r]
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const uint8_t* row = kB + (32 * grp + 16 * mt + g + 8 * rr) * KB * 4;
-        if constexpr (KB == 1) {
-          const uint32_t x = code_pass(lds32(row), qd >> 1) >> (16 * (qd & 1));
-          cb[mt][rr][0][0] = e2m1_pair_lo(x);
-          cb[mt][rr][0][1] = e2m1_pair_lo(x >> 8);
-        } else {
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-          for (int s = 0; s < KB; s += 2) {
-            const int pos = 4 * KB * qd + 4 * s;
+        for (int rr = 0; rr < 2; ++rr) {
+          const uint8_t* row = kB + (32 * grp + 16 * mt + g + 8 * rr) * KB * 4;
+          if constexpr (KB == 1) {
+            const uint32_t x = code_pass(lds32(row), qd >> 1) >> (16 * (qd & 1));
+            cb[mt][rr][0][0] = e2m1_pair_lo(x);
+            cb[mt][rr][0][1] = e2m1_pair_lo(x >> 8);
+          } else {
+            const int pos = 4 * KB * qd + 4 * sp;
             const uint32_t x = code_pass(lds32(row + (pos >> 4) * 4), (pos >> 3) & 1);
-            e2m1_pairs(x, cb[mt][rr][s][0], cb[mt][rr][s][1], cb[mt][rr][s + 1][0], cb[mt][rr][s + 1][1]);
+            e2m1_pairs(x, cb[mt][rr][0][0], cb[mt][rr][0][1], cb[mt][rr][SP - 1][0], cb[mt][rr][SP - 1][1]);
           }
         }
-      }
 #pragma unroll
-    for (int s = 0; s < KB; ++s) {
-      const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
-      // indices are < 128 in any record the library wrote; the mask keeps a corrupt
-      // record from reading outside the query rows
-      const int i00 = idx[j0] & 127, i01 = idx[j0 + 1] & 127, i10 = idx[j1] & 127, i11 = idx[j1 + 1] & 127;
-      const uint32_t s0 = to_f16x2(lds32(kbsc + j0 * 2), T()), s1 = to_f16x2(lds32(kbsc + j1 * 2), T());
-      uint32_t b[NT][2];
+      for (int ss = 0; ss < SP; ++ss) {
+        const int s = sp + ss;
+        const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
+        // indices are < 128 in any record the library wrote; the mask keeps a corrupt
+        // record from reading outside the query rows
+        const int i00 = idx[j0] & 127, i01 = idx[j0 + 1] & 127, i10 = idx[j1] & 127, i11 = idx[j1 + 1] & 127;
+        const uint32_t s0 = to_f16x2(lds32(kbsc + j0 * 2), T()), s1 = to_f16x2(lds32(kbsc + j1 * 2), T());
+        uint32_t b[NT][2];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int hB = (g >> 1) + 4 * nt;
-        uint32_t q0 = 0u, q1 = 0u;
-        if (hB < GQA) {
-          const uint16_t* qh = qs + hB * kHeadDim;
-          q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
-          q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hB = (g >> 1) + 4 * nt;
+          uint32_t q0 = 0u, q1 = 0u;
+          if (hB < GQA) {
+            const uint16_t* qh = qs + hB * kHeadDim;
+            q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
+            q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
+          }
+          b[nt][0] = fold_one(to_f16x2(q0, T()), s0, lq.negmask, __half());
+          b[nt][1] = fold_one(to_f16x2(q1, T()), s1, lq.negmask, __half());
         }
-        b[nt][0] = fold_one(to_f16x2(q0, T()), s0, lq.negmask, __half());
-        b[nt][1] = fold_one(to_f16x2(q1, T()), s1, lq.negmask, __half());
-      }
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const uint32_t a[4] = {cb[mt][0][s][0], cb[mt][1][s][0], cb[mt][0][s][1], cb[mt][1][s][1]};
+        for (int mt = 0; mt < 2; ++mt) {
+          const uint32_t a[4] = {cb[mt][0][ss][0], cb[mt][1][ss][0], cb[mt][0][ss][1], cb[mt][1][ss][1]};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+          for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+        }
       }
     }
   }
