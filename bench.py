@@ -45,8 +45,8 @@ WORKLOAD = "llama3_8b"
 # dram__bytes_write.sum from the ncu capture summarised in
 # profiles/decode_kernel_llama3_8b_layer.md), valid only for the kernel source it was taken
 # on: the bench reports it when the decode kernel source still hashes to this value.
-DECODE_TRAFFIC = {"source_sha256": "3cf4603468d8180a6f639505ad4626816094725d0a64f32aaf41a08874ddf016",
-                  "bytes": 50291456 + 8448}
+DECODE_TRAFFIC = {"source_sha256": "faad0b80dcde21ebc8028149ee6dae75d22c8f8f82b78c5f282825615040dbd1",
+                  "bytes": 50294016 + 100352}
 LAYERS = 32
 METRIC = "2-bit KV decode-attn GB/s & % of HBM peak; quantize tokens/s"
 
