@@ -67,15 +67,6 @@ __host__ __device__ __forceinline__ int key_meta_pos(int c) {
 __host__ __device__ __forceinline__ int boost_pos(int j, int KB) {
   return 4 * KB * ((j >> 1) & 3) + 4 * (j >> 4) + 2 * ((j >> 3) & 1) + (j & 1);
 }
-// Value code slot (16 * word + element) -> token (32g + 16a + 8u + 2q + f) and channel
-// (16m + 8v + w): word = ((2g + (m>>2))*32 + 4w + q)*4 + (m&3), element 8a + 2(2u+v) + f.
-__host__ __device__ __forceinline__ void value_at_slot(int slot, int& t, int& c) {
-  const int word = slot >> 4, e = slot & 15;
-  const int mm = word & 3, lane = (word >> 2) & 31, blk = word >> 7;
-  const int a = e >> 3, b = (e >> 1) & 3, f = e & 1;
-  t = 32 * (blk >> 1) + 16 * a + 8 * (b >> 1) + 2 * (lane & 3) + f;
-  c = 16 * (4 * (blk & 1) + mm) + 8 * (b & 1) + (lane >> 2);
-}
 // Value scale / zero position of token t = 32g + 8u + w: 32g + 4w + u.
 __host__ __device__ __forceinline__ int value_meta_pos(int t) {
   return (t & ~31) + 4 * (t & 7) + ((t >> 3) & 3);
@@ -132,33 +123,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Non-blocking test of the same condition.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Arrives once on `bar` (release semantics at CTA scope).
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
 // try_wait that may suspend the thread for up to `ns` nanoseconds while the phase is
 // incomplete (fewer spin iterations competing with the warps that compute).
 __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
@@ -209,10 +173,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ warp-level matrix ops
 
 // D += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulate.

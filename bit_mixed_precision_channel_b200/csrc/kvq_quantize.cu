@@ -367,8 +367,9 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   if (need_v) {
     uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
     for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) {
-      // element e = 8a + 2b + f of word i holds token t0 + 16a + 8(b >> 1) + f and
-      // channel c0 + 8(b & 1) (the inverse of value_at_slot), at bit elem_bit(e)
+      // value-code word i = ((2g + (m >> 2)) * 32 + 4w + q) * 4 + (m & 3): its element
+      // e = 8a + 2b + f holds token 32g + 2q + 16a + 8(b >> 1) + f and channel
+      // 16m + w + 8(b & 1), at bit elem_bit(e)
       const int mm = i & 3, ln = (i >> 2) & 31, blk = i >> 7;
       const uint8_t* base = cV + (32 * (blk >> 1) + 2 * (ln & 3)) * kHeadDim + 16 * (4 * (blk & 1) + mm) + (ln >> 2);
       uint32_t word = 0;
