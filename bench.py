@@ -455,13 +455,7 @@ def run_gpu(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": f"Llama-3-8B-shaped decode: batch {B} per GPU, {w.Hq} q / {w.Hkv} kv heads, "
-                               f"head_dim {D}, {w.context}-token prompts in pages of {P}, {w.k} of {D} key "
-                               f"channels boosted to 4 bit, residual window {P}, {L_layers} layers per step",
-                   "global_batch": B * world, "layers": L_layers, "seq_len": w.context,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {L_layers} layer caches, "
-                         f"{L_layers * B * w.Hkv * n_pages * payload / 1e9:.2f} GB of packed pages per GPU"},
+        "config": workload_config(w, L_layers, world, payload),
         "hbm_frac": round(value / world / peak, 4),
         "quantize": {"tokens_per_s": round(quant_tokens_per_s, 1), "ms_per_layer": round(q_ms, 4),
                      "gbs": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
@@ -488,6 +482,19 @@ def run_gpu(args):
 
 
 # ------------------------------------------------------------------ reference arm
+
+def workload_config(w, layers, world, payload):
+    """The bench's `config` object (both arms report the same one)."""
+    B, P, D = w.batch, w.P, w.D
+    n_pages = w.context // P
+    return {"workload": f"Llama-3-8B-shaped decode: batch {B} per GPU, {w.Hq} q / {w.Hkv} kv heads, "
+                        f"head_dim {D}, {w.context}-token prompts in pages of {P}, {w.k} of {D} key "
+                        f"channels boosted to 4 bit, residual window {P}, {layers} layers per step",
+            "global_batch": B * world, "layers": layers, "seq_len": w.context,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"inputs larger than L2: {layers} layer caches, "
+                  f"{layers * B * w.Hkv * n_pages * payload / 1e9:.2f} GB of packed pages per GPU"}
+
 
 def run_reference(args):
     """The oracle as the reference implementation: each step decodes a bounded sample
@@ -541,8 +548,7 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "Llama-3-8B-shaped decode layer (batch 16, 32 q / 8 kv heads, head_dim 128, "
-                                   "4096-token prompts, pages of 128, 25% boost), CPU oracle on a sample of units"},
+            "config": workload_config(w, args.layers, args.gpus, payload),
             "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
