@@ -111,6 +111,20 @@ def test_empty_and_residual_only_sequences():
     assert_attention_close(got[1:], want[1:], "residual only / pages only")
 
 
+def test_batch_above_one_pass_with_empty_runs():
+    """More sequences than threads in a CTA (the weight line is summed in passes and the
+    per-sequence lengths are cached from the located sequence on), with long runs of empty
+    sequences that the item lists skip, some of them longer than the cache."""
+    cfg = kb.Config(num_q_heads=4, num_kv_heads=1, page_tokens=32, num_boost=16)
+    lens = [0] * 420
+    for b, L in {0: 100, 1: 33, 150: 257, 151: 0, 290: 1, 291: 64, 419: 95}.items():
+        lens[b] = L
+    got, want, _ = _run(cfg, lens, seed=31)
+    live = [b for b, L in enumerate(lens) if L]
+    assert (np.delete(got, live, axis=0) == 0).all()
+    assert_attention_close(got[live], want[live], "batch 420 with empty runs")
+
+
 def test_shuffled_physical_pages():
     cfg = kb.Config(num_q_heads=4, num_kv_heads=2, page_tokens=128, num_boost=16)
     got, want, cache = _run(cfg, [128 * 20 + 50, 128 * 15], seed=13, shuffle=True)
