@@ -303,26 +303,27 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
     }
   }
 
-  // ---- a3: values, two tokens per warp (a half-warp each, 8 channels per lane)
+  // ---- a3: values, four tokens per warp (a quarter-warp each, 16 channels per lane)
   if (need_v) {
     using T2 = typename Pair<T>::type;
-    const int warp = tid >> 5, lane = tid & 31, hl = lane & 15;
+    const int warp = tid >> 5, lane = tid & 31, ql = lane & 7;
     uint16_t* vs_out = reinterpret_cast<uint16_t*>(rec + p.L.v_scale);
     uint16_t* vz_out = reinterpret_cast<uint16_t*>(rec + p.L.v_zero);
-    for (int t0 = 2 * warp; t0 < P; t0 += 2 * (kQThreads / 32)) {
-      const int t = t0 + (lane >> 4);
-      const uint4 raw = lds128(Vs + t * kHeadDim + 8 * hl);
-      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+    for (int t0 = 4 * warp; t0 < P; t0 += 4 * (kQThreads / 32)) {
+      const int t = t0 + (lane >> 3);
+      const uint16_t* row = Vs + t * kHeadDim + 16 * ql;
+      const uint4 r0 = lds128(row), r1 = lds128(row + 8);
+      const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
       T2 lo = u32_as_pair(wv[0], T()), hi = lo;
 #pragma unroll
-      for (int i = 1; i < 4; ++i) {
+      for (int i = 1; i < 8; ++i) {
         lo = __hmin2(lo, u32_as_pair(wv[i], T()));
         hi = __hmax2(hi, u32_as_pair(wv[i], T()));
       }
       float mn = fminf(bits_to_float(uint16_t(pair_as_u32(lo)), T()), bits_to_float(uint16_t(pair_as_u32(lo) >> 16), T()));
       float mx = fmaxf(bits_to_float(uint16_t(pair_as_u32(hi)), T()), bits_to_float(uint16_t(pair_as_u32(hi) >> 16), T()));
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) {
+      for (int off = 4; off > 0; off >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(kFull, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
       }
@@ -330,25 +331,26 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       float zero;
       const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
       const float rcp = quant_rcp(scale);
-      uint32_t packed[2] = {0u, 0u};
+      uint32_t packed[4] = {0u, 0u, 0u, 0u};
       bool redo = rcp == 0.0f && scale != 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
         bool near;
         packed[i >> 2] |= (quant_bits_fma(x, zero, rcp, near) & 0xffu) << (8 * (i & 3));
         redo |= near;
       }
       if (redo) {  // near a rounding boundary: the IEEE divide decides
-        packed[0] = packed[1] = 0u;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) packed[i] = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
           const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
           packed[i >> 2] |= uint32_t(quant_code(x, zero, scale, 3)) << (8 * (i & 3));
         }
       }
-      *reinterpret_cast<uint2*>(cV + t * kHeadDim + 8 * hl) = make_uint2(packed[0], packed[1]);
-      if (hl == 0) {
+      *reinterpret_cast<uint4*>(cV + t * kHeadDim + 16 * ql) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      if (ql == 0) {
         vs_out[value_meta_pos(t)] = sb;
         vz_out[value_meta_pos(t)] = zb;
       }
