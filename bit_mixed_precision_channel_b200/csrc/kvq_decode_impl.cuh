@@ -5,7 +5,8 @@
 // Work decomposition (balanced streaming).  Every (sequence b, kv head h) is a unit;
 // its items are its pages, grouped into 128-token stages (1, 2 or 4 pages), followed by
 // its residual tokens in pieces of 16.  Item weights count 32-token groups (a full
-// stage weighs 4, a residual piece 1).  Units are laid end to end in (b, h) order and
+// stage weighs 4, a residual piece kPieceWeight, the merge at a unit's end kMergeWeight,
+// all as measured).  Units are laid end to end in (b, h) order and
 // the resulting weight line is cut into one equal range per CTA, one CTA per resident
 // slot of the GPU (SMs x CTAs per SM); a CTA processes the items that start inside its
 // range, so every SM receives the same amount of work whatever the sequence lengths.
