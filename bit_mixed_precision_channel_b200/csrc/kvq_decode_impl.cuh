@@ -14,12 +14,14 @@
 // partial (max, sum, unnormalised output); the last contributor of a unit merges the
 // partials (log-sum-exp), so there is no second launch.
 //
-// Data movement.  Warp 0 fills a 3-stage shared-memory ring with one cp.async.bulk per
-// page record (L2 evict-first hint), one bulk copy per residual row, and the unit's
-// query heads with the unit's first stage; completion is tracked with "full"
-// mbarriers, release with "empty" mbarriers, and every wait is bounded.  Each warp owns
-// one 32-token group of a page stage and runs its own online softmax; warps meet only
-// at the end of a unit.
+// Data movement.  A 3-stage shared-memory ring holds page records (one cp.async.bulk per
+// record, L2 evict-first hint) or residual pieces (16-byte cp.async into padded rows,
+// zero-filled past the last token); a unit's query heads travel with its first item.
+// Completion is tracked with "full" mbarriers and every wait is bounded.  Warp 0 issues
+// the first three items of a segment; afterwards the warp that releases a stage last
+// (an acquire-release counter per stage) refills it with the item three places ahead.
+// Each warp owns one 32-token group of a page stage and runs its own online softmax;
+// warps meet only at the end of a unit.
 //
 // Arithmetic.  The 2-bit codes never become scaled values.  The scales are folded into
 // the other operand of each product, and the codes go to the tensor cores as they are
@@ -845,6 +847,8 @@ __device__ __forceinline__ void merge_heads(const float* pu, size_t slot, int nc
 
 // One warp: counts this contributor in for unit u and, if it is the last of the
 // contributors i0..i1, merges their partial states (log-sum-exp) into the output.
+// (Written out rather than through merge_heads: inlined into the item loop, the helper
+// changes the loop's register allocation enough to spill at 128 registers.)
 template <int GQA>
 __device__ __forceinline__ void merge_partials(const DecodeParams& p, int u, int i0, int i1, float* outu, int lane) {
   uint32_t arrived = 0;
