@@ -176,6 +176,31 @@ def _cuda(*tensors):
             raise ValueError("kvq calls take CUDA tensors (device memory)")
 
 
+def _need(name: str, t, dtype=None, numel: int | None = None, dim: int | None = None):
+    """The library takes plain pointers: a tensor must be dense, of the element type the
+    call reads, and at least as large as the call's extent."""
+    if t is None:
+        return
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, the call reads {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions, not {t.dim()}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, the call reads {numel}")
+
+
+def _need_source(name: str, src, cfg: Config, n_pages: int):
+    if src is None:
+        return
+    extent = 0
+    if n_pages > 0:
+        extent = ((n_pages - 1) * src.page_stride + (cfg.page_tokens - 1) * src.token_stride +
+                  (cfg.num_kv_heads - 1) * src.head_stride + cfg.head_dim)
+    _need(name, src.tensor, torch_dtype(cfg.dtype), extent)
+
+
 def status_string(status: int) -> str:
     return load().kvq_status_string(status).decode()
 
@@ -195,6 +220,11 @@ def page_bytes(cfg: Config) -> int:
 
 
 def _quant(fn, cfg, src_k, src_v, dst_pages, pool, err, stream):
+    _need("dst_pages", dst_pages, torch.int32)
+    _need("pool", pool, torch.uint8)
+    _need("err", err, torch.int32, 1)
+    _need_source("k source", src_k, cfg, dst_pages.numel())
+    _need_source("v source", src_v, cfg, dst_pages.numel())
     _cuda(dst_pages, pool, err)
     pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
     L = load()
@@ -230,8 +260,15 @@ def quantize_pages(cfg: Config, k: Source, v: Source, dst_pages: torch.Tensor, p
 
 
 def append_token(cfg: Config, k_new, v_new, res_k, res_v, res_len, err=None, stream=None):
-    _cuda(k_new, v_new, res_k, res_v, res_len, err)
     batch = res_len.numel()
+    dt, H, P, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.page_tokens, cfg.head_dim
+    _need("res_len", res_len, torch.int32)
+    _need("k_new", k_new, dt, batch * H * D)
+    _need("v_new", v_new, dt, batch * H * D)
+    _need("res_k", res_k, dt, batch * H * P * D)
+    _need("res_v", res_v, dt, batch * H * P * D)
+    _need("err", err, torch.int32, 1)
+    _cuda(k_new, v_new, res_k, res_v, res_len, err)
     _check("kvq_append_token", load().kvq_append_token(
         ctypes.byref(cfg.c()), batch, k_new.data_ptr(), v_new.data_ptr(), res_k.data_ptr(),
         res_v.data_ptr(), res_len.data_ptr(), _ptr(err), _stream(stream)))
@@ -239,8 +276,16 @@ def append_token(cfg: Config, k_new, v_new, res_k, res_v, res_len, err=None, str
 
 def flush_residual(cfg: Config, res_k, res_v, res_len, new_page, page_table, num_pages, pool,
                    err=None, stream=None):
-    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err)
+    _need("page_table", page_table, torch.int32, dim=2)
     batch, max_pages = page_table.shape
+    dt, H, P, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.page_tokens, cfg.head_dim
+    _need("res_k", res_k, dt, batch * H * P * D)
+    _need("res_v", res_v, dt, batch * H * P * D)
+    for name, t in (("res_len", res_len), ("new_page", new_page), ("num_pages", num_pages)):
+        _need(name, t, torch.int32, batch)
+    _need("pool", pool, torch.uint8)
+    _need("err", err, torch.int32, 1)
+    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err)
     pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
     _check("kvq_flush_residual", load().kvq_flush_residual(
         ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
@@ -252,8 +297,24 @@ def decode_workspace_bytes(cfg: Config, batch: int, max_pages: int) -> int:
     return int(load().kvq_decode_workspace_bytes(ctypes.byref(cfg.c()), batch, max_pages))
 
 
+def _need_decode(cfg: Config, pool, q, page_table, num_pages, res_k, res_v, res_len, out, err):
+    _need("page_table", page_table, torch.int32, dim=2)
+    batch = page_table.shape[0]
+    dt, H, P, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.page_tokens, cfg.head_dim
+    _need("pool", pool, torch.uint8)
+    _need("q", q, dt, batch * cfg.num_q_heads * D)
+    _need("out", out, torch.float32, batch * cfg.num_q_heads * D)
+    _need("num_pages", num_pages, torch.int32, batch)
+    _need("res_len", res_len, torch.int32, batch)
+    _need("res_k", res_k, dt, batch * H * P * D)
+    _need("res_v", res_v, dt, batch * H * P * D)
+    _need("err", err, torch.int32, 1)
+
+
 def decode_attention(cfg: Config, pool, q, page_table, num_pages, res_k, res_v, res_len, out,
                      workspace, sm_scale: float | None = None, err=None, stream=None):
+    _need_decode(cfg, pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
+    _need("workspace", workspace, torch.uint8)
     _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, workspace, err)
     batch, max_pages = page_table.shape
     if sm_scale is None:
@@ -272,6 +333,7 @@ def decode_attention_static(cfg: Config, pool, q, page_table, num_pages, res_k, 
     scratch is the library's own static 16 MiB device buffer (no workspace argument).
     Calls on one device share that buffer, so they must not overlap on the GPU; the
     first call on a device must not be made during stream capture."""
+    _need_decode(cfg, pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
     _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
     batch, max_pages = page_table.shape
     if sm_scale is None:
