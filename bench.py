@@ -101,7 +101,7 @@ def whole_job_gbs(world, bytes_per_rank, ms):
 def decode_bytes(w, payload, n_pages, res_len):
     """Algorithmic bytes of one decode-attention launch (one layer): packed pages
     (codes + scales + zeros + boost indices), the fp16 residual K and V, the query,
-    the fp32 output and the page table entries."""
+    the fp32 output, the page table entries and the two lengths of every sequence."""
     B, Hkv, Hq, D = w.batch, w.Hkv, w.Hq, w.D
     return (B * Hkv * n_pages * payload + B * Hkv * res_len * 2 * D * 2 + B * Hq * D * 2 + B * Hq * D * 4
             + 4 * B * n_pages + 8 * B)
