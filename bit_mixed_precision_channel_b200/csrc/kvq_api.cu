@@ -27,8 +27,8 @@ static int sm_count() {
   return n;
 }
 
-// Decode workspace: one partial slot per (worker, unit) pair that can occur — worker i
-// and unit u write slot i + u — then one arrival counter per unit.
+// Decode workspace: one partial slot per (CTA, unit) pair that can occur — CTA i and
+// unit u write slot i + u — then one arrival counter per unit.
 struct Plan {
   int ctas;
   size_t part_bytes, cnt_bytes;
@@ -39,7 +39,7 @@ static Plan decode_plan(const kvq_config* cfg, int batch) {
   const size_t units = size_t(batch) * cfg->num_kv_heads;
   Plan pl;
   pl.ctas = sm_count() * decode_ctas_per_sm(gqa, cfg->dtype, cfg->num_boost / 16, cfg->page_tokens);
-  pl.part_bytes = (size_t(pl.ctas) * kDecodeWorkersPerCta + units) * gqa * (kHeadDim + 4) * sizeof(float);
+  pl.part_bytes = (size_t(pl.ctas) + units) * gqa * (kHeadDim + 4) * sizeof(float);
   pl.part_bytes = (pl.part_bytes + 255) / 256 * 256;
   pl.cnt_bytes = units * sizeof(uint32_t);
   return pl;
@@ -236,13 +236,11 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(pool) || !aligned16(q) || !aligned16(res_k) || !aligned16(res_v) || !aligned16(workspace))
     return KVQ_ERR_INVALID_ARG;
-  // the kernel's work line (32-token groups, weighted 32-token residual pieces and a
+  // the kernel's work line (32-token groups, weighted 16-token residual pieces and a
   // merge weight per (sequence, kv head)) is indexed with 32-bit integers
-  const long long line =
-      (long long)batch * cfg->num_kv_heads *
-      ((long long)max_pages * (cfg->page_tokens / 32) +
-       (long long)kDecodePieceWeight * ((cfg->page_tokens + kDecodePieceTokens - 1) / kDecodePieceTokens) +
-       kDecodeMergeWeight);
+  const long long line = (long long)batch * cfg->num_kv_heads *
+                         ((long long)max_pages * (cfg->page_tokens / 32) +
+                          (long long)kDecodePieceWeight * ((cfg->page_tokens + 15) / 16) + kDecodeMergeWeight);
   if (line >= (1ll << 31)) return KVQ_ERR_INVALID_ARG;
   const Plan pl = decode_plan(cfg, batch);
   if (workspace_bytes < pl.part_bytes + pl.cnt_bytes) return KVQ_ERR_CAPACITY;

@@ -1,69 +1,53 @@
-// kvq_decode_impl.cuh — decode attention over the paged 2-bit cache on the fifth-
-// generation tensor cores (tcgen05) of sm_100a.  Kernel templates;
-// kvq_decode_<dtype>_g<GQA>.cu instantiate them, kvq_decode.cu holds the host side.
+// kvq_decode_impl.cuh — decode attention over the paged 2-bit cache, sm_100a.
+// Kernel templates; kvq_decode_<dtype>_g<GQA>.cu instantiate them, kvq_decode.cu
+// holds the host side.
 //
-// Workers.  A CTA holds two warpgroups of 128 threads, and each warpgroup is an
-// independent worker: it owns a ring of shared-memory stages, a region of tensor
-// memory, its shared-memory operand buffers and its own range of the work line.  The
-// two warpgroups of a CTA never wait for one another between the prologue and the
-// end of the kernel.
+// Work decomposition (balanced streaming).  Every (sequence b, kv head h) is a unit;
+// its items are its pages, grouped into 128-token stages (1, 2 or 4 pages), followed by
+// its residual tokens in pieces of 16.  Item weights count 32-token groups (a full
+// stage weighs 4, a residual piece kPieceWeight, the merge at a unit's end kMergeWeight,
+// all as measured).  Units are laid end to end in (b, h) order and
+// the resulting weight line is cut into one equal range per CTA, one CTA per resident
+// slot of the GPU (SMs x CTAs per SM); a CTA processes the items that start inside its
+// range, so every SM receives the same amount of work whatever the sequence lengths.
+// A CTA that finishes a unit writes either the output (when it saw the whole unit) or a
+// partial (max, sum, unnormalised output); the last contributor of a unit merges the
+// partials (log-sum-exp), so there is no second launch.
 //
-// Work line.  Every (sequence b, kv head h) is a unit; its items are its pages in
-// 128-token stages (1, 2 or 4 records), then its residual tokens in pieces of 32.
-// Item weights: a stage weighs 4, a residual piece kPieceWeight, and a unit's end adds
-// kMergeWeight.  The units are laid end to end and the line is cut into one equal
-// range per worker; a worker takes the items that start in its range.  A worker that
-// ends a unit it did not see whole writes a partial softmax state; the last
-// contributor of a unit merges the partials (log-sum-exp) in the same launch.
+// Data movement.  A 3-stage shared-memory ring holds page records (one cp.async.bulk per
+// record, L2 evict-first hint) or residual pieces (16-byte cp.async into padded rows,
+// zero-filled past the last token); a unit's query heads travel with its first item.
+// Completion is tracked with "full" mbarriers and every wait is bounded.  Warp 0 issues
+// the first three items of a segment; afterwards the warp that releases a stage last
+// (an acquire-release counter per stage) refills it with the item three places ahead.
+// Each warp owns one 32-token group of a page stage and runs its own online softmax;
+// warps meet only at the end of a unit.
 //
-// Arithmetic of a 128-token page stage (thread t of the warpgroup is token t for keys
-// and channel t for values; tensor-memory lane t belongs to the same thread):
-//   keys   A_K[t][c]    = codes of plane A (c < 128) and plane B (c >= 128) as
-//                         fp16 0.5 * code (the FP4 conversion), written to tensor memory
-//          B_s[c][n]    = q'_h[c] * sA[c][g] split into fp16 (hi, lo), n = (g, part, h)
-//          B_b[j][n]    = q'_h[idx(j)] * sB[j][g], the same for plane B
-//          B_z[c][n]    = q'_h[c] * zA[c][g]
-//          S[t][n]      = A_K x (B_s ; B_b) + 0.5 x B_z      (all fp32 in tensor memory)
-//   so that 2 * (S[t][g(t), hi, h] + S[t][g(t), lo, h]) = q'_h . K^_t exactly up to fp32
-//   rounding.  q' = q * 2^-e_h with e_h chosen per (unit, head) so that |q'| < 1: the
-//   folded operands then never exceed the key scales (fp16 caches cannot overflow).
-//   values A_V[c][t]    = 0.5 * value code of token t, channel c (tensor memory)
-//          B_p[t][n]    = p_h[t] * sV[t] * 2^-F split into fp16 (hi, lo), n = (part, h)
-//          O[c][n]     += A_V x B_p                          (fp32, across the unit)
-//   and the value zero points and the softmax sum stay per thread:
-//          zv_h += p_h[t] * zV[t],   l_h += p_h[t].
-// Online softmax (log2 units) with a running maximum M_h per worker that moves only
-// when a logit exceeds it by more than kLazy; then every thread rescales its own
-// partial sums and its own lane of O.  F (>= 0) keeps p * sV * 2^-F below 2^15.
-// Residual pieces use the raw key and value rows (cache dtype) as A with B = q'
-// (exact) and B = 0.5 * p * 2^-F; their products run in the cache dtype.
-//
-// Synchronisation inside a worker: two warpgroup barriers per item (operands ready
-// for the QK product; probabilities ready for the PV product, which also ORs the
-// "maximum must move" votes), tcgen05 commits to two mbarriers, and one bulk-copy
-// mbarrier per stage.  Every mbarrier wait is bounded; a timeout sets
-// KVQ_DEV_ERR_TIMEOUT and the worker stops after waiting (bounded) for its copies and
-// products in flight.
+// Arithmetic.  The 2-bit codes never become scaled values.  The scales are folded into
+// the other operand of each product, and the codes go to the tensor cores as they are
+// (Kitty abstract: page dequantization kernels; MiniKV proposed method: dequantization
+// fused into the attention matmul):
+//   q.k_t = sum_c codeA[t,c] (q_c sA_c) + sum_j codeB[t,j] (q_idx(j) sB_j) + sum_c q_c zA_c
+//   sum_t p_t v_t[c] = sum_t codeV[t,c] (p_t sV_t) + sum_t p_t zV_t
+// Codes reach the tensor cores exactly as 0.5 * code through the FP4 (e2m1) conversion;
+// the folded operands are carried as fp16 high and low parts (hi = fp16(x),
+// lo = fp16(x - hi)).  The eight columns of an m16n8k16 product hold four query heads,
+// each as an adjacent (hi, lo) column pair, so a lane's two accumulator columns are the
+// two parts of one head: the logits need no shuffle, and the (hi, lo) pair of
+// p * sV is one register that movmatrix turns into the B fragment of the PV product.
 #pragma once
 #include <algorithm>
 
 #include "kvq_internal.cuh"
-#include "kvq_tc.cuh"
 
 namespace kvq {
-namespace dec {
 
-constexpr int kWG = 2;                   // workers (warpgroups) per CTA
-constexpr int kThreads = 128 * kWG;
-constexpr int kStageBytes = 16384;       // one 128-token page stage or one residual piece
-constexpr int kPieceTokens = 32;         // residual tokens per piece
-constexpr int kResV = 8192;              // value rows of a residual piece in its stage
-constexpr int kSegItems = 64;            // items listed per segment
-constexpr int kSeqCache = 512;           // sequences whose lengths the prologue keeps
-constexpr float kLazy = 8.0f;            // log2 margin before the running maximum moves
+constexpr int kStages = 3;
+constexpr int kDecodeThreads = 128;
+constexpr int kResRowBytes = 272;  // residual row in shared memory: 256 bytes + 16 pad
+constexpr int kPieceTokens = 16;   // residual tokens per item
 constexpr int kPieceWeight = kDecodePieceWeight;
 constexpr int kMergeWeight = kDecodeMergeWeight;
-constexpr int kSmemPerWorker = 104 * 1024;
 
 // Compile-time offsets of one record (the same values as make_layout).
 template <int P, int KB>
@@ -82,173 +66,401 @@ struct Rec {
   static constexpr uint32_t record = (payload + 127u) / 128u * 128u;
 };
 
-constexpr int round16(int x) { return (x + 15) / 16 * 16; }
-constexpr int cmax(int a, int b) { return a > b ? a : b; }
-constexpr int cmin(int a, int b) { return a < b ? a : b; }
-
-// Shapes, tensor-memory columns and shared-memory offsets of one instantiation.
-template <int GQA, int KB, int P>
-struct Cfg {
-  static constexpr int PPS = 128 / P;                  // pages per stage
-  static constexpr int NG = P / 32;                    // key groups per page
-  static constexpr int NQK = cmax(16, 8 * GQA);        // QK columns: 4 groups x (hi, lo) x heads
-  static constexpr int LBO_QK = NQK / 8 * 128;
-  static constexpr int LBO_PV = 256;                   // PV / residual-QK B operands: N = 16
-  static constexpr int AQ = 64 + 8 * KB;               // key A columns
-  static constexpr int AV = 64;                        // value A columns
-  static constexpr int COLS_SPLIT = round16(AQ + AV + NQK + 16);
-  static constexpr bool SPLIT = 16 + kWG * COLS_SPLIT <= 512;  // separate key and value A regions
-  static constexpr int COLS = SPLIT ? COLS_SPLIT : round16(cmax(AQ, AV) + NQK + 16);
-  static constexpr int C_AQ = 0, C_AV = SPLIT ? AQ : 0, C_S = SPLIT ? AQ + AV : cmax(AQ, AV), C_O = C_S + NQK;
-  static_assert(16 + kWG * COLS <= 512, "tensor memory");
-  // shared memory of one worker
-  static constexpr int BQK = 128 * NQK * 2;
-  static constexpr int BQB = 16 * KB * NQK * 2;
-  static constexpr int FIXED = 2 * BQK + BQB + 4096 + 4096 + 128 * GQA * 2;
-  static constexpr int NS = cmin(4, (kSmemPerWorker - FIXED) / (kStageBytes + GQA * 256));
-  static_assert(NS >= 2, "shared memory");
-  static constexpr int O_RING = 0;
-  static constexpr int O_Q = O_RING + NS * kStageBytes;
-  static constexpr int O_BQK = O_Q + NS * GQA * 256;
-  static constexpr int O_BZ = O_BQK + BQK;
-  static constexpr int O_BQB = O_BZ + BQK;
-  static constexpr int O_BPV = O_BQB + BQB;
-  static constexpr int O_BQR = O_BPV + 4096;
-  static constexpr int O_QH = O_BQR + 4096;
-  static constexpr int BYTES = (O_QH + 128 * GQA * 2 + 1023) / 1024 * 1024;
-  static_assert(BYTES <= kSmemPerWorker, "shared memory");
+// Dynamic shared memory of one CTA: kStages stages (page records, or the K and V rows
+// of a residual piece), then the merge buffer [4 warps][GQA][128] fp32.
+template <int GQA, int P, int KB>
+struct Smem {
+  static constexpr uint32_t body = std::max<uint32_t>((128 / P) * Rec<P, KB>::record, 2 * kPieceTokens * kResRowBytes);
+  static constexpr uint32_t stage = (body + 127u) / 128u * 128u;
+  static constexpr uint32_t merge = kStages * stage;
+  static constexpr uint32_t bytes = merge + 4u * GQA * 128u * 4u;
 };
 
-// ---------------------------------------------------------------- small helpers
+// ---------------------------------------------------------------- operand builders
 
-__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory"); }
-// Barrier of the warpgroup that also returns the OR of `pred` over its threads.
-__device__ __forceinline__ bool wg_sync_or(int wg, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"(uint32_t(pred)), "r"(wg + 1)
-      : "memory");
-  return r != 0;
-}
-
-__device__ __forceinline__ uint32_t u16_at(const uint8_t* p) { return *reinterpret_cast<const uint16_t*>(p); }
-
-// A 16-bit value of the cache dtype as fp32 (exact).
-__device__ __forceinline__ float t_to_f(uint32_t b, __half) { return __half2float(__ushort_as_half(uint16_t(b))); }
-__device__ __forceinline__ float t_to_f(uint32_t b, __nv_bfloat16) { return __uint_as_float(b << 16); }
-// A 16-bit value of the cache dtype as an fp16 pair (x, x): exact for fp16; for bf16
-// exact inside fp16's normal range.
-__device__ __forceinline__ uint32_t t_bcast_h2(uint32_t b, __half) { return (b & 0xffffu) | (b << 16); }
-__device__ __forceinline__ uint32_t t_bcast_h2(uint32_t b, __nv_bfloat16) {
-  const float x = __uint_as_float(b << 16);
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(x));
-  return d;
-}
-// Two floats as a pair of the given 16-bit type (low half = a).
-__device__ __forceinline__ uint32_t pack2(float a, float b, __half) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(b), "f"(a));
-  return d;
-}
-__device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16) {
-  uint32_t d;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(b), "f"(a));
-  return d;
-}
-__device__ __forceinline__ float2 unpack2(uint32_t u, __half) { return __half22float2(u32_as_h2(u)); }
-__device__ __forceinline__ float2 unpack2(uint32_t u, __nv_bfloat16) {
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
-// (hi, lo) pairs of (a, b) in the 16-bit type U: hi = U(x), lo = U(x - hi).
-template <typename U>
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  hi = pack2(a, b, U());
-  const float2 h = unpack2(hi, U());
-  lo = pack2(a - h.x, b - h.y, U());
-}
-// Products q * s of an fp16 query pair and a broadcast fp16 scale, as (hi, lo) fp16
-// pairs: hi = fp16(q s), lo = q s - hi (exact: the rest of a product of two fp16 values).
-__device__ __forceinline__ void fold2(uint32_t q2, uint32_t s2, uint32_t& hi, uint32_t& lo) {
+// One part of the folded query operand, chosen per lane without a branch:
+// hfma2(q, s, -fp16(q*s) * m) is fp16(q*s) for m = 0 (hi lanes) and the exact rest
+// q*s - fp16(q*s) for m = 1 (lo lanes); the product of two fp16 values is exact in fp32.
+__device__ __forceinline__ uint32_t fold_one(uint32_t q2, uint32_t s2, uint32_t negmask, __half) {
   const __half2 q = u32_as_h2(q2), s = u32_as_h2(s2);
   const __half2 h = __hmul2(q, s);
-  hi = h2_as_u32(h);
-  lo = h2_as_u32(__hfma2(q, s, __hneg2(h)));
+  return h2_as_u32(__hfma2(q, s, __hmul2(h, u32_as_h2(negmask))));
 }
-__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // e in [-126, 127]
+// Two cache-dtype values as an fp16 pair.  bf16 values are exact in fp16 inside its
+// normal range (8 significant bits fit in 11), which is where the kernel carries bf16
+// queries, scales and zero points: the folded products then use the fp16 path above.
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t x, __half) { return x; }
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t x, __nv_bfloat16) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(__uint_as_float(x & 0xffff0000u)), "f"(__uint_as_float(x << 16)));
+  return d;
+}
 
-// Folded operand row of one key group: GQA heads x (hi, lo) as GQA 32-bit words.
-// Layout n = part * GQA + h (GQA >= 2: hi pairs then lo pairs); GQA 1: (hi, lo).
-template <int GQA>
-struct GroupRow {
-  uint32_t w[GQA];
+// (hi, lo) of x as one register: low half = hi, high half = lo.
+__device__ __forceinline__ uint32_t hilo(float x, __half) {
+  const float hf = __half2float(__float2half_rn(x));
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x - hf), "f"(hf));
+  return d;
+}
+__device__ __forceinline__ uint32_t hilo(float x, __nv_bfloat16) {
+  const float hf = __bfloat162float(__float2bfloat16_rn(x));
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x - hf), "f"(hf));
+  return d;
+}
+
+// Two 16-bit values of a register as floats.
+__device__ __forceinline__ float2 t2_to_float2(uint32_t u, __half) { return __half22float2(u32_as_h2(u)); }
+__device__ __forceinline__ float2 t2_to_float2(uint32_t u, __nv_bfloat16) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// ---------------------------------------------------------------- per-warp state
+
+template <int NT>
+struct WarpState {
+  float o[8][NT][4];  // PV accumulator: rows = channels 16*mc + g (+8), cols (hi, lo) of head qd + 4*nt
+  float m[NT], l[NT], zv[NT];
 };
-template <int GQA>
-__device__ __forceinline__ GroupRow<GQA> fold_group(const uint32_t (&q2)[(GQA + 1) / 2], uint32_t s2) {
-  GroupRow<GQA> r;
-  if constexpr (GQA == 1) {
-    uint32_t hi, lo;
-    fold2(q2[0], s2, hi, lo);
-    r.w[0] = (hi & 0xffffu) | (lo << 16);
-  } else {
-#pragma unroll
-    for (int i = 0; i < GQA / 2; ++i) fold2(q2[i], s2, r.w[i], r.w[GQA / 2 + i]);
+
+// Query pairs of this lane in fp16: head (g/2) + 4 nt, channels 16 s + 2 qd (+1) for
+// j = 0 and 8 more for j = 1.  They are the B column g of the code products (with the
+// part g % 2 chosen by negmask) and, stored as register quads, the A operand of the
+// zero-point product, whose rows are heads:
+//   NT = 2: quad s = {q(0,s,0), q(1,s,0), q(0,s,1), q(1,s,1)}: rows g / g+8 = heads
+//           g/2 and g/2 + 4 at k-step s;
+//   NT = 1: quad i = {q(0,i,0), q(0,i+4,0), q(0,i,1), q(0,i+4,1)}: rows g / g+8 = head
+//           g/2 at k-steps i and i + 4.
+template <int NT>
+struct LaneQ {
+  uint32_t qa[NT == 2 ? 8 : 4][4];
+  uint32_t negmask;  // fp16x2 -1 for lo-part lanes (odd g), 0 otherwise
+  __device__ __forceinline__ uint32_t& qv(int nt, int s, int j) {
+    return NT == 2 ? qa[s][2 * j + nt] : qa[s & 3][2 * j + (s >> 2)];
   }
-  return r;
-}
-// Stores the four group rows of one K-row (channel or boosted row) of a QK B operand:
-// the GQA words of group g start at column 2 * GQA * g.
-template <int GQA, int LBO>
-__device__ __forceinline__ void store_qk_row(uint8_t* B, int row, const GroupRow<GQA> (&g)[4]) {
-  uint32_t v[4 * GQA];
+  __device__ __forceinline__ uint32_t qv(int nt, int s, int j) const {
+    return NT == 2 ? qa[s][2 * j + nt] : qa[s & 3][2 * j + (s >> 2)];
+  }
+};
+
+template <int NT>
+__device__ __forceinline__ void reset_state(WarpState<NT>& st) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int mc = 0; mc < 8; ++mc)
 #pragma unroll
-    for (int j = 0; j < GQA; ++j) v[GQA * i + j] = g[i].w[j];
-  uint8_t* base = B + (row >> 3) * LBO + (row & 7) * 16;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-  for (int c = 0; c < GQA; ++c)
-    *reinterpret_cast<uint4*>(base + c * 128) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-}
-// Stores one K-row of an N = 16 B operand (probabilities or the residual query):
-// `words` 32-bit words (2 * words values) from column 0 on; the other columns are zero.
-template <int NW>
-__device__ __forceinline__ void store_n16_row(uint8_t* B, int row, const uint32_t (&v)[NW]) {
-  uint8_t* base = B + (row >> 3) * 256 + (row & 7) * 16;
-  if constexpr (NW <= 4) {
-    uint32_t x[4] = {0u, 0u, 0u, 0u};
+      for (int i = 0; i < 4; ++i) st.o[mc][nt][i] = 0.0f;
 #pragma unroll
-    for (int i = 0; i < NW; ++i) x[i] = v[i];
-    *reinterpret_cast<uint4*>(base) = make_uint4(x[0], x[1], x[2], x[3]);
-  } else {
-    *reinterpret_cast<uint4*>(base) = make_uint4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<uint4*>(base + 128) = make_uint4(v[4], v[5], v[6], v[7]);
+  for (int nt = 0; nt < NT; ++nt) {
+    st.m[nt] = -INFINITY;
+    st.l[nt] = 0.0f;
+    st.zv[nt] = 0.0f;
   }
 }
 
-// Converts one code word (16 codes) to 8 tensor-memory columns of fp16 pairs, in
-// natural element order: column 4a + b holds elements 8a + 2b (low) and 8a + 2b + 1.
-__device__ __forceinline__ void word_to_cols(uint32_t w, uint32_t* c) {
-  e2m1_pairs(code_pass(w, 0), c[0], c[1], c[2], c[3]);
-  e2m1_pairs(code_pass(w, 1), c[4], c[5], c[6], c[7]);
+// Online-softmax update from MT x 2 logits per head part of this lane (log2 units).  The
+// running maximum moves only when a logit exceeds it by more than 8, so probabilities
+// stay below 2^8 and most groups skip the rescale of the accumulators.
+template <int NT, int MT>
+__device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)[MT][NT][2]) {
+  // the lanes' own maxima decide whether any head can move; only then are they reduced
+  float mx[NT];
+  bool big = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    mx[nt] = L[0][nt][0];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) mx[nt] = fmaxf(mx[nt], fmaxf(L[mt][nt][0], L[mt][nt][1]));
+    big |= mx[nt] > st.m[nt] + 8.0f;
+  }
+  if (!__any_sync(kFull, big)) return;
+  float alpha[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    mx[nt] = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 4));
+    mx[nt] = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 8));
+    mx[nt] = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 16));
+    alpha[nt] = 1.0f;
+    if (mx[nt] > st.m[nt] + 8.0f) {
+      alpha[nt] = ex2(st.m[nt] - mx[nt]);  // 0 on the first group (m = -inf)
+      st.m[nt] = mx[nt];
+      st.l[nt] *= alpha[nt];
+      st.zv[nt] *= alpha[nt];
+    }
+  }
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= alpha[nt];
 }
 
-// ---------------------------------------------------------------- work line
+// ---------------------------------------------------------------- one quantized group
 
+// Tokens [32 grp, 32 grp + 32) of the page record `rec` (shared memory), for the lane
+// (g, qd): QK^T over planes A and B and the zero points, online softmax, then PV.
+template <typename T, int GQA, int KB, int P>
+__device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const LaneQ<(GQA > 4 ? 2 : 1)>& lq,
+                                           const uint16_t* qs, WarpState<(GQA > 4 ? 2 : 1)>& st, int lane,
+                                           float c_log2) {
+  constexpr int NT = GQA > 4 ? 2 : 1;
+  using R = Rec<P, KB>;
+  const int g = lane >> 2, qd = lane & 3;
+  float acc[2][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
+
+  // -- plane A: rows 32 grp + 16 mt + 8 r + g, words 2qd and 2qd+1 (channels of k-steps
+  //    0..3 and 4..7); scales of k-steps 2i, 2i+1 are 16 bytes at 64 i + 16 qd --
+  const uint8_t* kA = rec + R::k_codes + (32 * grp + g) * 32 + 8 * qd;
+  uint2 w[2][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) w[mt][r] = lds64(kA + (16 * mt + 8 * r) * 32);
+  const uint8_t* ksc = rec + R::k_scale + grp * 256 + 16 * qd;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 sc = lds128(ksc + 64 * i);
+    uint32_t c[2][2][4];  // [mt][row][byte]: byte 2jj + r -> k-step 2i + jj, A register (r ? 2 : 0) + row
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        e2m1_pairs(code_pass((i >> 1) ? w[mt][r].y : w[mt][r].x, i & 1), c[mt][r][0], c[mt][r][1], c[mt][r][2],
+                   c[mt][r][3]);
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int s = 2 * i + jj;
+      uint32_t b[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        b[nt][0] = fold_one(lq.qv(nt, s, 0), to_f16x2(jj ? sc.z : sc.x, T()), lq.negmask, __half());
+        b[nt][1] = fold_one(lq.qv(nt, s, 1), to_f16x2(jj ? sc.w : sc.y, T()), lq.negmask, __half());
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t a[4] = {c[mt][0][2 * jj], c[mt][1][2 * jj], c[mt][0][2 * jj + 1], c[mt][1][2 * jj + 1]};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+      }
+    }
+  }
+
+  // -- plane B: low bits of the boosted channels; rows 16s + 8r + 2qd + f of this lane sit
+  //    at positions 4 KB qd + 4s + 2r + f of each token row --
+  if constexpr (KB > 0) {
+    const uint8_t* kB = rec + R::kb_codes;
+    const uint8_t* idx = rec + R::boost_idx;
+    const uint8_t* kbsc = rec + R::kb_scale + grp * (32 * KB);
+    // k-steps in pairs: the codes of two k-steps sit in one word of each token row, so at
+    // most 16 code registers are live whatever KB is
+    constexpr int SP = KB == 1 ? 1 : 2;
+#pragma unroll
+    for (int sp = 0; sp < KB; sp += SP) {
+      uint32_t cb[2][2][SP][2];  // [mt][row][s - sp][r]
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const uint8_t* row = kB + (32 * grp + 16 * mt + g + 8 * rr) * KB * 4;
+          if constexpr (KB == 1) {
+            const uint32_t x = code_pass(lds32(row), qd >> 1) >> (16 * (qd & 1));
+            cb[mt][rr][0][0] = e2m1_pair_lo(x);
+            cb[mt][rr][0][1] = e2m1_pair_lo(x >> 8);
+          } else {
+            const int pos = 4 * KB * qd + 4 * sp;
+            const uint32_t x = code_pass(lds32(row + (pos >> 4) * 4), (pos >> 3) & 1);
+            e2m1_pairs(x, cb[mt][rr][0][0], cb[mt][rr][0][1], cb[mt][rr][SP - 1][0], cb[mt][rr][SP - 1][1]);
+          }
+        }
+#pragma unroll
+      for (int ss = 0; ss < SP; ++ss) {
+        const int s = sp + ss;
+        const int j0 = 16 * s + 2 * qd, j1 = j0 + 8;
+        // indices are < 128 in any record the library wrote; the mask keeps a corrupt
+        // record from reading outside the query rows
+        const int i00 = idx[j0] & 127, i01 = idx[j0 + 1] & 127, i10 = idx[j1] & 127, i11 = idx[j1 + 1] & 127;
+        const uint32_t s0 = to_f16x2(lds32(kbsc + j0 * 2), T()), s1 = to_f16x2(lds32(kbsc + j1 * 2), T());
+        uint32_t b[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hB = (g >> 1) + 4 * nt;
+          uint32_t q0 = 0u, q1 = 0u;
+          if (hB < GQA) {
+            const uint16_t* qh = qs + hB * kHeadDim;
+            q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
+            q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
+          }
+          b[nt][0] = fold_one(to_f16x2(q0, T()), s0, lq.negmask, __half());
+          b[nt][1] = fold_one(to_f16x2(q1, T()), s1, lq.negmask, __half());
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const uint32_t a[4] = {cb[mt][0][ss][0], cb[mt][1][ss][0], cb[mt][0][ss][1], cb[mt][1][ss][1]};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a, b[nt][0], b[nt][1], __half());
+        }
+      }
+    }
+  }
+
+  // -- zero points: Z[h] = sum_c q[h][c] * zA[c], with the query quads as A (rows are
+  //    heads) and the zero points as B (every column the same); the 16 bytes at
+  //    64 i + 16 qd are the B pairs of k-steps 2i and 2i+1 --
+  float zh[NT];
+  {
+    const uint8_t* kz = rec + R::k_zero + grp * 256 + 16 * qd;
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 zz = lds128(kz + 64 * i);
+      const uint32_t b0[2] = {to_f16x2(zz.x, T()), to_f16x2(zz.z, T())};
+      const uint32_t b1[2] = {to_f16x2(zz.y, T()), to_f16x2(zz.w, T())};
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int s = 2 * i + jj;
+        if constexpr (NT == 2) {
+          mma_16816(z0, lq.qa[s], b0[jj], b1[jj], __half());  // rows g: head g/2, g+8: head g/2 + 4
+        } else if (s < 4) {
+          mma_16816(z0, lq.qa[s], b0[jj], b1[jj], __half());  // rows g: k-step s
+        } else {
+          mma_16816(z1, lq.qa[s - 4], b0[jj], b1[jj], __half());  // rows g+8: k-step s
+        }
+      }
+    }
+    // this lane holds Z of head g/2 (+4); head qd (+4) sits in lane 8 qd
+    if constexpr (NT == 2) {
+      zh[0] = __shfl_sync(kFull, z0[0], 8 * qd);
+      zh[1] = __shfl_sync(kFull, z0[2], 8 * qd);
+    } else {
+      zh[0] = __shfl_sync(kFull, z0[0] + z1[2], 8 * qd);
+    }
+  }
+
+  // -- logits (log2 units) of tokens 16 mt + 8 r + g for head qd + 4 nt; the code
+  //    products carry a factor 0.5 --
+  const float cc = c_log2 * kCodeScale;
+  float L[2][NT][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        L[mt][nt][r] = fmaf(acc[mt][nt][2 * r] + acc[mt][nt][2 * r + 1], cc, zh[nt] * c_log2);
+  softmax_step<NT, 2>(st, L);
+
+  // -- probabilities times the value scales, as (hi, lo) pairs -> B operand of PV.
+  //    Value scale/zero positions 32 grp + 4 g + u hold tokens 8u + g --
+  const uint2 vsr = lds64(rec + R::v_scale + (32 * grp + 4 * g) * 2);
+  const uint2 vzr = lds64(rec + R::v_zero + (32 * grp + 4 * g) * 2);
+  const float2 s01 = t2_to_float2(vsr.x, T()), s23 = t2_to_float2(vsr.y, T());
+  const float2 z01 = t2_to_float2(vzr.x, T()), z23 = t2_to_float2(vzr.y, T());
+  const float sv[4] = {s01.x, s01.y, s23.x, s23.y}, zv[4] = {z01.x, z01.y, z23.x, z23.y};
+  uint32_t pb[2][NT][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int u = 2 * mt + r;
+        const float pr = ex2(L[mt][nt][r] - st.m[nt]);
+        st.l[nt] += pr;
+        st.zv[nt] = fmaf(pr, zv[u], st.zv[nt]);
+        pb[mt][nt][r] = movmatrix_trans(hilo(pr * sv[u], __half()));
+      }
+
+  // -- P V: words ((2 grp + n) * 32 + lane) * 4 + mm hold channel tile 4n + mm of this
+  //    lane; pass ks of a word is k-step ks, bytes in A-register order --
+  const uint8_t* vq = rec + R::v_codes + (64 * grp + lane) * 16;
+  const uint4 v0 = lds128(vq), v1 = lds128(vq + 512);
+  const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      e2m1_pairs(code_pass(vw[mc], ks), a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[ks][nt][0], pb[ks][nt][1], __half());
+    }
+}
+
+// ---------------------------------------------------------------- residual tokens
+
+// One piece of n <= 16 residual tokens staged in shared memory as K rows then V rows
+// (272-byte rows; rows n..15 hold zeros).  The PV operand carries 0.5 * p so
+// that the accumulator stays in the units of the code products.
+template <typename T, int GQA>
+__device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t* Vr, int n, const uint16_t* qs,
+                                               WarpState<(GQA > 4 ? 2 : 1)>& st, int lane, float c_log2) {
+  constexpr int NT = GQA > 4 ? 2 : 1;
+  const int g = lane >> 2, li = lane >> 3, lr = lane & 7;
+  const bool lo = g & 1;  // lo-part columns get no query: the raw query is exact
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    uint32_t a[4];
+    ldmatrix_x4(a, smem_addr(Kr + (lr + 8 * (li & 1)) * kResRowBytes + (16 * s + 8 * (li >> 1)) * 2));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      // the raw query in the cache dtype (exact); lo-part columns get none
+      const int hB = (g >> 1) + 4 * nt, qd = lane & 3;
+      const bool use = !lo && hB < GQA;
+      const uint32_t b0 = use ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd) : 0u;
+      const uint32_t b1 = use ? lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8) : 0u;
+      mma_16816(acc[nt], a, b0, b1, T());
+    }
+  }
+  float L[1][NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+      L[0][nt][r] = (g + 8 * r) < n ? (acc[nt][2 * r] + acc[nt][2 * r + 1]) * c_log2 : -INFINITY;
+  softmax_step<NT, 1>(st, L);
+  uint32_t pb[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float pr = ex2(L[0][nt][r] - st.m[nt]);
+      st.l[nt] += pr;
+      pb[nt][r] = movmatrix_trans(hilo(0.5f * pr, T()));
+    }
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc) {
+    uint32_t a[4];
+    ldmatrix_x4_trans(a, smem_addr(Vr + (lr + 8 * (li >> 1)) * kResRowBytes + (16 * mc + 8 * (li & 1)) * 2));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mma_16816(st.o[mc][nt], a, pb[nt][0], pb[nt][1], T());
+  }
+}
+
+// ---------------------------------------------------------------- work items
+
+// Position on the weight line: unit (b, h), item k of the unit, start weight s.  Every
+// warp walks the same sequence of items, so the loop structure (and every barrier in
+// it) is identical in all warps even when a copy fails.  Weights are 32-bit: the host
+// rejects shapes whose line could reach 2^31.
 struct Cursor {
   int b, h, k;
   int np, rl, nst, nres;  // pages, residual tokens, page stages, residual pieces of b
   int s, ubase;           // start weight of item k and of the unit
 };
-
-template <int P>
-__device__ __forceinline__ int unit_weight_of(int np, int rl) {
-  const int items = np * (P / 32) + kPieceWeight * ((rl + kPieceTokens - 1) / kPieceTokens);
-  return items > 0 ? items + kMergeWeight : 0;
-}
 
 // Unit weight of sequence b (-1 when its lengths are invalid), with its pages and
 // residual tokens (0 when invalid).
@@ -261,80 +473,77 @@ __device__ __forceinline__ int seq_weight(const DecodeParams& p, int b, int& np,
     rl = 0;
     return -1;
   }
-  return unit_weight_of<P>(np, rl);
+  const int items = np * (P / 32) + kPieceWeight * ((rl + kPieceTokens - 1) / kPieceTokens);
+  return items > 0 ? items + kMergeWeight : 0;
 }
 
 template <int P>
-__device__ __forceinline__ int unit_weight(const Cursor& c) {
-  return unit_weight_of<P>(c.np, c.rl);
-}
-
-__device__ __forceinline__ int owner_of(int s, int W, int C) { return int(floor(double(s) * C / W)); }
-__device__ __forceinline__ int range_start(int i, int W, int C) { return int(ceil(double(W) * i / C)); }
-
-// Partial softmax state of one (worker, unit) slot and head: unnormalised output [128],
-// then the maximum and the sum (floats 128, 129), padded to 16 bytes.
-constexpr int kPartStride = kHeadDim + 4;
-
-enum : uint32_t { kDescRes = 1u << 8, kDescFirst = 1u << 9, kDescLast = 1u << 10 };
-
-struct ItemDesc {
-  uint32_t w;   // bits 0-7: pages in the stage or residual tokens; kDescRes, kDescFirst,
-                // kDescLast; bits 16-31: stage or piece index within the unit
-  int b, h;
-  uint32_t io;  // first and last contributing worker of the unit (low, high 16 bits)
-};
-
-struct UnitSpan {
-  int off, b, h, k0, n, np, rl, first, last;
-  uint32_t io;
-};
-
-// Lengths the prologue keeps for the whole CTA.
-struct CtaCtl {
-  uint32_t tmem;
-  int red[kThreads / 32];
-  int2 seq[kSeqCache];   // (pages, residual tokens) of sequence b (b < kSeqCache)
-  int b0[kWG], base0[kWG];
-};
-
-// Control state of one worker.
-template <int P>
-struct WgCtl {
-  uint64_t full[4];
-  uint64_t bar_s, bar_pv;
-  Cursor cur;
-  int nseg, more, nspan, issued, abort_flag;
-  float red[4][24];
-  UnitSpan span[16];
-  ItemDesc desc[kSegItems];
-  int ids[kSegItems][128 / P];
-};
-
-// Pages and residual tokens of sequence b (from the CTA cache when it holds b).
-template <int P>
-__device__ __forceinline__ int seq_info(const DecodeParams& p, const CtaCtl& cc, int b, int& np, int& rl) {
-  if (b < kSeqCache) {
-    const int2 v = cc.seq[b];
-    np = v.x;
-    rl = v.y;
-    return unit_weight_of<P>(np, rl);
+__device__ __forceinline__ void cursor_load_seq(const DecodeParams& p, Cursor& c) {
+  // skip sequences without items; c.b == batch marks the end of the line
+  while (c.b < p.batch) {
+    if (seq_weight<P>(p, c.b, c.np, c.rl) > 0) break;
+    ++c.b;
   }
-  return max(0, seq_weight<P>(p, b, np, rl));
-}
-
-template <int P>
-__device__ __forceinline__ void cursor_load_seq(const DecodeParams& p, const CtaCtl& cc, Cursor& c) {
-  while (c.b < p.batch && seq_info<P>(p, cc, c.b, c.np, c.rl) == 0) ++c.b;
   if (c.b >= p.batch) c.np = c.rl = 0;
   c.nst = (c.np * P + 127) / 128;
   c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
 }
 
+// Weight of item k of the current unit: pages of the stage x groups per page, or 1.
+template <int P>
+__device__ __forceinline__ int item_weight(const Cursor& c) {
+  if (c.k < c.nst) return min(128 / P, c.np - c.k * (128 / P)) * (P / 32);
+  return kPieceWeight;
+}
+// Weight of a unit: its items, then the merge weight (0 for a unit without items).
+template <int P>
+__device__ __forceinline__ int unit_weight(const Cursor& c) {
+  const int items = c.np * (P / 32) + kPieceWeight * c.nres;
+  return items > 0 ? items + kMergeWeight : 0;
+}
+
+template <int P>
+__device__ __forceinline__ int unit_weight_of(int2 v) {
+  const int items = v.x * (P / 32) + kPieceWeight * ((v.y + kPieceTokens - 1) / kPieceTokens);
+  return items > 0 ? items + kMergeWeight : 0;
+}
+
+template <int P>
+__device__ __forceinline__ void cursor_next(const DecodeParams& p, Cursor& c) {
+  c.s += item_weight<P>(c);
+  if (++c.k < c.nst + c.nres) return;
+  c.k = 0;
+  c.s += kMergeWeight;
+  c.ubase = c.s;
+  if (++c.h < p.Hkv) return;
+  c.h = 0;
+  ++c.b;
+  cursor_load_seq<P>(p, c);
+}
+
+// CTA that owns weight position s: the one whose range [ceil(W i / C), ceil(W (i+1) / C))
+// contains it.
+// Both are exact in double: the products stay below 2^53 and a quotient that is not an
+// integer is at least 1/(W C) away from one, far above the rounding error.
+__device__ __forceinline__ int owner_cta(int s, int W, int C) { return int(floor(double(s) * C / W)); }
+__device__ __forceinline__ int range_start(int i, int W, int C) { return int(ceil(double(W) * i / C)); }
+
+// Owners of positions on the weight line: the line is cut into Cs equal ranges and CTA
+// i owns range i.  Every range is at least 4 long, so every owner between a unit's
+// first and last owner holds an item of the unit.
+struct Owners {
+  int W, Cs;
+  __device__ __forceinline__ int of(int s) const { return owner_cta(s, W, Cs); }
+};
+
+// Partial softmax state of one (CTA, unit) slot and head: unnormalised output [128],
+// then the maximum and the sum (floats 128, 129), padded to 16 bytes.
+constexpr int kPartStride = kHeadDim + 4;
+
 // Moves the cursor from offset `ou` of its unit to the first item that starts at or
 // after it, or to the first item of the next unit.
 template <int P>
-__device__ __forceinline__ void cursor_seek(const DecodeParams& p, const CtaCtl& cc, Cursor& c, int ou) {
+__device__ __forceinline__ void cursor_seek(const DecodeParams& p, Cursor& c, int ou) {
   if (c.nst > 0 && ou <= 4 * (c.nst - 1)) {
     c.k = (ou + 3) / 4;
     c.s = c.ubase + 4 * c.k;
@@ -352,19 +561,103 @@ __device__ __forceinline__ void cursor_seek(const DecodeParams& p, const CtaCtl&
   if (++c.h < p.Hkv) return;
   c.h = 0;
   ++c.b;
-  cursor_load_seq<P>(p, cc, c);
+  cursor_load_seq<P>(p, c);
 }
 
-// Lists the next segment of the worker's items (all 128 threads of the worker).
+
+__device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Shared-memory atomic add with acquire-release semantics at CTA scope.
+__device__ __forceinline__ int atomic_add_acq_rel_cta(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], %2;" : "=r"(old) : "r"(smem_addr(p)), "r"(v) : "memory");
+  return old;
+}
+
+// Device-scope atomic add with acquire-release semantics.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+
+// ---------------------------------------------------------------- item descriptors
+
+// A CTA walks its range in segments of up to kSegItems items.  Before a segment, the
+// CTA lists its items in shared memory (all threads, page ids loaded in parallel), so
+// that issuing the copies of an item and consuming it need no further bookkeeping.
+constexpr int kSegItems = 128;
+constexpr int kSeqCache = 128;  // (pages, residual) of the sequences from the first one on
+
+enum : uint32_t { kDescRes = 1u << 8, kDescFirst = 1u << 9, kDescLast = 1u << 10 };
+
+struct ItemDesc {
+  uint32_t w;   // bits 0-7: pages in the stage or residual tokens; kDescRes, kDescFirst,
+                // kDescLast; bits 11-12: query slot; bits 16-31: stage or piece index
+  int b, h;     // unit
+  uint32_t io;  // first and last contributing CTA of the unit (low, high 16 bits), kDescLast only
+};
+
+// Unit spans of one segment, found by one thread walking the line.
+struct UnitSpan {
+  int off;        // first item of the span within the segment
+  int b, h, k0;   // unit and its first item in the span
+  int n;          // items of the span
+  int np, rl;
+  int first, last;  // span starts / ends the unit's part in this CTA
+  int qslot;
+  uint32_t io;
+};
+
+// Pages and residual tokens of sequence b: from the cache filled during the scan, else
+// from global memory.  Returns the unit weight (0 for empty or invalid lengths).
 template <int P>
-__device__ __forceinline__ void build_segment(const DecodeParams& p, const CtaCtl& cc, WgCtl<P>& wc, int hi,
-                                              int W, int C, int wt, int wg, bool worker_first) {
+__device__ __forceinline__ int seq_info(const DecodeParams& p, int b, int b0, const int2* s_seq, int& np, int& rl) {
+  if (b0 >= 0 && b - b0 >= 0 && b - b0 < kSeqCache) {
+    const int2 v = s_seq[b - b0];
+    np = v.x;
+    rl = v.y;
+    return unit_weight_of<P>(v);
+  }
+  return max(0, seq_weight<P>(p, b, np, rl));
+}
+
+// ---------------------------------------------------------------- the kernel
+
+// Shared state of one CTA besides the stages.
+template <int GQA, int P>
+struct CtaShared {
+  uint64_t full_bar[kStages];  // stage filled (bulk-copy bytes landed)
+  int rel[kStages];            // warps that released the stage's current item
+  int red[4];
+  int b0, base0, abort_flag, issued, arrived;
+  int tail_u;         // unit whose split merge waits for the end of the range, or -1
+  uint32_t tail_io;   // its first and last contributors
+  int pref[kSeqCache];         // exclusive prefix of the weights (x kv heads), one-pass case
+  int nseg, more, nspan, uord, qslot_cont;
+  Cursor cur;                  // first item of the next segment
+  float m[4][GQA], l[4][GQA], zv[4][GQA];
+  int2 seq[kSeqCache];
+  UnitSpan span[32];
+  ItemDesc desc[kSegItems];
+  int ids[kSegItems][128 / P];
+  __align__(16) uint16_t q[3][GQA * kHeadDim];  // query heads of the last 3 units
+};
+
+// Lists the next segment of this CTA's items (all threads).  One thread walks the units
+// from sh.cur; then every thread fills one descriptor and loads its page ids.
+template <int GQA, int KB, int P>
+__device__ __forceinline__ void build_segment(const DecodeParams& p, CtaShared<GQA, P>& sh, int hi, const Owners& ow,
+                                              int tid, bool one_pass) {
   constexpr int PPC = 128 / P, GPP = P / 32;
-  if (wt == 0) {
-    Cursor c = wc.cur;
-    int n = 0, ns = 0;
-    while (c.s < hi && n < kSegItems && ns < 16) {
+  if (tid == 0) {
+    Cursor c = sh.cur;
+    int n = 0, ns = 0, uord = sh.uord, qcont = sh.qslot_cont;
+    const bool cta_first = sh.uord < 0;  // no unit started yet: the range's first segment
+    while (c.s < hi && n < kSegItems && ns < 32) {
       const int nitems = c.nst + c.nres;
+      // items of the unit that start before hi
       int kend = nitems;
       const int kst = min(c.nst, max(0, hi - c.ubase + 3) / 4);
       if (kst < c.nst) {
@@ -374,7 +667,7 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, const CtaCt
         kend = c.nst + min(c.nres, max(0, (hi - r0 + kPieceWeight - 1) / kPieceWeight));
       }
       const int cnt = min(kend - c.k, kSegItems - n);
-      UnitSpan& sp = wc.span[ns];
+      UnitSpan& sp = sh.span[ns];
       sp.off = n;
       sp.b = c.b;
       sp.h = c.h;
@@ -382,16 +675,17 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, const CtaCt
       sp.n = cnt;
       sp.np = c.np;
       sp.rl = c.rl;
-      sp.first = (c.k == 0) || (worker_first && n == 0);
+      sp.first = (c.k == 0) || (cta_first && n == 0);
       sp.last = (c.k + cnt == kend);
+      if (sp.first) qcont = (++uord) % 3;
+      sp.qslot = qcont;
       const int uw = unit_weight<P>(c);
       const int last_start =
           c.ubase + uw - kMergeWeight - (c.nres > 0 ? kPieceWeight : (c.np - (c.nst - 1) * PPC) * GPP);
-      sp.io = uint32_t(owner_of(c.ubase, W, C)) | (uint32_t(owner_of(last_start, W, C)) << 16);
+      sp.io = uint32_t(ow.of(c.ubase)) | (uint32_t(ow.of(last_start)) << 16);
       n += cnt;
       ++ns;
       c.k += cnt;
-      worker_first = false;
       if (c.k == nitems) {
         c.s = c.ubase + uw;
         c.ubase = c.s;
@@ -399,7 +693,11 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, const CtaCt
         if (++c.h == p.Hkv) {
           c.h = 0;
           ++c.b;
-          cursor_load_seq<P>(p, cc, c);
+          // next sequence with items
+          while (c.b < p.batch && seq_info<P>(p, c.b, one_pass ? 0 : sh.b0, sh.seq, c.np, c.rl) == 0) ++c.b;
+          if (c.b >= p.batch) c.np = c.rl = 0;
+          c.nst = (c.np * P + 127) / 128;
+          c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
         }
       } else if (c.k == kend) {
         c.s = hi;  // the range ends inside this unit
@@ -407,24 +705,26 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, const CtaCt
         c.s = c.ubase + (c.k < c.nst ? 4 * c.k : c.np * GPP + kPieceWeight * (c.k - c.nst));
       }
     }
-    wc.cur = c;
-    wc.nseg = n;
-    wc.nspan = ns;
-    wc.more = c.s < hi;
+    sh.cur = c;
+    sh.nseg = n;
+    sh.nspan = ns;
+    sh.more = c.s < hi;
+    sh.uord = uord;
+    sh.qslot_cont = qcont;
   }
-  wg_sync(wg);
-  const int n = wc.nseg, ns = wc.nspan;
-  for (int t = wt; t < n; t += 128) {
+  __syncthreads();
+  const int n = sh.nseg, ns = sh.nspan;
+  for (int t = tid; t < n; t += kDecodeThreads) {
     int si = 0;
-    while (si + 1 < ns && wc.span[si + 1].off <= t) ++si;
-    const UnitSpan& sp = wc.span[si];
+    while (si + 1 < ns && sh.span[si + 1].off <= t) ++si;
+    const UnitSpan& sp = sh.span[si];
     const int k = sp.k0 + (t - sp.off);
     const int nst = (sp.np * P + 127) / 128;
     ItemDesc d;
     d.b = sp.b;
     d.h = sp.h;
     d.io = sp.io;
-    uint32_t w = 0;
+    uint32_t w = uint32_t(sp.qslot) << 11;
     if (sp.first && t == sp.off) w |= kDescFirst;
     if (sp.last && t == sp.off + sp.n - 1) w |= kDescLast;
     if (k < nst) {
@@ -436,52 +736,70 @@ __device__ __forceinline__ void build_segment(const DecodeParams& p, const CtaCt
           flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
           id = 0;
         }
-        wc.ids[t][i] = id;
+        sh.ids[t][i] = id;
       }
     } else {
       const int j = k - nst;
       w |= uint32_t(min(kPieceTokens, sp.rl - kPieceTokens * j)) | kDescRes | (uint32_t(j) << 16);
     }
-    d.w = w;
-    wc.desc[t] = d;
+    sh.desc[t] = d;
+    sh.desc[t].w = w;
   }
-  wg_sync(wg);
+  __syncthreads();
 }
 
-// Issues the copies of segment item t (global item number x) into stage x % NS: the
-// page records or the residual rows, and the unit's query heads with its first item.
-// One thread.
+// Issues the copies of item x (descriptor slot t of the segment) into stage x % kStages:
+// the page records or residual rows, and the unit's query heads with its first item.
+// All lanes of the calling warp take part.
 template <int GQA, int KB, int P>
-__device__ __forceinline__ void issue_item(const DecodeParams& p, WgCtl<P>& wc, uint8_t* ws, int x, int t,
-                                           uint64_t policy) {
+__device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA, P>& sh, uint8_t* smem, int x, int t,
+                                           uint64_t policy, int lane) {
   using R = Rec<P, KB>;
-  using C = Cfg<GQA, KB, P>;
-  const ItemDesc d = wc.desc[t];
-  const int st = x % C::NS, n = d.w & 0xff;
+  using S = Smem<GQA, P, KB>;
+  const ItemDesc d = sh.desc[t];
+  const int st = x % kStages, n = d.w & 0xff;
   const bool res = d.w & kDescRes, first = d.w & kDescFirst;
-  uint8_t* sb = ws + C::O_RING + st * kStageBytes;
-  const uint32_t bytes = (res ? 2u * uint32_t(n) * 256u : uint32_t(n) * R::payload) + (first ? GQA * 256u : 0u);
-  tc::fence_async_smem();
-  mbar_arrive_expect_tx(&wc.full[st], bytes);
+  uint8_t* sb = smem + st * S::stage;
+  const uint32_t bytes = (res ? 0u : uint32_t(n) * R::payload) + (first ? GQA * 256u : 0u);
+  if (lane == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (!res) mbar_arrive_expect_tx(&sh.full_bar[st], bytes);
+    atomicAdd(&sh.issued, 1);
+  }
+  __syncwarp();
   if (!res) {
-    for (int i = 0; i < n; ++i)
-      bulk_g2s(sb + i * R::record, p.pool + (size_t(wc.ids[t][i]) * p.Hkv + d.h) * R::record, R::payload,
-               &wc.full[st], policy);
+    if (lane < n)
+      bulk_g2s(sb + lane * R::record, p.pool + (size_t(sh.ids[t][lane]) * p.Hkv + d.h) * R::record, R::payload,
+               &sh.full_bar[st], policy);
   } else {
-    const size_t row0 = (size_t(d.b) * p.Hkv + d.h) * P + size_t(kPieceTokens) * (d.w >> 16);
-    bulk_g2s(sb, p.res_k + row0 * kHeadDim, uint32_t(n) * 256u, &wc.full[st], policy);
-    bulk_g2s(sb + kResV, p.res_v + row0 * kHeadDim, uint32_t(n) * 256u, &wc.full[st], policy);
+    // residual rows: 16-byte asynchronous copies into the padded rows, zero-filled past
+    // the last token; each lane's copies arrive on the stage's barrier when they land
+    const int t0 = kPieceTokens * int(d.w >> 16);
+    const uint16_t* kr = p.res_k + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+    const uint16_t* vr = p.res_v + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+#pragma unroll 4
+    for (int i = lane; i < 2 * kPieceTokens * 16; i += 32) {
+      const int which = i >> 8, row = (i >> 4) & 15, chunk = i & 15;
+      const uint16_t* src = (which ? vr : kr) + (row < n ? row : 0) * kHeadDim + chunk * 8;
+      cp_async16(sb + (which * kPieceTokens + row) * kResRowBytes + chunk * 16, src, row < n ? 16u : 0u);
+    }
+    cp_async_arrive(&sh.full_bar[st]);
   }
-  if (first) {
+  if (res) {
+    // every lane's asynchronous arrival is registered: now the one expected arrival
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(&sh.full_bar[st], bytes);
+    __syncwarp();
+  }
+  if (first && lane == 31) {
     const uint16_t* src = p.q + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
-    bulk_g2s(ws + C::O_Q + st * GQA * 256, src, GQA * 256u, &wc.full[st], policy);
+    bulk_g2s(sh.q[(d.w >> 11) & 3], src, GQA * 256u, &sh.full_bar[st], policy);
   }
-  ++wc.issued;
 }
 
 // Merges heads h0 .. h0 + HC - 1 of the nc partial states at pu (log-sum-exp) into outu.
 // One warp; lane i holds channels 4i .. 4i + 3.
-template <int HC>
+template <int HC, int UNROLL>
 __device__ __forceinline__ void merge_heads(const float* pu, size_t slot, int nc, int h0, float* outu, int lane) {
   float Mh[HC], Lh[HC];
   float4 Oh[HC];
@@ -497,7 +815,8 @@ __device__ __forceinline__ void merge_heads(const float* pu, size_t slot, int nc
     Lh[h] = 0.0f;
     Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-#pragma unroll 4
+  // every contributor's loads of a batch are in flight together
+#pragma unroll UNROLL
   for (int i = 0; i < nc; ++i) {
     const float* pi = pu + i * slot + h0 * kPartStride;
     float mi[HC], li[HC];
@@ -526,668 +845,105 @@ __device__ __forceinline__ void merge_heads(const float* pu, size_t slot, int nc
   }
 }
 
-__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-// ---------------------------------------------------------------- one worker
-
-// Per-thread softmax state of the current unit.
+// One warp: counts this contributor in for unit u and, if it is the last of the
+// contributors i0..i1, merges their partial states (log-sum-exp) into the output.
+// (Written out rather than through merge_heads: inlined into the item loop, the helper
+// changes the loop's register allocation enough to spill at 128 registers.)
 template <int GQA>
-struct State {
-  float M[GQA];   // running maximum (log2 units), the same in every thread of the worker
-  float l[GQA];   // this thread's share of the softmax sum
-  float zv[GQA];  // this thread's share of sum p * value zero point
-  int F;          // value-operand exponent
-  float vlim;     // 2^(7 + F): value scales at or above it need a larger F
-  float fsc;      // 2^-F
-  bool pv;        // O holds products of this unit
-};
-
-template <typename T, int GQA, int KB, int P>
-__device__ __forceinline__ void worker_run(const DecodeParams& p, const CtaCtl& cc, WgCtl<P>& wc, uint8_t* ws,
-                                           uint32_t tmem, int W, int Cw, int worker, int wg, int wt) {
-  using R = Rec<P, KB>;
-  using C = Cfg<GQA, KB, P>;
-  constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
-  constexpr int NQ2 = (GQA + 1) / 2;
-  constexpr uint32_t ID_QK = tc::idesc_f16(C::NQK, false);
-  constexpr uint32_t ID_PV = tc::idesc_f16(16, false);
-  constexpr uint32_t ID_RES = tc::idesc_f16(16, BF);
-  const int wwarp = wt >> 5, lane = wt & 31;
-  const uint32_t tbase = tmem + 16 + uint32_t(wg * C::COLS);  // this worker's columns
-  const uint32_t tl = tc::lane_addr(tbase, wwarp, 0);          // this thread's lane quarter
-  const uint32_t t_ones = tmem;                                // columns 0..7: fp16 0.5
-  uint8_t* const bqk = ws + C::O_BQK;
-  uint8_t* const bz = ws + C::O_BZ;
-  uint8_t* const bqb = ws + C::O_BQB;
-  uint8_t* const bpv = ws + C::O_BPV;
-  uint8_t* const bqr = ws + C::O_BQR;
-  uint16_t* const qh = reinterpret_cast<uint16_t*>(ws + C::O_QH);
-  const uint32_t a_bqk = smem_addr(bqk), a_bz = smem_addr(bz), a_bqb = smem_addr(bqb), a_bpv = smem_addr(bpv),
-                 a_bqr = smem_addr(bqr);
-  const uint64_t policy = l2_evict_first_policy();
-  const int lo = range_start(worker, W, Cw), hi = range_start(worker + 1, W, Cw);
-
-  // locate the first item: the prologue found the sequence holding position lo
-  if (wt == 0) {
-    Cursor c;
-    c.b = cc.b0[wg];
-    seq_info<P>(p, cc, c.b, c.np, c.rl);
-    c.nst = (c.np * P + 127) / 128;
-    c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
-    c.k = 0;
-    const int wseq = unit_weight<P>(c);
-    const int off = lo - cc.base0[wg];
-    c.h = off / wseq;
-    c.ubase = cc.base0[wg] + c.h * wseq;
-    cursor_seek<P>(p, cc, c, off - c.h * wseq);
-    wc.cur = c;
-    wc.issued = 0;
-    wc.abort_flag = 0;
-  }
-  wg_sync(wg);
-
-  State<GQA> stt;
-  uint32_t q2[NQ2];    // this thread's channel of q' as fp16 pairs (heads 2i, 2i + 1)
-  float cq[GQA], cr[GQA];  // logit factors: pages (2 * c * 2^e), residual (c * 2^e)
-  int x = 0;               // items of this worker so far
-  uint32_t ps = 0, ppv = 0;  // parities of bar_s and bar_pv
-  bool pv_pending = false;   // a PV product was issued and not yet waited for
-  bool worker_first = true;
-  bool failed = false;
-
-  auto wait_pv = [&]() {
-    if (pv_pending) {
-      if (!mbar_wait_bounded(&wc.bar_pv, ppv)) failed = true;
-      __syncwarp();
-      ppv ^= 1u;
-      pv_pending = false;
+__device__ __forceinline__ void merge_partials(const DecodeParams& p, int u, int i0, int i1, float* outu, int lane) {
+  uint32_t arrived = 0;
+  if (lane == 0) arrived = atomic_add_acq_rel_gpu(p.cnt + u, 1u);
+  arrived = __shfl_sync(kFull, arrived, 0);
+  const int nc = i1 - i0 + 1;
+  if (arrived != uint32_t(nc - 1)) return;
+  const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
+  const size_t slot = size_t(GQA) * kPartStride;  // floats per contributor
+  // up to four heads at a time, so that every contributor's loads are in flight together
+  constexpr int HC = GQA < 4 ? GQA : 4;
+#pragma unroll
+  for (int h0 = 0; h0 < GQA; h0 += HC) {
+    float Mh[HC], Lh[HC];
+    float4 Oh[HC];
+#pragma unroll
+    for (int h = 0; h < HC; ++h) Mh[h] = -INFINITY;
+    for (int i = lane; i < nc; i += 32)
+#pragma unroll
+      for (int h = 0; h < HC; ++h) Mh[h] = fmaxf(Mh[h], __ldcg(pu + i * slot + (h0 + h) * kPartStride + kHeadDim));
+#pragma unroll
+    for (int h = 0; h < HC; ++h) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) Mh[h] = fmaxf(Mh[h], __shfl_xor_sync(kFull, Mh[h], off));
+      Lh[h] = 0.0f;
+      Oh[h] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-  };
-
-  while (true) {
-    build_segment<P>(p, cc, wc, hi, W, Cw, wt, wg, worker_first);
-    worker_first = false;
-    const int nseg = wc.nseg;
-    if (wt == 0)
-      for (int t = 0; t < min(C::NS, nseg); ++t) issue_item<GQA, KB, P>(p, wc, ws, x + t, t, policy);
-    for (int t = 0; t < nseg; ++t) {
-      const int xi = x + t, st = xi % C::NS;
-      const uint32_t par = uint32_t(xi / C::NS) & 1u;
-      const ItemDesc d = wc.desc[t];
-      const uint8_t* sb = ws + C::O_RING + st * kStageBytes;
-      const bool res = d.w & kDescRes;
-      const int n = d.w & 0xff;
-      if (!mbar_wait_bounded(&wc.full[st], par)) failed = true;
-      __syncwarp();
-
-      // ---------------------------------------------------------- unit start
-      if (d.w & kDescFirst) {
-        const uint8_t* qs = ws + C::O_Q + st * GQA * 256;
-        float qf[GQA];
+#pragma unroll 4
+    for (int i = 0; i < nc; ++i) {
+      const float* pi = pu + i * slot + h0 * kPartStride;
+      float mi[HC], li[HC];
+      float4 oi[HC];
 #pragma unroll
-        for (int h = 0; h < GQA; ++h) qf[h] = t_to_f(u16_at(qs + h * 256 + 2 * wt), T());
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          const uint32_t mb = __reduce_max_sync(kFull, __float_as_uint(fabsf(qf[h])));
-          if (lane == 0) wc.red[wwarp][h] = __uint_as_float(mb);
-        }
-        wg_sync(wg);
-        float qp[GQA];
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          const float m = fmaxf(fmaxf(wc.red[0][h], wc.red[1][h]), fmaxf(wc.red[2][h], wc.red[3][h]));
-          // |q'| = |q| * 2^-e < 1; e kept inside the normal exponent range
-          int e = m > 0.0f ? int((__float_as_uint(m) >> 23) & 0xff) - 126 : 0;
-          e = min(max(e, -125), 125);
-          qp[h] = qf[h] * pow2f(-e);
-          cq[h] = 2.0f * p.c_log2 * pow2f(e);
-          cr[h] = p.c_log2 * pow2f(e);
-        }
-        if constexpr (GQA == 1) {
-          q2[0] = pack2(qp[0], 0.0f, __half());
-        } else {
-#pragma unroll
-          for (int i = 0; i < GQA / 2; ++i) q2[i] = pack2(qp[2 * i], qp[2 * i + 1], __half());
-        }
-        // q' in fp16 for the plane-B gathers, in the cache dtype for the residual product
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) qh[wt * GQA + h] = __half_as_ushort(__float2half_rn(qp[h]));
-        {
-          uint32_t v[(GQA + 1) / 2];
-          if constexpr (GQA == 1) {
-            v[0] = pack2(qp[0], 0.0f, T());
-          } else {
-#pragma unroll
-            for (int i = 0; i < GQA / 2; ++i) v[i] = pack2(qp[2 * i], qp[2 * i + 1], T());
-          }
-          store_n16_row(bqr, wt, v);
-        }
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          stt.M[h] = -INFINITY;
-          stt.l[h] = 0.0f;
-          stt.zv[h] = 0.0f;
-        }
-        stt.F = 0;
-        stt.vlim = 128.0f;
-        stt.fsc = 1.0f;
-        stt.pv = false;
-        tc::fence_async_smem();
-        wg_sync(wg);  // q' visible to every thread (plane B) and, through the fence, to the products
+      for (int h = 0; h < HC; ++h) {
+        mi[h] = __ldcg(pi + h * kPartStride + kHeadDim);
+        li[h] = __ldcg(pi + h * kPartStride + kHeadDim + 1);
+        oi[h] = __ldcg(reinterpret_cast<const float4*>(pi + h * kPartStride) + lane);
       }
-
-      float L[GQA];     // this thread's token logits (log2 units), -inf when masked
-      float sv = 0.0f;  // value scale of the token (pages)
-      float zvt = 0.0f; // value zero point of the token (pages)
-      bool valid;
-      if (!res) {
-        // ---------------------------------------------------------- page stage
-        const int npg = n;
-        const int r_t = wt / P, tk = wt % P;  // record and token of this thread's token
-        valid = r_t < npg;
-        if (!C::SPLIT) wait_pv();  // the value product still reads the shared A region
-        {
-          // keys of token wt: plane A words (two blocks of four), plane B words
-          const uint8_t* rk = sb + r_t * R::record;
-          const uint4 a0 = lds128(rk + R::k_codes + 16 * tk);
-          const uint4 a1 = lds128(rk + R::k_codes + 16 * P + 16 * tk);
-          uint32_t cv[32];
-          word_to_cols(a0.x, cv);
-          word_to_cols(a0.y, cv + 8);
-          word_to_cols(a0.z, cv + 16);
-          word_to_cols(a0.w, cv + 24);
-          tc::st<32>(tl + C::C_AQ, cv);
-          word_to_cols(a1.x, cv);
-          word_to_cols(a1.y, cv + 8);
-          word_to_cols(a1.z, cv + 16);
-          word_to_cols(a1.w, cv + 24);
-          tc::st<32>(tl + C::C_AQ + 32, cv);
-          if constexpr (KB == 1) {
-            uint32_t cb[8];
-            word_to_cols(lds32(rk + R::kb_codes + 4 * tk), cb);
-            tc::st<8>(tl + C::C_AQ + 64, cb);
-          } else if constexpr (KB == 2) {
-            const uint2 b0 = lds64(rk + R::kb_codes + 8 * tk);
-            uint32_t cb[16];
-            word_to_cols(b0.x, cb);
-            word_to_cols(b0.y, cb + 8);
-            tc::st<16>(tl + C::C_AQ + 64, cb);
-          } else if constexpr (KB >= 4) {
 #pragma unroll
-            for (int blk = 0; blk < KB / 4; ++blk) {
-              const uint4 b0 = lds128(rk + R::kb_codes + blk * 16 * P + 16 * tk);
-              word_to_cols(b0.x, cv);
-              word_to_cols(b0.y, cv + 8);
-              word_to_cols(b0.z, cv + 16);
-              word_to_cols(b0.w, cv + 24);
-              tc::st<32>(tl + C::C_AQ + 64 + 32 * blk, cv);
-            }
-          }
-        }
-        {
-          // folded query of channel wt: plane-A scales and zero points, 4 groups
-          uint32_t sbits[4], zbits[4];
-          if constexpr (P == 128) {
-            const uint2 s = lds64(sb + R::k_scale + 8 * wt), z = lds64(sb + R::k_zero + 8 * wt);
-            sbits[0] = s.x; sbits[1] = s.x >> 16; sbits[2] = s.y; sbits[3] = s.y >> 16;
-            zbits[0] = z.x; zbits[1] = z.x >> 16; zbits[2] = z.y; zbits[3] = z.y >> 16;
-          } else if constexpr (P == 64) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const uint32_t s = lds32(sb + r * R::record + R::k_scale + 4 * wt);
-              const uint32_t z = lds32(sb + r * R::record + R::k_zero + 4 * wt);
-              sbits[2 * r] = s; sbits[2 * r + 1] = s >> 16;
-              zbits[2 * r] = z; zbits[2 * r + 1] = z >> 16;
-            }
-          } else {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              sbits[r] = u16_at(sb + r * R::record + R::k_scale + 2 * wt);
-              zbits[r] = u16_at(sb + r * R::record + R::k_zero + 2 * wt);
-            }
-          }
-          GroupRow<GQA> gs[4], gz[4];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            // groups of records past the stage's pages hold stale bytes: zero operands
-            const bool gv = (g / C::NG) < npg;
-            gs[g] = fold_group<GQA>(q2, gv ? t_bcast_h2(sbits[g] & 0xffffu, T()) : 0u);
-            gz[g] = fold_group<GQA>(q2, gv ? t_bcast_h2(zbits[g] & 0xffffu, T()) : 0u);
-          }
-          store_qk_row<GQA, C::LBO_QK>(bqk, wt, gs);
-          store_qk_row<GQA, C::LBO_QK>(bz, wt, gz);
-        }
-        if constexpr (KB > 0) {
-          if (wt < 16 * KB) {
-            // plane B: boosted row wt of each record, with that record's channel index
-            GroupRow<GQA> gb[4];
-#pragma unroll
-            for (int r = 0; r < C::PPS; ++r) {
-              const uint8_t* rr = sb + r * R::record;
-              const bool rv = r < npg;
-              const int ch = rv ? (rr[R::boost_idx + wt] & 127) : 0;
-              uint32_t qb[NQ2];
-              if constexpr (GQA == 1) {
-                qb[0] = qh[ch];
-              } else if constexpr (GQA == 2) {
-                qb[0] = lds32(qh + 2 * ch);
-              } else if constexpr (GQA == 4) {
-                const uint2 v = lds64(qh + 4 * ch);
-                qb[0] = v.x;
-                qb[1] = v.y;
-              } else {
-                const uint4 v = lds128(qh + 8 * ch);
-                qb[0] = v.x;
-                qb[1] = v.y;
-                qb[2] = v.z;
-                qb[3] = v.w;
-              }
-#pragma unroll
-              for (int g2 = 0; g2 < C::NG; ++g2) {
-                const uint32_t sbb = rv ? u16_at(rr + R::kb_scale + (wt * C::NG + g2) * 2) : 0u;
-                gb[r * C::NG + g2] = fold_group<GQA>(qb, rv ? t_bcast_h2(sbb, T()) : 0u);
-              }
-            }
-            store_qk_row<GQA, C::LBO_QK>(bqb, wt, gb);
-          }
-        }
-        tc::wait_st();
-        tc::fence_async_smem();
-        tc::fence_before();
-        failed = wg_sync_or(wg, failed);
-        if (failed) break;
-        if (wt == 0) {
-          tc::fence_after();
-          const uint32_t dS = tbase + C::C_S;
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            tc::mma(dS, tbase + C::C_AQ + 8 * s, tc::smem_desc(a_bqk + s * 2 * C::LBO_QK, C::LBO_QK, 128), ID_QK,
-                    s > 0);
-#pragma unroll
-          for (int s = 0; s < KB; ++s)
-            tc::mma(dS, tbase + C::C_AQ + 64 + 8 * s, tc::smem_desc(a_bqb + s * 2 * C::LBO_QK, C::LBO_QK, 128),
-                    ID_QK, 1);
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            tc::mma(dS, t_ones, tc::smem_desc(a_bz + s * 2 * C::LBO_QK, C::LBO_QK, 128), ID_QK, 1);
-          tc::commit(&wc.bar_s);
-        }
-        if (!mbar_wait_bounded(&wc.bar_s, ps)) failed = true;
-        __syncwarp();
-        ps ^= 1u;
-        tc::fence_after();
-        // logits of token wt: its group's columns (group = warp of the worker)
-        uint32_t sr[2 * GQA];
-        if constexpr (GQA == 4) {
-          tc::ld<8>(tl + C::C_S + wwarp * 8, sr);
-        } else if constexpr (GQA == 8) {
-          tc::ld<16>(tl + C::C_S + wwarp * 16, sr);
-        } else if constexpr (GQA == 2) {
-          tc::ld<4>(tl + C::C_S + wwarp * 4, sr);
-        } else {
-          tc::ld<2>(tl + C::C_S + wwarp * 2, sr);
-        }
-        // values of channel wt -> A_V (after the previous value product has finished)
-        if (C::SPLIT) wait_pv();
-        {
-          uint32_t cv[32];
-          if constexpr (P == 128) {
-            const uint4 v0 = lds128(sb + R::v_codes + 16 * wt), v1 = lds128(sb + R::v_codes + 2048 + 16 * wt);
-            word_to_cols(v0.x, cv);
-            word_to_cols(v0.y, cv + 8);
-            word_to_cols(v0.z, cv + 16);
-            word_to_cols(v0.w, cv + 24);
-            tc::st<32>(tl + C::C_AV, cv);
-            word_to_cols(v1.x, cv);
-            word_to_cols(v1.y, cv + 8);
-            word_to_cols(v1.z, cv + 16);
-            word_to_cols(v1.w, cv + 24);
-            tc::st<32>(tl + C::C_AV + 32, cv);
-          } else if constexpr (P == 64) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const uint4 v0 = lds128(sb + r * R::record + R::v_codes + 16 * wt);
-              word_to_cols(v0.x, cv);
-              word_to_cols(v0.y, cv + 8);
-              word_to_cols(v0.z, cv + 16);
-              word_to_cols(v0.w, cv + 24);
-              tc::st<32>(tl + C::C_AV + 32 * r, cv);
-            }
-          } else {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const uint2 v0 = lds64(sb + r * R::record + R::v_codes + 8 * wt);
-              uint32_t c16[16];
-              word_to_cols(v0.x, c16);
-              word_to_cols(v0.y, c16 + 8);
-              tc::st<16>(tl + C::C_AV + 16 * r, c16);
-            }
-          }
-        }
-        // the token's value scale and zero point
-        {
-          const uint8_t* rv = sb + r_t * R::record;
-          sv = valid ? t_to_f(u16_at(rv + R::v_scale + 2 * tk), T()) : 0.0f;
-          zvt = valid ? t_to_f(u16_at(rv + R::v_zero + 2 * tk), T()) : 0.0f;
-        }
-        tc::wait_ld();
-#pragma unroll
-        for (int h = 0; h < GQA; ++h)
-          L[h] = valid ? (__uint_as_float(sr[h]) + __uint_as_float(sr[GQA + h])) * cq[h] : -INFINITY;
-      } else {
-        // ---------------------------------------------------------- residual piece
-        valid = wt < n;
-        if (!C::SPLIT) wait_pv();
-        if (wwarp == 0) {
-          // key row `lane` of the piece (rows >= n are stale and masked below)
-          const uint8_t* kr = sb + lane * 256;
-          uint32_t cv[32];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint4 v = lds128(kr + half * 128 + 16 * i);
-              cv[4 * i] = v.x;
-              cv[4 * i + 1] = v.y;
-              cv[4 * i + 2] = v.z;
-              cv[4 * i + 3] = v.w;
-            }
-            tc::st<32>(tl + C::C_AQ + 32 * half, cv);
-          }
-        }
-        tc::wait_st();
-        tc::fence_before();
-        failed = wg_sync_or(wg, failed);
-        if (failed) break;
-        if (wt == 0) {
-          tc::fence_after();
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            tc::mma(tbase + C::C_S, tbase + C::C_AQ + 8 * s, tc::smem_desc(a_bqr + s * 512, 256, 128), ID_RES, s > 0);
-          tc::commit(&wc.bar_s);
-        }
-        if (!mbar_wait_bounded(&wc.bar_s, ps)) failed = true;
-        __syncwarp();
-        ps ^= 1u;
-        tc::fence_after();
-        uint32_t sr[GQA];
-        if (wwarp == 0) {
-          if constexpr (GQA == 1) {
-            tc::ld<1>(tl + C::C_S, sr);
-          } else if constexpr (GQA == 2) {
-            tc::ld<2>(tl + C::C_S, sr);
-          } else if constexpr (GQA == 4) {
-            tc::ld<4>(tl + C::C_S, sr);
-          } else {
-            tc::ld<8>(tl + C::C_S, sr);
-          }
-        }
-        // values: channel wt of the piece's n tokens -> A_V columns 0..15
-        if (C::SPLIT) wait_pv();
-        {
-          uint32_t cv[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint32_t v0 = 2 * i < n ? u16_at(sb + kResV + (2 * i) * 256 + 2 * wt) : 0u;
-            const uint32_t v1 = 2 * i + 1 < n ? u16_at(sb + kResV + (2 * i + 1) * 256 + 2 * wt) : 0u;
-            cv[i] = v0 | (v1 << 16);
-          }
-          tc::st<16>(tl + C::C_AV, cv);
-        }
-        if (wwarp == 0) tc::wait_ld();
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) L[h] = valid ? __uint_as_float(sr[h]) * cr[h] : -INFINITY;
-      }
-
-      // ---------------------------------------------------------- softmax, PV operand
-      bool ex = valid && !(sv < stt.vlim);
-#pragma unroll
-      for (int h = 0; h < GQA; ++h) ex |= !(L[h] <= stt.M[h] + kLazy);
-      float pr[GQA];
-      auto write_pv_row = [&]() {
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) pr[h] = valid ? ex2(L[h] - stt.M[h]) : 0.0f;
-        if (!res) {
-          float xv[GQA];
-#pragma unroll
-          for (int h = 0; h < GQA; ++h) xv[h] = pr[h] * sv * stt.fsc;
-          uint32_t v[GQA];
-          if constexpr (GQA == 1) {
-            uint32_t hi, lo;
-            split2<__half>(xv[0], 0.0f, hi, lo);
-            v[0] = (hi & 0xffffu) | (lo << 16);
-          } else {
-#pragma unroll
-            for (int i = 0; i < GQA / 2; ++i) split2<__half>(xv[2 * i], xv[2 * i + 1], v[i], v[GQA / 2 + i]);
-          }
-          store_n16_row(bpv, wt, v);
-        } else if (wwarp == 0) {
-          float xv[GQA];
-#pragma unroll
-          for (int h = 0; h < GQA; ++h) xv[h] = 0.5f * pr[h] * stt.fsc;
-          uint32_t v[GQA];
-          if constexpr (GQA == 1) {
-            uint32_t hi, lo;
-            split2<T>(xv[0], 0.0f, hi, lo);
-            v[0] = (hi & 0xffffu) | (lo << 16);
-          } else {
-#pragma unroll
-            for (int i = 0; i < GQA / 2; ++i) split2<T>(xv[2 * i], xv[2 * i + 1], v[i], v[GQA / 2 + i]);
-          }
-          store_n16_row(bpv, wt, v);
-        }
-      };
-      write_pv_row();
-      tc::wait_st();
-      tc::fence_async_smem();
-      tc::fence_before();
-      const bool any = wg_sync_or(wg, ex || failed);
-      if (any) {
-        failed = wg_sync_or(wg, failed);
-        if (failed) break;
-        // ---- slow path: the running maximum or the value exponent moves
-        float mx[GQA];
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          float v = L[h];
-          if (v != v || v == INFINITY) {  // NaN or +inf: an operand left the supported range
-            flag_error(p.err, KVQ_DEV_ERR_RANGE);
-            v = -INFINITY;
-            L[h] = -INFINITY;
-          }
-          mx[h] = v;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], off));
-        }
-        float svm = valid ? sv : 0.0f;
-        if (!(svm < INFINITY)) {
-          flag_error(p.err, KVQ_DEV_ERR_RANGE);
-          svm = 0.0f;
-          sv = 0.0f;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) svm = fmaxf(svm, __shfl_xor_sync(kFull, svm, off));
-        if (lane == 0) {
-#pragma unroll
-          for (int h = 0; h < GQA; ++h) wc.red[wwarp][h] = mx[h];
-          wc.red[wwarp][GQA] = svm;
-        }
-        wg_sync(wg);
-        float alpha[GQA];
-        int Fn = stt.F;
-        {
-          const float s4 = fmaxf(fmaxf(wc.red[0][GQA], wc.red[1][GQA]), fmaxf(wc.red[2][GQA], wc.red[3][GQA]));
-          if (s4 >= stt.vlim) {
-            // s4 in [2^e, 2^(e+1)): F = e - 6 keeps s4 * 2^(8 - F) below 2^15
-            const int e = int((__float_as_uint(s4) >> 23) & 0xff) - 127;
-            Fn = max(stt.F, min(e - 6, 120));
-          }
-        }
-        const float beta = pow2f(stt.F - Fn);
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          const float mp = fmaxf(fmaxf(wc.red[0][h], wc.red[1][h]), fmaxf(wc.red[2][h], wc.red[3][h]));
-          const float Mn = fmaxf(stt.M[h], mp);
-          alpha[h] = stt.M[h] == -INFINITY ? 0.0f : ex2(stt.M[h] - Mn);
-          stt.M[h] = Mn;
-          stt.l[h] *= alpha[h];
-          stt.zv[h] *= alpha[h];
-        }
-        if (stt.pv) {
-          // rescale this thread's lane of O (the last value product has completed)
-          wait_pv();
-          uint32_t o[16];
-          tc::ld<16>(tl + C::C_O, o);
-          tc::wait_ld();
-#pragma unroll
-          for (int h = 0; h < GQA; ++h) {
-            const float f = alpha[h] * beta;
-            o[h] = __float_as_uint(__uint_as_float(o[h]) * f);
-            o[GQA + h] = __float_as_uint(__uint_as_float(o[GQA + h]) * f);
-          }
-          tc::st<16>(tl + C::C_O, o);
-        }
-        stt.F = Fn;
-        stt.vlim = pow2f(min(7 + Fn, 127));
-        stt.fsc = pow2f(-Fn);
-        write_pv_row();
-        tc::wait_st();
-        tc::fence_async_smem();
-        tc::fence_before();
-        wg_sync(wg);  // also keeps wc.red from being overwritten early
-      }
-      // ---------------------------------------------------------- PV product
-      if (wt == 0) {
-        tc::fence_after();
-        if (!res) {
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            tc::mma(tbase + C::C_O, tbase + C::C_AV + 8 * s, tc::smem_desc(a_bpv + s * 512, 256, 128), ID_PV,
-                    (stt.pv || s > 0) ? 1u : 0u);
-        } else {
-#pragma unroll
-          for (int s = 0; s < 2; ++s)
-            tc::mma(tbase + C::C_O, tbase + C::C_AV + 8 * s, tc::smem_desc(a_bpv + s * 512, 256, 128), ID_RES,
-                    (stt.pv || s > 0) ? 1u : 0u);
-        }
-        tc::commit(&wc.bar_pv);
-        // the stage is free (every thread has passed the barrier above): refill it
-        if (t + C::NS < nseg) issue_item<GQA, KB, P>(p, wc, ws, xi + C::NS, t + C::NS, policy);
-      }
-      pv_pending = true;
-      stt.pv = true;
-#pragma unroll
-      for (int h = 0; h < GQA; ++h) {
-        stt.l[h] += pr[h];
-        stt.zv[h] = fmaf(pr[h], zvt, stt.zv[h]);
-      }
-
-      // ---------------------------------------------------------- unit end
-      if (d.w & kDescLast) {
-        wait_pv();
-        tc::fence_after();
-        uint32_t o[16];
-        tc::ld<16>(tl + C::C_O, o);
-        float ls[GQA], zs[GQA];
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          ls[h] = stt.l[h];
-          zs[h] = stt.zv[h];
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-            ls[h] += __shfl_xor_sync(kFull, ls[h], off);
-            zs[h] += __shfl_xor_sync(kFull, zs[h], off);
-          }
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int h = 0; h < GQA; ++h) {
-            wc.red[wwarp][h] = ls[h];
-            wc.red[wwarp][8 + h] = zs[h];
-          }
-        }
-        tc::wait_ld();
-        wg_sync(wg);
-        const int u = d.b * p.Hkv + d.h;
-        const int i0 = int(d.io & 0xffffu), i1 = int(d.io >> 16);
-        const bool sole = i0 == i1;
-        float* outu = p.out + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
-        float* part_me = p.part + (size_t(worker) + u) * GQA * kPartStride;
-        const float of = pow2f(stt.F + 1);
-#pragma unroll
-        for (int h = 0; h < GQA; ++h) {
-          const float Lh = wc.red[0][h] + wc.red[1][h] + wc.red[2][h] + wc.red[3][h];
-          const float Zh = wc.red[0][8 + h] + wc.red[1][8 + h] + wc.red[2][8 + h] + wc.red[3][8 + h];
-          const float O = (__uint_as_float(o[h]) + __uint_as_float(o[GQA + h])) * of + Zh;
-          if (sole) {
-            outu[h * kHeadDim + wt] = Lh > 0.0f ? O / Lh : 0.0f;
-          } else {
-            float* pp = part_me + h * kPartStride;
-            pp[wt] = O;
-            if (wt == 0) {
-              pp[kHeadDim] = stt.M[h];
-              pp[kHeadDim + 1] = Lh;
-            }
-          }
-        }
-        stt.pv = false;
-        if (!sole) {
-          // the last of the contributors i0..i1 merges their partials.  The barrier
-          // orders every thread's partial writes before the counter update (a release
-          // at device scope); the merging worker acquires it.
-          wg_sync(wg);
-          if (wt == 0) wc.red[0][23] = __int_as_float(int(atomic_add_acq_rel_gpu(p.cnt + u, 1u)));
-          wg_sync(wg);
-          const int nc = i1 - i0 + 1;
-          if (__float_as_int(wc.red[0][23]) == nc - 1) {
-            const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
-            for (int h = wwarp; h < GQA; h += 4) merge_heads<1>(pu, size_t(GQA) * kPartStride, nc, h, outu, lane);
-            if (wt == 0) p.cnt[u] = 0u;  // ready for the next launch
-          }
-        }
-        wg_sync(wg);  // wc.red is reused by the next unit
+      for (int h = 0; h < HC; ++h) {
+        const float f = Mh[h] == -INFINITY ? 0.0f : ex2(mi[h] - Mh[h]);
+        Lh[h] += f * li[h];
+        Oh[h].x += f * oi[h].x;
+        Oh[h].y += f * oi[h].y;
+        Oh[h].z += f * oi[h].z;
+        Oh[h].w += f * oi[h].w;
       }
     }
-    if (failed) break;
-    x += nseg;
-    if (!wc.more) break;
-  }
-
-  if (failed) {
-    // a wait gave up: flag it, then wait (bounded) for this worker's copies and
-    // products in flight before the shared and tensor memory are released
-    if (wt == 0) {
-      flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
-      const int issued = wc.issued;
-      for (int y = max(0, issued - C::NS); y < issued; ++y)
-        mbar_wait_bounded(&wc.full[y % C::NS], uint32_t(y / C::NS) & 1u);
+#pragma unroll
+    for (int h = 0; h < HC; ++h) {
+      const float inv = Lh[h] > 0.0f ? 1.0f / Lh[h] : 0.0f;
+      reinterpret_cast<float4*>(outu + (h0 + h) * kHeadDim)[lane] =
+          make_float4(Oh[h].x * inv, Oh[h].y * inv, Oh[h].z * inv, Oh[h].w * inv);
     }
-    if (pv_pending) mbar_wait_bounded(&wc.bar_pv, ppv);
   }
+  if (lane == 0) p.cnt[u] = 0u;  // ready for the next launch
 }
 
-// ---------------------------------------------------------------- the kernel
+// The same with the whole CTA, for a unit end that is the CTA's last item (all four
+// warps are free): thread 96 counts in; if the CTA is the last contributor, warp w
+// merges heads w, w + 4, ...
+template <int GQA>
+__device__ __noinline__ void merge_partials_cta(const DecodeParams& p, int* flag, int u, int i0, int i1, float* outu,
+                                                   int warp, int lane) {
+  const int nc = i1 - i0 + 1;
+  if (warp == 3 && lane == 0) *flag = int(atomic_add_acq_rel_gpu(p.cnt + u, 1u));
+  named_sync();  // the count (and, through it, the other contributors' partials) is seen by all
+  if (*flag != nc - 1) return;
+  const float* pu = p.part + (size_t(i0) + u) * GQA * kPartStride;
+  for (int h = warp; h < GQA; h += 4) merge_heads<1, 8>(pu, size_t(GQA) * kPartStride, nc, h, outu, lane);
+  if (warp == 3 && lane == 0) p.cnt[u] = 0u;  // ready for the next launch
+}
 
 template <typename T, int GQA, int KB, int P>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
-  using C = Cfg<GQA, KB, P>;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ CtaCtl cc;
-  __shared__ WgCtl<P> wctl[kWG];
+__global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
+    decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int NT = GQA > 4 ? 2 : 1;
+  using R = Rec<P, KB>;
+  using S = Smem<GQA, P, KB>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ CtaShared<GQA, P> sh;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int wg = tid >> 7, wt = tid & 127;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
   const int cta = blockIdx.x;
+  // the grid fills every resident slot at once, so the next kernel in the stream may be
+  // scheduled right away: its CTAs take the slots this grid releases
   pdl_wait();
+  pdl_trigger();
 
   // ---------------------------------------------------------------- 1. the weight line
-  // Total weight W, and the lengths of the first kSeqCache sequences.
-  int W = 0;
-  for (int base = 0; base < p.batch; base += kThreads) {
+  // Total weight W; with one sequence per thread (batch <= 128) the per-sequence prefix
+  // and lengths stay in shared memory for locating any position later.
+  int W = 0, x0 = 0, np0 = 0, rl0 = 0;
+  const bool one_pass = p.batch <= kDecodeThreads;
+  for (int base = 0; base < p.batch; base += kDecodeThreads) {
     const int b = base + tid;
     int x = 0;
     if (b < p.batch) {
@@ -1199,125 +955,282 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         for (int i = 0; i < p.Hq * kHeadDim / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       x = max(w, 0) * p.Hkv;
-      if (b < kSeqCache) cc.seq[b] = make_int2(np, rl);
+      np0 = np;
+      rl0 = rl;
     }
+    x0 = x;
     int incl = x;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(kFull, incl, off);
       if (lane >= off) incl += y;
     }
-    if (lane == 31) cc.red[warp] = incl;
+    if (lane == 31) sh.red[warp] = incl;
     __syncthreads();
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) W += cc.red[w];
+    if (one_pass) {
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += sh.red[w];
+      if (b < p.batch) {
+        sh.pref[b] = before + incl - x;
+        sh.seq[b] = make_int2(np0, rl0);
+      }
+    }
+    W += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
     __syncthreads();
   }
   if (W == 0) return;
-  const int n_workers = p.n_ctas * kWG;
-  const int Cw = min(n_workers, max(1, W / 4));  // every range at least one stage long
-  if (cta * kWG >= Cw) return;
 
-  // ---------------------------------------------------------------- 2. locate the ranges
-  // Sequence holding the first position of each worker's range: a second scan of the
-  // weights (from the cache where it holds them).
-  if (tid < kWG) {
-    cc.b0[tid] = -1;
-    cc.base0[tid] = 0;
-  }
-  {
-    int run = 0;
-    for (int base = 0; base < p.batch; base += kThreads) {
-      const int b = base + tid;
-      int x = 0;
-      if (b < p.batch) {
-        int np, rl;
-        x = (b < kSeqCache ? unit_weight_of<P>(cc.seq[b].x, cc.seq[b].y) : max(seq_weight<P>(p, b, np, rl), 0)) *
-            p.Hkv;
-      }
-      int incl = x;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, off);
-        if (lane >= off) incl += y;
-      }
-      __syncthreads();  // the previous round's reads of cc.red are done
-      if (lane == 31) cc.red[warp] = incl;
-      __syncthreads();
-      int start = run + incl - x;
-      for (int w = 0; w < warp; ++w) start += cc.red[w];
-#pragma unroll
-      for (int w = 0; w < kThreads / 32; ++w) run += cc.red[w];
-#pragma unroll
-      for (int g = 0; g < kWG; ++g) {
-        const int pos = range_start(cta * kWG + g, W, Cw);
-        if (x > 0 && start <= pos && pos < start + x) {
-          cc.b0[g] = b;
-          cc.base0[g] = start;
-        }
-      }
-    }
-  }
-
-  // ---------------------------------------------------------------- 3. resources
-  if (warp == 0) tc::alloc(&cc.tmem, 512);
+  // At most W/4 CTAs take part, so that every range is at least one full stage long.
+  Owners ow;
+  ow.W = W;
+  ow.Cs = min(p.n_ctas, max(1, W / 4));
+  if (cta >= ow.Cs) return;
   if (tid == 0) {
-    for (int g = 0; g < kWG; ++g) {
-      for (int s = 0; s < 4; ++s) mbar_init(&wctl[g].full[s], 1);
-      mbar_init(&wctl[g].bar_s, 1);
-      mbar_init(&wctl[g].bar_pv, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      sh.rel[s] = 0;
     }
     fence_mbar_init();
+    sh.abort_flag = 0;
+    sh.issued = 0;
+    sh.tail_u = -1;
   }
-  // operand buffers start at zero (their padding columns are never written again)
-  for (int g = 0; g < kWG; ++g) {
-    uint4* z = reinterpret_cast<uint4*>(smem + g * C::BYTES + C::O_BQK);
-    for (int i = tid; i < (C::O_QH - C::O_BQK) / 16; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
-  }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tmem = cc.tmem;
-  if (warp < 4) {
-    // columns 0..7 of every lane: fp16 0.5, the A operand of the zero-point product
-    uint32_t h[8];
+
+  // Moves sh.cur to the first item at or after position pos (all threads).
+  auto locate = [&](int pos) {
+    if (one_pass) {
+      __syncthreads();
+      if (tid < p.batch) {
+        const int st0 = sh.pref[tid], w = unit_weight_of<P>(sh.seq[tid]) * p.Hkv;
+        if (w > 0 && st0 <= pos && pos < st0 + w) {
+          sh.b0 = tid;
+          sh.base0 = st0;
+        }
+      }
+    } else {
+      int run = 0;
+      for (int base = 0; base < p.batch; base += kDecodeThreads) {
+        const int b = base + tid;
+        int x = 0;
+        if (b < p.batch) x = max(seq_weight<P>(p, b, np0, rl0), 0) * p.Hkv;
+        int incl = x;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) h[i] = 0x38003800u;
-    tc::st<8>(tc::lane_addr(tmem, warp, 0), h);
-    tc::wait_st();
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(kFull, incl, off);
+          if (lane >= off) incl += y;
+        }
+        if (lane == 31) sh.red[warp] = incl;
+        __syncthreads();
+        int before = run;
+        for (int w = 0; w < warp; ++w) before += sh.red[w];
+        const int end = before + incl, start = end - x;
+        if (x > 0 && start <= pos && pos < end) {
+          sh.b0 = b;
+          sh.base0 = start;
+        }
+        run += sh.red[0] + sh.red[1] + sh.red[2] + sh.red[3];
+        __syncthreads();
+      }
+      // lengths of the sequences from the located one on
+      for (int i = tid; i < kSeqCache && sh.b0 + i < p.batch; i += kDecodeThreads) {
+        int np, rl;
+        seq_weight<P>(p, sh.b0 + i, np, rl);
+        sh.seq[i] = make_int2(np, rl);
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      Cursor c;
+      c.b = sh.b0;
+      const int2 v = sh.seq[one_pass ? sh.b0 : 0];
+      c.np = v.x;
+      c.rl = v.y;
+      c.nst = (c.np * P + 127) / 128;
+      c.nres = (c.rl + kPieceTokens - 1) / kPieceTokens;
+      c.k = 0;
+      const int wseq = unit_weight<P>(c);
+      const int off = pos - sh.base0;
+      c.h = off / wseq;
+      c.ubase = sh.base0 + c.h * wseq;
+      cursor_seek<P>(p, c, off - c.h * wseq);
+      sh.cur = c;
+      sh.uord = -1;
+      sh.qslot_cont = 0;
+    }
+    __syncthreads();
+  };
+
+  // ---------------------------------------------------------------- 2. items
+  LaneQ<NT> lq;
+  WarpState<NT> st;
+  float* sO = reinterpret_cast<float*>(smem + S::merge);  // [4][GQA][128]
+  const uint64_t policy = l2_evict_first_policy();
+  int x = 0;  // items of this CTA so far
+  const int owner = cta;
+  const int lo = range_start(cta, ow.W, ow.Cs), hi = range_start(cta + 1, ow.W, ow.Cs);
+  {
+    locate(lo);
+    while (true) {
+      build_segment<GQA, P>(p, sh, hi, ow, tid, one_pass);
+      const int nseg = sh.nseg;
+      if (warp == 0)
+        for (int t = 0; t < min(kStages, nseg); ++t) issue_item<GQA, KB, P>(p, sh, smem, x + t, t, policy, lane);
+      int stg = x % kStages;
+      uint32_t par = uint32_t(x / kStages) & 1u;
+      for (int t = 0; t < nseg; ++t) {
+        const int xi = x + t;
+        const ItemDesc d = sh.desc[t];
+        bool ok = !*reinterpret_cast<volatile int*>(&sh.abort_flag);
+        if (ok && !mbar_wait_bounded(&sh.full_bar[stg], par)) {
+          if (lane == 0) flag_error(p.err, KVQ_DEV_ERR_TIMEOUT);
+          sh.abort_flag = 1;
+          ok = false;
+        }
+        ok = __all_sync(kFull, ok);
+        const uint8_t* sb = smem + stg * S::stage;
+        const uint16_t* qs = sh.q[(d.w >> 11) & 3];
+        const int n = d.w & 0xff;
+        if (d.w & kDescFirst) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const int hB = (g >> 1) + 4 * nt;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+              lq.qv(nt, s, 0) = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd), T()) : 0u;
+              lq.qv(nt, s, 1) = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8), T()) : 0u;
+            }
+          }
+          lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
+          reset_state(st);
+        }
+        if (ok) {
+          if (!(d.w & kDescRes)) {
+            const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
+            if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
+          } else if (int(d.w >> 16) % 4 == warp) {
+            residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, qs, st, lane, p.c_log2);
+          }
+        }
+        // release the stage; the last warp to release it refills it with item xi + kStages
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomic_add_acq_rel_cta(&sh.rel[stg], 1);
+        prev = __shfl_sync(kFull, prev, 0);
+        if (prev == 3) {
+          if (lane == 0) sh.rel[stg] = 0;
+          if (t + kStages < nseg) issue_item<GQA, KB, P>(p, sh, smem, xi + kStages, t + kStages, policy, lane);
+        }
+        if (++stg == kStages) {
+          stg = 0;
+          par ^= 1u;
+        }
+
+        if (d.w & kDescLast) {
+          // ---- merge the four warps' states for this unit
+          named_sync();  // the previous merge no longer reads the merge buffer
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float l = st.l[nt], zv = st.zv[nt];
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+              l += __shfl_xor_sync(kFull, l, off);
+              zv += __shfl_xor_sync(kFull, zv, off);
+            }
+            const int head = qd + 4 * nt;
+            if (g == 0 && head < GQA) {
+              sh.m[warp][head] = st.m[nt];
+              sh.l[warp][head] = l;
+              sh.zv[warp][head] = zv;
+            }
+            if (head < GQA) {
+#pragma unroll
+              for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                  sO[(warp * GQA + head) * kHeadDim + 16 * mc + g + 8 * r] =
+                      st.o[mc][nt][2 * r] + st.o[mc][nt][2 * r + 1];
+            }
+          }
+          named_sync();
+          const int u = d.b * p.Hkv + d.h;
+          const int i0 = int(d.io & 0xffffu), i1 = int(d.io >> 16);
+          const bool sole = i0 == i1;
+          float* outu = p.out + (size_t(d.b) * p.Hq + size_t(d.h) * GQA) * kHeadDim;
+          float* part_me = p.part + (size_t(owner) + u) * GQA * kPartStride;
+          for (int e = tid; e < GQA * kHeadDim; e += kDecodeThreads) {
+            const int h = e >> 7, ch = e & 127;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, sh.m[w][h]);
+            float Ls = 0.0f, O = 0.0f;
+            if (M != -INFINITY) {
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const float f = ex2(sh.m[w][h] - M);
+                Ls += f * sh.l[w][h];
+                O += f * (kCodeScale * sO[(w * GQA + h) * kHeadDim + ch] + sh.zv[w][h]);
+              }
+            }
+            if (sole) {
+              outu[e] = Ls > 0.0f ? O / Ls : 0.0f;
+            } else {
+              float* pp = part_me + h * kPartStride;
+              pp[ch] = O;
+              if (ch == 0) {
+                pp[kHeadDim] = M;
+                pp[kHeadDim + 1] = Ls;
+              }
+            }
+          }
+          if (!sole) {
+            // ---- split merge: the last of the contributors i0..i1 merges their partials.
+            // The barrier orders every thread's partial writes before the counter update,
+            // which is a release at device scope; the merging CTA acquires it.
+            named_sync();
+            if (t == nseg - 1 && !sh.more) {
+              // the CTA's last item: all warps merge, after the loop
+              if (tid == 0) {
+                sh.tail_u = u;
+                sh.tail_io = d.io;
+              }
+            } else if (warp == 3) {
+              merge_partials<GQA>(p, u, i0, i1, outu, lane);
+            }
+          }
+        }
+      }
+      x += nseg;
+      if (!sh.more) break;
+      __syncthreads();  // every item of the segment is consumed before its slots are reused
+    }
   }
-  tc::fence_async_smem();
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  // the grid fills every SM: the next kernel in the stream may be scheduled now
-  pdl_trigger();
 
-  // ---------------------------------------------------------------- 4. the workers
-  const int worker = cta * kWG + wg;
-  if (worker < Cw && cc.b0[wg] >= 0)
-    worker_run<T, GQA, KB, P>(p, cc, wctl[wg], smem + wg * C::BYTES, tmem, W, Cw, worker, wg, wt);
+  named_sync();
+  if (sh.tail_u >= 0) {
+    const int u = sh.tail_u, b = u / p.Hkv, h = u - b * p.Hkv;
+    const uint32_t io = sh.tail_io;
+    merge_partials_cta<GQA>(p, &sh.arrived, u, int(io & 0xffffu), int(io >> 16),
+                            p.out + (size_t(b) * p.Hq + size_t(h) * GQA) * kHeadDim, warp, lane);
+  }
 
-  // ---------------------------------------------------------------- 5. leave
-  tc::fence_before();
+  // ---------------------------------------------------------------- 3. leave
   __syncthreads();
-  if (warp == 0) {
-    tc::fence_after();
-    tc::dealloc(tmem, 512);
+  if (sh.abort_flag && warp == 0) {
+    // copies may still be in flight after a timeout: wait for them (bounded) before the
+    // shared memory is released; the output is undefined and the error word says why
+    const int issued = sh.issued;
+    for (int y = max(0, issued - kStages); y < issued; ++y) {
+      if (lane == 0) mbar_wait_bounded(&sh.full_bar[y % kStages], uint32_t(y / kStages) & 1u);
+    }
   }
 }
 
 // ---------------------------------------------------------------- per-instantiation host side
 
 template <typename T, int GQA, int KB, int P>
-constexpr int smem_bytes() {
-  return kWG * Cfg<GQA, KB, P>::BYTES;
-}
-
-template <typename T, int GQA, int KB, int P>
 cudaError_t prepare_decode() {
   static int seen[64];
-  return ensure_dynamic_smem(decode_kernel<T, GQA, KB, P>, smem_bytes<T, GQA, KB, P>(), seen);
+  return ensure_dynamic_smem(decode_kernel<T, GQA, KB, P>, int(Smem<GQA, P, KB>::bytes), seen);
 }
 
 // Calls f.template operator()<KB, P>() for one (kb, P).
@@ -1348,8 +1261,8 @@ struct DecodeOcc {
   cudaError_t operator()() {
     cudaError_t e = prepare_decode<T, GQA, KB, P>();
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, decode_kernel<T, GQA, KB, P>, kThreads,
-                                                         smem_bytes<T, GQA, KB, P>());
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, decode_kernel<T, GQA, KB, P>, kDecodeThreads,
+                                                         Smem<GQA, P, KB>::bytes);
   }
 };
 
@@ -1362,20 +1275,18 @@ struct DecodeRun {
     if (p.L.record != Rec<P, KB>::record || p.L.payload != Rec<P, KB>::payload) return cudaErrorInvalidValue;
     cudaError_t e = prepare_decode<T, GQA, KB, P>();
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_kernel<T, GQA, KB, P>, dim3(p.n_ctas), dim3(kThreads), smem_bytes<T, GQA, KB, P>(),
+    return launch_pdl(decode_kernel<T, GQA, KB, P>, dim3(p.n_ctas), dim3(kDecodeThreads), Smem<GQA, P, KB>::bytes,
                       stream, p);
   }
 };
 
-}  // namespace dec
-
 // One translation unit per (dtype, GQA) defines these two entry points.
 #define KVQ_DECODE_INSTANCE(NAME, T, GQA)                                                       \
   cudaError_t decode_occupancy_##NAME(int kb, int P, int* n) {                                 \
-    return dec::dispatch_kb_p(kb, P, dec::DecodeOcc<T, GQA>{n});                                \
+    return dispatch_kb_p(kb, P, DecodeOcc<T, GQA>{n});                                          \
   }                                                                                             \
   cudaError_t decode_launch_##NAME(const DecodeParams& p, cudaStream_t stream) {               \
-    return dec::dispatch_kb_p(p.KB, p.P, dec::DecodeRun<T, GQA>{p, stream});                    \
+    return dispatch_kb_p(p.KB, p.P, DecodeRun<T, GQA>{p, stream});                              \
   }
 
 }  // namespace kvq

@@ -15,13 +15,12 @@
 namespace kvq {
 
 // Weights of the decode kernel's work line, in units of one 32-token page group (a page
-// stage of 128 tokens weighs 4): a 32-token residual piece, and the merge at the end
-// of a (sequence, KV head), which is given weight where no item starts.
+// stage of 128 tokens weighs 4).  Measured on B200 (per-CTA traces regressed on the
+// items each CTA held): a 16-token residual piece, which one warp processes while the
+// stage waits for it, costs about as much time as three page groups; the merge at the
+// end of a (sequence, KV head) is given extra weight where no item starts.
 constexpr int kDecodePieceWeight = 3;
-constexpr int kDecodeMergeWeight = 4;
-constexpr int kDecodePieceTokens = 32;
-// Independent workers (warpgroups) per decode CTA; one CTA per SM.
-constexpr int kDecodeWorkersPerCta = 2;
+constexpr int kDecodeMergeWeight = 6;
 
 constexpr int kHeadDim = 128;
 constexpr int kKeyGroup = 32;
@@ -54,13 +53,23 @@ inline Layout make_layout(int P, int D, int k, int G) {
   return L;
 }
 
-// Index of word w of row r in a code section of R rows of W words (see the page-record
-// description in kvq.h): the words of a row go in blocks of V = min(W, 4), and block b
-// of every row precedes block b + 1 of any row, so that consecutive rows' blocks are
-// consecutive 16-byte (or 8- or 4-byte) vectors.
-__host__ __device__ __forceinline__ int word_index(int r, int w, int W, int R) {
-  const int V = W < 4 ? W : 4;
-  return (w / V) * V * R + V * r + (w % V);
+// Storage order of the packed rows (see the page-record description in kvq.h).
+// Key channel c = 16s + 8r + 2q + f  <->  plane-A code position 32q + 4s + 2r + f.
+__host__ __device__ __forceinline__ int key_pos(int c) {
+  return 32 * ((c >> 1) & 3) + 4 * (c >> 4) + 2 * ((c >> 3) & 1) + (c & 1);
+}
+// ... and k_scale / k_zero position 32*(s>>1) + 8q + 4*(s&1) + 2r + f.
+__host__ __device__ __forceinline__ int key_meta_pos(int c) {
+  const int s = c >> 4;
+  return 32 * (s >> 1) + 8 * ((c >> 1) & 3) + 4 * (s & 1) + 2 * ((c >> 3) & 1) + (c & 1);
+}
+// Boosted row j = 16s + 8r + 2q + f  <->  position 4*KB*q + 4s + 2r + f.
+__host__ __device__ __forceinline__ int boost_pos(int j, int KB) {
+  return 4 * KB * ((j >> 1) & 3) + 4 * (j >> 4) + 2 * ((j >> 3) & 1) + (j & 1);
+}
+// Value scale / zero position of token t = 32g + 8u + w: 32g + 4w + u.
+__host__ __device__ __forceinline__ int value_meta_pos(int t) {
+  return (t & ~31) + 4 * (t & 7) + ((t >> 3) & 3);
 }
 // Bit of element e = 8a + 2b + f inside a code word: 8b + 4f + 2a.
 __host__ __device__ __forceinline__ int elem_bit(int e) {

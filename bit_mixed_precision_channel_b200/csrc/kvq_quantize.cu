@@ -249,17 +249,17 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         const int c = c0 + e;
         j[e] = row_of[c];
         qmax[e] = j[e] >= 0 ? 15 : 3;
-        pc[e] = c;
-        pj[e] = j[e] >= 0 ? j[e] : 0;
+        pc[e] = key_pos(c);
+        pj[e] = j[e] >= 0 ? boost_pos(j[e], k / 16) : 0;
         uint16_t sb, zb;
         scale[e] = quant_params<T>(bits_to_float(uint16_t(lob >> (16 * e)), T()),
                                    bits_to_float(uint16_t(hib >> (16 * e)), T()), qmax[e], sb, zb, zero[e]);
         rcp[e] = quant_rcp(scale[e]);
-        // plane A of a boosted channel carries the high bits: scale 4*s4 (exact);
-        // scale and zero entries are [channel or boosted row][group]
-        ks_out[c * n_groups + g] = j[e] >= 0 ? exact_bits(4.0f * scale[e], T()) : sb;
-        kz_out[c * n_groups + g] = zb;
-        if (j[e] >= 0) kbs_out[j[e] * n_groups + g] = sb;
+        // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
+        const int pm = key_meta_pos(c);
+        ks_out[g * kHeadDim + pm] = j[e] >= 0 ? exact_bits(4.0f * scale[e], T()) : sb;
+        kz_out[g * kHeadDim + pm] = zb;
+        if (j[e] >= 0) kbs_out[g * k + j[e]] = sb;
       }
       // codes of the group's 32 tokens; plane A gets code >> 2 for a boosted channel (its
       // low bits go to plane B) and the code itself otherwise; a channel that is not
@@ -351,34 +351,36 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       }
       *reinterpret_cast<uint4*>(cV + t * kHeadDim + 16 * ql) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       if (ql == 0) {
-        vs_out[t] = sb;
-        vz_out[t] = zb;
+        vs_out[value_meta_pos(t)] = sb;
+        vz_out[value_meta_pos(t)] = zb;
       }
     }
   }
   __syncthreads();
 
-  // ---- pack the code planes into the record: position p of a row is element p % 16
-  //      of the row's word p / 16; word w of row r sits at word_index(r, w, W, R)
+  // ---- pack the code planes into the record
   if (mode & kModeKeys) {
     uint32_t* kA = reinterpret_cast<uint32_t*>(rec + p.L.k_codes);
-    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads)
-      kA[word_index(i >> 3, i & 7, kHeadDim / 16, P)] = pack16(cA + 16 * i);
+    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) kA[i] = pack16(cA + 16 * i);
     const int kbw = k / 16;
     uint32_t* kB = reinterpret_cast<uint32_t*>(rec + p.L.kb_codes);
-    for (int i = tid; i < P * kbw; i += kQThreads) kB[word_index(i / kbw, i % kbw, kbw, P)] = pack16(cB + 16 * i);
+    for (int i = tid; i < P * kbw; i += kQThreads) kB[i] = pack16(cB + 16 * i);
   }
   if (need_v) {
-    // value rows are channels, their positions tokens
     uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
-    const int vw = P / 16;
-    for (int i = tid; i < kHeadDim * vw; i += kQThreads) {
-      const int c = i / vw, w = i % vw;
-      const uint8_t* base = cV + (16 * w) * kHeadDim + c;
+    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) {
+      // value-code word i = ((2g + (m >> 2)) * 32 + 4w + q) * 4 + (m & 3): its element
+      // e = 8a + 2b + f holds token 32g + 2q + 16a + 8(b >> 1) + f and channel
+      // 16m + w + 8(b & 1), at bit elem_bit(e)
+      const int mm = i & 3, ln = (i >> 2) & 31, blk = i >> 7;
+      const uint8_t* base = cV + (32 * (blk >> 1) + 2 * (ln & 3)) * kHeadDim + 16 * (4 * (blk & 1) + mm) + (ln >> 2);
       uint32_t word = 0;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) word |= uint32_t(base[e * kHeadDim] & 3u) << elem_bit(e);
-      vq[word_index(c, w, vw, kHeadDim)] = word;
+      for (int e = 0; e < 16; ++e) {
+        const int a = e >> 3, b = (e >> 1) & 3, f = e & 1;
+        word |= uint32_t(base[(16 * a + 8 * (b >> 1) + f) * kHeadDim + 8 * (b & 1)] & 3u) << elem_bit(e);
+      }
+      vq[i] = word;
     }
   }
   pdl_trigger();

@@ -131,7 +131,6 @@ typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 #define KVQ_DEV_ERR_TABLE_FULL   4  /* flush with no free page-table slot or no destination page      */
 #define KVQ_DEV_ERR_TIMEOUT      8  /* a bounded wait for an asynchronous copy gave up                */
 #define KVQ_DEV_ERR_LENGTH      16  /* num_pages[b] or res_len[b] outside its valid range             */
-#define KVQ_DEV_ERR_RANGE       32  /* decode: a folded operand left the fp16 range (see kvq_decode_attention) */
 
 /* Shape and precision of one attention layer's KV cache.
  * Supported: head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8};
