@@ -23,8 +23,9 @@ What it follows (web pages on the method, by title and section):
 
 Readings where the pages are silent (listed again in the design notes):
 scale = (max-min)/(2^b-1) in fp32, rounded up to the storage type; zero = min;
-a fixed storage order inside the packed rows (see kvq_oracle.c: elem_shift,
-word_index; channels of key rows and tokens of value rows in natural order);
+a fixed storage order of channels and tokens inside the packed rows (see
+kvq_oracle.c: elem_shift, key_pos, key_meta_pos, boost_pos, value_slot,
+value_meta_pos);
 round half to even; clamp; scale 0 gives code 0; magnitude = max |x| over the page;
 ties to the lower channel index; boost set per (page, KV head); 4-bit code =
 4*hi + lo; key groups aligned to the page start; residual flushed when it holds a
@@ -83,10 +84,12 @@ def lib():
         L.kvqo_quant_group.restype = None
         L.kvqo_quant_group.argtypes = [u16p, ctypes.c_int, ctypes.c_long, ctypes.c_int,
                                        ctypes.c_int, u8p, u16p, u16p]
-        L.kvqo_elem_shift.restype = ctypes.c_int
-        L.kvqo_elem_shift.argtypes = [ctypes.c_int]
-        L.kvqo_word_index.restype = ctypes.c_long
-        L.kvqo_word_index.argtypes = [ctypes.c_int] * 4
+        for name in ("kvqo_elem_shift", "kvqo_key_pos", "kvqo_key_meta_pos", "kvqo_value_meta_pos"):
+            getattr(L, name).restype = ctypes.c_int
+            getattr(L, name).argtypes = [ctypes.c_int]
+        for name in ("kvqo_boost_pos", "kvqo_value_slot"):
+            getattr(L, name).restype = ctypes.c_int
+            getattr(L, name).argtypes = [ctypes.c_int, ctypes.c_int]
         L.kvqo_layout.restype = None
         L.kvqo_layout.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(ctypes.c_long)]
         L.kvqo_select_boost.restype = None
@@ -152,9 +155,29 @@ def elem_shift(e: int) -> int:
     return lib().kvqo_elem_shift(e)
 
 
-def word_index(r: int, w: int, W: int, R: int) -> int:
-    """Index of word w of row r in a code section of R rows of W words each."""
-    return int(lib().kvqo_word_index(r, w, W, R))
+def key_pos(c: int) -> int:
+    """Storage position of key channel c in plane-A code rows."""
+    return lib().kvqo_key_pos(c)
+
+
+def key_meta_pos(c: int) -> int:
+    """Storage position of key channel c in the plane-A scale and zero rows."""
+    return lib().kvqo_key_meta_pos(c)
+
+
+def boost_pos(j: int, KB: int) -> int:
+    """Storage position of boosted row j in plane-B rows (KB = boosted channels / 16)."""
+    return lib().kvqo_boost_pos(j, KB)
+
+
+def value_slot(t: int, c: int) -> int:
+    """Slot (16 * word + element) of the value code of token t, channel c."""
+    return lib().kvqo_value_slot(t, c)
+
+
+def value_meta_pos(t: int) -> int:
+    """Storage position of token t in the value scale and zero rows."""
+    return lib().kvqo_value_meta_pos(t)
 
 
 LAYOUT_KEYS = ("k_codes", "kb_codes", "v_codes", "k_scale", "k_zero", "kb_scale",

@@ -209,30 +209,70 @@ static int elem_shift(int e) {
   return 8 * b + 4 * f + 2 * a;
 }
 
-/* Index of word w (0..W-1) of row r (0..R-1) inside a code section of R rows of W
- * words.  Position p of a row is element p % 16 of the row's word p / 16 (channels
- * of a key row and tokens of a value row keep their natural order).  The words of
- * a row are taken in blocks of V = min(W, 4) consecutive words, and block b of every
- * row is stored before block b + 1 of any row:
- *   index = (w / V) * V * R + V * r + (w % V).
- * Key rows are tokens (R = P, W = D/16 for plane A and k/16 for plane B); value rows
- * are channels (R = D, W = P/16). */
-static long word_index(int r, int w, int W, int R) {
-  const int V = W < 4 ? W : 4;
-  return (long)(w / V) * V * R + (long)V * r + (w % V);
+/* Storage position of key channel c (0..127) inside a plane-A row and inside the
+ * plane-A scale and zero rows.  Writing c = 16s + 8r + 2q + f (s in 0..7, r, f in
+ * {0,1}, q in 0..3), the position is 32q + 4s + 2r + f. */
+static int key_pos(int c) {
+  const int s = c >> 4, r = (c >> 3) & 1, q = (c >> 1) & 3, f = c & 1;
+  return 32 * q + 4 * s + 2 * r + f;
+}
+
+/* Storage position of boosted row j (0..k-1) inside a plane-B row, KB = k/16:
+ * j = 16s + 8r + 2q + f -> 4*KB*q + 4s + 2r + f. */
+static int boost_pos(int j, int KB) {
+  const int s = j >> 4, r = (j >> 3) & 1, q = (j >> 1) & 3, f = j & 1;
+  return 4 * KB * q + 4 * s + 2 * r + f;
+}
+
+/* Storage position of key channel c inside the plane-A scale and zero rows:
+ * c = 16s + 8r + 2q + f -> 32*(s >> 1) + 8q + 4*(s & 1) + 2r + f. */
+static int key_meta_pos(int c) {
+  const int s = c >> 4, r = (c >> 3) & 1, q = (c >> 1) & 3, f = c & 1;
+  return 32 * (s >> 1) + 8 * q + 4 * (s & 1) + 2 * r + f;
+}
+
+/* Slot (16 * word + element) of the value code of token t (0..P-1) and channel c
+ * (0..127) inside the value-code section.  Writing t = 32g + 16a + 8u + 2q + f and
+ * c = 16m + 8v + w (a, u, v, f in {0,1}, q in 0..3, w in 0..7, m in 0..7), the code is
+ * element 8a + 2(2u + v) + f of word ((2g + (m >> 2)) * 32 + 4w + q) * 4 + (m & 3). */
+static int value_slot(int t, int c) {
+  const int g = t >> 5, a = (t >> 4) & 1, u = (t >> 3) & 1, q = (t >> 1) & 3, f = t & 1;
+  const int m = c >> 4, v = (c >> 3) & 1, w = c & 7;
+  const int word = ((2 * g + (m >> 2)) * 32 + 4 * w + q) * 4 + (m & 3);
+  return 16 * word + 8 * a + 2 * (2 * u + v) + f;
+}
+
+/* Storage position of token t inside the value scale and zero rows:
+ * t = 32g + 8u + w (u in 0..3, w in 0..7) -> 32g + 4w + u. */
+static int value_meta_pos(int t) {
+  const int g = t >> 5, u = (t >> 3) & 3, w = t & 7;
+  return 32 * g + 4 * w + u;
 }
 
 int kvqo_elem_shift(int e) { return elem_shift(e); }
-long kvqo_word_index(int r, int w, int W, int R) { return word_index(r, w, W, R); }
+int kvqo_key_pos(int c) { return key_pos(c); }
+int kvqo_boost_pos(int j, int KB) { return boost_pos(j, KB); }
+int kvqo_key_meta_pos(int c) { return key_meta_pos(c); }
+int kvqo_value_slot(int t, int c) { return value_slot(t, c); }
+int kvqo_value_meta_pos(int t) { return value_meta_pos(t); }
 
-/* Writes / reads the 2-bit code at position pos of row `row` of a section of R rows
- * of W words. */
-static void put2(uint32_t* words, int row, int W, int R, int pos, unsigned code) {
-  words[word_index(row, pos / 16, W, R)] |= (uint32_t)(code & 3u) << elem_shift(pos % 16);
+/* Writes / reads the 2-bit code at storage position pos of row `row` (words_per_row
+ * words of 16 elements each). */
+static void put2(uint32_t* words, int row, int words_per_row, int pos, unsigned code) {
+  words[row * words_per_row + pos / 16] |= (uint32_t)(code & 3u) << elem_shift(pos % 16);
 }
 
-static unsigned get2(const uint32_t* words, int row, int W, int R, int pos) {
-  return (words[word_index(row, pos / 16, W, R)] >> elem_shift(pos % 16)) & 3u;
+static unsigned get2(const uint32_t* words, int row, int words_per_row, int pos) {
+  return (words[row * words_per_row + pos / 16] >> elem_shift(pos % 16)) & 3u;
+}
+
+/* Same for a section addressed by slot = 16 * word + element. */
+static void put2s(uint32_t* words, int slot, unsigned code) {
+  words[slot / 16] |= (uint32_t)(code & 3u) << elem_shift(slot % 16);
+}
+
+static unsigned get2s(const uint32_t* words, int slot) {
+  return (words[slot / 16] >> elem_shift(slot % 16)) & 3u;
 }
 
 /* -------------------------------------------------------------- boost selection (a1) */
@@ -293,42 +333,40 @@ void kvqo_quantize_page(const uint16_t* K, const uint16_t* V, long tok_stride, i
   for (int c = 0; c < D; ++c) row_of[c] = -1;
   for (int j = 0; j < k; ++j) row_of[bidx[j]] = j;
 
-  /* a2: keys, per channel and per group of G tokens.  Code rows are tokens;
-   * scale and zero rows are channels (plane A) or boosted rows (plane B), one entry
-   * per group. */
+  /* a2: keys, per channel and per group of G tokens */
   uint8_t* codes = (uint8_t*)malloc((size_t)(P > D ? P : D));
-  const int kw = D / 16, kbw = k / 16, ng = P / G;
-  for (int g = 0; g < ng; ++g) {
+  const int kw = D / 16, kbw = k / 16;
+  for (int g = 0; g < P / G; ++g) {
     for (int c = 0; c < D; ++c) {
       const uint16_t* col = K + (long)g * G * tok_stride + c;
       uint16_t sb, zb;
       int j = row_of[c];
+      const int pc = key_pos(c);
       if (j < 0) {
         kvqo_quant_group(col, G, tok_stride, 2, dtype, codes, &sb, &zb);
-        for (int t = 0; t < G; ++t) put2(kA, g * G + t, kw, P, c, codes[t]);
-        ks[c * ng + g] = sb;
+        for (int t = 0; t < G; ++t) put2(kA, g * G + t, kw, pc, codes[t]);
+        ks[g * D + key_meta_pos(c)] = sb;
       } else {
         kvqo_quant_group(col, G, tok_stride, 4, dtype, codes, &sb, &zb);
         for (int t = 0; t < G; ++t) {
-          put2(kA, g * G + t, kw, P, c, codes[t] >> 2);
-          put2(kB, g * G + t, kbw, P, j, codes[t] & 3);
+          put2(kA, g * G + t, kw, pc, codes[t] >> 2);
+          put2(kB, g * G + t, kbw, boost_pos(j, kbw), codes[t] & 3);
         }
         /* plane A carries the high bits with four times the 4-bit scale (exact) */
-        ks[c * ng + g] = dt_round(4.0 * dt_value(sb, dtype), dtype, 0);
-        kbs[j * ng + g] = sb;
+        ks[g * D + key_meta_pos(c)] = dt_round(4.0 * dt_value(sb, dtype), dtype, 0);
+        kbs[g * k + j] = sb;
       }
-      kz[c * ng + g] = zb;
+      kz[g * D + key_meta_pos(c)] = zb;
     }
   }
 
-  /* a3: values, per token over all D channels.  Code rows are channels, positions
-   * tokens. */
+  /* a3: values, per token over all D channels */
   for (int t = 0; t < P; ++t) {
     uint16_t sb, zb;
     kvqo_quant_group(V + (long)t * tok_stride, D, 1, 2, dtype, codes, &sb, &zb);
-    for (int c = 0; c < D; ++c) put2(vq, c, P / 16, D, t, codes[c]);
-    vs[t] = sb;
-    vz[t] = zb;
+    for (int c = 0; c < D; ++c) put2s(vq, value_slot(t, c), codes[c]);
+    vs[value_meta_pos(t)] = sb;
+    vz[value_meta_pos(t)] = zb;
   }
   free(codes);
   free(row_of);
@@ -348,25 +386,27 @@ void kvqo_dequantize_page(const uint8_t* rec, int P, int D, int G, int k, int dt
   const uint16_t* vs = (const uint16_t*)(rec + L.v_scale);
   const uint16_t* vz = (const uint16_t*)(rec + L.v_zero);
   const uint8_t* bidx = rec + L.boost_idx;
-  const int kw = D / 16, kbw = k / 16, ng = P / G;
+  const int kw = D / 16, kbw = k / 16;
   if (Khat) {
     for (int t = 0; t < P; ++t) {
       int g = t / G;
       for (int c = 0; c < D; ++c) {
-        unsigned a = get2(kA, t, kw, P, c);
-        Khat[t * D + c] = a * dt_value(ks[c * ng + g], dtype) + dt_value(kz[c * ng + g], dtype);
+        const int pm = key_meta_pos(c);
+        unsigned a = get2(kA, t, kw, key_pos(c));
+        Khat[t * D + c] = a * dt_value(ks[g * D + pm], dtype) + dt_value(kz[g * D + pm], dtype);
       }
       for (int j = 0; j < k; ++j) {
-        unsigned b = get2(kB, t, kbw, P, j);
-        Khat[t * D + bidx[j]] += b * dt_value(kbs[j * ng + g], dtype);
+        unsigned b = get2(kB, t, kbw, boost_pos(j, kbw));
+        Khat[t * D + bidx[j]] += b * dt_value(kbs[g * k + j], dtype);
       }
     }
   }
   if (Vhat) {
     for (int t = 0; t < P; ++t)
       for (int c = 0; c < D; ++c) {
-        unsigned v = get2(vq, c, P / 16, D, t);
-        Vhat[t * D + c] = v * dt_value(vs[t], dtype) + dt_value(vz[t], dtype);
+        unsigned v = get2s(vq, value_slot(t, c));
+        const int pv = value_meta_pos(t);
+        Vhat[t * D + c] = v * dt_value(vs[pv], dtype) + dt_value(vz[pv], dtype);
       }
   }
 }

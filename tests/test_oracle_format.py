@@ -31,39 +31,82 @@ def _shift(e):
     return 8 * ((e >> 1) & 3) + 4 * (e & 1) + 2 * (e >> 3)
 
 
-def _word_index(r, w, W, R):
-    """word w of row r of a section of R rows of W words: (w // V) * V * R + V * r + w % V,
-    V = min(W, 4)"""
-    V = min(W, 4)
-    r, w = np.asarray(r), np.asarray(w)
-    return (w // V) * V * R + V * r + w % V
+def _key_channel(p):
+    """inverse of the key storage order: position 32q + 4s + 2r + f -> channel 16s + 8r + 2q + f"""
+    p = np.asarray(p)
+    q, s, r, f = p >> 5, (p >> 2) & 7, (p >> 1) & 1, p & 1
+    return 16 * s + 8 * r + 2 * q + f
 
 
-def _section_rows(words, W, R):
-    """section of R rows of W words -> [R][16 * W] codes by position (natural order)"""
+def _boost_row(p, KB):
+    p = np.asarray(p)
+    q, rem = p // (4 * KB), p % (4 * KB)
+    s, r, f = rem >> 2, (rem >> 1) & 1, rem & 1
+    return 16 * s + 8 * r + 2 * q + f
+
+
+def _key_meta_channel(p):
+    """inverse of the scale/zero order: position 32i + 8q + 4j + 2r + f -> channel 16(2i + j) + 8r + 2q + f"""
+    p = np.asarray(p)
+    i, q, j, r, f = p >> 5, (p >> 3) & 3, (p >> 2) & 1, (p >> 1) & 1, p & 1
+    return 16 * (2 * i + j) + 8 * r + 2 * q + f
+
+
+def _value_token_channel(slot):
+    """inverse of the value-code order: slot 16*word + element -> (token, channel), with
+    word = ((2g + n) * 32 + 4w + q) * 4 + mm, element = 8a + 2(2u + v) + f,
+    token 32g + 16a + 8u + 2q + f, channel 16(4n + mm) + 8v + w"""
+    slot = np.asarray(slot)
+    word, e = slot >> 4, slot & 15
+    mm, lane, blk = word & 3, (word >> 2) & 31, word >> 7
+    g, n = blk >> 1, blk & 1
+    w, q = lane >> 2, lane & 3
+    a, b, f = e >> 3, (e >> 1) & 3, e & 1
+    u, v = b >> 1, b & 1
+    return 32 * g + 16 * a + 8 * u + 2 * q + f, 16 * (4 * n + mm) + 8 * v + w
+
+
+def _value_meta_token(p):
+    """inverse of the value scale/zero order: position 32g + 4w + u -> token 32g + 8u + w"""
+    p = np.asarray(p)
+    g, w, u = p >> 5, (p >> 2) & 7, p & 3
+    return 32 * g + 8 * u + w
+
+
+def _words_to_positions(words):
+    """[rows][n_words] uint32 -> [rows][16 * n_words] codes by storage position"""
     w = np.asarray(words, np.uint32)
-    rr, ww = np.meshgrid(np.arange(R), np.arange(W), indexing="ij")
-    rows = w[_word_index(rr, ww, W, R)]  # [R][W]
     e = np.arange(16)
-    return ((rows[..., None] >> _shift(e).astype(np.uint32)) & 3).reshape(R, 16 * W)
+    return ((w[..., None] >> _shift(e).astype(np.uint32)) & 3).reshape(w.shape[0], -1)
 
 
 def _decode_record(rec, P, k, dtype):
     """-> dict of planes in natural order: kA [P][128], kB [P][k], v [P][128], scales..."""
     L = oracle.layout(P, 128, k, 32)
-    KB, ng = k // 16, P // 32
+    KB = k // 16
     u16 = lambda a, b: rec[a:b].view(np.uint16)
-    kA = _section_rows(rec[L["k_codes"]:L["kb_codes"]].view(np.uint32), 8, P).astype(np.int64)
+    kA_pos = _words_to_positions(rec[L["k_codes"]:L["kb_codes"]].view(np.uint32).reshape(P, 8))
+    kA = np.zeros((P, 128), np.int64)
+    kA[:, _key_channel(np.arange(128))] = kA_pos
     kB = np.zeros((P, k), np.int64)
     if k:
-        kB = _section_rows(rec[L["kb_codes"]:L["v_codes"]].view(np.uint32), KB, P).astype(np.int64)
-    v = _section_rows(rec[L["v_codes"]:L["k_scale"]].view(np.uint32), P // 16, 128).T.astype(np.int64)
-    return dict(kA=kA, kB=kB, v=v,
-                ks=u16(L["k_scale"], L["k_zero"]).reshape(128, ng).T,
-                kz=u16(L["k_zero"], L["kb_scale"]).reshape(128, ng).T,
-                kbs=u16(L["kb_scale"], L["v_scale"]).reshape(k, ng).T,
-                vs=u16(L["v_scale"], L["v_zero"]), vz=u16(L["v_zero"], L["boost_idx"]),
-                idx=rec[L["boost_idx"]:L["boost_idx"] + k])
+        kB_pos = _words_to_positions(rec[L["kb_codes"]:L["v_codes"]].view(np.uint32).reshape(P, KB))
+        kB[:, _boost_row(np.arange(k), KB)] = kB_pos
+    v_slots = _words_to_positions(rec[L["v_codes"]:L["k_scale"]].view(np.uint32)[None, :])[0]
+    v = np.zeros((P, 128), np.int64)
+    tok, ch = _value_token_channel(np.arange(P * 128))
+    v[tok, ch] = v_slots
+    ks = np.zeros((P // 32, 128), np.uint16)
+    kz = np.zeros((P // 32, 128), np.uint16)
+    ks[:, _key_meta_channel(np.arange(128))] = u16(L["k_scale"], L["k_zero"]).reshape(P // 32, 128)
+    kz[:, _key_meta_channel(np.arange(128))] = u16(L["k_zero"], L["kb_scale"]).reshape(P // 32, 128)
+    vs = np.zeros(P, np.uint16)
+    vz = np.zeros(P, np.uint16)
+    vs[_value_meta_token(np.arange(P))] = u16(L["v_scale"], L["v_zero"])
+    vz[_value_meta_token(np.arange(P))] = u16(L["v_zero"], L["boost_idx"])
+    return dict(kA=kA, kB=kB, v=v, ks=ks, kz=kz,
+                kbs=u16(L["kb_scale"], L["v_scale"]).reshape(P // 32, k),
+                vs=vs, vz=vz, idx=rec[L["boost_idx"]:L["boost_idx"] + k])
 
 
 # -------------------------------------------------------------------------- pins
@@ -80,27 +123,43 @@ def test_layout_sizes_hand_worked(row):
     assert all(o % 16 == 0 for o in offs[:-1])
 
 
-def test_word_index_hand_worked():
+def test_storage_positions_hand_worked():
     g = _golden()
-    for r, w, W, R, idx in g["word_index"]:
-        assert oracle.word_index(r, w, W, R) == idx
-        assert int(_word_index(r, w, W, R)) == idx
-    # every section's word order is a permutation of its words
-    for W in (1, 2, 4, 8):
-        for R in (32, 64, 128):
-            got = sorted(oracle.word_index(r, w, W, R) for r in range(R) for w in range(W))
-            assert got == list(range(W * R))
+    for c, p in g["key_pos"]:
+        assert oracle.key_pos(c) == p
+    for KB, j, p in g["boost_pos"]:
+        assert oracle.boost_pos(j, KB) == p
+    for c, p in g["key_meta_pos"]:
+        assert oracle.key_meta_pos(c) == p
+    for t, c, word, elem in g["value_slot"]:
+        assert oracle.value_slot(t, c) == 16 * word + elem
+    for t, p in g["value_meta_pos"]:
+        assert oracle.value_meta_pos(t) == p
+    # each order is a permutation, and inverts the decoder's reading of the rule
+    assert sorted(oracle.key_pos(c) for c in range(128)) == list(range(128))
+    assert all(_key_channel(oracle.key_pos(c)) == c for c in range(128))
+    for KB in (1, 2, 4, 8):
+        assert sorted(oracle.boost_pos(j, KB) for j in range(16 * KB)) == list(range(16 * KB))
+        assert all(_boost_row(oracle.boost_pos(j, KB), KB) == j for j in range(16 * KB))
+    assert sorted(oracle.key_meta_pos(c) for c in range(128)) == list(range(128))
+    assert all(_key_meta_channel(oracle.key_meta_pos(c)) == c for c in range(128))
+    slots = [oracle.value_slot(t, c) for t in range(128) for c in range(128)]
+    assert sorted(slots) == list(range(128 * 128))
+    tok, ch = _value_token_channel(np.array(slots))
+    assert (tok == np.repeat(np.arange(128), 128)).all() and (ch == np.tile(np.arange(128), 128)).all()
+    assert sorted(oracle.value_meta_pos(t) for t in range(128)) == list(range(128))
+    assert all(_value_meta_token(oracle.value_meta_pos(t)) == t for t in range(128))
     assert [oracle.elem_shift(e) for e in range(16)] == list(_shift(np.arange(16)))
 
 
 @pytest.mark.parametrize("case", _golden()["words"], ids=lambda c: c["word"])
 def test_key_word_packing_hand_worked(case):
-    """Word 0 of token row 0 holds key channels 0..15 (element e = channel e); give
+    """Word 0 of token row 0 holds the key channels stored at positions 0..15; give
     element e the code case["codes"][e] through a real page and read the word back."""
     cfg = oracle.Cfg(P=32, k=0)
     K = np.zeros((cfg.P, cfg.D), np.float32)
     for e, code in enumerate(case["codes"]):
-        c = e
+        c = int(_key_channel(e))
         K[0, c] = code
         K[1, c] = 3.0  # the group spans [0, 3]: scale 1, zero 0
     rec = oracle.quantize_page(syn.to_bits(K, F16), syn.to_bits(np.zeros_like(K), F16), cfg)
@@ -110,12 +169,14 @@ def test_key_word_packing_hand_worked(case):
 
 @pytest.mark.parametrize("case", _golden()["words"], ids=lambda c: c["word"])
 def test_value_word_packing_hand_worked(case):
-    """Word 0 of the value codes is word 0 of channel row 0: element e = token e."""
+    """Word 0 of the value codes holds element e = 8a + 2(2u + v) + f <-> token 16a + 8u + f,
+    channel 8v."""
     cfg = oracle.Cfg(P=32, k=0)
     V = np.zeros((cfg.P, cfg.D), np.float32)
     V[:, 1] = 3.0  # every token's range is [0, 3]: scale 1, zero 0
     for e, code in enumerate(case["codes"]):
-        V[e, 0] = code
+        a, b, f = e >> 3, (e >> 1) & 3, e & 1
+        V[16 * a + 8 * (b >> 1) + f, 8 * (b & 1)] = code
     rec = oracle.quantize_page(np.zeros((cfg.P, cfg.D), np.uint16), syn.to_bits(V, F16), cfg)
     L = oracle.layout(cfg.P, cfg.D, cfg.k, cfg.G)
     assert int(rec[L["v_codes"]:L["v_codes"] + 4].view(np.uint32)[0]) == int(case["word"], 16)
