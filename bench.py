@@ -42,9 +42,9 @@ import numpy as np  # noqa: E402
 
 WORKLOAD = "llama3_8b"
 # DRAM traffic of one decode launch of this workload (dram__bytes_read.sum +
-# dram__bytes_write.sum from the ncu capture summarised in
-# profiles/decode_kernel_llama3_8b_layer.md), valid only for the kernel source it was taken
-# on: the bench reports it when the decode kernel source still hashes to this value.
+# dram__bytes_write.sum from one ncu capture of the decode kernel), valid only for the
+# kernel source it was taken on: the bench reports it while the decode kernel source
+# still hashes to this value.
 DECODE_TRAFFIC = {"source_sha256": "2907ee8123ed9e830983202970f4c4daaee50fab223ba8799a67ab423954aabb",
                   "bytes": 50294016 + 100352}
 LAYERS = 32
@@ -59,6 +59,7 @@ def parse():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload measurements")
     return ap.parse_args()
 
 
@@ -469,6 +470,16 @@ def run_gpu(args):
         "gpu_launches": args.steps * L_layers * 4,
         "clocks": clock_info,
     }
+    if world == 1 and not args.no_configs:
+        cfgs = {WORKLOAD: {"decode_us_per_launch": round(attn_ms * 1e3, 2), "decode_gbs": round(achieved, 1),
+                           "frac": round(achieved / peak, 4), "bytes_per_launch": bytes_attn,
+                           "replicas": L_layers, "quantize_tokens_per_s": round(quant_tokens_per_s, 1),
+                           "quantize_gbs": result["quantize"]["gbs"]}}
+        cfgs[WORKLOAD + "_l2_flushed"] = l2_flushed_single(dev, peak)
+        cfgs["qwen3_8b_long"] = workload_bench("qwen3_8b_long", dev, peak)
+        cfgs["llama3_70b_batch"] = workload_bench("llama3_70b_batch", dev, peak)
+        cfgs["ragged_serving"] = workload_bench("ragged_serving", dev, peak, flush_steps=256)
+        result["configs"] = cfgs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # every step appended the same k_new / v_new, so the windows hold copies of them
         rk = np.repeat(kn[:, :, None, :], res_end, axis=2)
@@ -479,6 +490,194 @@ def run_gpu(args):
         del g_step, g_attn, g_e2e
         dist.destroy_process_group()
     return result if rank == 0 else None
+
+
+# ------------------------------------------------------------------ the other workloads
+
+def _device_prompts(w, lens, sigma_dev, gen, tdt, dev):
+    """Seeded synthetic prompts drawn on the device with the workload's distributions
+    (keys N(0,1) x per-channel sigma, values N(0,1)); the values differ from the numpy
+    streams the parity tests use, the distributions do not."""
+    for b, L in enumerate(lens):
+        K = (torch_randn((int(L), w.Hkv, w.D), gen, dev) * sigma_dev).to(tdt)
+        V = torch_randn((int(L), w.Hkv, w.D), gen, dev).to(tdt)
+        yield b, K, V
+
+
+def torch_randn(shape, gen, dev):
+    import torch
+    return torch.randn(shape, generator=gen, device=dev)
+
+
+def workload_bench(name, dev, peak, min_bytes=512e6, flush_steps=0, iters=20):
+    """Decode attention (and quantize) throughput of one workload on one GPU.
+    Replicas of the layer cache are added until the packed pages exceed min_bytes (four
+    times the L2), and the decode launches cycle through them."""
+    import torch
+
+    from bit_mixed_precision_channel_b200 import binding as kb
+    from bit_mixed_precision_channel_b200 import synthetic as syn
+    from bit_mixed_precision_channel_b200.cache import PagedKVCache
+
+    w = syn.WORKLOADS[name]
+    cfg = kb.Config(head_dim=w.D, num_q_heads=w.Hq, num_kv_heads=w.Hkv, page_tokens=w.P, key_group=w.G,
+                    num_boost=w.k, dtype=w.dtype)
+    tdt = kb.torch_dtype(w.dtype)
+    lens = syn.lengths(w)
+    B, P, H = w.batch, w.P, w.Hkv
+    payload = kb.page_layout(cfg)["payload_bytes"]
+    page_bytes = int(sum(lens // P)) * H * payload
+    # replicas cycle through identical lengths; the flush steps run on a single cache
+    replicas = 1 if flush_steps else max(1, math.ceil(min_bytes / page_bytes))
+    max_pages = int(max(lens) // P + flush_steps // P + 2)
+    pool_pages = int(sum(lens // P) + B * (flush_steps // P + 2))
+    sigma = torch.from_numpy(syn.key_channel_sigma(w)).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    caches = []
+    q_ms = 0.0
+    for r in range(replicas):
+        c = PagedKVCache(cfg, B, max_pages, pool_pages, device=dev, page_order=syn.page_order(w, pool_pages))
+        full_k, full_v, dsts = [], [], []
+        for b, K, V in _device_prompts(w, lens, sigma, gen, tdt, dev):
+            c.prefill(b, K, V)
+            n = int(lens[b]) // P
+            if r == 0 and n:
+                full_k.append(K[:n * P])
+                full_v.append(V[:n * P])
+                dsts += c.host_pages[b][:n]
+        if r == 0:
+            # quantize: every full page of the workload in one launch, into the pages the
+            # prefill assigned (the same records again)
+            fk, fv = torch.cat(full_k), torch.cat(full_v)
+            dst = torch.tensor(dsts, dtype=torch.int32, device=dev)
+            srck, srcv = kb.Source.token_major(fk, cfg), kb.Source.token_major(fv, cfg)
+            for _ in range(2):
+                kb.quantize_pages(cfg, srck, srcv, dst, c.pool, c.err)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(5):
+                kb.quantize_pages(cfg, srck, srcv, dst, c.pool, c.err)
+            e1.record()
+            torch.cuda.synchronize()
+            q_ms = e0.elapsed_time(e1) / 5
+            n_tok = int(fk.shape[0])
+            del fk, fv, full_k, full_v
+        caches.append(c)
+    q = (torch_randn((B, w.Hq, w.D), gen, dev)).to(tdt)
+    out = torch.empty(B, w.Hq, w.D, device=dev)
+    res = {}
+    # flush rate (ragged serving): eager decode steps, the flush calls timed alone
+    if flush_steps:
+        c = caches[0]
+        kn = (torch_randn((B, H, w.D), gen, dev) * sigma).to(tdt)
+        vn = torch_randn((B, H, w.D), gen, dev).to(tdt)
+        flushed, f_ms = 0, 0.0
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(flush_steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for s in range(flush_steps):
+            fl = c.reserve_flush_pages()
+            c.append(kn, vn)
+            ev[s][0].record()
+            c.flush()
+            ev[s][1].record()
+            c.attend(q, out)
+            c.commit_host(fl)
+            flushed += len(fl)
+        t1.record()
+        torch.cuda.synchronize()
+        f_ms = sum(a.elapsed_time(b) for a, b in ev)
+        res["flush"] = {"steps": flush_steps, "flushed_pages": flushed * H, "flush_ms_total": round(f_ms, 3),
+                        "flush_ms_per_step": round(f_ms / flush_steps, 4),
+                        "flushed_page_heads_per_s": round(flushed * H / (f_ms * 1e-3), 1),
+                        "step_ms_eager": round(t0.elapsed_time(t1) / flush_steps, 4),
+                        "what": "append + flush + attend per step; the flush calls (quantize of full "
+                                "windows + page-table commit) timed with events around them"}
+        assert c.check_errors() == 0
+    for c in caches:
+        c.attend(q, out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in caches:
+            c.attend(q, out)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / iters / replicas
+    c = caches[0]
+    nps = c.num_pages.cpu().numpy().astype(np.int64)
+    rls = c.res_len.cpu().numpy().astype(np.int64)
+    nbytes = int(H * (nps * payload).sum() + H * rls.sum() * 2 * w.D * 2 + B * w.Hq * w.D * (2 + 4)
+                 + 4 * nps.sum() + 8 * B)
+    for c in caches:
+        assert c.check_errors() == 0
+    res.update({"decode_us_per_launch": round(ms * 1e3, 2), "decode_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4), "bytes_per_launch": nbytes,
+                "replicas": replicas, "tokens": int(lens.sum()),
+                "quantize_tokens_per_s": round(n_tok / (q_ms * 1e-3), 1),
+                "quantize_gbs": round((n_tok * H * w.D * 2 * 2 + (n_tok // P) * H * payload) / (q_ms * 1e-3) / 1e9, 1),
+                "quantize_ms": round(q_ms, 4)})
+    del caches, g
+    torch.cuda.empty_cache()
+    return res
+
+
+def l2_flushed_single(dev, peak, iters=20):
+    """Config 2 with one layer cache (50 MB, inside the L2) and a 512 MB write between
+    the timed launches, outside the timed region, so every launch reads from HBM."""
+    import torch
+
+    from bit_mixed_precision_channel_b200 import binding as kb
+    from bit_mixed_precision_channel_b200 import synthetic as syn
+    from bit_mixed_precision_channel_b200.cache import PagedKVCache
+
+    w = syn.WORKLOADS[WORKLOAD]
+    cfg = kb.Config(head_dim=w.D, num_q_heads=w.Hq, num_kv_heads=w.Hkv, page_tokens=w.P, key_group=w.G,
+                    num_boost=w.k, dtype=w.dtype)
+    tdt = kb.torch_dtype(w.dtype)
+    B, P, H = w.batch, w.P, w.Hkv
+    payload = kb.page_layout(cfg)["payload_bytes"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    sigma = torch.from_numpy(syn.key_channel_sigma(w)).to(dev)
+    c = PagedKVCache(cfg, B, w.context // P + 2, B * (w.context // P + 2), device=dev)
+    K = (torch_randn((B, w.context, H, w.D), gen, dev) * sigma).to(tdt)
+    V = torch_randn((B, w.context, H, w.D), gen, dev).to(tdt)
+    c.prefill_batch(K, V)
+    del K, V
+    q = torch_randn((B, w.Hq, w.D), gen, dev).to(tdt)
+    out = torch.empty(B, w.Hq, w.D, device=dev)
+    scrub = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        c.attend(q, out)
+    tot = 0.0
+    for _ in range(iters):
+        scrub.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        c.attend(q, out)
+        b.record()
+        torch.cuda.synchronize()
+        tot += a.elapsed_time(b)
+    ms = tot / iters
+    nbytes = B * H * (w.context // P) * payload + B * w.Hq * w.D * 6 + 4 * B * (w.context // P) + 8 * B
+    assert c.check_errors() == 0
+    return {"decode_us_per_launch": round(ms * 1e3, 2), "decode_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4), "bytes_per_launch": nbytes,
+            "what": "one layer cache, a 512 MB write between launches (outside the timed region), "
+                    "each launch timed alone with events"}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -498,7 +697,8 @@ def workload_config(w, layers, world, payload):
 
 def run_reference(args):
     """The oracle as the reference implementation: each step decodes a bounded sample
-    (8 sequence x kv-head units) of the same workload on the host cores."""
+    (one sequence x kv-head unit per host thread, at least 8) of the same workload on the
+    host cores."""
     import concurrent.futures as cf
 
     import oracle
@@ -513,7 +713,8 @@ def run_reference(args):
     n_pages = w.context // P
     sigma = syn.key_channel_sigma(w)
     threads = max(1, min(os.cpu_count() or 1, 32))
-    units = [(b, h) for b in range(2) for h in range(w.Hkv)][:8]
+    # at least one unit per thread, so that every host core has work
+    units = [(b, h) for b in range(w.batch) for h in range(w.Hkv)][:max(threads, 8)]
     Ks = {b: syn.keys(w, b, 0, w.context, sigma) for b in {u[0] for u in units}}
     Vs = {b: syn.values(w, b, 0, w.context) for b in Ks}
     pools = {}

@@ -22,7 +22,7 @@ __all__ = [
     "decode_workspace_bytes", "decode_attention", "decode_attention_static", "STATIC_SCRATCH_BYTES",
     "F16", "BF16", "torch_dtype",
     "DEV_ERR_PAGE_RANGE", "DEV_ERR_RESIDUAL", "DEV_ERR_TABLE_FULL", "DEV_ERR_TIMEOUT",
-    "DEV_ERR_LENGTH",
+    "DEV_ERR_LENGTH", "DEV_ERR_RANGE",
 ]
 
 F16 = 0
@@ -32,6 +32,7 @@ DEV_ERR_RESIDUAL = 2
 DEV_ERR_TABLE_FULL = 4
 DEV_ERR_TIMEOUT = 8
 DEV_ERR_LENGTH = 16
+DEV_ERR_RANGE = 32
 STATIC_SCRATCH_BYTES = 16 << 20  # KVQ_STATIC_SCRATCH_BYTES
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -170,10 +171,28 @@ def _check(fn: str, status: int):
         raise KVQError(fn, status)
 
 
-def _cuda(*tensors):
+def _cuda(*tensors, stream=None):
+    """Every tensor must be device memory of one device, the current one: the library
+    launches on the current device and its stream, and a pointer into another GPU's
+    memory would fault there instead of failing cleanly."""
+    dev = None
     for t in tensors:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("kvq calls take CUDA tensors (device memory)")
+        if dev is None:
+            dev = t.device.index
+        elif t.device.index != dev:
+            raise ValueError(f"kvq calls take tensors of one device: cuda:{dev} and cuda:{t.device.index}")
+    if dev is None:
+        return
+    cur = torch.cuda.current_device()
+    if dev != cur:
+        raise ValueError(f"tensors are on cuda:{dev} but the current device is cuda:{cur}; "
+                         f"make the call under torch.cuda.device({dev})")
+    if stream is not None and getattr(stream, "device", None) is not None and stream.device.index != dev:
+        raise ValueError(f"stream of cuda:{stream.device.index} for tensors on cuda:{dev}")
 
 
 def _need(name: str, t, dtype=None, numel: int | None = None, dim: int | None = None):
@@ -225,7 +244,8 @@ def _quant(fn, cfg, src_k, src_v, dst_pages, pool, err, stream):
     _need("err", err, torch.int32, 1)
     _need_source("k source", src_k, cfg, dst_pages.numel())
     _need_source("v source", src_v, cfg, dst_pages.numel())
-    _cuda(dst_pages, pool, err)
+    _cuda(dst_pages, pool, err, src_k.tensor if src_k is not None else None,
+          src_v.tensor if src_v is not None else None, stream=stream)
     pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
     L = load()
     n = dst_pages.numel()
@@ -268,7 +288,7 @@ def append_token(cfg: Config, k_new, v_new, res_k, res_v, res_len, err=None, str
     _need("res_k", res_k, dt, batch * H * P * D)
     _need("res_v", res_v, dt, batch * H * P * D)
     _need("err", err, torch.int32, 1)
-    _cuda(k_new, v_new, res_k, res_v, res_len, err)
+    _cuda(k_new, v_new, res_k, res_v, res_len, err, stream=stream)
     _check("kvq_append_token", load().kvq_append_token(
         ctypes.byref(cfg.c()), batch, k_new.data_ptr(), v_new.data_ptr(), res_k.data_ptr(),
         res_v.data_ptr(), res_len.data_ptr(), _ptr(err), _stream(stream)))
@@ -285,7 +305,7 @@ def flush_residual(cfg: Config, res_k, res_v, res_len, new_page, page_table, num
         _need(name, t, torch.int32, batch)
     _need("pool", pool, torch.uint8)
     _need("err", err, torch.int32, 1)
-    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err)
+    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err, stream=stream)
     pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
     _check("kvq_flush_residual", load().kvq_flush_residual(
         ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
@@ -315,7 +335,7 @@ def decode_attention(cfg: Config, pool, q, page_table, num_pages, res_k, res_v, 
                      workspace, sm_scale: float | None = None, err=None, stream=None):
     _need_decode(cfg, pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
     _need("workspace", workspace, torch.uint8)
-    _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, workspace, err)
+    _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, workspace, err, stream=stream)
     batch, max_pages = page_table.shape
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(cfg.head_dim)
@@ -334,7 +354,7 @@ def decode_attention_static(cfg: Config, pool, q, page_table, num_pages, res_k, 
     Calls on one device share that buffer, so they must not overlap on the GPU; the
     first call on a device must not be made during stream capture."""
     _need_decode(cfg, pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
-    _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, err)
+    _cuda(pool, q, page_table, num_pages, res_k, res_v, res_len, out, err, stream=stream)
     batch, max_pages = page_table.shape
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(cfg.head_dim)

@@ -45,6 +45,28 @@ static Plan decode_plan(const kvq_config* cfg, int batch) {
   return pl;
 }
 
+// Every host-side check of a decode call except the workspace (shared by the
+// workspace and static-scratch entry points, so both reject the same calls before
+// enqueuing anything).
+kvq_status decode_check_args(const kvq_config* cfg, const void* pool, int64_t pool_pages, const void* q,
+                             int32_t batch, const int32_t* page_table, int32_t max_pages, const int32_t* num_pages,
+                             const void* res_k, const void* res_v, const int32_t* res_len, const float* out) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!pool || pool_pages <= 0 || !q || !num_pages || !res_k || !res_v || !res_len || !out) return KVQ_ERR_INVALID_ARG;
+  if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(q) || !aligned16(res_k) || !aligned16(res_v)) return KVQ_ERR_INVALID_ARG;
+  // the kernel's work line (32-token groups, weighted 16-token residual pieces and a
+  // merge weight per (sequence, kv head)) is indexed with 32-bit integers
+  const long long line = (long long)batch * cfg->num_kv_heads *
+                         ((long long)max_pages * (cfg->page_tokens / 32) +
+                          (long long)kDecodePieceWeight * ((cfg->page_tokens + 15) / 16) + kDecodeMergeWeight);
+  if (line >= (1ll << 31)) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
 }  // namespace kvq
 
 using namespace kvq;
@@ -227,21 +249,11 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
                                 const int32_t* num_pages, const void* res_k, const void* res_v,
                                 const int32_t* res_len, float sm_scale, float* out, void* workspace,
                                 size_t workspace_bytes, int32_t* err, cudaStream_t stream) {
-  const kvq_status s = kvq_check_config(cfg);
+  const kvq_status s = decode_check_args(cfg, pool, pool_pages, q, batch, page_table, max_pages, num_pages, res_k,
+                                         res_v, res_len, out);
   if (s != KVQ_OK) return s;
-  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
   if (batch == 0) return KVQ_OK;
-  if (!pool || pool_pages <= 0 || !q || !num_pages || !res_k || !res_v || !res_len || !out || !workspace)
-    return KVQ_ERR_INVALID_ARG;
-  if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
-  if (!aligned16(pool) || !aligned16(q) || !aligned16(res_k) || !aligned16(res_v) || !aligned16(workspace))
-    return KVQ_ERR_INVALID_ARG;
-  // the kernel's work line (32-token groups, weighted 16-token residual pieces and a
-  // merge weight per (sequence, kv head)) is indexed with 32-bit integers
-  const long long line = (long long)batch * cfg->num_kv_heads *
-                         ((long long)max_pages * (cfg->page_tokens / 32) +
-                          (long long)kDecodePieceWeight * ((cfg->page_tokens + 15) / 16) + kDecodeMergeWeight);
-  if (line >= (1ll << 31)) return KVQ_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
   const Plan pl = decode_plan(cfg, batch);
   if (workspace_bytes < pl.part_bytes + pl.cnt_bytes) return KVQ_ERR_CAPACITY;
   const int gqa = cfg->num_q_heads / cfg->num_kv_heads;

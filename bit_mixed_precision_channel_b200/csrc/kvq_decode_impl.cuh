@@ -96,6 +96,18 @@ __device__ __forceinline__ uint32_t to_f16x2(uint32_t x, __nv_bfloat16) {
   return d;
 }
 
+// A query pair of the cache dtype scaled by 2^-e, as fp16: for fp16 one exact product
+// (2^-e >= 2^-24 is an fp16 number); for bf16 through fp32, so that queries beyond
+// fp16's range are scaled before they are rounded.
+__device__ __forceinline__ uint32_t scale_q2(uint32_t q2, uint32_t sbq, float, __half) {
+  return h2_as_u32(__hmul2(u32_as_h2(q2), u32_as_h2(sbq)));
+}
+__device__ __forceinline__ uint32_t scale_q2(uint32_t q2, uint32_t, float sc, __nv_bfloat16) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(__uint_as_float(q2 & 0xffff0000u) * sc), "f"(__uint_as_float(q2 << 16) * sc));
+  return d;
+}
+
 // (hi, lo) of x as one register: low half = hi, high half = lo.
 __device__ __forceinline__ uint32_t hilo(float x, __half) {
   const float hf = __half2float(__float2half_rn(x));
@@ -122,6 +134,11 @@ template <int NT>
 struct WarpState {
   float o[8][NT][4];  // PV accumulator: rows = channels 16*mc + g (+8), cols (hi, lo) of head qd + 4*nt
   float m[NT], l[NT], zv[NT];
+  // value exponent: the PV operand carries p * sV * 2^-F, and F grows (rescaling o) before
+  // a value scale could push p * sV * 2^-F past fp16's range (p < 2^8 by the lazy maximum)
+  int F;
+  float fsc;   // 2^-F
+  float vlim;  // 2^(7 + F): value scales at or above it need a larger F
 };
 
 // Query pairs of this lane in fp16: head (g/2) + 4 nt, channels 16 s + 2 qd (+1) for
@@ -136,6 +153,12 @@ template <int NT>
 struct LaneQ {
   uint32_t qa[NT == 2 ? 8 : 4][4];
   uint32_t negmask;  // fp16x2 -1 for lo-part lanes (odd g), 0 otherwise
+  // The query enters the products as q' = q * 2^-e_h, e_h >= 0 the smallest power of two
+  // with max_c |q_h[c]| < 2^e_h (0 when the query is already below 1), so that a folded
+  // key operand q' * scale never exceeds the scale: no fp16 overflow for fp16 caches.
+  float cl[NT];      // sm_scale * log2(e) * 2^e of the logit head qd + 4 nt
+  uint32_t sbq[NT];  // fp16x2 2^-e of the B-column head (g / 2) + 4 nt (plane-B gathers)
+  float sq[NT];      // the same 2^-e as a float
   __device__ __forceinline__ uint32_t& qv(int nt, int s, int j) {
     return NT == 2 ? qa[s][2 * j + nt] : qa[s & 3][2 * j + (s >> 2)];
   }
@@ -158,13 +181,43 @@ __device__ __forceinline__ void reset_state(WarpState<NT>& st) {
     st.l[nt] = 0.0f;
     st.zv[nt] = 0.0f;
   }
+  st.F = 0;
+  st.fsc = 1.0f;
+  st.vlim = 128.0f;
+}
+
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // e in [-126, 127]
+
+// Raises the value exponent F of this warp so that a value scale sv stays below 2^(7+F)
+// (warp-uniform call); o is rescaled by 2^(F_old - F_new).  A scale that is not finite
+// means an input outside the supported range: flagged, and F stays.
+template <int NT>
+__device__ __forceinline__ void raise_value_exponent(WarpState<NT>& st, float sv, int32_t* err) {
+  float m = sv < INFINITY ? sv : 0.0f;
+  if (!(sv < INFINITY)) flag_error(err, KVQ_DEV_ERR_RANGE);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+  if (!(m >= st.vlim)) return;
+  // m in [2^e, 2^(e+1)): F = e - 6 keeps m * 2^(8 - F) below 2^15
+  const int e = int((__float_as_uint(m) >> 23) & 0xff) - 127;
+  const int Fn = max(st.F, min(e - 6, 100));
+  const float beta = pow2f(st.F - Fn);
+#pragma unroll
+  for (int mc = 0; mc < 8; ++mc)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) st.o[mc][nt][i] *= beta;
+  st.F = Fn;
+  st.fsc = pow2f(-Fn);
+  st.vlim = pow2f(min(7 + Fn, 127));
 }
 
 // Online-softmax update from MT x 2 logits per head part of this lane (log2 units).  The
 // running maximum moves only when a logit exceeds it by more than 8, so probabilities
 // stay below 2^8 and most groups skip the rescale of the accumulators.
 template <int NT, int MT>
-__device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)[MT][NT][2]) {
+__device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)[MT][NT][2], int32_t* err) {
   // the lanes' own maxima decide whether any head can move; only then are they reduced
   float mx[NT];
   bool big = false;
@@ -173,9 +226,12 @@ __device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)
     mx[nt] = L[0][nt][0];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) mx[nt] = fmaxf(mx[nt], fmaxf(L[mt][nt][0], L[mt][nt][1]));
-    big |= mx[nt] > st.m[nt] + 8.0f;
+    big |= !(mx[nt] <= st.m[nt] + 8.0f);  // also true for a NaN logit
   }
   if (!__any_sync(kFull, big)) return;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+    if (!(mx[nt] < INFINITY) && mx[nt] != -INFINITY) flag_error(err, KVQ_DEV_ERR_RANGE);
   float alpha[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -205,7 +261,7 @@ __device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&L)
 template <typename T, int GQA, int KB, int P>
 __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const LaneQ<(GQA > 4 ? 2 : 1)>& lq,
                                            const uint16_t* qs, WarpState<(GQA > 4 ? 2 : 1)>& st, int lane,
-                                           float c_log2) {
+                                           int32_t* err) {
   constexpr int NT = GQA > 4 ? 2 : 1;
   using R = Rec<P, KB>;
   const int g = lane >> 2, qd = lane & 3;
@@ -299,8 +355,9 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
             q0 = uint32_t(qh[i00]) | (uint32_t(qh[i01]) << 16);
             q1 = uint32_t(qh[i10]) | (uint32_t(qh[i11]) << 16);
           }
-          b[nt][0] = fold_one(to_f16x2(q0, T()), s0, lq.negmask, __half());
-          b[nt][1] = fold_one(to_f16x2(q1, T()), s1, lq.negmask, __half());
+          // the gathered query scaled to q' = q * 2^-e (exact unless q' is an fp16 subnormal)
+          b[nt][0] = fold_one(scale_q2(q0, lq.sbq[nt], lq.sq[nt], T()), s0, lq.negmask, __half());
+          b[nt][1] = fold_one(scale_q2(q1, lq.sbq[nt], lq.sq[nt], T()), s1, lq.negmask, __half());
         }
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
@@ -346,8 +403,7 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
   }
 
   // -- logits (log2 units) of tokens 16 mt + 8 r + g for head qd + 4 nt; the code
-  //    products carry a factor 0.5 --
-  const float cc = c_log2 * kCodeScale;
+  //    products carry a factor 0.5, and the query its scale 2^-e --
   float L[2][NT][2];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -355,8 +411,8 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int r = 0; r < 2; ++r)
-        L[mt][nt][r] = fmaf(acc[mt][nt][2 * r] + acc[mt][nt][2 * r + 1], cc, zh[nt] * c_log2);
-  softmax_step<NT, 2>(st, L);
+        L[mt][nt][r] = fmaf(acc[mt][nt][2 * r] + acc[mt][nt][2 * r + 1], lq.cl[nt] * kCodeScale, zh[nt] * lq.cl[nt]);
+  softmax_step<NT, 2>(st, L, err);
 
   // -- probabilities times the value scales, as (hi, lo) pairs -> B operand of PV.
   //    Value scale/zero positions 32 grp + 4 g + u hold tokens 8u + g --
@@ -365,6 +421,8 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
   const float2 s01 = t2_to_float2(vsr.x, T()), s23 = t2_to_float2(vsr.y, T());
   const float2 z01 = t2_to_float2(vzr.x, T()), z23 = t2_to_float2(vzr.y, T());
   const float sv[4] = {s01.x, s01.y, s23.x, s23.y}, zv[4] = {z01.x, z01.y, z23.x, z23.y};
+  if (__any_sync(kFull, !(fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3])) < st.vlim)))
+    raise_value_exponent(st, fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3])), err);
   uint32_t pb[2][NT][2];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -376,7 +434,7 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
         const float pr = ex2(L[mt][nt][r] - st.m[nt]);
         st.l[nt] += pr;
         st.zv[nt] = fmaf(pr, zv[u], st.zv[nt]);
-        pb[mt][nt][r] = movmatrix_trans(hilo(pr * sv[u], __half()));
+        pb[mt][nt][r] = movmatrix_trans(hilo(pr * sv[u] * st.fsc, __half()));
       }
 
   // -- P V: words ((2 grp + n) * 32 + lane) * 4 + mm hold channel tile 4n + mm of this
@@ -402,7 +460,8 @@ __device__ __forceinline__ void page_group(const uint8_t* rec, int grp, const La
 // that the accumulator stays in the units of the code products.
 template <typename T, int GQA>
 __device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t* Vr, int n, const uint16_t* qs,
-                                               WarpState<(GQA > 4 ? 2 : 1)>& st, int lane, float c_log2) {
+                                               WarpState<(GQA > 4 ? 2 : 1)>& st, int lane, float c_log2,
+                                               int32_t* err) {
   constexpr int NT = GQA > 4 ? 2 : 1;
   const int g = lane >> 2, li = lane >> 3, lr = lane & 7;
   const bool lo = g & 1;  // lo-part columns get no query: the raw query is exact
@@ -431,7 +490,7 @@ __device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t*
 #pragma unroll
     for (int r = 0; r < 2; ++r)
       L[0][nt][r] = (g + 8 * r) < n ? (acc[nt][2 * r] + acc[nt][2 * r + 1]) * c_log2 : -INFINITY;
-  softmax_step<NT, 1>(st, L);
+  softmax_step<NT, 1>(st, L, err);
   uint32_t pb[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -439,7 +498,7 @@ __device__ __forceinline__ void residual_piece(const uint8_t* Kr, const uint8_t*
     for (int r = 0; r < 2; ++r) {
       const float pr = ex2(L[0][nt][r] - st.m[nt]);
       st.l[nt] += pr;
-      pb[nt][r] = movmatrix_trans(hilo(0.5f * pr, T()));
+      pb[nt][r] = movmatrix_trans(hilo(0.5f * pr * st.fsc, T()));
     }
 #pragma unroll
   for (int mc = 0; mc < 8; ++mc) {
@@ -1091,13 +1150,42 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
         const uint16_t* qs = sh.q[(d.w >> 11) & 3];
         const int n = d.w & 0xff;
         if (d.w & kDescFirst) {
+          // query scale exponent of every head (each warp computes all of them)
+          int eh[GQA];
+#pragma unroll
+          for (int h = 0; h < GQA; ++h) {
+            const uint2 v = lds64(qs + h * kHeadDim + 4 * lane);
+            const float2 a = t2_to_float2(v.x, T()), b2 = t2_to_float2(v.y, T());
+            const float m = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b2.x), fabsf(b2.y)));
+            const uint32_t mb = __reduce_max_sync(kFull, __float_as_uint(m));
+            const int e = int((mb >> 23) & 0xff) - 126;  // max |q| < 2^e
+            if (e > 24 && lane == 0) flag_error(p.err, KVQ_DEV_ERR_RANGE);
+            eh[h] = min(max(e, 0), 24);
+          }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const int hB = (g >> 1) + 4 * nt;
+            const int hB = (g >> 1) + 4 * nt, hL = qd + 4 * nt;
+            int eB = 0, eL = 0;
+#pragma unroll
+            for (int h = 0; h < GQA; ++h) {
+              eB = h == hB ? eh[h] : eB;
+              eL = h == hL ? eh[h] : eL;
+            }
+            lq.cl[nt] = p.c_log2 * pow2f(eL);
+            const float sc = pow2f(-eB);
+            lq.sbq[nt] = h2_as_u32(__float2half2_rn(sc));
+            lq.sq[nt] = sc;
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-              lq.qv(nt, s, 0) = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd), T()) : 0u;
-              lq.qv(nt, s, 1) = hB < GQA ? to_f16x2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8), T()) : 0u;
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                uint32_t x = 0u;
+                if (hB < GQA) {
+                  const float2 v = t2_to_float2(lds32(qs + hB * kHeadDim + 16 * s + 2 * qd + 8 * j), T());
+                  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(v.y * sc), "f"(v.x * sc));
+                }
+                lq.qv(nt, s, j) = x;
+              }
             }
           }
           lq.negmask = (g & 1) ? 0xbc00bc00u : 0u;  // fp16x2 (-1, -1) on lo-part lanes
@@ -1106,9 +1194,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
         if (ok) {
           if (!(d.w & kDescRes)) {
             const int pw = (32 * warp) / P, grp = ((32 * warp) % P) / 32;
-            if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.c_log2);
+            if (pw < n) page_group<T, GQA, KB, P>(sb + pw * R::record, grp, lq, qs, st, lane, p.err);
           } else if (int(d.w >> 16) % 4 == warp) {
-            residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, qs, st, lane, p.c_log2);
+            residual_piece<T, GQA>(sb, sb + kPieceTokens * kResRowBytes, n, qs, st, lane, p.c_log2, p.err);
           }
         }
         // release the stage; the last warp to release it refills it with item xi + kStages
@@ -1148,7 +1236,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
 #pragma unroll
                 for (int r = 0; r < 2; ++r)
                   sO[(warp * GQA + head) * kHeadDim + 16 * mc + g + 8 * r] =
-                      st.o[mc][nt][2 * r] + st.o[mc][nt][2 * r + 1];
+                      (st.o[mc][nt][2 * r] + st.o[mc][nt][2 * r + 1]) * pow2f(st.F);
             }
           }
           named_sync();

@@ -51,13 +51,19 @@ extern "C" kvq_status kvq_decode_attention_static(const kvq_config* cfg, const v
                                                   int32_t max_pages, const int32_t* num_pages, const void* res_k,
                                                   const void* res_v, const int32_t* res_len, float sm_scale,
                                                   float* out, int32_t* err, cudaStream_t stream) {
-  const kvq_status s = kvq_check_config(cfg);
+  // every argument is checked before the scratch is touched or anything is enqueued
+  const kvq_status s = kvq::decode_check_args(cfg, pool, pool_pages, q, batch, page_table, max_pages, num_pages,
+                                              res_k, res_v, res_len, out);
   if (s != KVQ_OK) return s;
-  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
-  if (batch == 0) return KVQ_OK;
+  void* scratch = nullptr;
+  if (batch == 0) {
+    // nothing to compute: only look the scratch up, so that a caller can resolve it
+    // (and, with lazy module loading, have the module loaded) before its own memory
+    // pool claims the device and before any stream capture
+    return scratch_address(&scratch);
+  }
   const size_t need = kvq_decode_workspace_bytes(cfg, batch, max_pages);
   if (need == 0 || need > kScratchBytes) return KVQ_ERR_CAPACITY;
-  void* scratch = nullptr;
   const kvq_status a = scratch_address(&scratch);
   if (a != KVQ_OK) return a;
   // The scratch keeps whatever the previous call left.  The arrival counters (the

@@ -357,5 +357,8 @@ inline cudaError_t ensure_dynamic_smem(Kernel kernel, int bytes, int (&seen)[64]
   return e;
 }
 size_t decode_main_bytes(int P, int GQA, uint32_t rec_bytes);
+kvq_status decode_check_args(const kvq_config* cfg, const void* pool, int64_t pool_pages, const void* q,
+                             int32_t batch, const int32_t* page_table, int32_t max_pages, const int32_t* num_pages,
+                             const void* res_k, const void* res_v, const int32_t* res_len, const float* out);
 
 }  // namespace kvq

@@ -131,6 +131,8 @@ typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 #define KVQ_DEV_ERR_TABLE_FULL   4  /* flush with no free page-table slot or no destination page      */
 #define KVQ_DEV_ERR_TIMEOUT      8  /* a bounded wait for an asynchronous copy gave up                */
 #define KVQ_DEV_ERR_LENGTH      16  /* num_pages[b] or res_len[b] outside its valid range             */
+#define KVQ_DEV_ERR_RANGE       32  /* decode: an operand outside the range the kernel carries (see
+                                       kvq_decode_attention, "Precision")                             */
 
 /* Shape and precision of one attention layer's KV cache.
  * Supported: head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8};
@@ -263,12 +265,17 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_config* cfg, int32_t batch, 
  * see kvq_decode_workspace_bytes for its zero-counter contract.
  * A sequence with no tokens at all (num_pages[b] == 0 and res_len[b] == 0) gets an
  * all-zero output row.
- * Precision: inside the kernel q*scale (keys) and p*scale (values) are carried as an
- * fp16 high part plus an fp16 low part, so |q| * key scale must stay below the fp16
- * maximum (65504); codes are exact.  Accumulation is fp32.  For bf16 caches the query,
- * the key scales and the key zero points enter the tensor cores as fp16: they must lie
- * within fp16's range (|x| <= 65504), where bf16 values are exact in fp16 down to 2^-14
- * and keep fewer bits below it (fp16 subnormals). */
+ * Precision and range: the codes enter the tensor-core products exactly; the scales are
+ * folded into the other operand, carried as an fp16 high part plus an fp16 low part, and
+ * products accumulate in fp32.  Each query head enters as q * 2^-e with e >= 0 the
+ * smallest power of two above max |q| (e = 0 when |q| < 1), so a folded key operand
+ * never exceeds its key scale: for fp16 caches no folded operand can overflow.  The
+ * value operand p * sV is carried as p * sV * 2^-F with a per-warp exponent F that grows
+ * before a value scale could overflow it.  bf16 caches: key scales and zero points enter
+ * the products as fp16 — exact down to 2^-14, with an absolute error below 2^-25 under
+ * it; a key scale or zero point above 65504 in magnitude (keys of magnitude above about
+ * 10^5), or a query above 2^24, is outside the supported range and sets
+ * KVQ_DEV_ERR_RANGE (the output is then undefined), as does any non-finite input. */
 KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t pool_pages,
                                 const void* q, int32_t batch,
                                 const int32_t* page_table, int32_t max_pages,
@@ -295,11 +302,19 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool,
  * rejected with KVQ_ERR_CAPACITY before anything is enqueued.
  * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  * The first call on each device looks up the buffer's device address
- * (cudaGetSymbolAddress) with that device current; make that first call outside any
- * stream capture.  Each call clears the buffer's arrival counters on `stream` before
- * the kernel runs; the rest keeps the previous call's contents.  All calls on a device
- * share the one buffer, so two calls whose executions overlap on the GPU (different
- * streams without ordering between them) race and give undefined results. */
+ * (cudaGetSymbolAddress) with that device current.  With lazy module loading (the CUDA
+ * default since 12.2) that lookup is also what loads the library's device code and
+ * commits the buffer's memory, so it can fail with KVQ_ERR_CUDA on a device whose memory
+ * is already taken: call once with batch = 0 (every other argument may be NULL or zero
+ * except cfg) early — before the caller's pool claims the device and outside any stream
+ * capture; that call only resolves the buffer.  The address is cached per device for the
+ * life of the process: after cudaDeviceReset or a re-created primary context the entry
+ * point must not be called again on that device.
+ * Each call clears the buffer's arrival counters on `stream` before the kernel runs; the
+ * rest keeps the previous call's contents.  All calls on a device share the one buffer,
+ * so two calls whose executions overlap on the GPU (different streams without ordering
+ * between them) race and give undefined results.  Invalid arguments are rejected before
+ * the buffer is looked up or cleared, exactly as kvq_decode_attention rejects them. */
 KVQ_API kvq_status kvq_decode_attention_static(const kvq_config* cfg, const void* pool, int64_t pool_pages,
                                                const void* q, int32_t batch,
                                                const int32_t* page_table, int32_t max_pages,

@@ -60,3 +60,29 @@ def test_append_rejects_a_short_window():
     tok = torch.zeros(B, 2, 128, dtype=torch.float16)
     with pytest.raises(ValueError, match="res_k"):
         kb.append_token(CFG, tok, tok, res, res, torch.zeros(B, dtype=torch.int32))
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor on a machine without a GPU: only what the device
+    check reads."""
+
+    def __init__(self, index):
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+
+
+def test_tensors_of_another_device_are_refused(monkeypatch):
+    """A call whose tensors live on a GPU other than the current one is refused on the
+    host (the kernels would run on the current GPU with the other GPU's pointers)."""
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    kb._cuda(_FakeCuda(0), None, _FakeCuda(0))  # one device, the current one: accepted
+    with pytest.raises(ValueError, match="current device is cuda:0"):
+        kb._cuda(_FakeCuda(1), _FakeCuda(1))
+    with pytest.raises(ValueError, match="tensors of one device"):
+        kb._cuda(_FakeCuda(0), _FakeCuda(1))
+
+    class _Stream:
+        device = torch.device("cuda", 1)
+
+    with pytest.raises(ValueError, match="stream of cuda:1"):
+        kb._cuda(_FakeCuda(0), stream=_Stream())

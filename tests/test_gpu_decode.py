@@ -18,17 +18,17 @@ from _kv import assert_attention_close, oracle_unit, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(rng, L, cfg, outlier_scale=(8.0, 20.0)):
+def _inputs(rng, L, cfg, outlier_scale=(8.0, 20.0), k_scale=1.0, v_scale=1.0):
     H, D = cfg.num_kv_heads, cfg.head_dim
     sig = np.exp(rng.standard_normal((H, D))).astype(np.float32)
     for h in range(H):
         sig[h, rng.choice(D, 5, replace=False)] *= rng.uniform(*outlier_scale, 5)
-    K = syn.to_bits(rng.standard_normal((L, H, D)).astype(np.float32) * sig, cfg.dtype)
-    V = syn.to_bits(rng.standard_normal((L, H, D)).astype(np.float32), cfg.dtype)
+    K = syn.to_bits(rng.standard_normal((L, H, D)).astype(np.float32) * sig * k_scale, cfg.dtype)
+    V = syn.to_bits(rng.standard_normal((L, H, D)).astype(np.float32) * v_scale, cfg.dtype)
     return K, V
 
 
-def _run(cfg, lens, seed, max_pages=None, shuffle=False, q_scale=1.0):
+def _run(cfg, lens, seed, max_pages=None, shuffle=False, q_scale=1.0, k_scale=1.0, v_scale=1.0, expect_err=0):
     """Prefill sequences of the given lengths, attend once; returns (out, oracle out)."""
     rng = np.random.default_rng(seed)
     P = cfg.page_tokens
@@ -39,7 +39,7 @@ def _run(cfg, lens, seed, max_pages=None, shuffle=False, q_scale=1.0):
     cache = PagedKVCache(cfg, B, max_pages, pool_pages, page_order=page_order)
     inputs = []
     for b, L in enumerate(lens):
-        K, V = _inputs(rng, L, cfg)
+        K, V = _inputs(rng, L, cfg, k_scale=k_scale, v_scale=v_scale)
         inputs.append((K, V))
         if L:
             cache.prefill(b, to_dev(K, cfg.dtype), to_dev(V, cfg.dtype))
@@ -49,8 +49,10 @@ def _run(cfg, lens, seed, max_pages=None, shuffle=False, q_scale=1.0):
     q_dev = to_dev(q, cfg.dtype)
     cache.attend(q_dev, out)
     torch.cuda.synchronize()
-    assert cache.err.item() == 0
+    assert cache.err.item() == expect_err
     got = out.cpu().numpy()
+    if expect_err:
+        return got, None, cache
     want = np.zeros_like(got, dtype=np.float64)
     g = cfg.gqa
     for b, L in enumerate(lens):
@@ -161,3 +163,32 @@ def test_bad_lengths_flag_error():
     cache.attend(q, out)
     torch.cuda.synchronize()
     assert cache.err.item() & kb.DEV_ERR_LENGTH
+
+
+# ---------------------------------------------------------------- operand range
+
+def test_large_queries_are_scaled_into_range():
+    """fp16 cache, queries of magnitude ~10^4: q * key scale reaches ~10^5, past fp16's
+    largest value.  The kernel carries q * 2^-e per head (|q * 2^-e| < 1), so the folded
+    operands stay finite and the result matches the oracle (a nearly one-hot softmax)."""
+    cfg = kb.Config(num_q_heads=4, num_kv_heads=2, page_tokens=128, num_boost=32)
+    got, want, _ = _run(cfg, [128 * 6 + 40, 300], seed=41, q_scale=3000.0)
+    assert_attention_close(got, want, "queries of magnitude 1e4")
+
+
+@pytest.mark.parametrize("dtype", [kb.F16, kb.BF16])
+def test_large_values_use_the_value_exponent(dtype):
+    """Values of magnitude ~3000 (value scales ~2700): p * scale would pass 65504 in the
+    fp16 PV operand without the per-warp value exponent.  Both sides are divided by the
+    value magnitude before the comparison, so the tolerance applies to unit-sized values."""
+    cfg = kb.Config(num_q_heads=8, num_kv_heads=2, page_tokens=128, num_boost=16, dtype=dtype)
+    got, want, _ = _run(cfg, [128 * 9 + 100, 77], seed=43, v_scale=1000.0)
+    assert_attention_close(got / 1000.0, want / 1000.0, "values of magnitude 3e3")
+
+
+def test_bf16_key_scales_beyond_fp16_flag_range():
+    """bf16 keys of magnitude ~10^6: their scales and zero points cannot enter the fp16
+    operands.  The call raises KVQ_DEV_ERR_RANGE instead of returning a silently wrong
+    output."""
+    cfg = kb.Config(num_q_heads=4, num_kv_heads=1, page_tokens=128, num_boost=32, dtype=kb.BF16)
+    _run(cfg, [128 * 3 + 5], seed=45, k_scale=1e6, expect_err=kb.DEV_ERR_RANGE)

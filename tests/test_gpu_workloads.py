@@ -1,12 +1,15 @@
 """Full-size parity on the five seeded workloads, in the launch configuration the
 benchmark times (PagedKVCache.step: append, flush, attend).
 
-The GPU runs every sequence and every decode step of the workload.  The oracle
-follows a sample of sequences through the same steps (its own quantization of the
-raw inputs, its own residual bookkeeping) and is compared at sampled steps:
-every record of the sampled sequences must match byte for byte, and their attention
-outputs must be within the method's tolerance."""
+The GPU runs every sequence and every decode step of the workload.  Every record
+the GPU wrote (prefill pages and pages flushed during the steps, of every sequence and
+KV head) must equal, byte for byte, the oracle's quantization of the same raw tokens.
+The oracle also follows a sample of sequences through the same steps (its own
+residual bookkeeping and fp64 attention), and their attention outputs must be within
+the method's tolerance at sampled steps."""
+import concurrent.futures as cf
 import math
+import os
 
 import numpy as np
 import pytest
@@ -27,6 +30,38 @@ def _check_steps(steps):
     if steps > 8:
         s.add(steps // 2)
     return sorted(s)
+
+
+def check_all_records(w: syn.Workload, cfg, cache, lens, steps, sigma):
+    """Every page of every sequence: the token stream of sequence b is its prompt followed
+    by the token it appended at each step, and page i of b holds stream tokens
+    [i P, (i + 1) P) whether it was written at prefill or by a flush."""
+    oc = ocfg(cfg)
+    P, B, H = w.P, w.batch, w.Hkv
+    payload = kb.page_layout(cfg)["payload_bytes"]
+    pool = cache.pool.view(cache.pool_pages, H, -1).cpu().numpy()
+    step_k = np.stack([syn.step_tokens(w, s, sigma)[0] for s in range(steps)], axis=1) if steps else None
+    step_v = np.stack([syn.step_tokens(w, s, sigma)[1] for s in range(steps)], axis=1) if steps else None
+
+    def check_seq(b):
+        L = int(lens[b])
+        K, V = syn.keys(w, b, 0, L, sigma), syn.values(w, b, 0, L)
+        if steps:
+            K, V = np.concatenate([K, step_k[b]]), np.concatenate([V, step_v[b]])
+        bad = []
+        for i, pg in enumerate(cache.host_pages[b]):
+            for h in range(H):
+                want = oracle.quantize_page(K[i * P:(i + 1) * P, h], V[i * P:(i + 1) * P, h], oc)[:payload]
+                if not np.array_equal(pool[pg, h, :payload], want):
+                    bad.append((b, i, h))
+        return len(cache.host_pages[b]) * H, bad
+
+    with cf.ThreadPoolExecutor(max(1, min(32, os.cpu_count() or 1))) as ex:
+        res = list(ex.map(check_seq, range(B)))
+    n = sum(r[0] for r in res)
+    bad = [x for r in res for x in r[1]]
+    assert not bad, f"{w.name}: {len(bad)} of {n} records differ, first (seq, page, head) {bad[0]}"
+    return n
 
 
 def run_workload(w: syn.Workload, steps: int | None = None, lengths=None):
@@ -71,7 +106,9 @@ def run_workload(w: syn.Workload, steps: int | None = None, lengths=None):
                     n_checked += 1
     torch.cuda.synchronize()
     assert cache.err.item() == 0
-    # every record of the sampled sequences, prefill and flushed pages alike
+    n_records = check_all_records(w, cfg, cache, lens, steps, sigma)
+    assert n_records == sum(len(p) for p in cache.host_pages) * w.Hkv
+    # the sampled sequences' page lists and records also agree with the oracle's bookkeeping
     payload = kb.page_layout(cfg)["payload_bytes"]
     recs = cache.pool.view(pool_pages, w.Hkv, -1)
     for i, b in enumerate(sampled):
