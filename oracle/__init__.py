@@ -97,6 +97,13 @@ def lib():
                                         ctypes.c_int, ctypes.c_int, u8p]
         L.kvqo_quantize_page.restype = None
         L.kvqo_quantize_page.argtypes = [u16p, u16p, ctypes.c_long] + [ctypes.c_int] * 5 + [u8p]
+        f32p = ctypes.POINTER(ctypes.c_float)
+        L.kvqo_quantize_page_ex.restype = None
+        L.kvqo_quantize_page_ex.argtypes = [u16p, u16p, ctypes.c_long] + [ctypes.c_int] * 5 + [
+            f32p, ctypes.c_int, u8p]
+        L.kvqo_select_boost_query.restype = None
+        L.kvqo_select_boost_query.argtypes = [u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              f32p, ctypes.c_int, u8p]
         L.kvqo_dequantize_page.restype = None
         L.kvqo_dequantize_page.argtypes = [u8p] + [ctypes.c_int] * 5 + [f64p, f64p]
         L.kvqo_decode_unit.restype = None
@@ -217,6 +224,35 @@ def select_boost(K_bits: np.ndarray, k: int, dtype: int) -> np.ndarray:
     idx = np.zeros(k, np.uint8)
     lib().kvqo_select_boost(_p(K, ctypes.c_uint16), D, P, D, k, dtype, _p(idx, ctypes.c_uint8))
     return idx
+
+
+def select_boost_query(K_bits: np.ndarray, n: int, weight: np.ndarray, dtype: int) -> np.ndarray:
+    """Query-aware boosted channels of one page (MixKVQ reading): K_bits [P][D], weight
+    float32[D] -> ascending uint8[n]."""
+    K = np.ascontiguousarray(K_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(weight, dtype=np.float32)
+    P, D = K.shape
+    idx = np.zeros(n, np.uint8)
+    lib().kvqo_select_boost_query(_p(K, ctypes.c_uint16), D, P, D, n, _p(w, ctypes.c_float), dtype,
+                                  _p(idx, ctypes.c_uint8))
+    return idx
+
+
+def quantize_page_ex(K_bits: np.ndarray, V_bits: np.ndarray, cfg: Cfg, n_boost: int | None = None,
+                     weight: np.ndarray | None = None) -> np.ndarray:
+    """quantize_page with n_boost <= cfg.k boosted channels (the per-head boost count)
+    and, when weight is given, the query-aware ranking."""
+    K = np.ascontiguousarray(K_bits, dtype=np.uint16)
+    V = np.ascontiguousarray(V_bits, dtype=np.uint16)
+    assert K.shape == (cfg.P, cfg.D) and V.shape == (cfg.P, cfg.D)
+    n = cfg.k if n_boost is None else int(n_boost)
+    assert 0 <= n <= cfg.k
+    w = None if weight is None else np.ascontiguousarray(weight, dtype=np.float32)
+    rec = np.zeros(cfg.record_bytes, np.uint8)
+    lib().kvqo_quantize_page_ex(_p(K, ctypes.c_uint16), _p(V, ctypes.c_uint16), cfg.D, cfg.P, cfg.D, cfg.G,
+                                cfg.k, n, None if w is None else _p(w, ctypes.c_float), cfg.dtype,
+                                _p(rec, ctypes.c_uint8))
+    return rec
 
 
 def quantize_page(K_bits: np.ndarray, V_bits: np.ndarray, cfg: Cfg) -> np.ndarray:

@@ -308,13 +308,64 @@ void kvqo_select_boost(const uint16_t* K, long tok_stride, int P, int D, int k, 
   free(taken);
 }
 
+/* Query-aware selection (MixKVQ summary on fugumt.com, Abstract: key channels are
+ * ranked by their intrinsic quantization difficulty together with their relevance to
+ * the query).  Reading: the difficulty of channel c is its range over the page,
+ * r_c = fl32(max_t K[t][c] - min_t K[t][c]) (the 2-bit step, and so the error, grows
+ * with it); the relevance is a caller-given weight w_c >= 0 (for example the mean |q_c|
+ * of the query heads that share the KV head); score_c = fl32(w_c * r_c), each in fp32
+ * with one rounding.  The n channels with the highest score are boosted, ties to the
+ * lower channel index, returned in ascending channel order. */
+void kvqo_select_boost_query(const uint16_t* K, long tok_stride, int P, int D, int n, const float* w,
+                             int dtype, uint8_t* idx) {
+  float* score = (float*)malloc(sizeof(float) * D);
+  char* taken = (char*)calloc(D, 1);
+  for (int c = 0; c < D; ++c) {
+    float mn = (float)dt_value(K[c], dtype), mx = mn;
+    for (int t = 1; t < P; ++t) {
+      const float v = (float)dt_value(K[t * tok_stride + c], dtype);
+      if (v < mn) mn = v;
+      if (v > mx) mx = v;
+    }
+    volatile float range = mx - mn;
+    volatile float sc = w[c] * range;
+    score[c] = sc;
+  }
+  for (int r = 0; r < n; ++r) {
+    int best = -1;
+    for (int c = 0; c < D; ++c) {
+      if (taken[c]) continue;
+      if (best < 0 || score[c] > score[best]) best = c;  /* strict: lower index wins ties */
+    }
+    taken[best] = 1;
+  }
+  int j = 0;
+  for (int c = 0; c < D; ++c)
+    if (taken[c]) idx[j++] = (uint8_t)c;
+  free(score);
+  free(taken);
+}
+
 /* ------------------------------------------------------------- page quantization */
 
 /* Quantizes one page of one KV head into a record (a1 + a2 + a3).
  * K, V: [P][D] 16-bit patterns with token stride tok_stride (elements).
  * rec: record_bytes bytes; padding is left zero. */
+void kvqo_quantize_page_ex(const uint16_t* K, const uint16_t* V, long tok_stride, int P, int D,
+                           int G, int k, int n_boost, const float* w, int dtype, uint8_t* rec);
+
 void kvqo_quantize_page(const uint16_t* K, const uint16_t* V, long tok_stride, int P, int D,
                         int G, int k, int dtype, uint8_t* rec) {
+  kvqo_quantize_page_ex(K, V, tok_stride, P, D, G, k, k, NULL, dtype, rec);
+}
+
+/* The same with the options of the per-head boost count and the query-aware ranking:
+ * the record is laid out for k plane-B rows, but only n_boost <= k channels are boosted
+ * (rows n_boost..k-1 of plane B, their scales and their boost indices stay zero, so they
+ * add nothing to a dequantized key); w = NULL ranks by magnitude, otherwise by
+ * kvqo_select_boost_query. */
+void kvqo_quantize_page_ex(const uint16_t* K, const uint16_t* V, long tok_stride, int P, int D,
+                           int G, int k, int n_boost, const float* w, int dtype, uint8_t* rec) {
   layout_t L = make_layout(P, D, k, G);
   memset(rec, 0, (size_t)L.record);
   uint32_t* kA = (uint32_t*)(rec + L.k_codes);
@@ -328,10 +379,13 @@ void kvqo_quantize_page(const uint16_t* K, const uint16_t* V, long tok_stride, i
   uint8_t* bidx = rec + L.boost_idx;
 
   /* a1: boosted channels */
-  kvqo_select_boost(K, tok_stride, P, D, k, dtype, bidx);
+  if (w)
+    kvqo_select_boost_query(K, tok_stride, P, D, n_boost, w, dtype, bidx);
+  else
+    kvqo_select_boost(K, tok_stride, P, D, n_boost, dtype, bidx);
   int* row_of = (int*)malloc(sizeof(int) * D); /* plane-B row of a boosted channel, else -1 */
   for (int c = 0; c < D; ++c) row_of[c] = -1;
-  for (int j = 0; j < k; ++j) row_of[bidx[j]] = j;
+  for (int j = 0; j < n_boost; ++j) row_of[bidx[j]] = j;
 
   /* a2: keys, per channel and per group of G tokens */
   uint8_t* codes = (uint8_t*)malloc((size_t)(P > D ? P : D));
