@@ -480,6 +480,7 @@ def run_gpu(args):
         cfgs["llama3_70b_batch"] = workload_bench("llama3_70b_batch", dev, peak)
         cfgs["ragged_serving"] = workload_bench("ragged_serving", dev, peak, flush_steps=256)
         result["configs"] = cfgs
+        result["vs_fp16_dense"] = compare_dense(dev, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # every step appended the same k_new / v_new, so the windows hold copies of them
         rk = np.repeat(kn[:, :, None, :], res_end, axis=2)
@@ -678,6 +679,91 @@ def l2_flushed_single(dev, peak, iters=20):
             "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4), "bytes_per_launch": nbytes,
             "what": "one layer cache, a 512 MB write between launches (outside the timed region), "
                     "each launch timed alone with events"}
+
+
+def compare_dense(dev, peak, iters=20):
+    """The 8B-shaped layer (batch 16, 32 q / 8 kv heads, 4096 tokens, pages of 128) on the
+    same kernel and work line: 2-bit keys and values with 0 (KIVI), 16 and 32 (Kitty, 12.5%
+    and 25%) boosted key channels, and the unquantized fp16 cache.  Decode attention only,
+    each variant over replicas totalling at least 512 MB of cache."""
+    import torch
+
+    from bit_mixed_precision_channel_b200 import binding as kb
+    from bit_mixed_precision_channel_b200 import synthetic as syn
+    from bit_mixed_precision_channel_b200.cache import PagedKVCache
+
+    w = syn.WORKLOADS[WORKLOAD]
+    B, P, H, D, L = w.batch, w.P, w.Hkv, w.D, w.context
+    n = L // P
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    sigma = torch.from_numpy(syn.key_channel_sigma(w)).to(dev)
+    K = (torch_randn((B, L, H, D), gen, dev) * sigma).half()
+    V = torch_randn((B, L, H, D), gen, dev).half()
+    q = torch_randn((B, w.Hq, D), gen, dev).half()
+    out = torch.empty(B, w.Hq, D, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def time_graph(fns, replicas):
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for f in fns:
+                f()
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(iters):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters / replicas
+
+    res = {}
+    for k in (0, 16, 32):
+        cfg = kb.Config(head_dim=D, num_q_heads=w.Hq, num_kv_heads=H, page_tokens=P, key_group=w.G, num_boost=k,
+                        dtype=w.dtype)
+        payload = kb.page_layout(cfg)["payload_bytes"]
+        reps = max(1, math.ceil(512e6 / (B * H * n * payload)))
+        caches = [PagedKVCache(cfg, B, n + 1, B * (n + 1), device=dev) for _ in range(reps)]
+        for c in caches:
+            c.prefill_batch(K, V)
+        ms = time_graph([(lambda c=c: c.attend(q, out)) for c in caches], reps)
+        nbytes = B * H * n * payload + B * w.Hq * D * 6 + 4 * B * n + 8 * B
+        res[f"2bit_k{k}"] = {"decode_us_per_launch": round(ms * 1e3, 2), "bytes_per_launch": nbytes,
+                             "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "decode_tokens_per_s": round(B / (ms * 1e-3), 1),
+                             "kv_bytes_per_token_head": round(payload / P, 2)}
+        del caches
+    cfg = kb.Config(head_dim=D, num_q_heads=w.Hq, num_kv_heads=H, page_tokens=P, key_group=w.G, num_boost=32,
+                    dtype=w.dtype)
+    page_bytes = B * H * n * kb.dense_page_bytes(cfg)
+    reps = max(1, math.ceil(512e6 / page_bytes))
+    table = torch.arange(B * n, dtype=torch.int32, device=dev).view(B, n)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    ws = torch.zeros(kb.decode_workspace_bytes(cfg, B, n), dtype=torch.uint8, device=dev)
+    # [B][n][P][H][D] -> pages [B * n][H][2][P][D]
+    pages = torch.stack([K.view(B, n, P, H, D), V.view(B, n, P, H, D)], dim=3)  # [B][n][P][2][H][D]
+    pool = pages.permute(0, 1, 4, 3, 2, 5).contiguous().view(-1)
+    pools = [pool] + [pool.clone() for _ in range(reps - 1)]
+    ms = time_graph([(lambda p=p: kb.decode_attention_dense(cfg, p, q, table, lens, out, ws)) for p in pools], reps)
+    nbytes = B * H * n * kb.dense_page_bytes(cfg) + B * w.Hq * D * 6 + 4 * B * n + 8 * B
+    res["fp16_dense"] = {"decode_us_per_launch": round(ms * 1e3, 2), "bytes_per_launch": nbytes,
+                         "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "decode_tokens_per_s": round(B / (ms * 1e-3), 1),
+                         "kv_bytes_per_token_head": 512.0}
+    dense_us = res["fp16_dense"]["decode_us_per_launch"]
+    for key in ("2bit_k0", "2bit_k16", "2bit_k32"):
+        res[key]["speedup_vs_fp16_dense"] = round(dense_us / res[key]["decode_us_per_launch"], 3)
+        res[key]["kv_bytes_ratio_vs_fp16_dense"] = round(512.0 / res[key]["kv_bytes_per_token_head"], 2)
+    res["what"] = ("one decode-attention launch per layer at batch 16, 4096-token prompts; the same kernel and "
+                   "work line for every variant, the fp16 cache read through its page table in 16-token pieces")
+    del pools, pool, pages, K, V
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------ reference arm

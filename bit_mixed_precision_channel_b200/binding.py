@@ -20,6 +20,7 @@ __all__ = [
     "page_layout", "page_bytes", "select_boost_channels", "quantize_page_keys",
     "quantize_values", "quantize_pages", "append_token", "flush_residual",
     "decode_workspace_bytes", "decode_attention", "decode_attention_static", "STATIC_SCRATCH_BYTES",
+    "quantize_pages_ex", "dense_page_bytes", "decode_attention_dense",
     "F16", "BF16", "torch_dtype",
     "DEV_ERR_PAGE_RANGE", "DEV_ERR_RESIDUAL", "DEV_ERR_TABLE_FULL", "DEV_ERR_TIMEOUT",
     "DEV_ERR_LENGTH", "DEV_ERR_RANGE",
@@ -58,6 +59,10 @@ class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "k_codes", "kb_codes", "v_codes", "k_scale", "k_zero", "kb_scale", "v_scale", "v_zero",
         "boost_idx", "payload_bytes", "record_bytes")]
+
+
+class _BoostOptions(ctypes.Structure):
+    _fields_ = [("query_weight", ctypes.c_void_p), ("boost_per_head", ctypes.c_void_p)]
 
 
 class _Source(ctypes.Structure):
@@ -145,6 +150,16 @@ def load():
         L.kvq_append_token.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp, vp]
         L.kvq_flush_residual.restype = ctypes.c_int
         L.kvq_flush_residual.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, i32, vp, vp, i64, vp, vp]
+        L.kvq_dense_page_bytes.restype = sz
+        L.kvq_dense_page_bytes.argtypes = [cfgp]
+        L.kvq_decode_attention_dense.restype = ctypes.c_int
+        L.kvq_decode_attention_dense.argtypes = [cfgp, vp, i64, vp, i32, vp, i32, vp, ctypes.c_float, vp, vp, sz,
+                                                 vp, vp]
+        optp = ctypes.POINTER(_BoostOptions)
+        L.kvq_quantize_pages_ex.restype = ctypes.c_int
+        L.kvq_quantize_pages_ex.argtypes = [cfgp, _Source, _Source, vp, i32, vp, i64, optp, vp, vp]
+        L.kvq_flush_residual_ex.restype = ctypes.c_int
+        L.kvq_flush_residual_ex.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, i32, vp, vp, i64, optp, vp, vp]
         L.kvq_decode_workspace_bytes.restype = sz
         L.kvq_decode_workspace_bytes.argtypes = [cfgp, i32, i32]
         L.kvq_decode_attention.restype = ctypes.c_int
@@ -238,7 +253,17 @@ def page_bytes(cfg: Config) -> int:
     return int(load().kvq_page_bytes(ctypes.byref(cfg.c())))
 
 
-def _quant(fn, cfg, src_k, src_v, dst_pages, pool, err, stream):
+def _boost_options(cfg: Config, query_weight, boost_per_head):
+    """Checks and marshals the boost options (device float32 [Hkv][D] weights, device
+    int32 [Hkv] counts); None for both gives a null pointer (the plain behaviour)."""
+    _need("query_weight", query_weight, torch.float32, cfg.num_kv_heads * cfg.head_dim)
+    _need("boost_per_head", boost_per_head, torch.int32, cfg.num_kv_heads)
+    if query_weight is None and boost_per_head is None:
+        return None
+    return ctypes.byref(_BoostOptions(_ptr(query_weight), _ptr(boost_per_head)))
+
+
+def _quant(fn, cfg, src_k, src_v, dst_pages, pool, err, stream, query_weight=None, boost_per_head=None):
     _need("dst_pages", dst_pages, torch.int32)
     _need("pool", pool, torch.uint8)
     _need("err", err, torch.int32, 1)
@@ -249,7 +274,12 @@ def _quant(fn, cfg, src_k, src_v, dst_pages, pool, err, stream):
     pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
     L = load()
     n = dst_pages.numel()
-    if fn == "kvq_quantize_pages":
+    if fn == "kvq_quantize_pages_ex":
+        _cuda(query_weight, boost_per_head, pool, stream=stream)
+        st = L.kvq_quantize_pages_ex(ctypes.byref(cfg.c()), src_k.c(), src_v.c(), dst_pages.data_ptr(), n,
+                                     pool.data_ptr(), pool_pages, _boost_options(cfg, query_weight, boost_per_head),
+                                     _ptr(err), _stream(stream))
+    elif fn == "kvq_quantize_pages":
         st = L.kvq_quantize_pages(ctypes.byref(cfg.c()), src_k.c(), src_v.c(), dst_pages.data_ptr(), n,
                                   pool.data_ptr(), pool_pages, _ptr(err), _stream(stream))
     else:
@@ -279,6 +309,13 @@ def quantize_pages(cfg: Config, k: Source, v: Source, dst_pages: torch.Tensor, p
     _quant("kvq_quantize_pages", cfg, k, v, dst_pages, pool, err, stream)
 
 
+def quantize_pages_ex(cfg: Config, k: Source, v: Source, dst_pages: torch.Tensor, pool: torch.Tensor,
+                      err: torch.Tensor | None = None, stream=None, query_weight=None, boost_per_head=None):
+    """quantize_pages with the boost options: query_weight (float32 [Hkv][D], the
+    query-aware ranking) and boost_per_head (int32 [Hkv], boosted channels per head)."""
+    _quant("kvq_quantize_pages_ex", cfg, k, v, dst_pages, pool, err, stream, query_weight, boost_per_head)
+
+
 def append_token(cfg: Config, k_new, v_new, res_k, res_v, res_len, err=None, stream=None):
     batch = res_len.numel()
     dt, H, P, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.page_tokens, cfg.head_dim
@@ -295,7 +332,7 @@ def append_token(cfg: Config, k_new, v_new, res_k, res_v, res_len, err=None, str
 
 
 def flush_residual(cfg: Config, res_k, res_v, res_len, new_page, page_table, num_pages, pool,
-                   err=None, stream=None):
+                   err=None, stream=None, query_weight=None, boost_per_head=None):
     _need("page_table", page_table, torch.int32, dim=2)
     batch, max_pages = page_table.shape
     dt, H, P, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.page_tokens, cfg.head_dim
@@ -305,12 +342,20 @@ def flush_residual(cfg: Config, res_k, res_v, res_len, new_page, page_table, num
         _need(name, t, torch.int32, batch)
     _need("pool", pool, torch.uint8)
     _need("err", err, torch.int32, 1)
-    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err, stream=stream)
+    _cuda(res_k, res_v, res_len, new_page, page_table, num_pages, pool, err, query_weight, boost_per_head,
+          stream=stream)
     pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
-    _check("kvq_flush_residual", load().kvq_flush_residual(
-        ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
-        new_page.data_ptr(), page_table.data_ptr(), max_pages, num_pages.data_ptr(), pool.data_ptr(),
-        pool_pages, _ptr(err), _stream(stream)))
+    opts = _boost_options(cfg, query_weight, boost_per_head)
+    if opts is None:
+        _check("kvq_flush_residual", load().kvq_flush_residual(
+            ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
+            new_page.data_ptr(), page_table.data_ptr(), max_pages, num_pages.data_ptr(), pool.data_ptr(),
+            pool_pages, _ptr(err), _stream(stream)))
+    else:
+        _check("kvq_flush_residual_ex", load().kvq_flush_residual_ex(
+            ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
+            new_page.data_ptr(), page_table.data_ptr(), max_pages, num_pages.data_ptr(), pool.data_ptr(),
+            pool_pages, opts, _ptr(err), _stream(stream)))
 
 
 def decode_workspace_bytes(cfg: Config, batch: int, max_pages: int) -> int:
@@ -363,3 +408,30 @@ def decode_attention_static(cfg: Config, pool, q, page_table, num_pages, res_k, 
         ctypes.byref(cfg.c()), pool.data_ptr(), pool_pages, q.data_ptr(), batch, page_table.data_ptr(),
         max_pages, num_pages.data_ptr(), res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
         float(sm_scale), out.data_ptr(), _ptr(err), _stream(stream)))
+
+
+def dense_page_bytes(cfg: Config) -> int:
+    return int(load().kvq_dense_page_bytes(ctypes.byref(cfg.c())))
+
+
+def decode_attention_dense(cfg: Config, pool, q, page_table, seq_len, out, workspace,
+                           sm_scale: float | None = None, err=None, stream=None):
+    """Decode attention over an unquantized paged cache (the full-precision baseline):
+    pool dtype [pool_pages][Hkv][2][P][D], page_table int32 [B][max_pages], seq_len int32 [B]."""
+    dt = torch_dtype(cfg.dtype)
+    _need("page_table", page_table, torch.int32, dim=2)
+    batch, max_pages = page_table.shape
+    _need("pool", pool, dt)
+    _need("seq_len", seq_len, torch.int32, batch)
+    _need("q", q, dt, batch * cfg.num_q_heads * cfg.head_dim)
+    _need("out", out, torch.float32, batch * cfg.num_q_heads * cfg.head_dim)
+    _need("workspace", workspace, torch.uint8)
+    _need("err", err, torch.int32, 1)
+    _cuda(pool, q, page_table, seq_len, out, workspace, err, stream=stream)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(cfg.head_dim)
+    pool_pages = pool.numel() * 2 // (cfg.num_kv_heads * dense_page_bytes(cfg))
+    _check("kvq_decode_attention_dense", load().kvq_decode_attention_dense(
+        ctypes.byref(cfg.c()), pool.data_ptr(), pool_pages, q.data_ptr(), batch, page_table.data_ptr(),
+        max_pages, seq_len.data_ptr(), float(sm_scale), out.data_ptr(), workspace.data_ptr(),
+        workspace.numel(), _ptr(err), _stream(stream)))

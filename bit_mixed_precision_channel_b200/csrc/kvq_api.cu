@@ -133,7 +133,7 @@ size_t kvq_page_bytes(const kvq_config* cfg) {
 
 static kvq_status quantize_common(const kvq_config* cfg, kvq_source k, kvq_source v, int mode,
                                   const int32_t* dst_pages, int32_t n_pages, void* pool, int64_t pool_pages,
-                                  int32_t* err, cudaStream_t stream) {
+                                  int32_t* err, cudaStream_t stream, const kvq_boost_options* opts = nullptr) {
   const kvq_status s = kvq_check_config(cfg);
   if (s != KVQ_OK) return s;
   if (n_pages < 0) return KVQ_ERR_INVALID_ARG;
@@ -164,7 +164,18 @@ static kvq_status quantize_common(const kvq_config* cfg, kvq_source k, kvq_sourc
   p.err = err;
   p.mode = mode;
   p.flush = 0;
+  if (opts) {
+    p.qw = opts->query_weight;
+    p.kh = opts->boost_per_head;
+  }
   return cuda_status(launch_quantize(p, n_pages, cfg->dtype, stream));
+}
+
+kvq_status kvq_quantize_pages_ex(const kvq_config* cfg, kvq_source k, kvq_source v, const int32_t* dst_pages,
+                                 int32_t n_pages, void* pool, int64_t pool_pages, const kvq_boost_options* opts,
+                                 int32_t* err, cudaStream_t stream) {
+  return quantize_common(cfg, k, v, kModeSelect | kModeKeys | kModeValues, dst_pages, n_pages, pool, pool_pages,
+                         err, stream, opts);
 }
 
 kvq_status kvq_select_boost_channels(const kvq_config* cfg, kvq_source k, const int32_t* dst_pages,
@@ -201,10 +212,23 @@ kvq_status kvq_append_token(const kvq_config* cfg, int32_t batch, const void* k_
                                    cfg->page_tokens, err, stream));
 }
 
+kvq_status kvq_flush_residual_ex(const kvq_config* cfg, int32_t batch, const void* res_k, const void* res_v,
+                                 int32_t* res_len, const int32_t* new_page, int32_t* page_table, int32_t max_pages,
+                                 int32_t* num_pages, void* pool, int64_t pool_pages, const kvq_boost_options* opts,
+                                 int32_t* err, cudaStream_t stream);
+
 kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch, const void* res_k, const void* res_v,
                               int32_t* res_len, const int32_t* new_page, int32_t* page_table, int32_t max_pages,
                               int32_t* num_pages, void* pool, int64_t pool_pages, int32_t* err,
                               cudaStream_t stream) {
+  return kvq_flush_residual_ex(cfg, batch, res_k, res_v, res_len, new_page, page_table, max_pages, num_pages, pool,
+                               pool_pages, nullptr, err, stream);
+}
+
+kvq_status kvq_flush_residual_ex(const kvq_config* cfg, int32_t batch, const void* res_k, const void* res_v,
+                                 int32_t* res_len, const int32_t* new_page, int32_t* page_table, int32_t max_pages,
+                                 int32_t* num_pages, void* pool, int64_t pool_pages, const kvq_boost_options* opts,
+                                 int32_t* err, cudaStream_t stream) {
   const kvq_status s = kvq_check_config(cfg);
   if (s != KVQ_OK) return s;
   if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
@@ -232,6 +256,10 @@ kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch, const void* 
   p.res_len = res_len;
   p.num_pages = num_pages;
   p.max_pages = max_pages;
+  if (opts) {
+    p.qw = opts->query_weight;
+    p.kh = opts->boost_per_head;
+  }
   cudaError_t e = launch_quantize(p, batch, cfg->dtype, stream);
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
   return cuda_status(launch_flush_commit(res_len, new_page, page_table, max_pages, num_pages, pool_pages, batch, P,
@@ -281,6 +309,53 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   p.n_ctas = pl.ctas;
   p.err = err;
   return cuda_status(launch_decode(p, gqa, cfg->dtype, stream));
+}
+
+size_t kvq_dense_page_bytes(const kvq_config* cfg) {
+  if (kvq_check_config(cfg) != KVQ_OK) return 0;
+  return size_t(2) * cfg->page_tokens * cfg->head_dim * 2;
+}
+
+kvq_status kvq_decode_attention_dense(const kvq_config* cfg, const void* pool, int64_t pool_pages, const void* q,
+                                      int32_t batch, const int32_t* page_table, int32_t max_pages,
+                                      const int32_t* seq_len, float sm_scale, float* out, void* workspace,
+                                      size_t workspace_bytes, int32_t* err, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!pool || pool_pages <= 0 || !q || !seq_len || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+  if (max_pages > 0 && !page_table) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(q) || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+  // pieces of 16 tokens are numbered with 16 bits; the work line is indexed with 32
+  const long long tokens = (long long)max_pages * cfg->page_tokens;
+  if (tokens > 16ll * 65535) return KVQ_ERR_INVALID_ARG;
+  if ((long long)batch * cfg->num_kv_heads * (kDecodePieceWeight * ((tokens + 15) / 16) + kDecodeMergeWeight) >=
+      (1ll << 31))
+    return KVQ_ERR_INVALID_ARG;
+  const Plan pl = decode_plan(cfg, batch);
+  if (workspace_bytes < pl.part_bytes + pl.cnt_bytes) return KVQ_ERR_CAPACITY;
+  DecodeParams p{};
+  p.pool = static_cast<const uint8_t*>(pool);
+  p.pool_pages = pool_pages;
+  p.Hkv = cfg->num_kv_heads;
+  p.P = cfg->page_tokens;
+  p.k = cfg->num_boost;
+  p.KB = cfg->num_boost / 16;
+  p.L = make_layout(cfg->page_tokens, cfg->head_dim, cfg->num_boost, cfg->key_group);
+  p.q = static_cast<const uint16_t*>(q);
+  p.batch = batch;
+  p.Hq = cfg->num_q_heads;
+  p.page_table = page_table;
+  p.max_pages = max_pages;
+  p.seq_len = seq_len;
+  p.c_log2 = sm_scale * 1.4426950408889634f;
+  p.out = out;
+  p.part = static_cast<float*>(workspace);
+  p.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.part_bytes);
+  p.n_ctas = pl.ctas;
+  p.err = err;
+  return cuda_status(launch_decode(p, cfg->num_q_heads / cfg->num_kv_heads, cfg->dtype, stream));
 }
 
 }  // extern "C"

@@ -523,11 +523,18 @@ struct Cursor {
 
 // Unit weight of sequence b (-1 when its lengths are invalid), with its pages and
 // residual tokens (0 when invalid).
+// In dense mode (p.seq_len set) a sequence has no quantized pages: all its tokens are
+// read as raw rows through its page table, in the residual pieces' path.
 template <int P>
 __device__ __forceinline__ int seq_weight(const DecodeParams& p, int b, int& np, int& rl) {
-  np = __ldcg(p.num_pages + b);
-  rl = __ldcg(p.res_len + b);
-  if (np < 0 || np > p.max_pages || rl < 0 || rl > P) {
+  if (p.seq_len) {
+    np = 0;
+    rl = __ldcg(p.seq_len + b);
+  } else {
+    np = __ldcg(p.num_pages + b);
+    rl = __ldcg(p.res_len + b);
+  }
+  if (np < 0 || np > p.max_pages || rl < 0 || rl > (p.seq_len ? p.max_pages * P : P)) {
     np = 0;
     rl = 0;
     return -1;
@@ -834,8 +841,22 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, CtaShared<GQA,
     // residual rows: 16-byte asynchronous copies into the padded rows, zero-filled past
     // the last token; each lane's copies arrive on the stage's barrier when they land
     const int t0 = kPieceTokens * int(d.w >> 16);
-    const uint16_t* kr = p.res_k + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
-    const uint16_t* vr = p.res_v + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+    const uint16_t* kr;
+    const uint16_t* vr;
+    if (p.seq_len) {
+      // dense: page t0 / P of the sequence holds K rows then V rows ([2][P][128]); a piece
+      // never crosses a page (P is a multiple of the piece length)
+      int id = __ldcg(p.page_table + size_t(d.b) * p.max_pages + t0 / P);
+      if (id < 0 || id >= p.pool_pages) {
+        if (lane == 0) flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
+        id = 0;
+      }
+      kr = reinterpret_cast<const uint16_t*>(p.pool) + ((size_t(id) * p.Hkv + d.h) * 2 * P + t0 % P) * kHeadDim;
+      vr = kr + size_t(P) * kHeadDim;
+    } else {
+      kr = p.res_k + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+      vr = p.res_v + ((size_t(d.b) * p.Hkv + d.h) * P + t0) * kHeadDim;
+    }
 #pragma unroll 4
     for (int i = lane; i < 2 * kPieceTokens * 16; i += 32) {
       const int which = i >> 8, row = (i >> 4) & 15, chunk = i & 15;

@@ -305,6 +305,8 @@ struct QuantParams {
   const int32_t* res_len;
   const int32_t* num_pages;
   int max_pages;
+  const float* qw;     // query-aware ranking weights [Hkv][128], or null (magnitude ranking)
+  const int32_t* kh;   // boosted channels per kv head [Hkv] (each <= k), or null (k for all)
 };
 
 // Decode attention (a6 + a7).
@@ -327,6 +329,9 @@ struct DecodeParams {
   uint32_t* cnt;  // [batch * Hkv] arrival counters
   int n_ctas;     // grid size: SMs x resident CTAs per SM
   int32_t* err;
+  // dense mode: tokens per sequence; pool then holds raw pages [pool_pages][Hkv][2][P][128]
+  // (K rows, V rows) of the cache dtype, and num_pages / res_len / res_k / res_v are unused
+  const int32_t* seq_len;
 };
 
 cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream);

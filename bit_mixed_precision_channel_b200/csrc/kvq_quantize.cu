@@ -146,6 +146,16 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   int* warp_cnt = row_of + kHeadDim;
   uint16_t* Vs = reinterpret_cast<uint16_t*>(smem);
   uint8_t* cV = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);
+  // boosted channels of this kv head: k, or the per-head count (plane-B rows kb..k-1,
+  // their scales and indices then stay zero)
+  int kb = k;
+  if (p.kh && need_k) {
+    kb = p.kh[h];
+    if (kb < 0 || kb > k) {
+      if (tid == 0) flag_error(p.err, KVQ_DEV_ERR_LENGTH);
+      kb = kb < 0 ? 0 : k;
+    }
+  }
 
   // ---- stage the page tiles (rows of 128 x 16-bit = 16 x 16 bytes)
   if (need_k) {
@@ -167,22 +177,47 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   // ---- a1: boosted channels (or read them back from the record)
   if (mode & kModeSelect) {
     using T2 = typename Pair<T>::type;
-    // score_c = max |K[t][c]|: thread = (channel pair tid / 4, token quarter tid % 4),
-    // packed abs/max (exact), then the four quarters by shuffles
+    // score_c = max |K[t][c]| (magnitude), or fp32(w_c * fp32(max - min)) (query-aware):
+    // thread = (channel pair tid / 4, token quarter tid % 4), packed abs/min/max (exact),
+    // then the four quarters by shuffles
     {
       const int pr = tid >> 2, qt = tid & 3;
       const uint32_t* col = reinterpret_cast<const uint32_t*>(Ks) + pr;
       const int tq = P / 4;
-      T2 m = __habs2(u32_as_pair(col[qt * tq * (kHeadDim / 2)], T()));
+      if (!p.qw) {
+        T2 m = __habs2(u32_as_pair(col[qt * tq * (kHeadDim / 2)], T()));
 #pragma unroll 8
-      for (int t = 1; t < tq; ++t) m = __hmax2(m, __habs2(u32_as_pair(col[(qt * tq + t) * (kHeadDim / 2)], T())));
-      uint32_t mb = pair_as_u32(m);
+        for (int t = 1; t < tq; ++t) m = __hmax2(m, __habs2(u32_as_pair(col[(qt * tq + t) * (kHeadDim / 2)], T())));
+        uint32_t mb = pair_as_u32(m);
 #pragma unroll
-      for (int off = 1; off < 4; off <<= 1)
-        mb = pair_as_u32(__hmax2(u32_as_pair(mb, T()), u32_as_pair(__shfl_xor_sync(kFull, mb, off), T())));
-      if (qt == 0) {
-        score[2 * pr] = bits_to_float(uint16_t(mb), T());
-        score[2 * pr + 1] = bits_to_float(uint16_t(mb >> 16), T());
+        for (int off = 1; off < 4; off <<= 1)
+          mb = pair_as_u32(__hmax2(u32_as_pair(mb, T()), u32_as_pair(__shfl_xor_sync(kFull, mb, off), T())));
+        if (qt == 0) {
+          score[2 * pr] = bits_to_float(uint16_t(mb), T());
+          score[2 * pr + 1] = bits_to_float(uint16_t(mb >> 16), T());
+        }
+      } else {
+        T2 lo = u32_as_pair(col[qt * tq * (kHeadDim / 2)], T()), hi = lo;
+#pragma unroll 8
+        for (int t = 1; t < tq; ++t) {
+          const T2 v = u32_as_pair(col[(qt * tq + t) * (kHeadDim / 2)], T());
+          lo = __hmin2(lo, v);
+          hi = __hmax2(hi, v);
+        }
+        uint32_t lb = pair_as_u32(lo), hb = pair_as_u32(hi);
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1) {
+          lb = pair_as_u32(__hmin2(u32_as_pair(lb, T()), u32_as_pair(__shfl_xor_sync(kFull, lb, off), T())));
+          hb = pair_as_u32(__hmax2(u32_as_pair(hb, T()), u32_as_pair(__shfl_xor_sync(kFull, hb, off), T())));
+        }
+        if (qt == 0) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float range = __fsub_rn(bits_to_float(uint16_t(hb >> (16 * e)), T()),
+                                          bits_to_float(uint16_t(lb >> (16 * e)), T()));
+            score[2 * pr + e] = __fmul_rn(p.qw[h * kHeadDim + 2 * pr + e], range);
+          }
+        }
       }
     }
     __syncthreads();
@@ -199,7 +234,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         rank += (so > sc) || (so == sc && o < c);
       }
       rank += __shfl_xor_sync(kFull, rank, 1);
-      const bool boosted = rank < k;
+      const bool boosted = rank < kb;
       // plane-B row of a boosted channel: boosted channels with a lower index before it
       const unsigned ballot = __ballot_sync(kFull, boosted && half == 0);
       if ((tid & 31) == 0) warp_cnt[tid >> 5] = __popc(ballot);
@@ -211,12 +246,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
         row_of[c] = row;
         if (row >= 0) rec[p.L.boost_idx + row] = uint8_t(c);
       }
+      if (tid >= kb && tid < k) rec[p.L.boost_idx + tid] = 0;  // unused rows
     }
     __syncthreads();
   } else if (mode & kModeKeys) {
     if (tid < kHeadDim) row_of[tid] = -1;
     __syncthreads();
-    if (tid < k) {
+    if (tid < kb) {
       const int c = rec[p.L.boost_idx + tid];
       if (c < kHeadDim) row_of[c] = tid;
     }
@@ -231,6 +267,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
     uint16_t* ks_out = reinterpret_cast<uint16_t*>(rec + p.L.k_scale);
     uint16_t* kz_out = reinterpret_cast<uint16_t*>(rec + p.L.k_zero);
     uint16_t* kbs_out = reinterpret_cast<uint16_t*>(rec + p.L.kb_scale);
+    if (kb < k) {
+      // plane-B rows kb..k-1 carry no channel: zero codes and zero scales
+      for (int i = tid; i < P * k; i += kQThreads) cB[i] = 0;
+      for (int i = tid; i < n_groups * (k - kb); i += kQThreads)
+        kbs_out[(i / (k - kb)) * k + kb + i % (k - kb)] = 0;
+      __syncthreads();
+    }
     for (int task = tid; task < n_groups * (kHeadDim / 2); task += kQThreads) {
       const int g = task / (kHeadDim / 2), c0 = 2 * (task % (kHeadDim / 2));
       const uint32_t* col = reinterpret_cast<const uint32_t*>(Ks + g * kKeyGroup * kHeadDim + c0);

@@ -130,7 +130,7 @@ typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 #define KVQ_DEV_ERR_RESIDUAL     2  /* append into a full residual window                            */
 #define KVQ_DEV_ERR_TABLE_FULL   4  /* flush with no free page-table slot or no destination page      */
 #define KVQ_DEV_ERR_TIMEOUT      8  /* a bounded wait for an asynchronous copy gave up                */
-#define KVQ_DEV_ERR_LENGTH      16  /* num_pages[b] or res_len[b] outside its valid range             */
+#define KVQ_DEV_ERR_LENGTH      16  /* num_pages[b], res_len[b] or a per-head boost count out of range */
 #define KVQ_DEV_ERR_RANGE       32  /* decode: an operand outside the range the kernel carries (see
                                        kvq_decode_attention, "Precision")                             */
 
@@ -214,6 +214,34 @@ KVQ_API kvq_status kvq_quantize_pages(const kvq_config* cfg, kvq_source k, kvq_s
                               void* pool, int64_t pool_pages, int32_t* err,
                               cudaStream_t stream);
 
+/* Options of the boost-channel choice, for kvq_quantize_pages_ex and
+ * kvq_flush_residual_ex (NULL options, or NULL fields, give the plain calls' behaviour).
+ *  query_weight   — query-aware ranking (MixKVQ summary on fugumt.com, Abstract: key
+ *                   channels chosen by intrinsic quantization difficulty together with
+ *                   query relevance).  Reading: device float[num_kv_heads][head_dim] of
+ *                   non-negative relevance weights w (for example the mean |q| of a
+ *                   channel over the query heads of the kv head and recent steps); a
+ *                   channel's score is fp32(w_c * fp32(max_t K - min_t K)) over the page
+ *                   (its range, which sets its 2-bit error), the highest scores are
+ *                   boosted, ties to the lower channel index.  NULL: magnitude (max |K|).
+ *  boost_per_head — per-head boost count (notes.yuuk.io wiki "KVキャッシュ量子化", open
+ *                   questions: per-head or adaptive boost ratios).  Device int32
+ *                   [num_kv_heads], each in [0, num_boost]: head h boosts that many
+ *                   channels; the record keeps its num_boost plane-B rows and the unused
+ *                   ones (codes, scales, indices) are zero, so decode attention reads
+ *                   them unchanged and they add nothing.  A count outside the range sets
+ *                   KVQ_DEV_ERR_LENGTH and is clamped.  NULL: num_boost for every head. */
+typedef struct {
+  const float* query_weight;
+  const int32_t* boost_per_head;
+} kvq_boost_options;
+
+/* kvq_quantize_pages with boost options. */
+KVQ_API kvq_status kvq_quantize_pages_ex(const kvq_config* cfg, kvq_source k, kvq_source v,
+                                         const int32_t* dst_pages, int32_t n_pages,
+                                         void* pool, int64_t pool_pages, const kvq_boost_options* opts,
+                                         int32_t* err, cudaStream_t stream);
+
 /* a4 — streaming append into the full-precision residual window (KIVI section 3:
  * recent tokens stay in full precision and new tokens are appended without touching
  * quantized pages).  k_new, v_new: dtype [batch][Hkv][D].  For every b, writes the
@@ -240,6 +268,14 @@ KVQ_API kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch,
                               int32_t max_pages, int32_t* num_pages,
                               void* pool, int64_t pool_pages, int32_t* err,
                               cudaStream_t stream);
+
+/* kvq_flush_residual with boost options (the flushed pages' channel choice). */
+KVQ_API kvq_status kvq_flush_residual_ex(const kvq_config* cfg, int32_t batch,
+                                         const void* res_k, const void* res_v, int32_t* res_len,
+                                         const int32_t* new_page, int32_t* page_table,
+                                         int32_t max_pages, int32_t* num_pages,
+                                         void* pool, int64_t pool_pages, const kvq_boost_options* opts,
+                                         int32_t* err, cudaStream_t stream);
 
 /* Scratch bytes kvq_decode_attention needs for (cfg, batch, max_pages) on the current
  * device (max_pages does not change it).  The workspace holds the partial softmax
@@ -284,6 +320,28 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool,
                                 float sm_scale, float* out,
                                 void* workspace, size_t workspace_bytes,
                                 int32_t* err, cudaStream_t stream);
+
+/* Bytes of one (page, KV head) record of a dense cache: K rows then V rows, dtype
+ * [2][page_tokens][head_dim]; 0 if cfg is not supported. */
+KVQ_API size_t kvq_dense_page_bytes(const kvq_config* cfg);
+
+/* Decode attention over an unquantized (fp16 / bf16) paged cache, on the same kernel,
+ * work line and split-K merge as kvq_decode_attention: the comparison point of the 2-bit
+ * cache (KIVI article on aibr.jp, section 4, and the Kitty summary's Abstract compare
+ * against full-precision KV; this call is that baseline on this hardware).
+ * pool: dtype [pool_pages][num_kv_heads][2][page_tokens][head_dim] (K rows, V rows);
+ * page_table: int32 [batch][max_pages]; seq_len: device int32 [batch], tokens of each
+ * sequence (0 <= seq_len[b] <= max_pages * page_tokens, the first ceil(seq_len[b] /
+ * page_tokens) table entries valid); q, out, sm_scale, workspace (the size
+ * kvq_decode_workspace_bytes gives), err and stream as for kvq_decode_attention.
+ * Products run in the cache dtype with fp32 accumulation; num_boost and key_group of cfg
+ * are not used.  max_pages * page_tokens must not exceed 1048560. */
+KVQ_API kvq_status kvq_decode_attention_dense(const kvq_config* cfg, const void* pool, int64_t pool_pages,
+                                              const void* q, int32_t batch,
+                                              const int32_t* page_table, int32_t max_pages,
+                                              const int32_t* seq_len, float sm_scale, float* out,
+                                              void* workspace, size_t workspace_bytes,
+                                              int32_t* err, cudaStream_t stream);
 
 /* Size of the library's built-in decode scratch (see kvq_decode_attention_static). */
 #define KVQ_STATIC_SCRATCH_BYTES (16u << 20)
