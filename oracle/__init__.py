@@ -101,6 +101,10 @@ def lib():
         L.kvqo_quantize_page_ex.restype = None
         L.kvqo_quantize_page_ex.argtypes = [u16p, u16p, ctypes.c_long] + [ctypes.c_int] * 5 + [
             f32p, ctypes.c_int, u8p]
+        L.kvqo_prefill_attention.restype = None
+        L.kvqo_prefill_attention.argtypes = [u16p, u16p, u16p] + [ctypes.c_int] * 5 + [ctypes.c_double, f64p, f64p]
+        L.kvqo_retain.restype = ctypes.c_int
+        L.kvqo_retain.argtypes = [f64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p]
         L.kvqo_select_boost_query.restype = None
         L.kvqo_select_boost_query.argtypes = [u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               f32p, ctypes.c_int, u8p]
@@ -253,6 +257,31 @@ def quantize_page_ex(K_bits: np.ndarray, V_bits: np.ndarray, cfg: Cfg, n_boost: 
                                 cfg.k, n, None if w is None else _p(w, ctypes.c_float), cfg.dtype,
                                 _p(rec, ctypes.c_uint8))
     return rec
+
+
+def prefill_attention(Q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray, dtype: int,
+                      sm_scale: float):
+    """Causal prefill attention and cumulative attention scores (MiniKV reading):
+    Q [L][Hq][D], K and V [L][Hkv][D] patterns -> (O fp64 [L][Hq][D], A fp64 [Hkv][L])."""
+    Q = np.ascontiguousarray(Q_bits, dtype=np.uint16)
+    K = np.ascontiguousarray(K_bits, dtype=np.uint16)
+    V = np.ascontiguousarray(V_bits, dtype=np.uint16)
+    L, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    O = np.zeros((L, Hq, D), np.float64)
+    A = np.zeros((Hkv, L), np.float64)
+    lib().kvqo_prefill_attention(_p(Q, ctypes.c_uint16), _p(K, ctypes.c_uint16), _p(V, ctypes.c_uint16), L, Hq,
+                                 Hkv, D, dtype, float(sm_scale), _p(O, ctypes.c_double), _p(A, ctypes.c_double))
+    return O, A
+
+
+def retain(A_row: np.ndarray, n_heavy: int, n_recent: int) -> np.ndarray:
+    """Kept positions of one KV head: the last n_recent, plus the n_heavy best-scored
+    of the others (ties to the lower position), ascending."""
+    a = np.ascontiguousarray(A_row, dtype=np.float64)
+    keep = np.zeros(max(1, a.size), np.int32)
+    n = lib().kvqo_retain(_p(a, ctypes.c_double), a.size, n_heavy, n_recent, _p(keep, ctypes.c_int32))
+    return keep[:n]
 
 
 def quantize_page(K_bits: np.ndarray, V_bits: np.ndarray, cfg: Cfg) -> np.ndarray:

@@ -538,3 +538,74 @@ void kvqo_decode_unit(const uint8_t* pool, int Hkv, int head, const int32_t* pag
   free(Vh);
   free(qd);
 }
+
+/* ------------------------------------------------------- prefill with token retention */
+
+/* Prefill attention with cumulative attention scores (MiniKV summary on f-binder,
+ * section "proposed method": the prompt is processed at prefill, the tokens to keep are
+ * chosen by cumulative attention score, and a two-stage selective flash-attention
+ * kernel returns the usual attention output together with those scores in linear
+ * memory).  Reading: causal self-attention over the L prompt tokens; for query head h
+ * (KV head h / gqa) and position i,
+ *   O[i][h] = sum_{j <= i} softmax_j(sm_scale * q_i . k_j) v_j,
+ * and the cumulative score of key token j of KV head kvh is the attention it receives,
+ * summed over every query position and over the gqa query heads of that KV head:
+ *   A[kvh][j] = sum_{h in kvh} sum_{i >= j} P_h[i][j].
+ * Q: [L][Hq][D], K and V: [L][Hkv][D] 16-bit patterns; O: [L][Hq][D], A: [Hkv][L] (fp64). */
+void kvqo_prefill_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int L, int Hq, int Hkv,
+                            int D, int dtype, double sm_scale, double* O, double* A) {
+  const int gqa = Hq / Hkv;
+  double* s = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+  for (int i = 0; i < Hkv * L; ++i) A[i] = 0.0;
+  for (int h = 0; h < Hq; ++h) {
+    const int kvh = h / gqa;
+    for (int i = 0; i < L; ++i) {
+      double m = -INFINITY;
+      for (int j = 0; j <= i; ++j) {
+        double d = 0.0;
+        for (int c = 0; c < D; ++c)
+          d += dt_value(Q[((long)i * Hq + h) * D + c], dtype) * dt_value(K[((long)j * Hkv + kvh) * D + c], dtype);
+        s[j] = d * sm_scale;
+        if (s[j] > m) m = s[j];
+      }
+      double l = 0.0;
+      for (int j = 0; j <= i; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+      }
+      double* o = O + ((long)i * Hq + h) * D;
+      for (int c = 0; c < D; ++c) o[c] = 0.0;
+      for (int j = 0; j <= i; ++j) {
+        const double p = s[j] / l;
+        A[(long)kvh * L + j] += p;
+        for (int c = 0; c < D; ++c) o[c] += p * dt_value(V[((long)j * Hkv + kvh) * D + c], dtype);
+      }
+    }
+  }
+  free(s);
+}
+
+/* Token retention (MiniKV summary, "proposed method": heavy hitters by cumulative
+ * attention score and a recent window, 25% of the budget each by default).  Reading:
+ * the last n_recent positions are kept; among the other positions the n_heavy with the
+ * highest score are kept, ties to the lower position.  Writes the kept positions in
+ * ascending order and returns their number (min(L, n_recent + n_heavy)). */
+int kvqo_retain(const double* A, int L, int n_heavy, int n_recent, int32_t* keep) {
+  if (n_recent > L) n_recent = L;
+  const int cut = L - n_recent;  /* positions [cut, L) are the recent window */
+  if (n_heavy > cut) n_heavy = cut;
+  char* taken = (char*)calloc(L > 0 ? L : 1, 1);
+  for (int r = 0; r < n_heavy; ++r) {
+    int best = -1;
+    for (int j = 0; j < cut; ++j) {
+      if (taken[j]) continue;
+      if (best < 0 || A[j] > A[best]) best = j;  /* strict: lower position wins ties */
+    }
+    taken[best] = 1;
+  }
+  int n = 0;
+  for (int j = 0; j < L; ++j)
+    if (j >= cut || taken[j]) keep[n++] = j;
+  free(taken);
+  return n;
+}
