@@ -21,6 +21,7 @@ __all__ = [
     "quantize_values", "quantize_pages", "append_token", "flush_residual",
     "decode_workspace_bytes", "decode_attention", "decode_attention_static", "STATIC_SCRATCH_BYTES",
     "quantize_pages_ex", "dense_page_bytes", "decode_attention_dense",
+    "prefill_workspace_bytes", "prefill_attention", "retain_tokens", "gather_tokens",
     "F16", "BF16", "torch_dtype",
     "DEV_ERR_PAGE_RANGE", "DEV_ERR_RESIDUAL", "DEV_ERR_TABLE_FULL", "DEV_ERR_TIMEOUT",
     "DEV_ERR_LENGTH", "DEV_ERR_RANGE",
@@ -155,6 +156,14 @@ def load():
         L.kvq_decode_attention_dense.restype = ctypes.c_int
         L.kvq_decode_attention_dense.argtypes = [cfgp, vp, i64, vp, i32, vp, i32, vp, ctypes.c_float, vp, vp, sz,
                                                  vp, vp]
+        L.kvq_prefill_workspace_bytes.restype = sz
+        L.kvq_prefill_workspace_bytes.argtypes = [cfgp, i32]
+        L.kvq_prefill_attention.restype = ctypes.c_int
+        L.kvq_prefill_attention.argtypes = [cfgp, vp, vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp]
+        L.kvq_retain_tokens.restype = ctypes.c_int
+        L.kvq_retain_tokens.argtypes = [cfgp, vp, i32, i32, i32, vp, vp, vp]
+        L.kvq_gather_tokens.restype = ctypes.c_int
+        L.kvq_gather_tokens.argtypes = [cfgp, vp, vp, i32, vp, i32, vp, vp, vp, vp]
         optp = ctypes.POINTER(_BoostOptions)
         L.kvq_quantize_pages_ex.restype = ctypes.c_int
         L.kvq_quantize_pages_ex.argtypes = [cfgp, _Source, _Source, vp, i32, vp, i64, optp, vp, vp]
@@ -435,3 +444,54 @@ def decode_attention_dense(cfg: Config, pool, q, page_table, seq_len, out, works
         ctypes.byref(cfg.c()), pool.data_ptr(), pool_pages, q.data_ptr(), batch, page_table.data_ptr(),
         max_pages, seq_len.data_ptr(), float(sm_scale), out.data_ptr(), workspace.data_ptr(),
         workspace.numel(), _ptr(err), _stream(stream)))
+
+
+def prefill_workspace_bytes(cfg: Config, L: int) -> int:
+    return int(load().kvq_prefill_workspace_bytes(ctypes.byref(cfg.c()), L))
+
+
+def prefill_attention(cfg: Config, q, k, v, out, scores, workspace, sm_scale: float | None = None, stream=None):
+    """Causal prefill attention with cumulative attention scores: q [L][Hq][D], k, v
+    [L][Hkv][D] (cache dtype), out fp32 [L][Hq][D], scores fp32 [Hkv][L]."""
+    dt, D = torch_dtype(cfg.dtype), cfg.head_dim
+    L = q.shape[0]
+    _need("q", q, dt, L * cfg.num_q_heads * D)
+    _need("k", k, dt, L * cfg.num_kv_heads * D)
+    _need("v", v, dt, L * cfg.num_kv_heads * D)
+    _need("out", out, torch.float32, L * cfg.num_q_heads * D)
+    _need("scores", scores, torch.float32, cfg.num_kv_heads * L)
+    _need("workspace", workspace, torch.uint8)
+    _cuda(q, k, v, out, scores, workspace, stream=stream)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    _check("kvq_prefill_attention", load().kvq_prefill_attention(
+        ctypes.byref(cfg.c()), q.data_ptr(), k.data_ptr(), v.data_ptr(), L, float(sm_scale), out.data_ptr(),
+        scores.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def retain_tokens(cfg: Config, scores, n_heavy: int, n_recent: int, keep, n_keep, stream=None):
+    """Heavy hitters plus recent window per KV head: keep int32 [Hkv][L], n_keep int32 [Hkv]."""
+    L = scores.shape[-1]
+    _need("scores", scores, torch.float32, cfg.num_kv_heads * L)
+    _need("keep", keep, torch.int32, cfg.num_kv_heads * L)
+    _need("n_keep", n_keep, torch.int32, cfg.num_kv_heads)
+    _cuda(scores, keep, n_keep, stream=stream)
+    _check("kvq_retain_tokens", load().kvq_retain_tokens(
+        ctypes.byref(cfg.c()), scores.data_ptr(), L, n_heavy, n_recent, keep.data_ptr(), n_keep.data_ptr(),
+        _stream(stream)))
+
+
+def gather_tokens(cfg: Config, k, v, keep, n: int, k_out, v_out, err=None, stream=None):
+    """k_out[t][h] = k[keep[h][t]][h] (and v) for t < n: [n][Hkv][D] of the cache dtype."""
+    dt, H, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.head_dim
+    L = k.shape[0]
+    _need("k", k, dt, L * H * D)
+    _need("v", v, dt, L * H * D)
+    _need("keep", keep, torch.int32, H * L)
+    _need("k_out", k_out, dt, n * H * D)
+    _need("v_out", v_out, dt, n * H * D)
+    _need("err", err, torch.int32, 1)
+    _cuda(k, v, keep, k_out, v_out, err, stream=stream)
+    _check("kvq_gather_tokens", load().kvq_gather_tokens(
+        ctypes.byref(cfg.c()), k.data_ptr(), v.data_ptr(), L, keep.data_ptr(), n, k_out.data_ptr(),
+        v_out.data_ptr(), _ptr(err), _stream(stream)))

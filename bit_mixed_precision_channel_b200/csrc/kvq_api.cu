@@ -311,6 +311,47 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   return cuda_status(launch_decode(p, gqa, cfg->dtype, stream));
 }
 
+size_t kvq_prefill_workspace_bytes(const kvq_config* cfg, int32_t L) {
+  if (kvq_check_config(cfg) != KVQ_OK || L < 0) return 0;
+  return (size_t(cfg->num_q_heads) * size_t(L) * sizeof(float) + 255) / 256 * 256;
+}
+
+kvq_status kvq_prefill_attention(const kvq_config* cfg, const void* q, const void* k, const void* v, int32_t L,
+                                 float sm_scale, float* out, float* scores, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (L < 0) return KVQ_ERR_INVALID_ARG;
+  if (L == 0) return KVQ_OK;
+  if (!q || !k || !v || !out || !scores || !workspace) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return KVQ_ERR_INVALID_ARG;
+  if (workspace_bytes < kvq_prefill_workspace_bytes(cfg, L)) return KVQ_ERR_CAPACITY;
+  return cuda_status(launch_prefill(q, k, v, L, cfg->num_q_heads, cfg->num_kv_heads, sm_scale, cfg->dtype, out,
+                                    static_cast<float*>(workspace), scores, stream));
+}
+
+kvq_status kvq_retain_tokens(const kvq_config* cfg, const float* scores, int32_t L, int32_t n_heavy, int32_t n_recent,
+                             int32_t* keep, int32_t* n_keep, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (L < 0 || n_heavy < 0 || n_recent < 0) return KVQ_ERR_INVALID_ARG;
+  if (L == 0) return KVQ_OK;
+  if (!scores || !keep || !n_keep) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_retain(scores, L, cfg->num_kv_heads, n_heavy, n_recent, keep, n_keep, stream));
+}
+
+kvq_status kvq_gather_tokens(const kvq_config* cfg, const void* k, const void* v, int32_t L, const int32_t* keep,
+                             int32_t n, void* k_out, void* v_out, int32_t* err, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (L < 0 || n < 0 || n > L) return KVQ_ERR_INVALID_ARG;
+  if (n == 0) return KVQ_OK;
+  if (!k || !v || !keep || !k_out || !v_out) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_gather(k, v, cfg->num_kv_heads, L, keep, n, k_out, v_out, err, stream));
+}
+
 size_t kvq_dense_page_bytes(const kvq_config* cfg) {
   if (kvq_check_config(cfg) != KVQ_OK) return 0;
   return size_t(2) * cfg->page_tokens * cfg->head_dim * 2;

@@ -340,6 +340,12 @@ cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, voi
 cudaError_t launch_flush_commit(int32_t* res_len, const int32_t* new_page, int32_t* page_table, int max_pages,
                                 int32_t* num_pages, long long pool_pages, int batch, int P, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int gqa, int dtype, cudaStream_t stream);
+cudaError_t launch_prefill(const void* q, const void* k, const void* v, int L, int Hq, int Hkv, float sm_scale,
+                           int dtype, float* out, float* lse, float* score, cudaStream_t stream);
+cudaError_t launch_retain(const float* score, int L, int Hkv, int n_heavy, int n_recent, int32_t* keep,
+                          int32_t* n_keep, cudaStream_t stream);
+cudaError_t launch_gather(const void* k, const void* v, int Hkv, int L, const int32_t* keep, int n, void* k_out,
+                          void* v_out, int32_t* err, cudaStream_t stream);
 int decode_ctas_per_sm(int gqa, int dtype, int kb, int P);
 
 // Raises a kernel's dynamic shared-memory limit once per device and size, so that

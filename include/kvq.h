@@ -321,6 +321,46 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool,
                                 void* workspace, size_t workspace_bytes,
                                 int32_t* err, cudaStream_t stream);
 
+/* ---- MiniKV prefill: attention with cumulative scores, token retention, gather ----
+ * MiniKV summary (f-binder), "proposed method": the prompt is processed at prefill, the
+ * KV states to keep are chosen by cumulative attention score — heavy hitters — together
+ * with a recent window (25% of the budget each by default), and a two-stage selective
+ * flash-attention kernel returns the attention output and those scores in linear memory.
+ * The kept tokens are then quantized like any other (keys per channel, values per token).
+ * Reading: causal attention over the L prompt tokens; the cumulative score of key token
+ * j of KV head h is the attention it receives, summed over all query positions and over
+ * the query heads of h. */
+
+/* Workspace bytes of kvq_prefill_attention (the log2-sum-exp of every query row). */
+KVQ_API size_t kvq_prefill_workspace_bytes(const kvq_config* cfg, int32_t L);
+
+/* q: dtype [L][num_q_heads][head_dim]; k, v: dtype [L][num_kv_heads][head_dim];
+ * out: fp32 [L][num_q_heads][head_dim], out[i][h] = sum_{j <= i} softmax_j(sm_scale
+ * q_i . k_j) v_j (KV head h / (Hq/Hkv)); scores: fp32 [num_kv_heads][L] cumulative
+ * attention scores.  Two kernels (output and row log2-sum-exp; then the scores, by
+ * recomputing K Q^T per key block), memory linear in L.  Products in the cache dtype,
+ * fp32 accumulate; bf16 probabilities are carried as a high and a low bf16 part. */
+KVQ_API kvq_status kvq_prefill_attention(const kvq_config* cfg, const void* q, const void* k, const void* v,
+                                         int32_t L, float sm_scale, float* out, float* scores,
+                                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Token retention per KV head: the last n_recent positions plus the n_heavy positions of
+ * highest score among the others (ties to the lower position), written ascending to
+ * keep[h][0 .. n_keep[h]) (keep: device int32 [num_kv_heads][L], n_keep: device int32
+ * [num_kv_heads]; n_keep[h] = min(L, n_heavy + n_recent)).  Scores are the fp32 values of
+ * kvq_prefill_attention (non-negative); the decision is taken on them as given. */
+KVQ_API kvq_status kvq_retain_tokens(const kvq_config* cfg, const float* scores, int32_t L,
+                                     int32_t n_heavy, int32_t n_recent, int32_t* keep, int32_t* n_keep,
+                                     cudaStream_t stream);
+
+/* The kept tokens compacted, token-major: k_out[t][h] = k[keep[h][t]][h] (and v) for
+ * t < n, every KV head keeping n tokens (n = n_keep[h] of kvq_retain_tokens).  k_out and
+ * v_out are dtype [n][num_kv_heads][head_dim], the source layout of kvq_quantize_pages.
+ * A kept position outside [0, L) sets KVQ_DEV_ERR_LENGTH and copies token 0. */
+KVQ_API kvq_status kvq_gather_tokens(const kvq_config* cfg, const void* k, const void* v, int32_t L,
+                                     const int32_t* keep, int32_t n, void* k_out, void* v_out,
+                                     int32_t* err, cudaStream_t stream);
+
 /* Bytes of one (page, KV head) record of a dense cache: K rows then V rows, dtype
  * [2][page_tokens][head_dim]; 0 if cfg is not supported. */
 KVQ_API size_t kvq_dense_page_bytes(const kvq_config* cfg);
