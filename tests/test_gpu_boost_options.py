@@ -1,6 +1,6 @@
-"""GPU parity of the boost options (SURVEY rows f3 and f4 of the method's next steps):
-the query-aware channel ranking (the MixKVQ reading: channel range over the page times a
-query-relevance weight) and the per-head boost count.  Every record byte must equal the
+"""GPU parity of the boost options: the query-aware channel ranking (the MixKVQ
+reading: channel range over the page times a query-relevance weight) and the per-head
+boost count.  Every record byte must equal the
 oracle's, through the prefill quantizer and through the residual flush; decode attention
 over such records must match the oracle within the method's tolerance."""
 import math

@@ -1,4 +1,4 @@
-"""GPU parity of the MiniKV prefill path (SURVEY row f2): causal prefill attention with
+"""GPU parity of the MiniKV prefill path: causal prefill attention with
 cumulative attention scores, heavy-hitter + recent-window retention, the gather of the
 kept tokens and their quantization.
 
