@@ -310,8 +310,7 @@ def run_gpu(args):
 
     def device_step():
         for i, c in enumerate(caches):
-            c.append(kns[i], vns[i])
-            c.flush()
+            c.append_flush(kns[i], vns[i])
             c.attend(qs[i], outs[i])
 
     def attend_only():
@@ -366,8 +365,7 @@ def run_gpu(args):
                 landed.append(ev)
         for i, c in enumerate(caches):
             stream.wait_event(landed[i])
-            c.append(kns[i], vns[i])
-            c.flush()
+            c.append_flush(kns[i], vns[i])
             c.attend(qs[i], outs[i])
             ev = torch.cuda.Event()
             ev.record(stream)
@@ -591,9 +589,8 @@ def workload_bench(name, dev, peak, min_bytes=512e6, flush_steps=0, iters=20):
         t0.record()
         for s in range(flush_steps):
             fl = c.reserve_flush_pages()
-            c.append(kn, vn)
             ev[s][0].record()
-            c.flush()
+            c.append_flush(kn, vn)
             ev[s][1].record()
             c.attend(q, out)
             c.commit_host(fl)

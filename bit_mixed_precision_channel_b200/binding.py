@@ -151,6 +151,9 @@ def load():
         L.kvq_append_token.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp, vp]
         L.kvq_flush_residual.restype = ctypes.c_int
         L.kvq_flush_residual.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, i32, vp, vp, i64, vp, vp]
+        L.kvq_append_flush.restype = ctypes.c_int
+        L.kvq_append_flush.argtypes = [cfgp, i32, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i64,
+                                       ctypes.POINTER(_BoostOptions), vp, vp, vp]
         L.kvq_dense_page_bytes.restype = sz
         L.kvq_dense_page_bytes.argtypes = [cfgp]
         L.kvq_decode_attention_dense.restype = ctypes.c_int
@@ -365,6 +368,32 @@ def flush_residual(cfg: Config, res_k, res_v, res_len, new_page, page_table, num
             ctypes.byref(cfg.c()), batch, res_k.data_ptr(), res_v.data_ptr(), res_len.data_ptr(),
             new_page.data_ptr(), page_table.data_ptr(), max_pages, num_pages.data_ptr(), pool.data_ptr(),
             pool_pages, opts, _ptr(err), _stream(stream)))
+
+
+def append_flush(cfg: Config, k_new, v_new, res_k, res_v, res_len, new_page, page_table, num_pages, pool,
+                 counters, err=None, stream=None, query_weight=None, boost_per_head=None):
+    """append_token followed by flush_residual, in one launch (kvq_append_flush).
+    counters: int32[batch], zero before the first call; every call leaves it zero."""
+    _need("page_table", page_table, torch.int32, dim=2)
+    batch, max_pages = page_table.shape
+    dt, H, P, D = torch_dtype(cfg.dtype), cfg.num_kv_heads, cfg.page_tokens, cfg.head_dim
+    _need("k_new", k_new, dt, batch * H * D)
+    _need("v_new", v_new, dt, batch * H * D)
+    _need("res_k", res_k, dt, batch * H * P * D)
+    _need("res_v", res_v, dt, batch * H * P * D)
+    for name, t in (("res_len", res_len), ("new_page", new_page), ("num_pages", num_pages),
+                    ("counters", counters)):
+        _need(name, t, torch.int32, batch)
+    _need("pool", pool, torch.uint8)
+    _need("err", err, torch.int32, 1)
+    _cuda(k_new, v_new, res_k, res_v, res_len, new_page, page_table, num_pages, pool, counters, err,
+          query_weight, boost_per_head, stream=stream)
+    pool_pages = pool.numel() // (cfg.num_kv_heads * page_bytes(cfg))
+    opts = _boost_options(cfg, query_weight, boost_per_head)
+    _check("kvq_append_flush", load().kvq_append_flush(
+        ctypes.byref(cfg.c()), batch, k_new.data_ptr(), v_new.data_ptr(), res_k.data_ptr(), res_v.data_ptr(),
+        res_len.data_ptr(), new_page.data_ptr(), page_table.data_ptr(), max_pages, num_pages.data_ptr(),
+        pool.data_ptr(), pool_pages, opts, counters.data_ptr(), _ptr(err), _stream(stream)))
 
 
 def decode_workspace_bytes(cfg: Config, batch: int, max_pages: int) -> int:

@@ -38,6 +38,7 @@ class PagedKVCache:
         self.workspace = torch.zeros(max(ws, 256), dtype=torch.uint8, device=self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.new_page = torch.full((batch,), -1, dtype=torch.int32, device=self.device)
+        self.counters = torch.zeros(batch, dtype=torch.int32, device=self.device)  # append_flush arrivals
         # host mirrors used to hand out pages
         order = list(range(pool_pages)) if page_order is None else [int(x) for x in page_order]
         if sorted(order) != list(range(pool_pages)):
@@ -129,15 +130,19 @@ class PagedKVCache:
         kb.flush_residual(self.cfg, self.res_k, self.res_v, self.res_len, self.new_page, self.page_table,
                           self.num_pages, self.pool, self.err, stream)
 
+    def append_flush(self, k_new, v_new, stream=None):
+        """append then flush, in one launch."""
+        kb.append_flush(self.cfg, k_new, v_new, self.res_k, self.res_v, self.res_len, self.new_page,
+                        self.page_table, self.num_pages, self.pool, self.counters, self.err, stream)
+
     def attend(self, q, out, sm_scale=None, stream=None):
         kb.decode_attention(self.cfg, self.pool, q, self.page_table, self.num_pages, self.res_k, self.res_v,
                             self.res_len, out, self.workspace, sm_scale, self.err, stream)
 
     def step(self, q, k_new, v_new, out, sm_scale=None, stream=None):
-        """One decode step: append, flush full windows, attend."""
+        """One decode step: append and flush full windows (one launch), attend."""
         flushing = self.reserve_flush_pages()
-        self.append(k_new, v_new, stream)
-        self.flush(stream)
+        self.append_flush(k_new, v_new, stream)
         self.attend(q, out, sm_scale, stream)
         self.commit_host(flushing)
 

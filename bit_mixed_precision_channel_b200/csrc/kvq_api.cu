@@ -225,6 +225,52 @@ kvq_status kvq_flush_residual(const kvq_config* cfg, int32_t batch, const void* 
                                pool_pages, nullptr, err, stream);
 }
 
+kvq_status kvq_append_flush(const kvq_config* cfg, int32_t batch, const void* k_new, const void* v_new, void* res_k,
+                            void* res_v, int32_t* res_len, const int32_t* new_page, int32_t* page_table,
+                            int32_t max_pages, int32_t* num_pages, void* pool, int64_t pool_pages,
+                            const kvq_boost_options* opts, int32_t* counters, int32_t* err, cudaStream_t stream) {
+  const kvq_status s = kvq_check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || max_pages < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!k_new || !v_new || !res_k || !res_v || !res_len || !new_page || !page_table || !num_pages || !pool ||
+      pool_pages <= 0 || !counters)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(res_k) || !aligned16(res_v) || !aligned16(pool))
+    return KVQ_ERR_INVALID_ARG;
+  const int P = cfg->page_tokens, Hkv = cfg->num_kv_heads, D = cfg->head_dim;
+  QuantParams p{};
+  p.k_src = static_cast<const uint16_t*>(res_k);
+  p.v_src = static_cast<const uint16_t*>(res_v);
+  p.k_page_stride = p.v_page_stride = (long long)Hkv * P * D;
+  p.k_tok_stride = p.v_tok_stride = D;
+  p.k_head_stride = p.v_head_stride = (long long)P * D;
+  p.dst_pages = new_page;
+  p.pool = static_cast<uint8_t*>(pool);
+  p.pool_pages = pool_pages;
+  p.Hkv = Hkv;
+  p.P = P;
+  p.k = cfg->num_boost;
+  p.L = make_layout(P, D, cfg->num_boost, cfg->key_group);
+  p.err = err;
+  p.mode = kModeSelect | kModeKeys | kModeValues;
+  p.max_pages = max_pages;
+  if (opts) {
+    p.qw = opts->query_weight;
+    p.kh = opts->boost_per_head;
+  }
+  p.append = 1;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.res_k = static_cast<uint16_t*>(res_k);
+  p.res_v = static_cast<uint16_t*>(res_v);
+  p.res_len_w = res_len;
+  p.num_pages_w = num_pages;
+  p.page_table = page_table;
+  p.counters = counters;
+  return cuda_status(launch_quantize(p, batch, cfg->dtype, stream));
+}
+
 kvq_status kvq_flush_residual_ex(const kvq_config* cfg, int32_t batch, const void* res_k, const void* res_v,
                                  int32_t* res_len, const int32_t* new_page, int32_t* page_table, int32_t max_pages,
                                  int32_t* num_pages, void* pool, int64_t pool_pages, const kvq_boost_options* opts,

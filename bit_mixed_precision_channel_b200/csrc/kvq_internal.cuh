@@ -307,6 +307,17 @@ struct QuantParams {
   int max_pages;
   const float* qw;     // query-aware ranking weights [Hkv][128], or null (magnitude ranking)
   const int32_t* kh;   // boosted channels per kv head [Hkv] (each <= k), or null (k for all)
+  // append-and-flush mode (a4 + a5 in one launch): the new token, the writable window,
+  // lengths and page table, and one arrival counter per sequence
+  int append;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* res_k;
+  uint16_t* res_v;
+  int32_t* res_len_w;
+  int32_t* num_pages_w;
+  int32_t* page_table;
+  int32_t* counters;
 };
 
 // Decode attention (a6 + a7).

@@ -1,60 +1,52 @@
 // kvq_quantize.cu — page quantization (boost selection, two-plane keys, per-token
 // values), residual append and residual flush for sm_100a.
 //
-// One CTA quantizes one (page, kv head): it stages the page's K and V tiles
-// ([P][128] each) in shared memory with 16-byte loads, then
+// One CTA quantizes the keys of one (page, kv head) and another its values.  A CTA
+// stages its [P][128] tile in shared memory with 16-byte asynchronous copies, then
 //   a1  ranks channels by max |K| over the page (Kitty, Dynamic Channel-wise
-//       Precision Boost; magnitude heuristic per the notes.yuuk.io wiki page),
+//       Precision Boost; magnitude heuristic per the notes.yuuk.io wiki page), or by
+//       w_c * (max - min) (MixKVQ summary, Abstract: query relevance times the
+//       channel's quantization difficulty),
 //   a2  quantizes every (key group, channel) asymmetrically — 4 bits for boosted
 //       channels, split into a high plane and a low plane of 2-bit codes, 2 bits
 //       otherwise (KIVI per-channel keys; Kitty two uniform 2-bit tensors),
 //   a3  quantizes every token's values over the head dimension (KIVI per-token values),
-// and writes the packed record.  The quantizer's fp32 operations use explicit
-// round-to-nearest intrinsics in the order the ABI documents, so codes, scales and
-// zeros are bit-identical to any implementation of that definition.
+// and writes the packed record.  Scales and zeros use explicit round-to-nearest fp32
+// operations in the order the ABI documents, so codes, scales and zeros are
+// bit-identical to any implementation of that definition.
+//
+// The codes never pass through shared memory: ldmatrix hands each lane the sixteen
+// elements of one record word (the record's word order is the mma fragment order), the
+// code of each element comes from two fused multiply-adds with the group's reciprocal
+// bracketed from below and above (equal results prove the code; the rare element near
+// a rounding boundary is redone with the IEEE divide), and byte permutes pack the codes.
 #include "kvq_internal.cuh"
 
 namespace kvq {
 
 constexpr int kQThreads = 256;
 
-// Shared memory of one quantize CTA.  A CTA quantizes either the keys of a (page, kv
-// head) (selection and both planes) or its values, so that four CTAs fit on an SM.
+// Tiles in shared memory: token t's 128 channels are 16 chunks of 16 bytes, chunk j
+// stored at j ^ (t % 8), so the eight rows one ldmatrix matrix reads, or eight
+// consecutive tokens read at one chunk, fall on eight different bank groups.
+__device__ __forceinline__ uint32_t qtile_off(int t, int chunk) {
+  return uint32_t(t) * 256u + (uint32_t(chunk ^ (t & 7)) << 4);
+}
+
+// Shared memory of one quantize CTA: the tile, then the code constants
+// {-zero, r_lo, r_hi, scale} per (key group, channel) or per token, then (keys) the
+// plane-B row of each channel and the channel of each plane-B row.
 struct QSmem {
-  static size_t key_bytes(int P, int k) {
-    return size_t(P) * kHeadDim * 2        // K tile
-           + size_t(P) * kHeadDim          // plane-A codes [P][128]
-           + size_t(P) * (k > 0 ? k : 16)  // plane-B codes [P][k]
-           + 16                            // scratch byte of channels that are not boosted
-           + kHeadDim * 4 * 2 + 16 * 4;    // scores, plane-B row of each channel, warp counts
-  }
-  static size_t value_bytes(int P) {
-    return size_t(P) * kHeadDim * 2  // V tile
-           + size_t(P) * kHeadDim;   // value codes [P][128]
-  }
-  static size_t bytes(int P, int k, int mode) {
+  __host__ __device__ static size_t tile(int P) { return size_t(P) * kHeadDim * 2; }
+  static size_t key_bytes(int P) { return tile(P) + size_t(P / kKeyGroup) * kHeadDim * 16 + 2 * kHeadDim; }
+  static size_t value_bytes(int P) { return tile(P) + size_t(P) * 16; }
+  static size_t bytes(int P, int mode) {
     size_t b = 0;
-    if (mode & (kModeSelect | kModeKeys)) b = key_bytes(P, k);
+    if (mode & (kModeSelect | kModeKeys)) b = key_bytes(P);
     if (mode & kModeValues) b = b > value_bytes(P) ? b : value_bytes(P);
     return b;
   }
 };
-
-// 16 codes given by element order (one byte each) -> one word, element e = 8a + 2b + f
-// at bit 8b + 4f + 2a.  Bytes 4i..4i+3 (element 4i + m) land at bit
-// 16*(i & 1) + 2*(i >> 1) + 4*m.
-__device__ __forceinline__ uint32_t pack16(const uint8_t* c) {
-  const uint4 v = lds128(c);
-  const uint32_t q[4] = {v.x, v.y, v.z, v.w};
-  uint32_t w = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t x = q[i];
-    const uint32_t nib = (x & 0x3u) | ((x >> 4) & 0x30u) | ((x >> 8) & 0x300u) | ((x >> 12) & 0x3000u);
-    w |= nib << (16 * (i & 1) + 2 * (i >> 1));
-  }
-  return w;
-}
 
 // Quantizes one group with the documented fp32 op order; returns the scale as float
 // and writes scale/zero bits.  min/max are exact; a zero minimum is stored as +0.
@@ -70,6 +62,7 @@ __device__ __forceinline__ float quant_params(float mn, float mx, int qmax, uint
   return bits_to_float(sbits, T());
 }
 
+// The definition: code = clamp(rint((x - zero) / scale), 0, qmax) in fp32.
 __device__ __forceinline__ int quant_code(float x, float zero, float scale, int qmax) {
   if (scale == 0.0f) return 0;
   const float t = __fdiv_rn(__fsub_rn(x, zero), scale);
@@ -78,74 +71,83 @@ __device__ __forceinline__ int quant_code(float x, float zero, float scale, int 
   return int(r);
 }
 
-// Reciprocal of a group's scale for quant_bits_fma, or 0 when the fast path may not be
-// used (scale 0, or below the smallest normal float, where the approximate reciprocal
-// flushes).
-__device__ __forceinline__ float quant_rcp(float scale) {
-  if (!(scale >= 1.17549435e-38f)) return 0.0f;
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(scale));
-  return r;
-}
-
-// The code quant_code gives, bit for bit, without a divide in almost every case.
-// x - zero >= 0, and scale >= (max - min) / qmax (rounded up), so x - zero <= qmax * scale
-// and no code exceeds qmax: the clamp never acts.  fma(d, rcp, 1.5 * 2^23) rounds the
-// exact product d * rcp to an integer n held in the low byte of the result's bits
-// (0x4B400000 + n, returned).  d * rcp is within 2^-17 of the correctly rounded quotient
-// (rcp.approx: relative error below 2^-22; the divide: half an ulp, at most 2^-20), so n
-// is the code unless d * rcp lies within 2^-14 of a rounding boundary n +- 1/2.  There
-// `near` is set and the caller redoes the element with quant_code.  With rcp = 0
-// (scale 0) the code is 0, as quant_code gives.
-__device__ __forceinline__ uint32_t quant_bits_fma(float x, float zero, float rcp, bool& near) {
-  const float d = __fsub_rn(x, zero);
-  const float t = __fmaf_rn(d, rcp, 12582912.0f);
-  const float res = __fmaf_rn(d, rcp, -__fsub_rn(t, 12582912.0f));
-  near = !(fabsf(res) < 0.5f - 1.0f / 16384.0f);
-  return __float_as_uint(t);
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p) {
-  pdl_wait();
-  const int item = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  const int P = p.P, k = p.k;
-  int dst;
-  if (p.flush) {
-    if (p.res_len[item] != P) return;
-    dst = p.dst_pages[item];
-    const int np = p.num_pages[item];
-    if (dst < 0 || np < 0 || np >= p.max_pages) {
-      if (tid == 0 && h == 0) flag_error(p.err, KVQ_DEV_ERR_TABLE_FULL);
-      return;
-    }
+// Constants of the divide-free code of a group with scale s and zero z: {-z, r_lo,
+// r_hi, s}.  r_lo and r_hi lie 8 units in the last place below and above the correctly
+// rounded 1/s, so for d = x - z >= 0 the exact product d * r_lo is at most, and d * r_hi
+// at least, the rounded quotient fl(d / s) (each of 1/s -> rcp and d / s -> fl loses at
+// most 2^-24 relative; eight units are at least 8 * 2^-24).  Round-to-nearest-even is
+// monotone, so when d * r_lo and d * r_hi round to the same integer, fl(d / s) rounds
+// to it too: that is the code (the stored scale is rounded up, so no code exceeds qmax
+// and the clamp never acts).  Scale 0 gives r_lo = r_hi = 0 (every code 0, as the
+// definition gives); a scale whose reciprocal is not comfortably normal gives r_lo = 0,
+// r_hi = inf, which sends every element of the group to the exact path.
+__device__ __forceinline__ float4 code_consts(float zero, float scale) {
+  float rlo, rhi;
+  if (scale == 0.0f) {
+    rlo = rhi = 0.0f;
+  } else if (scale >= 0x1p-100f && scale <= 0x1p100f) {
+    const uint32_t rb = __float_as_uint(__frcp_rn(scale));
+    rlo = __uint_as_float(rb - 8u);
+    rhi = __uint_as_float(rb + 8u);
   } else {
-    dst = p.dst_pages[item];
+    rlo = 0.0f;
+    rhi = __uint_as_float(0x7f800000u);
   }
-  if (dst < 0 || dst >= p.pool_pages) {
-    if (tid == 0) flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
-    return;
-  }
-  uint8_t* rec = p.pool + (size_t(dst) * p.Hkv + h) * p.L.record;
+  return make_float4(-zero, rlo, rhi, scale);
+}
+
+// x - zero in fp32 with one rounding for both 16-bit elements of a pair (PTX
+// mixed-precision add: the 16-bit operand converts exactly, the sum rounds once).
+__device__ __forceinline__ void sub_pair(uint32_t w, float nz0, float nz1, float& d0, float& d1, __half) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %3;\n\tadd.rn.f32.f16 %1, h, %4;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "r"(w), "f"(nz0), "f"(nz1));
+}
+__device__ __forceinline__ void sub_pair(uint32_t w, float nz0, float nz1, float& d0, float& d1, __nv_bfloat16) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %3;\n\tadd.rn.f32.bf16 %1, h, %4;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "r"(w), "f"(nz0), "f"(nz1));
+}
+
+// Bits of fma(d, r, 1.5 * 2^23): for 0 <= d * r < 2^22 the result is 1.5 * 2^23 plus
+// d * r rounded to the nearest integer (ties to even), so its low byte is that integer.
+__device__ __forceinline__ uint32_t code_bits(float d, float r) {
+  return __float_as_uint(__fmaf_rn(d, r, 12582912.0f));
+}
+
+// Low bytes of four words -> one word, byte i from x_i.
+__device__ __forceinline__ uint32_t low_bytes(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  return __byte_perm(__byte_perm(x0, x1, 0x0040), __byte_perm(x2, x3, 0x0040), 0x5410);
+}
+
+// Total order of fp32 scores as unsigned integers (larger score -> larger key).
+__device__ __forceinline__ uint32_t order_key(float s) {
+  const uint32_t u = __float_as_uint(__fadd_rn(s, 0.0f));  // -0 -> +0, like a float compare
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Quantizes the window or page tile of (item, kv head h) into record rec: the key part
+// (z = 0) or the value part (z = gridDim.z - 1) of the requested modes.  last_k / last_v,
+// when given, replace the tile's last token (the token an append-and-flush just wrote).
+template <typename T>
+__device__ __forceinline__ void quantize_record(const QuantParams& p, int item, int h, uint8_t* rec,
+                                                const uint16_t* last_k, const uint16_t* last_v) {
+  const int tid = threadIdx.x;
+  const int P = p.P, k = p.k;
 
   // z = 0: the key part of the requested modes, z = gridDim.z - 1: the value part
   const int kmodes = blockIdx.z == 0 ? p.mode & (kModeSelect | kModeKeys) : 0;
   const int mode = kmodes | (blockIdx.z == gridDim.z - 1 ? p.mode & kModeValues : 0);
   const bool need_k = kmodes != 0;
-  const bool need_v = mode & kModeValues;
+  const bool need_v = (mode & kModeValues) && !need_k;
 
-  extern __shared__ __align__(16) uint8_t smem[];
-  // key part: K tile, plane A codes [token][key position], plane B codes [token][boost
-  // position], scores; value part: V tile, value codes [token][channel]
-  uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* cA = reinterpret_cast<uint8_t*>(Ks + P * kHeadDim);
-  uint8_t* cB = cA + P * kHeadDim;
-  uint8_t* cScratch = cB + P * (k > 0 ? k : 16);  // plane-B bytes of channels that are not boosted
-  float* score = reinterpret_cast<float*>(cScratch + 16);
-  int* row_of = reinterpret_cast<int*>(score + kHeadDim);
-  int* warp_cnt = row_of + kHeadDim;
-  uint16_t* Vs = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* cV = reinterpret_cast<uint8_t*>(Vs + P * kHeadDim);
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t tile = smem_addr(smem);
+  float4* qc = reinterpret_cast<float4*>(smem + QSmem::tile(P));  // keys [P/32][128], values [P]
+  int8_t* row_of = reinterpret_cast<int8_t*>(qc + (P / kKeyGroup) * kHeadDim);  // plane-B row of a channel
+  uint8_t* chan_of = reinterpret_cast<uint8_t*>(row_of + kHeadDim);             // channel of a plane-B row
   // boosted channels of this kv head: k, or the per-head count (plane-B rows kb..k-1,
   // their scales and indices then stay zero)
   int kb = k;
@@ -157,273 +159,473 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
     }
   }
 
-  // ---- stage the page tiles (rows of 128 x 16-bit = 16 x 16 bytes)
-  if (need_k) {
-    const uint16_t* src = p.k_src + item * p.k_page_stride + h * p.k_head_stride;
+  // ---- stage the tile (rows of 128 x 16-bit = 16 chunks of 16 bytes, swizzled)
+  {
+    const uint16_t* src = need_k ? p.k_src + item * p.k_page_stride + h * p.k_head_stride
+                                 : p.v_src + item * p.v_page_stride + h * p.v_head_stride;
+    const long long ts = need_k ? p.k_tok_stride : p.v_tok_stride;
+    const uint16_t* last = need_k ? last_k : last_v;
     for (int i = tid; i < P * 16; i += kQThreads) {
       const int t = i >> 4, c = i & 15;
-      reinterpret_cast<uint4*>(Ks)[i] = __ldg(reinterpret_cast<const uint4*>(src + t * p.k_tok_stride) + c);
+      const uint16_t* row = (last && t == P - 1) ? last : src + t * ts;
+      cp_async16(smem + qtile_off(t, c), row + c * 8, 16);
     }
-  }
-  if (need_v) {
-    const uint16_t* src = p.v_src + item * p.v_page_stride + h * p.v_head_stride;
-    for (int i = tid; i < P * 16; i += kQThreads) {
-      const int t = i >> 4, c = i & 15;
-      reinterpret_cast<uint4*>(Vs)[i] = __ldg(reinterpret_cast<const uint4*>(src + t * p.v_tok_stride) + c);
-    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   }
   __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
 
-  // ---- a1: boosted channels (or read them back from the record)
-  if (mode & kModeSelect) {
+  if (need_k) {
     using T2 = typename Pair<T>::type;
-    // score_c = max |K[t][c]| (magnitude), or fp32(w_c * fp32(max - min)) (query-aware):
-    // thread = (channel pair tid / 4, token quarter tid % 4), packed abs/min/max (exact),
-    // then the four quarters by shuffles
-    {
-      const int pr = tid >> 2, qt = tid & 3;
-      const uint32_t* col = reinterpret_cast<const uint32_t*>(Ks) + pr;
-      const int tq = P / 4;
-      if (!p.qw) {
-        T2 m = __habs2(u32_as_pair(col[qt * tq * (kHeadDim / 2)], T()));
+    const int NG = P / kKeyGroup;
+    // ---- exact min / max per (key group, channel pair), packed pairs (exact)
+    const int g1 = tid >> 6, c0 = 2 * (tid & 63);
+    const bool has_pair = g1 < NG;
+    uint32_t lob = 0, hib = 0;
+    uint32_t* mm = reinterpret_cast<uint32_t*>(qc);  // scratch [NG][min, max][64 pairs]
+    if (has_pair) {
+      const uint8_t* base = smem + (c0 & 7) * 2;
+      const int t0 = g1 * kKeyGroup;
+      T2 lo = u32_as_pair(lds32(base + qtile_off(t0, c0 >> 3)), T()), hi = lo;
 #pragma unroll 8
-        for (int t = 1; t < tq; ++t) m = __hmax2(m, __habs2(u32_as_pair(col[(qt * tq + t) * (kHeadDim / 2)], T())));
-        uint32_t mb = pair_as_u32(m);
+      for (int t = 1; t < kKeyGroup; ++t) {
+        const T2 v = u32_as_pair(lds32(base + qtile_off(t0 + t, c0 >> 3)), T());
+        lo = __hmin2(lo, v);
+        hi = __hmax2(hi, v);
+      }
+      lob = pair_as_u32(lo);
+      hib = pair_as_u32(hi);
+      if (mode & kModeSelect) {
+        mm[(2 * g1) * 64 + (tid & 63)] = lob;
+        mm[(2 * g1 + 1) * 64 + (tid & 63)] = hib;
+      }
+    }
+    __syncthreads();
+
+    // ---- a1: boosted channels (or read them back from the record)
+    if (mode & kModeSelect) {
+      if (warp == 0) {
+        // lane holds channels lane + 32 i; score from the page's exact min / max
+        uint32_t key[4];
 #pragma unroll
-        for (int off = 1; off < 4; off <<= 1)
-          mb = pair_as_u32(__hmax2(u32_as_pair(mb, T()), u32_as_pair(__shfl_xor_sync(kFull, mb, off), T())));
-        if (qt == 0) {
-          score[2 * pr] = bits_to_float(uint16_t(mb), T());
-          score[2 * pr + 1] = bits_to_float(uint16_t(mb >> 16), T());
+        for (int i = 0; i < 4; ++i) {
+          const int c = lane + 32 * i;
+          float mn = __int_as_float(0x7f800000), mx = -mn;
+          for (int g = 0; g < NG; ++g) {
+            mn = fminf(mn, bits_to_float(uint16_t(mm[(2 * g) * 64 + (c >> 1)] >> (16 * (c & 1))), T()));
+            mx = fmaxf(mx, bits_to_float(uint16_t(mm[(2 * g + 1) * 64 + (c >> 1)] >> (16 * (c & 1))), T()));
+          }
+          const float sc = p.qw ? __fmul_rn(p.qw[h * kHeadDim + c], __fsub_rn(mx, mn)) : fmaxf(fabsf(mn), fabsf(mx));
+          key[i] = order_key(sc);
         }
-      } else {
-        T2 lo = u32_as_pair(col[qt * tq * (kHeadDim / 2)], T()), hi = lo;
-#pragma unroll 8
-        for (int t = 1; t < tq; ++t) {
-          const T2 v = u32_as_pair(col[(qt * tq + t) * (kHeadDim / 2)], T());
-          lo = __hmin2(lo, v);
-          hi = __hmax2(hi, v);
-        }
-        uint32_t lb = pair_as_u32(lo), hb = pair_as_u32(hi);
+        // the kb largest keys, ties to the lower channel: kb rounds of a warp max
+        uint32_t sel = 0;
+        if (kb >= kHeadDim) {
+          sel = 0xfu;
+        } else {
+          uint32_t ek[4] = {key[0], key[1], key[2], key[3]};
+          for (int it = 0; it < kb; ++it) {
+            const uint32_t M = __reduce_max_sync(kFull, max(max(ek[0], ek[1]), max(ek[2], ek[3])));
+            uint32_t li = 255u;
 #pragma unroll
-        for (int off = 1; off < 4; off <<= 1) {
-          lb = pair_as_u32(__hmin2(u32_as_pair(lb, T()), u32_as_pair(__shfl_xor_sync(kFull, lb, off), T())));
-          hb = pair_as_u32(__hmax2(u32_as_pair(hb, T()), u32_as_pair(__shfl_xor_sync(kFull, hb, off), T())));
-        }
-        if (qt == 0) {
+            for (int i = 3; i >= 0; --i)
+              if (!((sel >> i) & 1u) && key[i] == M) li = uint32_t(lane + 32 * i);
+            const uint32_t I = __reduce_min_sync(kFull, li);
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float range = __fsub_rn(bits_to_float(uint16_t(hb >> (16 * e)), T()),
-                                          bits_to_float(uint16_t(lb >> (16 * e)), T()));
-            score[2 * pr + e] = __fmul_rn(p.qw[h * kHeadDim + 2 * pr + e], range);
+            for (int i = 0; i < 4; ++i)
+              if (uint32_t(lane + 32 * i) == I) {
+                sel |= 1u << i;
+                ek[i] = 0u;
+              }
+          }
+        }
+        // plane-B rows: the boosted channels in ascending order
+        int before = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool b = (sel >> i) & 1u;
+          const unsigned ball = __ballot_sync(kFull, b);
+          const int c = lane + 32 * i;
+          const int row = b ? before + __popc(ball & ((1u << lane) - 1u)) : -1;
+          row_of[c] = int8_t(row);
+          if (row >= 0) {
+            rec[p.L.boost_idx + row] = uint8_t(c);
+            chan_of[row] = uint8_t(c);
+          }
+          before += __popc(ball);
+        }
+        for (int j = kb + lane; j < k; j += 32) {  // unused rows
+          rec[p.L.boost_idx + j] = 0;
+          chan_of[j] = 0xff;
+        }
+      }
+    } else {
+      if (tid < kHeadDim) row_of[tid] = -1;
+      __syncthreads();
+      if (tid < k) {
+        const int c = tid < kb ? rec[p.L.boost_idx + tid] : 0xff;
+        chan_of[tid] = uint8_t(c < kHeadDim ? c : 0xff);
+        if (c < kHeadDim) row_of[c] = int8_t(tid);
+      }
+    }
+    __syncthreads();
+
+    if (mode & kModeKeys) {
+      uint16_t* ks_out = reinterpret_cast<uint16_t*>(rec + p.L.k_scale);
+      uint16_t* kz_out = reinterpret_cast<uint16_t*>(rec + p.L.k_zero);
+      uint16_t* kbs_out = reinterpret_cast<uint16_t*>(rec + p.L.kb_scale);
+      // ---- a2 constants: one thread per (group, channel pair), min / max still in registers
+      for (int i = tid; i < NG * (k - kb); i += kQThreads)  // rows kb..k-1 carry no channel
+        kbs_out[(i / (k - kb)) * k + kb + i % (k - kb)] = 0;
+      if (has_pair) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = c0 + e, j = row_of[c];
+          uint16_t sb, zb;
+          float zero;
+          const float scale = quant_params<T>(bits_to_float(uint16_t(lob >> (16 * e)), T()),
+                                              bits_to_float(uint16_t(hib >> (16 * e)), T()), j >= 0 ? 15 : 3, sb,
+                                              zb, zero);
+          // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
+          const int pm = key_meta_pos(c);
+          ks_out[g1 * kHeadDim + pm] = j >= 0 ? exact_bits(4.0f * scale, T()) : sb;
+          kz_out[g1 * kHeadDim + pm] = zb;
+          if (j >= 0) kbs_out[g1 * k + j] = sb;
+          qc[g1 * kHeadDim + c] = code_consts(zero, scale);
+        }
+      }
+      __syncthreads();
+
+      // ---- a2 plane A (and plane B when every channel is boosted: row j = channel j).
+      // Warp -> (group g, word half hh), 4 tokens per step; lane -> token tbase + lane / 8,
+      // word half a = (lane / 4) % 2, q = lane % 4.  Its eight elements are channels
+      // c(j, f) = 64hh + 32a + 8j + 2q + f, which sit at element 8a + 2j + f of record
+      // word 2q + hh of the token; the partner lane (a ^ 1) holds the other eight.
+      {
+        const bool all_b = kb == kHeadDim;
+        const int per = P / 16;
+        const int it0 = warp * per;
+        const int g = it0 >> 4, hh = (it0 >> 3) & 1;
+        const int a = (lane >> 2) & 1, q = lane & 3;
+        float nz[8], rlo[8], rhi[8];
+        uint32_t bm[2] = {0u, 0u};  // byte j = 0x3f where channel c(j, f) is boosted
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            const int c = 64 * hh + 32 * a + 8 * j + 2 * q + f;
+            const float4 v = qc[g * kHeadDim + c];
+            nz[2 * j + f] = v.x;
+            rlo[2 * j + f] = v.y;
+            rhi[2 * j + f] = v.z;
+            if (row_of[c] >= 0) bm[f] |= 0x3fu << (8 * j);
+          }
+        // ldmatrix: lane L gives row L % 8 of matrix L / 8 = j: token offset (L % 8) / 2,
+        // half (L % 8) % 2, chunk 8hh + 4 * half + j
+        const int rho = lane & 7;
+        const int chunk = 8 * hh + 4 * (rho & 1) + (lane >> 3);
+        uint32_t* kA = reinterpret_cast<uint32_t*>(rec + p.L.k_codes);
+        uint32_t* kB = reinterpret_cast<uint32_t*>(rec + p.L.kb_codes);
+        for (int it = 0; it < per; ++it) {
+          const int tbase = 32 * g + 4 * ((it0 + it) & 7);
+          uint32_t x[4];
+          ldmatrix_x4(x, tile + qtile_off(tbase + (rho >> 1), chunk));
+          uint32_t lo[8], acc = 0u;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float d0, d1;
+            sub_pair(x[j], nz[2 * j], nz[2 * j + 1], d0, d1, T());
+            lo[2 * j] = code_bits(d0, rlo[2 * j]);
+            lo[2 * j + 1] = code_bits(d1, rlo[2 * j + 1]);
+            acc |= (lo[2 * j] ^ code_bits(d0, rhi[2 * j])) | (lo[2 * j + 1] ^ code_bits(d1, rhi[2 * j + 1]));
+          }
+          uint32_t X0 = low_bytes(lo[0], lo[2], lo[4], lo[6]);  // element 8a + 2j, byte j
+          uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]);  // element 8a + 2j + 1
+          if (acc != 0u) {  // near a rounding boundary: the IEEE divide decides
+            X0 = X1 = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+              for (int f = 0; f < 2; ++f) {
+                const int c = 64 * hh + 32 * a + 8 * j + 2 * q + f;
+                const float xv = bits_to_float(uint16_t(x[j] >> (16 * f)), T());
+                const uint32_t code = uint32_t(
+                    quant_code(xv, -nz[2 * j + f], qc[g * kHeadDim + c].w, ((bm[f] >> (8 * j)) & 1u) ? 15 : 3));
+                (f ? X1 : X0) |= code << (8 * j);
+              }
+          }
+          // plane A: the code, or its high bits where the channel is boosted
+          const uint32_t A0 = (((X0 >> 2) & bm[0]) | (X0 & ~bm[0])) & 0x03030303u;
+          const uint32_t A1 = (((X1 >> 2) & bm[1]) | (X1 & ~bm[1])) & 0x03030303u;
+          const uint32_t wa = A0 + 16u * A1;
+          const uint32_t wa_other = __shfl_xor_sync(kFull, wa, 4);
+          const int t = tbase + (lane >> 3);
+          if (a == 0) kA[t * 8 + 2 * q + hh] = wa + 4u * wa_other;
+          if (all_b) {
+            const uint32_t wb = (X0 & 0x03030303u) + 16u * (X1 & 0x03030303u);
+            const uint32_t wb_other = __shfl_xor_sync(kFull, wb, 4);
+            if (a == 0) kB[t * 8 + 2 * q + hh] = wb + 4u * wb_other;
+          }
+        }
+      }
+
+      // ---- a2 plane B: the low bits of the boosted channels.  Task = (4 tokens of one
+      // group, plane-B word wb); its sixteen elements are rows j = 16s + 8r + 2q + f at
+      // word position 4(k/16)q + 4s + 2r + f - 16wb, gathered from their channels.
+      if (k > 0 && kb < kHeadDim) {
+        const int KW = k / 16;
+        const int n_tasks = KW * P / 4;
+        uint32_t* kB = reinterpret_cast<uint32_t*>(rec + p.L.kb_codes);
+        const int lg = 31 - __clz(4 * KW);  // log2(4 KW)
+        for (int task = tid; task < n_tasks; task += kQThreads) {
+          const int wb = task & (KW - 1), t0 = 4 * (task / KW), g = t0 >> 5;
+          uint32_t word[4] = {0u, 0u, 0u, 0u}, acc[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 1
+          for (int a = 0; a < 2; ++a) {
+            uint32_t co[8];
+            float nz[8], rlo[8], rhi[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {  // element e = 8a + i
+              const int pos = 16 * wb + 8 * a + i;
+              const int q = pos >> lg, rem = pos & ((1 << lg) - 1);
+              const int j = 16 * (rem >> 2) + 8 * ((rem >> 1) & 1) + 2 * q + (rem & 1);
+              const int c = chan_of[j];
+              if (c < kHeadDim) {
+                const float4 v = qc[g * kHeadDim + c];
+                nz[i] = v.x;
+                rlo[i] = v.y;
+                rhi[i] = v.z;
+                co[i] = uint32_t((c >> 3) << 4 | (c & 7) << 1);
+              } else {  // no channel: code 0
+                nz[i] = rlo[i] = rhi[i] = 0.0f;
+                co[i] = 0u;
+              }
+            }
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+              const int t = t0 + n;
+              const uint32_t sw = uint32_t(t & 7) << 4;
+              uint32_t lo[8];
+#pragma unroll
+              for (int i = 0; i < 8; i += 2) {
+                const uint32_t xl = *reinterpret_cast<const uint16_t*>(smem + t * 256 + (co[i] ^ sw));
+                const uint32_t xh = *reinterpret_cast<const uint16_t*>(smem + t * 256 + (co[i + 1] ^ sw));
+                float d0, d1;
+                sub_pair(xl | (xh << 16), nz[i], nz[i + 1], d0, d1, T());
+                lo[i] = code_bits(d0, rlo[i]);
+                lo[i + 1] = code_bits(d1, rlo[i + 1]);
+                acc[n] |= (lo[i] ^ code_bits(d0, rhi[i])) | (lo[i + 1] ^ code_bits(d1, rhi[i + 1]));
+              }
+              // element 8a + 2b + f at bit 8b + 4f + 2a
+              const uint32_t X0 = low_bytes(lo[0], lo[2], lo[4], lo[6]) & 0x03030303u;
+              const uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]) & 0x03030303u;
+              word[n] |= (X0 + 16u * X1) << (2 * a);
+            }
+          }
+#pragma unroll
+          for (int n = 0; n < 4; ++n) {
+            const int t = t0 + n;
+            if (acc[n] != 0u) {  // near a rounding boundary: the IEEE divide decides
+              word[n] = 0u;
+              for (int e = 0; e < 16; ++e) {
+                const int pos = 16 * wb + e;
+                const int q = pos >> lg, rem = pos & ((1 << lg) - 1);
+                const int j = 16 * (rem >> 2) + 8 * ((rem >> 1) & 1) + 2 * q + (rem & 1);
+                const int c = chan_of[j];
+                if (c >= kHeadDim) continue;
+                const float4 v = qc[g * kHeadDim + c];
+                const float xv = bits_to_float(
+                    *reinterpret_cast<const uint16_t*>(smem + qtile_off(t, c >> 3) + (c & 7) * 2), T());
+                word[n] |= uint32_t(quant_code(xv, -v.x, v.w, 15) & 3) << elem_bit(e);
+              }
+            }
+            kB[t * KW + wb] = word[n];
           }
         }
       }
     }
-    __syncthreads();
-    // rank of channel c: channels with a higher score, or an equal score and a lower
-    // index; two threads per channel (channels c' < 64 and >= 64), summed by a shuffle
-    {
-      const int c = tid >> 1, half = tid & 1;
-      const float sc = score[c];
-      int rank = 0;
-#pragma unroll 8
-      for (int i = 0; i < kHeadDim / 2; ++i) {
-        const int o = half * (kHeadDim / 2) + i;
-        const float so = score[o];
-        rank += (so > sc) || (so == sc && o < c);
-      }
-      rank += __shfl_xor_sync(kFull, rank, 1);
-      const bool boosted = rank < kb;
-      // plane-B row of a boosted channel: boosted channels with a lower index before it
-      const unsigned ballot = __ballot_sync(kFull, boosted && half == 0);
-      if ((tid & 31) == 0) warp_cnt[tid >> 5] = __popc(ballot);
-      __syncthreads();
-      if (half == 0) {
-        int before = 0;
-        for (int w = 0; w < (tid >> 5); ++w) before += warp_cnt[w];
-        const int row = boosted ? before + int(__popc(ballot & ((1u << (tid & 31)) - 1u))) : -1;
-        row_of[c] = row;
-        if (row >= 0) rec[p.L.boost_idx + row] = uint8_t(c);
-      }
-      if (tid >= kb && tid < k) rec[p.L.boost_idx + tid] = 0;  // unused rows
-    }
-    __syncthreads();
-  } else if (mode & kModeKeys) {
-    if (tid < kHeadDim) row_of[tid] = -1;
-    __syncthreads();
-    if (tid < kb) {
-      const int c = rec[p.L.boost_idx + tid];
-      if (c < kHeadDim) row_of[c] = tid;
-    }
-    __syncthreads();
   }
 
-  // ---- a2: keys, one task per (group, pair of adjacent channels): 32-bit loads and
-  //      packed min/max (exact) over the group's tokens
-  if (mode & kModeKeys) {
-    using T2 = typename Pair<T>::type;
-    const int n_groups = P / kKeyGroup;
-    uint16_t* ks_out = reinterpret_cast<uint16_t*>(rec + p.L.k_scale);
-    uint16_t* kz_out = reinterpret_cast<uint16_t*>(rec + p.L.k_zero);
-    uint16_t* kbs_out = reinterpret_cast<uint16_t*>(rec + p.L.kb_scale);
-    if (kb < k) {
-      // plane-B rows kb..k-1 carry no channel: zero codes and zero scales
-      for (int i = tid; i < P * k; i += kQThreads) cB[i] = 0;
-      for (int i = tid; i < n_groups * (k - kb); i += kQThreads)
-        kbs_out[(i / (k - kb)) * k + kb + i % (k - kb)] = 0;
-      __syncthreads();
-    }
-    for (int task = tid; task < n_groups * (kHeadDim / 2); task += kQThreads) {
-      const int g = task / (kHeadDim / 2), c0 = 2 * (task % (kHeadDim / 2));
-      const uint32_t* col = reinterpret_cast<const uint32_t*>(Ks + g * kKeyGroup * kHeadDim + c0);
-      T2 lo = u32_as_pair(col[0], T()), hi = lo;
-#pragma unroll 8
-      for (int t = 1; t < kKeyGroup; ++t) {
-        const T2 v = u32_as_pair(col[t * (kHeadDim / 2)], T());
-        lo = __hmin2(lo, v);
-        hi = __hmax2(hi, v);
-      }
-      const uint32_t lob = pair_as_u32(lo), hib = pair_as_u32(hi);
-      float scale[2], rcp[2], zero[2];
-      int qmax[2], j[2], pc[2], pj[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int c = c0 + e;
-        j[e] = row_of[c];
-        qmax[e] = j[e] >= 0 ? 15 : 3;
-        pc[e] = key_pos(c);
-        pj[e] = j[e] >= 0 ? boost_pos(j[e], k / 16) : 0;
-        uint16_t sb, zb;
-        scale[e] = quant_params<T>(bits_to_float(uint16_t(lob >> (16 * e)), T()),
-                                   bits_to_float(uint16_t(hib >> (16 * e)), T()), qmax[e], sb, zb, zero[e]);
-        rcp[e] = quant_rcp(scale[e]);
-        // plane A of a boosted channel carries the high bits: scale 4*s4 (exact)
-        const int pm = key_meta_pos(c);
-        ks_out[g * kHeadDim + pm] = j[e] >= 0 ? exact_bits(4.0f * scale[e], T()) : sb;
-        kz_out[g * kHeadDim + pm] = zb;
-        if (j[e] >= 0) kbs_out[g * k + j[e]] = sb;
-      }
-      // codes of the group's 32 tokens; plane A gets code >> 2 for a boosted channel (its
-      // low bits go to plane B) and the code itself otherwise; a channel that is not
-      // boosted writes its "plane B" byte to a scratch row.  Elements within 2^-14 of a
-      // rounding boundary (or of a group whose scale has no fast reciprocal) are redone
-      // with the IEEE divide afterwards.
-      uint8_t* a_base[2];
-      uint8_t* b_base[2];
-      int shift[2];
-      bool all_exact[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        a_base[e] = cA + g * kKeyGroup * kHeadDim + pc[e];
-        b_base[e] = j[e] >= 0 ? cB + g * kKeyGroup * k + pj[e] : cScratch;
-        shift[e] = j[e] >= 0 ? 2 : 0;
-        all_exact[e] = rcp[e] == 0.0f && scale[e] != 0.0f;
-      }
-      uint64_t redo = 0;
-#pragma unroll 8
-      for (int t = 0; t < kKeyGroup; ++t) {
-        const uint32_t w = col[t * (kHeadDim / 2)];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          // the low byte of the bits is the code (the packing keeps two bits per byte)
-          bool near;
-          const uint32_t bits = quant_bits_fma(bits_to_float(uint16_t(w >> (16 * e)), T()), zero[e], rcp[e], near);
-          redo |= uint64_t(near || all_exact[e]) << (2 * t + e);
-          a_base[e][t * kHeadDim] = uint8_t(bits >> shift[e]);
-          b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(bits);
-        }
-      }
-      while (redo) {
-        const int bit = __ffsll((long long)redo) - 1;
-        redo &= redo - 1;
-        const int t = bit >> 1, e = bit & 1;
-        const uint32_t code = uint32_t(quant_code(bits_to_float(uint16_t(col[t * (kHeadDim / 2)] >> (16 * e)), T()),
-                                                  zero[e], scale[e], qmax[e]));
-        a_base[e][t * kHeadDim] = uint8_t(code >> shift[e]);
-        b_base[e][t * (j[e] >= 0 ? k : 0)] = uint8_t(code);
-      }
-    }
-  }
-
-  // ---- a3: values, four tokens per warp (a quarter-warp each, 16 channels per lane)
   if (need_v) {
     using T2 = typename Pair<T>::type;
-    const int warp = tid >> 5, lane = tid & 31, ql = lane & 7;
     uint16_t* vs_out = reinterpret_cast<uint16_t*>(rec + p.L.v_scale);
     uint16_t* vz_out = reinterpret_cast<uint16_t*>(rec + p.L.v_zero);
-    for (int t0 = 4 * warp; t0 < P; t0 += 4 * (kQThreads / 32)) {
-      const int t = t0 + (lane >> 3);
-      const uint16_t* row = Vs + t * kHeadDim + 16 * ql;
-      const uint4 r0 = lds128(row), r1 = lds128(row + 8);
-      const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-      T2 lo = u32_as_pair(wv[0], T()), hi = lo;
+    // ---- a3 constants: two threads per token (64 channels each), packed min / max
+    {
+      const int t = tid >> 1, hf = tid & 1;
+      if (t < P) {  // whole warps
+        T2 lo, hi;
 #pragma unroll
-      for (int i = 1; i < 8; ++i) {
-        lo = __hmin2(lo, u32_as_pair(wv[i], T()));
-        hi = __hmax2(hi, u32_as_pair(wv[i], T()));
-      }
-      float mn = fminf(bits_to_float(uint16_t(pair_as_u32(lo)), T()), bits_to_float(uint16_t(pair_as_u32(lo) >> 16), T()));
-      float mx = fmaxf(bits_to_float(uint16_t(pair_as_u32(hi)), T()), bits_to_float(uint16_t(pair_as_u32(hi) >> 16), T()));
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = lds128(smem + qtile_off(t, 8 * hf + ((i + 4 * hf) & 7)));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int off = 4; off > 0; off >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(kFull, mn, off));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-      }
-      uint16_t sb, zb;
-      float zero;
-      const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
-      const float rcp = quant_rcp(scale);
-      uint32_t packed[4] = {0u, 0u, 0u, 0u};
-      bool redo = rcp == 0.0f && scale != 0.0f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
-        bool near;
-        packed[i >> 2] |= (quant_bits_fma(x, zero, rcp, near) & 0xffu) << (8 * (i & 3));
-        redo |= near;
-      }
-      if (redo) {  // near a rounding boundary: the IEEE divide decides
-#pragma unroll
-        for (int i = 0; i < 4; ++i) packed[i] = 0u;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float x = bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))), T());
-          packed[i >> 2] |= uint32_t(quant_code(x, zero, scale, 3)) << (8 * (i & 3));
+          for (int n = 0; n < 4; ++n) {
+            const T2 x = u32_as_pair(w[n], T());
+            if (i == 0 && n == 0) {
+              lo = hi = x;
+            } else {
+              lo = __hmin2(lo, x);
+              hi = __hmax2(hi, x);
+            }
+          }
+        }
+        float mn = fminf(bits_to_float(uint16_t(pair_as_u32(lo)), T()), bits_to_float(uint16_t(pair_as_u32(lo) >> 16), T()));
+        float mx = fmaxf(bits_to_float(uint16_t(pair_as_u32(hi)), T()), bits_to_float(uint16_t(pair_as_u32(hi) >> 16), T()));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        if (hf == 0) {
+          uint16_t sb, zb;
+          float zero;
+          const float scale = quant_params<T>(mn, mx, 3, sb, zb, zero);
+          vs_out[value_meta_pos(t)] = sb;
+          vz_out[value_meta_pos(t)] = zb;
+          qc[t] = code_consts(zero, scale);
         }
       }
-      *reinterpret_cast<uint4*>(cV + t * kHeadDim + 16 * ql) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      if (ql == 0) {
-        vs_out[value_meta_pos(t)] = sb;
-        vz_out[value_meta_pos(t)] = zb;
+    }
+    __syncthreads();
+
+    // ---- a3 codes.  Warp -> group g and P/32 consecutive channel blocks m; lane (w, q)
+    // builds record word ((2g + m/4) * 32 + lane) * 4 + m % 4, whose element
+    // e = 8a + 2b + f (b = 2u + v) is token 32g + 16a + 8u + 2q + f, channel 16m + 8v + w:
+    // exactly what ldmatrix.trans of the matrices (a, u, v) hands this lane.
+    {
+      const int NT = P / 32;
+      const int task0 = warp * NT, g = task0 >> 3;
+      const int q = lane & 3;
+      float nz[8], rlo[8], rhi[8];  // token (a, u, f) at index 4a + 2u + f
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 32 * g + 16 * (i >> 2) + 8 * ((i >> 1) & 1) + 2 * q + (i & 1);
+        const float4 v = qc[t];
+        nz[i] = v.x;
+        rlo[i] = v.y;
+        rhi[i] = v.z;
+      }
+      const int mi = lane >> 3, rho = lane & 7;
+      uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes) +
+                     ((2 * g + ((task0 & 7) >> 2)) * 32 + lane) * 4 + (task0 & 3);
+#pragma unroll 1
+      for (int n = 0; n < NT; ++n) {
+        const int m = (task0 + n) & 7;
+        uint32_t word = 0u, acc = 0u;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          uint32_t x[4];
+          ldmatrix_x4_trans(x, tile + qtile_off(32 * g + 16 * a + 8 * (mi >> 1) + rho, 2 * m + (mi & 1)));
+          uint32_t lo[8];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int ti = 4 * a + 2 * (b >> 1);
+            float d0, d1;
+            sub_pair(x[b], nz[ti], nz[ti + 1], d0, d1, T());
+            lo[2 * b] = code_bits(d0, rlo[ti]);
+            lo[2 * b + 1] = code_bits(d1, rlo[ti + 1]);
+            acc |= (lo[2 * b] ^ code_bits(d0, rhi[ti])) | (lo[2 * b + 1] ^ code_bits(d1, rhi[ti + 1]));
+          }
+          const uint32_t X0 = low_bytes(lo[0], lo[2], lo[4], lo[6]) & 0x03030303u;
+          const uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]) & 0x03030303u;
+          word += (X0 + 16u * X1) << (2 * a);
+        }
+        if (acc != 0u) {  // near a rounding boundary: the IEEE divide decides
+          word = 0u;
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            uint32_t x[4];
+            ldmatrix_x4_trans(x, tile + qtile_off(32 * g + 16 * a + 8 * (mi >> 1) + rho, 2 * m + (mi & 1)));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int b = i >> 1, f = i & 1;
+              const int t = 32 * g + 16 * a + 8 * (b >> 1) + 2 * q + f;
+              const float4 v = qc[t];
+              const float xv = bits_to_float(uint16_t(x[b] >> (16 * f)), T());
+              word |= uint32_t(quant_code(xv, -v.x, v.w, 3)) << elem_bit(8 * a + i);
+            }
+          }
+        }
+        vq[n] = word;
       }
     }
   }
-  __syncthreads();
+}
 
-  // ---- pack the code planes into the record
-  if (mode & kModeKeys) {
-    uint32_t* kA = reinterpret_cast<uint32_t*>(rec + p.L.k_codes);
-    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) kA[i] = pack16(cA + 16 * i);
-    const int kbw = k / 16;
-    uint32_t* kB = reinterpret_cast<uint32_t*>(rec + p.L.kb_codes);
-    for (int i = tid; i < P * kbw; i += kQThreads) kB[i] = pack16(cB + 16 * i);
-  }
-  if (need_v) {
-    uint32_t* vq = reinterpret_cast<uint32_t*>(rec + p.L.v_codes);
-    for (int i = tid; i < P * (kHeadDim / 16); i += kQThreads) {
-      // value-code word i = ((2g + (m >> 2)) * 32 + 4w + q) * 4 + (m & 3): its element
-      // e = 8a + 2b + f holds token 32g + 2q + 16a + 8(b >> 1) + f and channel
-      // 16m + w + 8(b & 1), at bit elem_bit(e)
-      const int mm = i & 3, ln = (i >> 2) & 31, blk = i >> 7;
-      const uint8_t* base = cV + (32 * (blk >> 1) + 2 * (ln & 3)) * kHeadDim + 16 * (4 * (blk & 1) + mm) + (ln >> 2);
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int a = e >> 3, b = (e >> 1) & 3, f = e & 1;
-        word |= uint32_t(base[(16 * a + 8 * (b >> 1) + f) * kHeadDim + 8 * (b & 1)] & 3u) << elem_bit(e);
+// Modes: quantize pages (dst_pages), flush full windows (flush), or append-and-flush
+// (append: a4 + a5 in one launch).  In the last, every CTA of sequence `item` appends its
+// row of the new token (z = 0: keys, z = 1: values of kv head h) at position res_len of
+// the window, and when the window is then full quantizes its part of the window into the
+// page new_page reserves.  The last of the sequence's 2 * Hkv CTAs to arrive writes the
+// lengths and the page-table entry, so every CTA has read the old length before it
+// changes.  The outcome, error bits included, is that of kvq_append_token followed by
+// kvq_flush_residual.
+template <typename T>
+__global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_constant__ QuantParams p) {
+  pdl_wait();
+  const int item = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int P = p.P;
+  int dst = -1, np = 0, r = 0;
+  bool go = false, app = false;
+  const uint16_t* last = nullptr;
+  if (p.append) {
+    const bool first = h == 0 && blockIdx.z == 0;
+    r = p.res_len_w[item];
+    if (r < 0 || r > P) {  // the append flags it; the flush skips a window that is not full
+      if (first && tid == 0) flag_error(p.err, r > P ? KVQ_DEV_ERR_RESIDUAL : KVQ_DEV_ERR_LENGTH);
+      return;
+    }
+    app = r < P;  // r == P: a full window left by an earlier skipped flush
+    if (!app && first && tid == 0) flag_error(p.err, KVQ_DEV_ERR_RESIDUAL);
+    const size_t hrow = size_t(item) * p.Hkv + h;
+    const uint16_t* src = (blockIdx.z == 0 ? p.k_new : p.v_new) + hrow * kHeadDim;
+    if (app && tid < 16)
+      reinterpret_cast<uint4*>(blockIdx.z == 0 ? p.res_k : p.res_v)[(hrow * P + r) * 16 + tid] =
+          reinterpret_cast<const uint4*>(src)[tid];
+    if (!app || r + 1 == P) {
+      dst = p.dst_pages[item];
+      np = p.num_pages_w[item];
+      if (dst < 0 || np < 0 || np >= p.max_pages) {
+        if (first && tid == 0) flag_error(p.err, KVQ_DEV_ERR_TABLE_FULL);
+      } else if (dst >= p.pool_pages) {
+        if (tid == 0) flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
+      } else {
+        go = true;
+        if (app) last = src;  // the token just appended, read from its source
       }
-      vq[i] = word;
+    }
+  } else {
+    if (p.flush) {
+      if (p.res_len[item] != P) return;
+      dst = p.dst_pages[item];
+      np = p.num_pages[item];
+      if (dst < 0 || np < 0 || np >= p.max_pages) {
+        if (tid == 0 && h == 0) flag_error(p.err, KVQ_DEV_ERR_TABLE_FULL);
+        return;
+      }
+    } else {
+      dst = p.dst_pages[item];
+    }
+    if (dst < 0 || dst >= p.pool_pages) {
+      if (tid == 0) flag_error(p.err, KVQ_DEV_ERR_PAGE_RANGE);
+      return;
+    }
+    go = true;
+  }
+  if (go) quantize_record<T>(p, item, h, p.pool + (size_t(dst) * p.Hkv + h) * p.L.record, last, last);
+  if (p.append) {
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      const int n = atomicAdd(p.counters + item, 1);
+      if (n == int(gridDim.y * gridDim.z) - 1) {
+        p.counters[item] = 0;
+        if (go) {
+          p.page_table[size_t(item) * p.max_pages + np] = dst;
+          p.num_pages_w[item] = np + 1;
+          p.res_len_w[item] = 0;
+        } else if (app) {
+          p.res_len_w[item] = r + 1;
+        }
+      }
     }
   }
   pdl_trigger();
@@ -480,7 +682,7 @@ __global__ void flush_commit_kernel(int32_t* res_len, const int32_t* new_page, i
 
 cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream) {
   if (n_items <= 0) return cudaSuccess;
-  const size_t smem = QSmem::bytes(p.P, p.k, p.mode);
+  const size_t smem = QSmem::bytes(p.P, p.mode);
   // keys and values of a page in separate CTAs when both are requested
   const bool both = (p.mode & (kModeSelect | kModeKeys)) && (p.mode & kModeValues);
   const dim3 grid(n_items, p.Hkv, both ? 2 : 1);

@@ -277,6 +277,26 @@ KVQ_API kvq_status kvq_flush_residual_ex(const kvq_config* cfg, int32_t batch,
                                          void* pool, int64_t pool_pages, const kvq_boost_options* opts,
                                          int32_t* err, cudaStream_t stream);
 
+/* a4 + a5 in one launch: for every b, kvq_append_token's append followed by
+ * kvq_flush_residual(_ex)'s flush of a window the append filled (KIVI section 3: the
+ * streaming append, and the residual quantized once a whole page has accumulated).  The
+ * arguments are those two calls' arguments together; the final window, lengths, page
+ * table, records and error bits equal what the two calls would leave, including a window
+ * that was already full (KVQ_DEV_ERR_RESIDUAL, then flushed if new_page[b] is valid).
+ * One CTA per (sequence, KV head, keys | values) appends its row and quantizes its part;
+ * the last of a sequence's CTAs to finish updates res_len, num_pages and page_table, so
+ * no CTA sees a length another has already changed.
+ * counters: device int32[batch], zero before the first call (clear once after
+ * allocating); every call leaves them zero.  opts may be NULL.  Errors as for the two
+ * calls; a NULL pointer or misaligned buffer returns KVQ_ERR_INVALID_ARG. */
+KVQ_API kvq_status kvq_append_flush(const kvq_config* cfg, int32_t batch,
+                                    const void* k_new, const void* v_new,
+                                    void* res_k, void* res_v, int32_t* res_len,
+                                    const int32_t* new_page, int32_t* page_table,
+                                    int32_t max_pages, int32_t* num_pages,
+                                    void* pool, int64_t pool_pages, const kvq_boost_options* opts,
+                                    int32_t* counters, int32_t* err, cudaStream_t stream);
+
 /* Scratch bytes kvq_decode_attention needs for (cfg, batch, max_pages) on the current
  * device (max_pages does not change it).  The workspace holds the partial softmax
  * states of sequences split across CTAs (one slot per pair of CTA and (sequence, KV

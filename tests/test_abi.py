@@ -29,7 +29,7 @@ def lib():
 def test_header_declares_the_expected_calls():
     names = _declared()
     for n in ["kvq_select_boost_channels", "kvq_quantize_page_keys", "kvq_quantize_values",
-              "kvq_quantize_pages", "kvq_append_token", "kvq_flush_residual", "kvq_decode_attention",
+              "kvq_quantize_pages", "kvq_append_token", "kvq_flush_residual", "kvq_append_flush", "kvq_decode_attention",
               "kvq_decode_workspace_bytes", "kvq_page_layout", "kvq_page_bytes", "kvq_check_config",
               "kvq_status_string"]:
         assert n in names
@@ -76,6 +76,13 @@ def test_calls_reject_bad_arguments_before_any_launch(lib):
     odd_stride = kb._Source(0x1000, 128 * 8 * 128, 8 * 128 + 1, 128)
     assert lib.kvq_quantize_pages(c, odd_stride, odd_stride, 0x100, 1, 0x1000, 1, None, None) == 1
     assert lib.kvq_flush_residual(c, 2, None, None, None, None, None, 4, None, None, 1, None, None) == 1
+    p16 = 0x1000
+    assert lib.kvq_append_flush(c, 2, p16, p16, p16, p16, p16, p16, p16, 4, p16, p16, 1, None, None, None,
+                                None) == 1  # no counters
+    assert lib.kvq_append_flush(c, 2, p16 + 8, p16, p16, p16, p16, p16, p16, 4, p16, p16, 1, None, p16, None,
+                                None) == 1  # misaligned token
+    assert lib.kvq_append_flush(c, 0, None, None, None, None, None, None, None, 4, None, None, 1, None, None,
+                                None, None) == 0
     assert lib.kvq_decode_attention(c, None, 1, None, 2, None, 4, None, None, None, None, 0.1, None, None, 0,
                                     None, None) == 1
     # workspace smaller than kvq_decode_workspace_bytes -> KVQ_ERR_CAPACITY
