@@ -474,7 +474,7 @@ def run_gpu(args):
                      "per_launch_bytes": bytes_attn, "ms_per_launch": round(attn_ms, 5)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": args.steps * L_layers * 4,
+        "gpu_launches": args.steps * L_layers * 2,  # append_flush + decode per layer
         "clocks": clock_info,
     }
     if world == 1 and not args.no_configs:

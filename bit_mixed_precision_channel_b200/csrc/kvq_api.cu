@@ -353,6 +353,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
   p.part = static_cast<float*>(workspace);
   p.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.part_bytes);
   p.n_ctas = pl.ctas;
+  p.n_sms = sm_count();
   p.err = err;
   return cuda_status(launch_decode(p, gqa, cfg->dtype, stream));
 }
@@ -441,6 +442,7 @@ kvq_status kvq_decode_attention_dense(const kvq_config* cfg, const void* pool, i
   p.part = static_cast<float*>(workspace);
   p.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.part_bytes);
   p.n_ctas = pl.ctas;
+  p.n_sms = sm_count();
   p.err = err;
   return cuda_status(launch_decode(p, cfg->num_q_heads / cfg->num_kv_heads, cfg->dtype, stream));
 }

@@ -594,6 +594,19 @@ __device__ __forceinline__ void cursor_next(const DecodeParams& p, Cursor& c) {
 __device__ __forceinline__ int owner_cta(int s, int W, int C) { return int(floor(double(s) * C / W)); }
 __device__ __forceinline__ int range_start(int i, int W, int C) { return int(ceil(double(W) * i / C)); }
 
+// Range index of CTA b.  The grid fills every resident slot at once and the hardware puts
+// CTA b on SM b mod S (S SMs, n = c * S CTAs), so SM s holds CTAs s, s + S, s + 2S, ...
+// Consecutive ranges are about a fifth of a unit long on the 8B-shaped layer, and S of
+// them span almost a whole number of units: CTAs s + jS would hold ranges at the same phase
+// of their units (all page stages, or all unit ends) and some SMs would get the heavy mix
+// four times.  Rotating block j of S ranges by j puts an SM's ranges j ranges apart in
+// phase.  (Any other placement only changes which ranges share an SM.)
+__device__ __forceinline__ int range_of_cta(int b, int n, int S) {
+  if (S <= 0 || n % S != 0) return b;
+  const int j = b / S, s = b - j * S;
+  return (s + j) % S + j * S;
+}
+
 // Owners of positions on the weight line: the line is cut into Cs equal ranges and CTA
 // i owns range i.  Every range is at least 4 long, so every owner between a unit's
 // first and last owner holds an item of the unit.
@@ -1012,7 +1025,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (GQA <= 4 ? 4 : 2))
   __shared__ CtaShared<GQA, P> sh;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
-  const int cta = blockIdx.x;
+  const int cta = range_of_cta(blockIdx.x, p.n_ctas, p.n_sms);
   // the grid fills every resident slot at once, so the next kernel in the stream may be
   // scheduled right away: its CTAs take the slots this grid releases
   pdl_wait();

@@ -339,6 +339,7 @@ struct DecodeParams {
   float* part;    // [n_ctas + batch * Hkv][GQA][128 + 4]: unnormalised output, max, sum
   uint32_t* cnt;  // [batch * Hkv] arrival counters
   int n_ctas;     // grid size: SMs x resident CTAs per SM
+  int n_sms;      // SMs of the device
   int32_t* err;
   // dense mode: tokens per sequence; pool then holds raw pages [pool_pages][Hkv][2][P][128]
   // (K rows, V rows) of the cache dtype, and num_pages / res_len / res_k / res_v are unused

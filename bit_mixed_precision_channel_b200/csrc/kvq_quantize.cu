@@ -528,19 +528,25 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
           const uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]) & 0x03030303u;
           word += (X0 + 16u * X1) << (2 * a);
         }
-        if (acc != 0u) {  // near a rounding boundary: the IEEE divide decides
-          word = 0u;
+        // Near a rounding boundary the IEEE divide decides.  The fragments are loaded again
+        // by the whole warp (ldmatrix is a warp-wide instruction and must not run in a
+        // branch that only some lanes take); the lanes that need it rebuild their word.
+        if (__any_sync(kFull, acc != 0u)) {
+          const bool redo = acc != 0u;
+          if (redo) word = 0u;
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
             uint32_t x[4];
             ldmatrix_x4_trans(x, tile + qtile_off(32 * g + 16 * a + 8 * (mi >> 1) + rho, 2 * m + (mi & 1)));
+            if (redo) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int b = i >> 1, f = i & 1;
-              const int t = 32 * g + 16 * a + 8 * (b >> 1) + 2 * q + f;
-              const float4 v = qc[t];
-              const float xv = bits_to_float(uint16_t(x[b] >> (16 * f)), T());
-              word |= uint32_t(quant_code(xv, -v.x, v.w, 3)) << elem_bit(8 * a + i);
+              for (int i = 0; i < 8; ++i) {
+                const int b = i >> 1, f = i & 1;
+                const int t = 32 * g + 16 * a + 8 * (b >> 1) + 2 * q + f;
+                const float4 v = qc[t];
+                const float xv = bits_to_float(uint16_t(x[b] >> (16 * f)), T());
+                word |= uint32_t(quant_code(xv, -v.x, v.w, 3)) << elem_bit(8 * a + i);
+              }
             }
           }
         }
