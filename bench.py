@@ -310,7 +310,8 @@ def run_gpu(args):
 
     def device_step():
         for i, c in enumerate(caches):
-            c.append_flush(kns[i], vns[i])
+            c.append(kns[i], vns[i])
+            c.flush()
             c.attend(qs[i], outs[i])
 
     def attend_only():
@@ -365,7 +366,8 @@ def run_gpu(args):
                 landed.append(ev)
         for i, c in enumerate(caches):
             stream.wait_event(landed[i])
-            c.append_flush(kns[i], vns[i])
+            c.append(kns[i], vns[i])
+            c.flush()
             c.attend(qs[i], outs[i])
             ev = torch.cuda.Event()
             ev.record(stream)
@@ -474,7 +476,7 @@ def run_gpu(args):
                      "per_launch_bytes": bytes_attn, "ms_per_launch": round(attn_ms, 5)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": args.steps * L_layers * 2,  # append_flush + decode per layer
+        "gpu_launches": args.steps * L_layers * 4,  # append, flush, commit, decode per layer
         "clocks": clock_info,
     }
     if world == 1 and not args.no_configs:
@@ -589,8 +591,9 @@ def workload_bench(name, dev, peak, min_bytes=512e6, flush_steps=0, iters=20):
         t0.record()
         for s in range(flush_steps):
             fl = c.reserve_flush_pages()
+            c.append(kn, vn)
             ev[s][0].record()
-            c.append_flush(kn, vn)
+            c.flush()
             ev[s][1].record()
             c.attend(q, out)
             c.commit_host(fl)

@@ -35,10 +35,13 @@ __device__ __forceinline__ uint32_t qtile_off(int t, int chunk) {
 
 // Shared memory of one quantize CTA: the tile, then the code constants
 // {-zero, r_lo, r_hi, scale} per (key group, channel) or per token, then (keys) the
-// plane-B row of each channel and the channel of each plane-B row.
+// plane-B row of each channel, the channel of each plane-B row, the ranking keys and
+// per-warp counts.
 struct QSmem {
   __host__ __device__ static size_t tile(int P) { return size_t(P) * kHeadDim * 2; }
-  static size_t key_bytes(int P) { return tile(P) + size_t(P / kKeyGroup) * kHeadDim * 16 + 2 * kHeadDim; }
+  static size_t key_bytes(int P) {
+    return tile(P) + size_t(P / kKeyGroup) * kHeadDim * 16 + 2 * kHeadDim + kHeadDim * 4 + 8 * 4;
+  }
   static size_t value_bytes(int P) { return tile(P) + size_t(P) * 16; }
   static size_t bytes(int P, int mode) {
     size_t b = 0;
@@ -115,6 +118,17 @@ __device__ __forceinline__ void sub_pair(uint32_t w, float nz0, float nz1, float
 // d * r rounded to the nearest integer (ties to even), so its low byte is that integer.
 __device__ __forceinline__ uint32_t code_bits(float d, float r) {
   return __float_as_uint(__fmaf_rn(d, r, 12582912.0f));
+}
+
+// The code of one element whose two bracketed products rounded to different integers;
+// k is the one from r_lo.  Inputs on the 16-bit grid often sit exactly on a rounding
+// boundary (d = (k + 1/2) s): the rounded quotient is then exactly k + 1/2 and rint takes
+// the even neighbour.  fma(-(k + 1/2), s, d) is the exact difference (one rounding of a
+// value that is either 0 or far above the smallest subnormal), so it tells a tie apart
+// without a divide; anything else is decided by the IEEE divide.
+__device__ __forceinline__ uint32_t fix_code(float d, float x, float nz, float scale, uint32_t k, int qmax) {
+  if (__fmaf_rn(-(float(k) + 0.5f), scale, d) == 0.0f) return k + (k & 1u);
+  return uint32_t(quant_code(x, -nz, scale, qmax));
 }
 
 // Low bytes of four words -> one word, byte i from x_i.
@@ -204,60 +218,60 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
 
     // ---- a1: boosted channels (or read them back from the record)
     if (mode & kModeSelect) {
-      if (warp == 0) {
-        // lane holds channels lane + 32 i; score from the page's exact min / max
-        uint32_t key[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = lane + 32 * i;
-          float mn = __int_as_float(0x7f800000), mx = -mn;
-          for (int g = 0; g < NG; ++g) {
-            mn = fminf(mn, bits_to_float(uint16_t(mm[(2 * g) * 64 + (c >> 1)] >> (16 * (c & 1))), T()));
-            mx = fmaxf(mx, bits_to_float(uint16_t(mm[(2 * g + 1) * 64 + (c >> 1)] >> (16 * (c & 1))), T()));
-          }
-          const float sc = p.qw ? __fmul_rn(p.qw[h * kHeadDim + c], __fsub_rn(mx, mn)) : fmaxf(fabsf(mn), fabsf(mx));
-          key[i] = order_key(sc);
+      uint32_t* keys = reinterpret_cast<uint32_t*>(chan_of + kHeadDim);  // [128]
+      int* warp_cnt = reinterpret_cast<int*>(keys + kHeadDim);           // [8]
+      if (tid < kHeadDim) {
+        // score from the page's exact min / max: max(|min|, |max|) (magnitude) or
+        // w * (max - min) (query-aware)
+        const int c = tid;
+        float mn = __int_as_float(0x7f800000), mx = -mn;
+        for (int g = 0; g < NG; ++g) {
+          mn = fminf(mn, bits_to_float(uint16_t(mm[(2 * g) * 64 + (c >> 1)] >> (16 * (c & 1))), T()));
+          mx = fmaxf(mx, bits_to_float(uint16_t(mm[(2 * g + 1) * 64 + (c >> 1)] >> (16 * (c & 1))), T()));
         }
-        // the kb largest keys, ties to the lower channel: kb rounds of a warp max
-        uint32_t sel = 0;
-        if (kb >= kHeadDim) {
-          sel = 0xfu;
-        } else {
-          uint32_t ek[4] = {key[0], key[1], key[2], key[3]};
-          for (int it = 0; it < kb; ++it) {
-            const uint32_t M = __reduce_max_sync(kFull, max(max(ek[0], ek[1]), max(ek[2], ek[3])));
-            uint32_t li = 255u;
-#pragma unroll
-            for (int i = 3; i >= 0; --i)
-              if (!((sel >> i) & 1u) && key[i] == M) li = uint32_t(lane + 32 * i);
-            const uint32_t I = __reduce_min_sync(kFull, li);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (uint32_t(lane + 32 * i) == I) {
-                sel |= 1u << i;
-                ek[i] = 0u;
-              }
-          }
+        // A magnitude is a 16-bit value widened to fp32, so its 13 low bits are zero:
+        // the channel index fills them and every key is unique (ties to the lower index).
+        keys[c] = p.qw ? order_key(__fmul_rn(p.qw[h * kHeadDim + c], __fsub_rn(mx, mn)))
+                       : (__float_as_uint(__fadd_rn(fmaxf(fabsf(mn), fabsf(mx)), 0.0f)) | uint32_t(127 - c));
+      }
+      __syncthreads();
+      // rank of channel c: channels ahead of it, two threads per channel (64 each)
+      const int c = tid >> 1, half = tid & 1;
+      const uint32_t kc = keys[c];
+      int rank = 0;
+      if (!p.qw) {
+#pragma unroll 4
+        for (int i = 0; i < 64; i += 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(keys + 64 * half + i);
+          rank += int(v.x > kc) + int(v.y > kc) + int(v.z > kc) + int(v.w > kc);
         }
-        // plane-B rows: the boosted channels in ascending order
+      } else {
+#pragma unroll 8
+        for (int i = 0; i < 64; ++i) {
+          const int o = 64 * half + i;
+          const uint32_t ko = keys[o];
+          rank += int(ko > kc || (ko == kc && o < c));
+        }
+      }
+      rank += __shfl_xor_sync(kFull, rank, 1);
+      const bool boosted = rank < kb;
+      // plane-B row of a boosted channel: boosted channels with a lower index before it
+      const unsigned ballot = __ballot_sync(kFull, boosted && half == 0);
+      if (lane == 0) warp_cnt[warp] = __popc(ballot);
+      __syncthreads();
+      if (half == 0) {
         int before = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const bool b = (sel >> i) & 1u;
-          const unsigned ball = __ballot_sync(kFull, b);
-          const int c = lane + 32 * i;
-          const int row = b ? before + __popc(ball & ((1u << lane) - 1u)) : -1;
-          row_of[c] = int8_t(row);
-          if (row >= 0) {
-            rec[p.L.boost_idx + row] = uint8_t(c);
-            chan_of[row] = uint8_t(c);
-          }
-          before += __popc(ball);
+        for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+        const int row = boosted ? before + __popc(ballot & ((1u << lane) - 1u)) : -1;
+        row_of[c] = int8_t(row);
+        if (row >= 0) {
+          rec[p.L.boost_idx + row] = uint8_t(c);
+          chan_of[row] = uint8_t(c);
         }
-        for (int j = kb + lane; j < k; j += 32) {  // unused rows
-          rec[p.L.boost_idx + j] = 0;
-          chan_of[j] = 0xff;
-        }
+      }
+      if (tid >= kb && tid < k) {  // unused rows
+        rec[p.L.boost_idx + tid] = 0;
+        chan_of[tid] = 0xff;
       }
     } else {
       if (tid < kHeadDim) row_of[tid] = -1;
@@ -341,17 +355,21 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
           }
           uint32_t X0 = low_bytes(lo[0], lo[2], lo[4], lo[6]);  // element 8a + 2j, byte j
           uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]);  // element 8a + 2j + 1
-          if (acc != 0u) {  // near a rounding boundary: the IEEE divide decides
-            X0 = X1 = 0u;
+          if (acc != 0u) {  // an element near a rounding boundary
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
               for (int f = 0; f < 2; ++f) {
-                const int c = 64 * hh + 32 * a + 8 * j + 2 * q + f;
+                uint32_t& X = f ? X1 : X0;
                 const float xv = bits_to_float(uint16_t(x[j] >> (16 * f)), T());
-                const uint32_t code = uint32_t(
-                    quant_code(xv, -nz[2 * j + f], qc[g * kHeadDim + c].w, ((bm[f] >> (8 * j)) & 1u) ? 15 : 3));
-                (f ? X1 : X0) |= code << (8 * j);
+                const float d = __fadd_rn(xv, nz[2 * j + f]);
+                const uint32_t k0 = (X >> (8 * j)) & 0xffu;
+                if (code_bits(d, rhi[2 * j + f]) != 0x4B400000u + k0) {
+                  const int c = 64 * hh + 32 * a + 8 * j + 2 * q + f;
+                  const uint32_t code = fix_code(d, xv, nz[2 * j + f], qc[g * kHeadDim + c].w, k0,
+                                                 ((bm[f] >> (8 * j)) & 1u) ? 15 : 3);
+                  X = (X & ~(0xffu << (8 * j))) | (code << (8 * j));
+                }
               }
           }
           // plane A: the code, or its high bits where the channel is boosted
@@ -379,7 +397,7 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
         const int lg = 31 - __clz(4 * KW);  // log2(4 KW)
         for (int task = tid; task < n_tasks; task += kQThreads) {
           const int wb = task & (KW - 1), t0 = 4 * (task / KW), g = t0 >> 5;
-          uint32_t word[4] = {0u, 0u, 0u, 0u}, acc[4] = {0u, 0u, 0u, 0u};
+          uint32_t word[4] = {0u, 0u, 0u, 0u};
 #pragma unroll 1
           for (int a = 0; a < 2; ++a) {
             uint32_t co[8];
@@ -396,7 +414,7 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
                 rlo[i] = v.y;
                 rhi[i] = v.z;
                 co[i] = uint32_t((c >> 3) << 4 | (c & 7) << 1);
-              } else {  // no channel: code 0
+              } else {  // no channel: code 0 (r_lo = r_hi = 0 never needs the fallback)
                 nz[i] = rlo[i] = rhi[i] = 0.0f;
                 co[i] = 0u;
               }
@@ -405,42 +423,40 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
             for (int n = 0; n < 4; ++n) {
               const int t = t0 + n;
               const uint32_t sw = uint32_t(t & 7) << 4;
-              uint32_t lo[8];
+              uint32_t lo[8], xp[4], acc = 0u;
 #pragma unroll
               for (int i = 0; i < 8; i += 2) {
                 const uint32_t xl = *reinterpret_cast<const uint16_t*>(smem + t * 256 + (co[i] ^ sw));
                 const uint32_t xh = *reinterpret_cast<const uint16_t*>(smem + t * 256 + (co[i + 1] ^ sw));
+                xp[i >> 1] = xl | (xh << 16);
                 float d0, d1;
-                sub_pair(xl | (xh << 16), nz[i], nz[i + 1], d0, d1, T());
+                sub_pair(xp[i >> 1], nz[i], nz[i + 1], d0, d1, T());
                 lo[i] = code_bits(d0, rlo[i]);
                 lo[i + 1] = code_bits(d1, rlo[i + 1]);
-                acc[n] |= (lo[i] ^ code_bits(d0, rhi[i])) | (lo[i + 1] ^ code_bits(d1, rhi[i + 1]));
+                acc |= (lo[i] ^ code_bits(d0, rhi[i])) | (lo[i + 1] ^ code_bits(d1, rhi[i + 1]));
+              }
+              uint32_t X0 = low_bytes(lo[0], lo[2], lo[4], lo[6]);
+              uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]);
+              if (acc != 0u) {  // an element near a rounding boundary
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  uint32_t& X = (i & 1) ? X1 : X0;
+                  const int sh = 8 * (i >> 1);
+                  const float xv = bits_to_float(uint16_t(xp[i >> 1] >> (16 * (i & 1))), T());
+                  const float d = __fadd_rn(xv, nz[i]);
+                  const uint32_t k0 = (X >> sh) & 0xffu;
+                  if (code_bits(d, rhi[i]) != 0x4B400000u + k0) {
+                    const int c = int((co[i] >> 4) << 3 | ((co[i] >> 1) & 7u));
+                    X = (X & ~(0xffu << sh)) | (fix_code(d, xv, nz[i], qc[g * kHeadDim + c].w, k0, 15) << sh);
+                  }
+                }
               }
               // element 8a + 2b + f at bit 8b + 4f + 2a
-              const uint32_t X0 = low_bytes(lo[0], lo[2], lo[4], lo[6]) & 0x03030303u;
-              const uint32_t X1 = low_bytes(lo[1], lo[3], lo[5], lo[7]) & 0x03030303u;
-              word[n] |= (X0 + 16u * X1) << (2 * a);
+              word[n] |= ((X0 & 0x03030303u) + 16u * (X1 & 0x03030303u)) << (2 * a);
             }
           }
 #pragma unroll
-          for (int n = 0; n < 4; ++n) {
-            const int t = t0 + n;
-            if (acc[n] != 0u) {  // near a rounding boundary: the IEEE divide decides
-              word[n] = 0u;
-              for (int e = 0; e < 16; ++e) {
-                const int pos = 16 * wb + e;
-                const int q = pos >> lg, rem = pos & ((1 << lg) - 1);
-                const int j = 16 * (rem >> 2) + 8 * ((rem >> 1) & 1) + 2 * q + (rem & 1);
-                const int c = chan_of[j];
-                if (c >= kHeadDim) continue;
-                const float4 v = qc[g * kHeadDim + c];
-                const float xv = bits_to_float(
-                    *reinterpret_cast<const uint16_t*>(smem + qtile_off(t, c >> 3) + (c & 7) * 2), T());
-                word[n] |= uint32_t(quant_code(xv, -v.x, v.w, 15) & 3) << elem_bit(e);
-              }
-            }
-            kB[t * KW + wb] = word[n];
-          }
+          for (int n = 0; n < 4; ++n) kB[(t0 + n) * KW + wb] = word[n];
         }
       }
     }
@@ -533,7 +549,6 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
         // branch that only some lanes take); the lanes that need it rebuild their word.
         if (__any_sync(kFull, acc != 0u)) {
           const bool redo = acc != 0u;
-          if (redo) word = 0u;
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
             uint32_t x[4];
@@ -541,11 +556,15 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
             if (redo) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const int b = i >> 1, f = i & 1;
-                const int t = 32 * g + 16 * a + 8 * (b >> 1) + 2 * q + f;
-                const float4 v = qc[t];
+                const int b = i >> 1, f = i & 1, ti = 4 * a + 2 * (b >> 1) + f, sh = elem_bit(8 * a + i);
                 const float xv = bits_to_float(uint16_t(x[b] >> (16 * f)), T());
-                word |= uint32_t(quant_code(xv, -v.x, v.w, 3)) << elem_bit(8 * a + i);
+                const float d = __fadd_rn(xv, nz[ti]);
+                const uint32_t k0 = (word >> sh) & 3u;
+                if (code_bits(d, rhi[ti]) != 0x4B400000u + k0) {
+                  const int t = 32 * g + 16 * a + 8 * (b >> 1) + 2 * q + f;
+                  const uint32_t code = fix_code(d, xv, nz[ti], qc[t].w, k0, 3);
+                  word = (word & ~(3u << sh)) | (code << sh);
+                }
               }
             }
           }
@@ -573,6 +592,8 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_con
   bool go = false, app = false;
   const uint16_t* last = nullptr;
   if (p.append) {
+    // the next kernel may be scheduled now: it reads nothing of ours before its own wait
+    pdl_trigger();
     const bool first = h == 0 && blockIdx.z == 0;
     r = p.res_len_w[item];
     if (r < 0 || r > P) {  // the append flags it; the flush skips a window that is not full
