@@ -45,8 +45,8 @@ WORKLOAD = "llama3_8b"
 # dram__bytes_write.sum from one ncu capture of the decode kernel), valid only for the
 # kernel source it was taken on: the bench reports it while the decode kernel source
 # still hashes to this value.
-DECODE_TRAFFIC = {"source_sha256": "2907ee8123ed9e830983202970f4c4daaee50fab223ba8799a67ab423954aabb",
-                  "bytes": 50294016 + 100352}
+DECODE_TRAFFIC = {"source_sha256": "0207a5f1d55e37f879fe053e08a049bbf13c710e2b7c307fb8b730a1a0cfdd68",
+                  "bytes": 50298880 + 22528}
 LAYERS = 32
 METRIC = "2-bit KV decode-attn GB/s & % of HBM peak; quantize tokens/s"
 
@@ -60,6 +60,10 @@ def parse():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-workload measurements")
+    ap.add_argument("--leg", default="main",
+                    help="main (the contract line), minikv (the MiniKV prefill leg alone), or "
+                         "decode:<workload> (one full-size cache, 5 decode launches: a short program "
+                         "for profiling one workload's decode kernel)")
     return ap.parse_args()
 
 
@@ -924,9 +928,50 @@ def run_reference(args):
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def decode_leg(name):
+    """One full-size cache of a workload and five decode launches (for a profiler to
+    capture the last ones); returns the workload's page bytes and launch count."""
+    import torch
+
+    from bit_mixed_precision_channel_b200 import binding as kb
+    from bit_mixed_precision_channel_b200 import synthetic as syn
+    from bit_mixed_precision_channel_b200.cache import PagedKVCache
+
+    dev = torch.device("cuda")
+    w = syn.WORKLOADS[name]
+    cfg = kb.Config(head_dim=w.D, num_q_heads=w.Hq, num_kv_heads=w.Hkv, page_tokens=w.P, key_group=w.G,
+                    num_boost=w.k, dtype=w.dtype)
+    tdt = kb.torch_dtype(w.dtype)
+    lens = syn.lengths(w)
+    P = w.P
+    pool_pages = int(sum(lens // P) + 2 * w.batch)
+    sigma = torch.from_numpy(syn.key_channel_sigma(w)).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    c = PagedKVCache(cfg, w.batch, int(max(lens) // P + 2), pool_pages, device=dev,
+                     page_order=syn.page_order(w, pool_pages))
+    for b, K, V in _device_prompts(w, lens, sigma, gen, tdt, dev):
+        c.prefill(b, K, V)
+    q = torch_randn((w.batch, w.Hq, w.D), gen, dev).to(tdt)
+    out = torch.empty(w.batch, w.Hq, w.D, device=dev)
+    for _ in range(5):
+        c.attend(q, out)
+    torch.cuda.synchronize()
+    assert c.check_errors() == 0
+    payload = kb.page_layout(cfg)["payload_bytes"]
+    return {"leg": "decode", "workload": name, "page_bytes": int(sum(lens // P)) * w.Hkv * payload,
+            "residual_tokens": int(sum(lens % P)), "launches": 5}
+
+
 def main():
     args = parse()
-    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if args.leg == "minikv":
+        import torch
+        res = {"leg": "minikv", **prefill_bench(torch.device("cuda"), peak_tensor())}
+    elif args.leg.startswith("decode:"):
+        res = decode_leg(args.leg.split(":", 1)[1])
+    else:
+        res = run_reference(args) if args.impl == "reference" else run_gpu(args)
     if res is not None:
         print(json.dumps(res), flush=True)
 
