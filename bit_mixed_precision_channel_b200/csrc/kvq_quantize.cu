@@ -145,11 +145,11 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 // Quantizes the window or page tile of (item, kv head h) into record rec: the key part
 // (z = 0) or the value part (z = gridDim.z - 1) of the requested modes.  last_k / last_v,
 // when given, replace the tile's last token (the token an append-and-flush just wrote).
-template <typename T>
+template <typename T, int P>
 __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, int h, uint8_t* rec,
                                                 const uint16_t* last_k, const uint16_t* last_v) {
   const int tid = threadIdx.x;
-  const int P = p.P, k = p.k;
+  const int k = p.k;
 
   // z = 0: the key part of the requested modes, z = gridDim.z - 1: the value part
   const int kmodes = blockIdx.z == 0 ? p.mode & (kModeSelect | kModeKeys) : 0;
@@ -583,11 +583,12 @@ __device__ __forceinline__ void quantize_record(const QuantParams& p, int item, 
 // lengths and the page-table entry, so every CTA has read the old length before it
 // changes.  The outcome, error bits included, is that of kvq_append_token followed by
 // kvq_flush_residual.
-template <typename T>
+// P (page tokens: 32, 64 or 128) is a template parameter so that every trip count, group
+// count and tile offset is a constant.
+template <typename T, int P>
 __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_constant__ QuantParams p) {
   pdl_wait();
   const int item = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  const int P = p.P;
   int dst = -1, np = 0, r = 0;
   bool go = false, app = false;
   const uint16_t* last = nullptr;
@@ -637,7 +638,7 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_con
     }
     go = true;
   }
-  if (go) quantize_record<T>(p, item, h, p.pool + (size_t(dst) * p.Hkv + h) * p.L.record, last, last);
+  if (go) quantize_record<T, P>(p, item, h, p.pool + (size_t(dst) * p.Hkv + h) * p.L.record, last, last);
   if (p.append) {
     __syncthreads();
     if (tid == 0) {
@@ -707,22 +708,32 @@ __global__ void flush_commit_kernel(int32_t* res_len, const int32_t* new_page, i
 
 // ------------------------------------------------------------------ host launchers
 
+template <typename T, int P>
+static cudaError_t launch_quantize_p(const QuantParams& p, dim3 grid, size_t smem, cudaStream_t stream) {
+  static int seen[64];
+  const cudaError_t e = ensure_dynamic_smem(quantize_kernel<T, P>, int(smem), seen);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(quantize_kernel<T, P>, grid, dim3(kQThreads), smem, stream, p);
+}
+
+template <typename T>
+static cudaError_t launch_quantize_t(const QuantParams& p, dim3 grid, size_t smem, cudaStream_t stream) {
+  switch (p.P) {
+    case 32: return launch_quantize_p<T, 32>(p, grid, smem, stream);
+    case 64: return launch_quantize_p<T, 64>(p, grid, smem, stream);
+    case 128: return launch_quantize_p<T, 128>(p, grid, smem, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_quantize(const QuantParams& p, int n_items, int dtype, cudaStream_t stream) {
   if (n_items <= 0) return cudaSuccess;
   const size_t smem = QSmem::bytes(p.P, p.mode);
   // keys and values of a page in separate CTAs when both are requested
   const bool both = (p.mode & (kModeSelect | kModeKeys)) && (p.mode & kModeValues);
   const dim3 grid(n_items, p.Hkv, both ? 2 : 1);
-  static int seen_bf16[64], seen_f16[64];
-  if (dtype == KVQ_BF16) {
-    const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__nv_bfloat16>, int(smem), seen_bf16);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_kernel<__nv_bfloat16>, grid, dim3(kQThreads), smem, stream, p);
-  } else {
-    const cudaError_t e = ensure_dynamic_smem(quantize_kernel<__half>, int(smem), seen_f16);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_kernel<__half>, grid, dim3(kQThreads), smem, stream, p);
-  }
+  return dtype == KVQ_BF16 ? launch_quantize_t<__nv_bfloat16>(p, grid, smem, stream)
+                           : launch_quantize_t<__half>(p, grid, smem, stream);
 }
 
 cudaError_t launch_append(const void* k_new, const void* v_new, void* res_k, void* res_v, int32_t* res_len,
