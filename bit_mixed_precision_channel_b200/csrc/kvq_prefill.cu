@@ -5,8 +5,10 @@
 // tokens to keep are chosen by their cumulative attention score (heavy hitters) together
 // with a recent window, and a two-stage selective flash-attention kernel returns the
 // attention output and those scores in linear memory.  Here:
-//   pass 1 (prefill_fwd)   causal flash attention, one CTA per (64 query rows, query
-//                          head): the output rows and each row's log2-sum-exp;
+//   pass 1 (prefill_fwd_tc) causal flash attention on the fifth-generation tensor cores
+//                          (tcgen05, accumulators in tensor memory), one CTA per (128
+//                          query rows, query head): the output rows and each row's
+//                          log2-sum-exp;
 //   pass 2 (prefill_score) one CTA per (64 key rows, KV head): recomputes K Q^T for the
 //                          query blocks at or after the key block and the query heads of
 //                          the KV head, turns it into probabilities with the rows'
@@ -16,10 +18,13 @@
 //                          lower position), ascending;
 //   gather_kernel          the kept tokens of every KV head, compacted token-major, ready
 //                          for the page quantizer.
-// Products run on the tensor cores (mma.sync m16n8k16, fp32 accumulate) with operands
-// in the cache dtype; fp16 probabilities carry 11 bits, bf16 ones are split into a high
-// and a low bf16 part.
+// Pass 1 runs on tcgen05 (M = N = 128 products, operands in the cache dtype, fp32
+// accumulators in tensor memory); pass 2 on mma.sync m16n8k16.  fp16 probabilities carry
+// 11 bits, bf16 ones are split into a high and a low bf16 part.
+#include <type_traits>
+
 #include "kvq_internal.cuh"
+#include "kvq_tc.cuh"
 
 namespace kvq {
 namespace pf {
@@ -92,151 +97,211 @@ struct PrefillParams {
   float* score;       // [Hkv][L]
 };
 
-// ---------------------------------------------------------------- pass 1
+// ---------------------------------------------------------------- pass 1 (tcgen05)
 
+constexpr int kTcRows = 128;                 // query rows per CTA, keys per block
+constexpr uint32_t kTcTile = kTcRows * 256;  // one [128][128] tile of the 16-bit dtype
+
+// Byte offset of 16-byte chunk c (8 elements) of row r in a tile built from the tensor
+// cores' core matrices: 8 rows x 16 bytes each, chunks 128 bytes apart, row groups 2048
+// bytes apart.  The same tile is a K-major operand (rows along M or N, chunks along K:
+// LBO = 128, SBO = 2048) and an MN-major one (rows along K, chunks along N: LBO = 2048,
+// SBO = 128).
+__device__ __forceinline__ uint32_t tco(int r, int c) { return uint32_t((r >> 3) * 2048 + c * 128 + (r & 7) * 16); }
+
+// Rows [0, valid) of a 128-row tile (row i at src + i * stride elements) into shared
+// memory with cp.async; rows at or past `valid` are zero-filled.
+__device__ __forceinline__ void load_tile_tc(uint8_t* dst, const uint16_t* src, long long stride, int valid, int tid,
+                                             int nthreads) {
+#pragma unroll 4
+  for (int i = tid; i < kTcRows * 16; i += nthreads) {
+    const int r = i >> 4, c = i & 15;
+    const bool ok = r < valid;
+    cp_async16(dst + tco(r, c), src + (ok ? r : 0) * stride + c * 8, ok ? 16u : 0u);
+  }
+}
+
+constexpr int kTcThreads = 128;  // one thread per query row
+
+// Causal flash attention on the fifth-generation tensor cores: one CTA per (128 query
+// rows, query head), thread t owns query row t (tensor-memory lane t).
+//   S = Q K^T   M = N = K = 128: Q and K from shared memory (K-major), S in tensor memory;
+//   softmax     each thread reads its row of S, masks the diagonal block, keeps a running
+//               maximum that is raised only when a block exceeds it by more than 2^8 (O is
+//               then rescaled), and writes the probabilities in the cache dtype back over S
+//               as the A operand of the next product (bf16: a high and a low part);
+//   O += P V    A = P from tensor memory, V from shared memory (MN-major), O in tensor
+//               memory.
+// Two CTAs share an SM (256 tensor-memory columns and 96 KB of shared memory each), so
+// one CTA's softmax runs while the other's products do.  The next K block loads while the
+// softmax and PV run, the next V block while the next QK and softmax run.  Every wait is
+// bounded; a CTA whose wait gives up writes NaN rows.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) prefill_fwd(const __grid_constant__ PrefillParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];  // Q tile | 2 x (K tile, V tile)
-  pdl_wait();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_fwd_tc(const __grid_constant__ PrefillParams p) {
+  constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
+  extern __shared__ __align__(128) uint8_t smem[];  // Q, K, V tiles
+  __shared__ uint64_t bar_s, bar_o;
+  __shared__ uint32_t tmem_base;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int qb = gridDim.x - 1 - blockIdx.x;  // the longest rows first
   const int h = blockIdx.y, kvh = h / p.gqa;
-  const int q0 = qb * kRows;
+  const int q0 = qb * kTcRows, row = q0 + tid;
   const long long qs = (long long)p.Hq * 128, ks_ = (long long)p.Hkv * 128;
   uint8_t* Qt = smem;
-  load_tile(Qt, p.q + (long long)q0 * qs + h * 128, qs, min(kRows, p.L - q0), tid);
-  load_tile(smem + kTile, p.k + kvh * 128, ks_, min(kRows, p.L), tid);
-  load_tile(smem + 2 * kTile, p.v + kvh * 128, ks_, min(kRows, p.L), tid);
+  uint8_t* Kt = smem + kTcTile;
+  uint8_t* Vt = smem + 2 * kTcTile;
+  if (warp == 0) tc::alloc(&tmem_base, 256);
+  if (tid == 0) {
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_o, 1);
+    fence_mbar_init();
+  }
+  pdl_wait();
+  load_tile_tc(Qt, p.q + (long long)q0 * qs + h * 128, qs, min(kTcRows, p.L - q0), tid, kTcThreads);
+  load_tile_tc(Kt, p.k + kvh * 128, ks_, min(kTcRows, p.L), tid, kTcThreads);
   cp_commit();
-
-  uint32_t qa[8][4];
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o[i][j] = 0.0f;
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
-  const int r0 = warp * 16;  // this warp's rows in the tile
-  const int row_g = q0 + r0 + g, row_g8 = row_g + 8;
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tS = tmem_base, tO = tmem_base + 128;
+  const uint32_t sQ = smem_addr(Qt), sK = smem_addr(Kt), sV = smem_addr(Vt);
+  constexpr uint32_t kIdQK = tc::idesc_f16(128, BF, false);
+  constexpr uint32_t kIdPV = tc::idesc_f16(128, BF, true);
+  float m = -INFINITY, l = 0.0f;
+  bool ok = true;
 
   for (int kb = 0; kb <= qb; ++kb) {
-    uint8_t* Kt = smem + kTile + (kb & 1) * 2 * kTile;
-    uint8_t* Vt = Kt + kTile;
-    if (kb < qb) {
-      uint8_t* Kn = smem + kTile + ((kb + 1) & 1) * 2 * kTile;
-      const int k0 = (kb + 1) * kRows;
-      load_tile(Kn, p.k + (long long)k0 * ks_ + kvh * 128, ks_, min(kRows, p.L - k0), tid);
-      load_tile(Kn + kTile, p.v + (long long)k0 * ks_ + kvh * 128, ks_, min(kRows, p.L - k0), tid);
-      cp_commit();
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
+    // the previous PV product is done: its P (over S) and the V buffer are free
+    if (kb > 0) {
+      ok = mbar_wait_bounded(&bar_o, uint32_t(kb - 1) & 1u) && ok;
+      tc::fence_after();
     }
+    const int k0 = kb * kTcRows;
+    load_tile_tc(Vt, p.v + (long long)k0 * ks_ + kvh * 128, ks_, min(kTcRows, p.L - k0), tid, kTcThreads);
+    cp_commit();
+    cp_wait<1>();  // Q and this K block landed
+    tc::fence_async_smem();
+    tc::fence_before();
     __syncthreads();
-    if (kb == 0) {
+    if (tid == 0) {
+      tc::fence_after();
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) ld_a(qa[ks], Qt, r0, ks, lane);
+      for (int s = 0; s < 8; ++s)
+        tc::mma_ss(tS, tc::smem_desc(sQ + s * 256, 128, 2048), tc::smem_desc(sK + s * 256, 128, 2048), kIdQK,
+                   s > 0 ? 1u : 0u);
+      tc::commit(&bar_s);
     }
-    // S = Q K^T: 16 rows x 64 keys per warp
-    float s[8][4];
+    ok = mbar_wait_bounded(&bar_s, uint32_t(kb) & 1u) && ok;
+    tc::fence_after();
+    // the K buffer is free: the next key block (an empty group after the last)
+    if (kb < qb)
+      load_tile_tc(Kt, p.k + (long long)(k0 + kTcRows) * ks_ + kvh * 128, ks_, min(kTcRows, p.L - k0 - kTcRows), tid,
+                   kTcThreads);
+    cp_commit();
+
+    // this thread's row of S: causal mask and key range (the diagonal block only: every
+    // key of an earlier block precedes every row); eight partial maxima of the raw scores
+    uint32_t sv[8][16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 8; ++i) tc::ld<16>(tc::lane_addr(tS, warp, 16 * i), sv[i]);
+    tc::wait_ld();
+    float mp[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) s[i][j] = 0.0f;
+    for (int i = 0; i < 8; ++i) {
+      mp[i] = -INFINITY;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t b[4];
-        ld_b_rows(b, Kt, 16 * np, ks, lane);
-        mma_16816(s[2 * np], qa[ks], b[0], b[1], T());
-        mma_16816(s[2 * np + 1], qa[ks], b[2], b[3], T());
-      }
-    // scale, causal mask and the key range
-    const int key0 = kb * kRows;
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int key = key0 + 8 * nt + 2 * qd + (j & 1);
-        const int row = (j >> 1) ? row_g8 : row_g;
-        const float x = (key <= row && key < p.L) ? s[nt][j] * p.c_log2 : -INFINITY;
-        s[nt][j] = x;
-        mx[j >> 1] = fmaxf(mx[j >> 1], x);
-      }
-    float alpha[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(kFull, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(kFull, mx[r], 2));
-      const float mn = fmaxf(m[r], mx[r]);
-      alpha[r] = mn == -INFINITY ? 1.0f : ex2(m[r] - mn);
-      m[r] = mn;
-      l[r] *= alpha[r];
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o[i][0] *= alpha[0];
-      o[i][1] *= alpha[0];
-      o[i][2] *= alpha[1];
-      o[i][3] *= alpha[1];
-    }
-    // probabilities -> A fragments of the PV product (S accumulators of n-tiles 2ks and
-    // 2ks + 1 form the A fragment of k-step ks)
-    uint32_t pa[4][4], pl[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float pv[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float mm = m[j >> 1];
-        pv[j] = mm == -INFINITY ? 0.0f : ex2(s[nt][j] - mm);
-        l[j >> 1] += pv[j];
-      }
-      const int ks = nt >> 1, hi = nt & 1;
-      pa[ks][2 * hi] = pk(pv[0], pv[1], T());
-      pa[ks][2 * hi + 1] = pk(pv[2], pv[3], T());
-      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        const float2 h0 = upk(pa[ks][2 * hi], T()), h1 = upk(pa[ks][2 * hi + 1], T());
-        pl[ks][2 * hi] = pk(pv[0] - h0.x, pv[1] - h0.y, T());
-        pl[ks][2 * hi + 1] = pk(pv[2] - h1.x, pv[3] - h1.y, T());
+      for (int j = 0; j < 16; ++j) {
+        if (kb == qb) {
+          const int key = k0 + 16 * i + j;
+          if (!(key <= row && key < p.L)) sv[i][j] = 0xff800000u;  // -inf
+        }
+        mp[i] = fmaxf(mp[i], __uint_as_float(sv[i][j]));
       }
     }
-    // O += P V: 16 rows x 128 channels per warp
+    const float mx =  // the scale is positive: the maximum of the scaled scores
+        fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+        p.c_log2;
+    // lazy running maximum; O (when it holds earlier blocks) is rescaled with it
+    float alpha = 1.0f;
+    if (mx > m + 8.0f) {
+      alpha = ex2(m - mx);  // m = -inf: 0
+      l *= alpha;
+      m = mx;
+    }
+    if (kb > 0 && __any_sync(kFull, alpha != 1.0f)) {
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
+      for (int i = 0; i < 8; ++i) {
+        uint32_t o[16];
+        tc::ld<16>(tc::lane_addr(tO, warp, 16 * i), o);
+        tc::wait_ld();
 #pragma unroll
-      for (int cp = 0; cp < 8; ++cp) {
-        uint32_t b[4];
-        ld_b_trans(b, Vt, 16 * ks, 16 * cp, lane);
-        mma_16816(o[2 * cp], pa[ks], b[0], b[1], T());
-        mma_16816(o[2 * cp + 1], pa[ks], b[2], b[3], T());
-        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-          mma_16816(o[2 * cp], pl[ks], b[0], b[1], T());
-          mma_16816(o[2 * cp + 1], pl[ks], b[2], b[3], T());
+        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+        tc::st<16>(tc::lane_addr(tO, warp, 16 * i), o);
+      }
+    }
+    // probabilities 2^(s c - m) over S (a masked -inf gives 0): column j holds keys 2j,
+    // 2j + 1 (bf16: low parts at 64 + j); m is finite from the first block on
+    const float nm = -m;
+    float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t ph[16], plo[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c = 32 * i + 2 * j;  // key offsets c, c + 1
+        const float p0 = ex2(__fmaf_rn(__uint_as_float(sv[c >> 4][c & 15]), p.c_log2, nm));
+        const float p1 = ex2(__fmaf_rn(__uint_as_float(sv[(c + 1) >> 4][(c + 1) & 15]), p.c_log2, nm));
+        lp[i] += p0 + p1;
+        ph[j] = pk(p0, p1, T());
+        if constexpr (BF) {
+          const float2 hv = upk(ph[j], T());
+          plo[j] = pk(p0 - hv.x, p1 - hv.y, T());
         }
       }
-    __syncthreads();  // the buffer is refilled two blocks later
+      tc::st<16>(tc::lane_addr(tS, warp, 16 * i), ph);
+      if constexpr (BF) tc::st<16>(tc::lane_addr(tS, warp, 64 + 16 * i), plo);
+    }
+    l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+    tc::wait_st();
+    cp_wait<1>();  // this V block landed (the next K block may still be in flight)
+    tc::fence_async_smem();
+    tc::fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc::fence_after();
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        tc::mma(tO, tS + 8 * s, tc::smem_desc(sV + s * 4096, 2048, 128), kIdPV, (kb > 0 || s > 0) ? 1u : 0u);
+      if constexpr (BF) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) tc::mma(tO, tS + 64 + 8 * s, tc::smem_desc(sV + s * 4096, 2048, 128), kIdPV, 1u);
+      }
+      tc::commit(&bar_o);
+    }
   }
+  ok = mbar_wait_bounded(&bar_o, uint32_t(qb) & 1u) && ok;
+  tc::fence_after();
   pdl_trigger();
-  // row sums across the quad, then the output and the log2-sum-exp
+  // the output row and its log2-sum-exp
+  const float inv = ok ? (l > 0.0f ? 1.0f / l : 0.0f) : __int_as_float(0x7fc00000);
+  float* orow = p.out + ((long long)row * p.Hq + h) * 128;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    l[r] += __shfl_xor_sync(kFull, l[r], 1);
-    l[r] += __shfl_xor_sync(kFull, l[r], 2);
+  for (int i = 0; i < 8; ++i) {
+    uint32_t o[16];
+    tc::ld<16>(tc::lane_addr(tO, warp, 16 * i), o);
+    tc::wait_ld();
+    if (row < p.L) {
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(orow + 16 * i + j) =
+            make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv, __uint_as_float(o[j + 2]) * inv,
+                        __uint_as_float(o[j + 3]) * inv);
+    }
   }
-  const float inv[2] = {l[0] > 0.0f ? 1.0f / l[0] : 0.0f, l[1] > 0.0f ? 1.0f / l[1] : 0.0f};
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = r ? row_g8 : row_g;
-    if (row >= p.L) continue;
-    float* orow = p.out + ((long long)row * p.Hq + h) * 128;
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-      *reinterpret_cast<float2*>(orow + 8 * nt + 2 * qd) = make_float2(o[nt][2 * r] * inv[r], o[nt][2 * r + 1] * inv[r]);
-    if (qd == 0) p.lse[(long long)h * p.L + row] = m[r] + __log2f(l[r]);
-  }
+  if (row < p.L) p.lse[(long long)h * p.L + row] = ok ? m + __log2f(l) : __int_as_float(0x7fc00000);
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::dealloc(tmem_base, 256);
 }
 
 // ---------------------------------------------------------------- pass 2
@@ -447,20 +512,21 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, int L, i
   p.lse = lse;
   p.score = score;
   const int nb = (L + pf::kRows - 1) / pf::kRows;
-  const size_t smem_fwd = 5 * pf::kTile, smem_score = 3 * pf::kTile + 2 * pf::kRows * sizeof(float);
+  const int nb_tc = (L + pf::kTcRows - 1) / pf::kTcRows;
+  const size_t smem_fwd = 3 * pf::kTcTile, smem_score = 3 * pf::kTile + 2 * pf::kRows * sizeof(float);
   static int seen[4][64];
   cudaError_t e;
   if (dtype == KVQ_BF16) {
-    if ((e = ensure_dynamic_smem(pf::prefill_fwd<__nv_bfloat16>, int(smem_fwd), seen[0])) != cudaSuccess) return e;
+    if ((e = ensure_dynamic_smem(pf::prefill_fwd_tc<__nv_bfloat16>, int(smem_fwd), seen[0])) != cudaSuccess) return e;
     if ((e = ensure_dynamic_smem(pf::prefill_score<__nv_bfloat16>, int(smem_score), seen[1])) != cudaSuccess) return e;
-    if ((e = launch_pdl(pf::prefill_fwd<__nv_bfloat16>, dim3(nb, Hq), dim3(pf::kThreads), smem_fwd, stream, p)) !=
+    if ((e = launch_pdl(pf::prefill_fwd_tc<__nv_bfloat16>, dim3(nb_tc, Hq), dim3(pf::kTcThreads), smem_fwd, stream, p)) !=
         cudaSuccess)
       return e;
     return launch_pdl(pf::prefill_score<__nv_bfloat16>, dim3(nb, Hkv), dim3(pf::kThreads), smem_score, stream, p);
   }
-  if ((e = ensure_dynamic_smem(pf::prefill_fwd<__half>, int(smem_fwd), seen[2])) != cudaSuccess) return e;
+  if ((e = ensure_dynamic_smem(pf::prefill_fwd_tc<__half>, int(smem_fwd), seen[2])) != cudaSuccess) return e;
   if ((e = ensure_dynamic_smem(pf::prefill_score<__half>, int(smem_score), seen[3])) != cudaSuccess) return e;
-  if ((e = launch_pdl(pf::prefill_fwd<__half>, dim3(nb, Hq), dim3(pf::kThreads), smem_fwd, stream, p)) != cudaSuccess)
+  if ((e = launch_pdl(pf::prefill_fwd_tc<__half>, dim3(nb_tc, Hq), dim3(pf::kTcThreads), smem_fwd, stream, p)) != cudaSuccess)
     return e;
   return launch_pdl(pf::prefill_score<__half>, dim3(nb, Hkv), dim3(pf::kThreads), smem_score, stream, p);
 }
