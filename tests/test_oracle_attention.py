@@ -157,3 +157,68 @@ def test_page_table_order_only_permutes_tokens():
     a = oracle.decode_unit(pool, cfg, 0, [0, 1, 2, 3], e, e, q, 0.2)
     b = oracle.decode_unit(pool, cfg, 0, [3, 1, 0, 2], e, e, q, 0.2)
     np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-14)
+
+
+def _grid_page(rng, P, k, G=32):
+    """One page [P][D] whose every key group and value row sits exactly on its own
+    quantization grid.  Keys of k channels span 15 steps of 1/8, 1/4 or 1/2 (a 4-bit
+    grid) with magnitudes of at least 1, the others span 3 steps of 1/16 or 1/8 (a
+    2-bit grid) below 0.4, so the magnitude ranking boosts exactly the k wide channels;
+    every value row spans 3 steps of 1/4, 1/2 or 1.  The step is drawn per group, so a
+    scale read from the wrong row or group changes the result.  All values are
+    multiples of 1/16 below 8: exact in fp16 and bf16."""
+    D = 128
+    wide = set(rng.choice(D, size=k, replace=False).tolist())
+    K = np.zeros((P, D))
+    for c in range(D):
+        for g in range(P // G):
+            if c in wide:
+                qmax, step, lo = 15, rng.choice([0.125, 0.25, 0.5]), 4
+            else:
+                qmax, step, lo = 3, rng.choice([0.0625, 0.125]), 0
+            codes = rng.integers(0, qmax + 1, G)
+            codes[rng.choice(G, 2, replace=False)] = [0, qmax]  # both ends: scale is exactly `step`
+            mn = -step * rng.integers(lo, lo + 4)
+            K[g * G:(g + 1) * G, c] = mn + codes * step
+    V = np.zeros((P, D))
+    for t in range(P):
+        step = rng.choice([0.25, 0.5, 1.0])
+        codes = rng.integers(0, 4, D)
+        codes[rng.choice(D, 2, replace=False)] = [0, 3]
+        V[t] = -step * rng.integers(0, 4) + step * codes
+    return K, V
+
+
+@pytest.mark.parametrize("dtype", [F16, BF16])
+@pytest.mark.parametrize("P,k", [(32, 0), (32, 16), (128, 32), (128, 128)])
+def test_grid_exact_pages_give_exact_attention_on_the_inputs(dtype, P, k):
+    """Keys on a 2/4-bit grid and values on a 2-bit grid are reproduced exactly by the
+    quantizer (grid recovery), so attention over the quantized pages plus an fp16
+    residual must equal exact attention over the raw inputs, here torch's fp64 SDPA,
+    to fp64 rounding.  No oracle dequantizer is involved on the expected side: a
+    plane, scale, zero, boost row or token-order mistake anywhere between the record
+    and the softmax shows up.  k = D is the all-channels 4-bit case, k = 0 plain
+    uniform 2 bits."""
+    rng = np.random.default_rng(50 + P + k + dtype)
+    cfg = oracle.Cfg(P=P, k=k, Hq=4, Hkv=2, dtype=dtype)
+    n_pages, res_len = 3, 5
+    pool = np.zeros((n_pages, cfg.Hkv, cfg.record_bytes), np.uint8)
+    raw = {}
+    for p in range(n_pages):
+        for h in range(cfg.Hkv):
+            K, V = _grid_page(rng, P, k)
+            Kb, Vb = syn.to_bits(K, dtype), syn.to_bits(V, dtype)
+            assert np.array_equal(oracle.values(Kb, dtype), K) and np.array_equal(oracle.values(Vb, dtype), V)
+            pool[p, h] = oracle.quantize_page(Kb, Vb, cfg)
+            raw[p, h] = (K, V)
+    order = [1, 2, 0]
+    sm = 1 / np.sqrt(cfg.D)
+    for h in range(cfg.Hkv):
+        rk = syn.to_bits(rng.standard_normal((res_len, cfg.D)), dtype)
+        rv = syn.to_bits(rng.standard_normal((res_len, cfg.D)), dtype)
+        q = syn.to_bits(rng.standard_normal((cfg.gqa, cfg.D)), dtype)
+        out = oracle.decode_unit(pool, cfg, h, order, rk, rv, q, sm)
+        Ks = np.concatenate([raw[p, h][0] for p in order] + [oracle.values(rk, dtype)])
+        Vs = np.concatenate([raw[p, h][1] for p in order] + [oracle.values(rv, dtype)])
+        want = _sdpa(oracle.values(q, dtype), Ks, Vs, sm)
+        np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-12)
