@@ -11,8 +11,11 @@ L2, so every step reads its pages from HBM.  Inputs are seeded synthetic tensors
 
 A step = for every layer: append the new token to the residual window, flush full
 windows, decode attention over pages + window (all rows of the hot path; the prompt
-pages were quantized once at prefill, whose rate is reported as "quantize").  The step
-is captured once in a CUDA graph and replayed.
+pages were quantized once at prefill, whose rate is reported as "quantize").  The host
+tracks the windows' lengths, so the flush is launched only on steps where a window
+fills (once every 128 steps; "flush_steps" counts them in the timed region, and the
+flush rate of the ragged workload is reported under configs).  Each kind of step
+(without / with flush) is captured once in a CUDA graph and replayed.
 
 value: decode-attention algorithmic bytes of all layers / step time (GB/s), whole job
 (summed over ranks for N > 1, each rank running its own batch: weak scaling).
@@ -312,10 +315,12 @@ def run_gpu(args):
     vns = [dev_bits(vn) for _ in range(L_layers)]
     outs = [torch.empty(B, w.Hq, D, device=dev) for _ in range(L_layers)]
 
-    def device_step():
+    def device_step(flush):
+        # the host knows which windows fill this step: the flush runs only then
         for i, c in enumerate(caches):
             c.append(kns[i], vns[i])
-            c.flush()
+            if flush:
+                c.flush()
             c.attend(qs[i], outs[i])
 
     def attend_only():
@@ -330,18 +335,24 @@ def run_gpu(args):
         for i, c in enumerate(caches):
             c.commit_host(flag_list[i])
 
+    def flushing(flag_list):
+        return any(len(f) > 0 for f in flag_list)
+
     flags = [None] * L_layers
     # eager warm-up (also sets kernel attributes before capture)
     for _ in range(2):
         host_step(flags)
-        device_step()
+        device_step(True)
         host_commit(flags)
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
-    g_step, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=stream):
-        device_step()
+    # one graph per step kind: without and with the flush of full windows
+    g_step = {False: torch.cuda.CUDAGraph(), True: torch.cuda.CUDAGraph()}
+    g_attn = torch.cuda.CUDAGraph()
+    for fl, graph in g_step.items():
+        with torch.cuda.graph(graph, stream=stream):
+            device_step(fl)
     with torch.cuda.graph(g_attn, stream=stream):
         attend_only()
     # e2e: host buffers in pinned memory, copies inside the graph
@@ -352,36 +363,38 @@ def run_gpu(args):
     # The copies run on two copy streams forked inside the graph: every layer's inputs go
     # up in layer order while earlier layers compute, and every layer's output comes back
     # while later layers compute.  Each step still moves all inputs and all outputs.
-    g_e2e = torch.cuda.CUDAGraph()
+    g_e2e = {False: torch.cuda.CUDAGraph(), True: torch.cuda.CUDAGraph()}
     up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    with torch.cuda.graph(g_e2e, stream=stream):
-        start = torch.cuda.Event()
-        start.record(stream)
-        up.wait_event(start)
-        down.wait_event(start)
-        landed, done = [], []
-        with torch.cuda.stream(up):
-            for i in range(L_layers):
-                qs[i].copy_(q_pin[i], non_blocking=True)
-                kns[i].copy_(kn_pin[i], non_blocking=True)
-                vns[i].copy_(vn_pin[i], non_blocking=True)
+    for fl, graph in g_e2e.items():
+        with torch.cuda.graph(graph, stream=stream):
+            start = torch.cuda.Event()
+            start.record(stream)
+            up.wait_event(start)
+            down.wait_event(start)
+            landed, done = [], []
+            with torch.cuda.stream(up):
+                for i in range(L_layers):
+                    qs[i].copy_(q_pin[i], non_blocking=True)
+                    kns[i].copy_(kn_pin[i], non_blocking=True)
+                    vns[i].copy_(vn_pin[i], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(up)
+                    landed.append(ev)
+            for i, c in enumerate(caches):
+                stream.wait_event(landed[i])
+                c.append(kns[i], vns[i])
+                if fl:
+                    c.flush()
+                c.attend(qs[i], outs[i])
                 ev = torch.cuda.Event()
-                ev.record(up)
-                landed.append(ev)
-        for i, c in enumerate(caches):
-            stream.wait_event(landed[i])
-            c.append(kns[i], vns[i])
-            c.flush()
-            c.attend(qs[i], outs[i])
-            ev = torch.cuda.Event()
-            ev.record(stream)
-            done.append(ev)
-        with torch.cuda.stream(down):
-            for i in range(L_layers):
-                down.wait_event(done[i])
-                out_pin[i].copy_(outs[i], non_blocking=True)
-        stream.wait_stream(down)
-        stream.wait_stream(up)
+                ev.record(stream)
+                done.append(ev)
+            with torch.cuda.stream(down):
+                for i in range(L_layers):
+                    down.wait_event(done[i])
+                    out_pin[i].copy_(outs[i], non_blocking=True)
+            stream.wait_stream(down)
+            stream.wait_stream(up)
     h2d_bytes = L_layers * (qh.nbytes + kn.nbytes + vn.nbytes)
     d2h_bytes = L_layers * B * w.Hq * D * 4
 
@@ -390,12 +403,14 @@ def run_gpu(args):
             dist.barrier()
 
     def timed(graph, n, warm, advance):
+        # graph: one graph, or (advance) a dict of the step graphs without / with flush
         for _ in range(warm):
             if advance:
                 host_step(flags)
-            graph.replay()
-            if advance:
+                graph[flushing(flags)].replay()
                 host_commit(flags)
+            else:
+                graph.replay()
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
@@ -404,9 +419,10 @@ def run_gpu(args):
         for _ in range(n):
             if advance:
                 host_step(flags)
-            graph.replay()
-            if advance:
+                graph[flushing(flags)].replay()
                 host_commit(flags)
+            else:
+                graph.replay()
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -429,7 +445,7 @@ def run_gpu(args):
         # main timed region: K decode steps over all layers
         for _ in range(args.warmup):
             host_step(flags)
-            g_step.replay()
+            g_step[flushing(flags)].replay()
             host_commit(flags)
         torch.cuda.synchronize()
         barrier()
@@ -437,9 +453,12 @@ def run_gpu(args):
         clocks.mark_start()
         ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev_a.record(stream)
+        flush_steps = 0
         for _ in range(args.steps):
             host_step(flags)
-            g_step.replay()
+            fl = flushing(flags)
+            flush_steps += fl
+            g_step[fl].replay()
             host_commit(flags)
         ev_b.record(stream)
         torch.cuda.synchronize()
@@ -480,7 +499,9 @@ def run_gpu(args):
                      "per_launch_bytes": bytes_attn, "ms_per_launch": round(attn_ms, 5)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": args.steps * L_layers * 4,  # append, flush, commit, decode per layer
+        # append and decode per layer; flush and commit per layer on steps where windows fill
+        "gpu_launches": args.steps * L_layers * 2 + flush_steps * L_layers * 2,
+        "flush_steps": flush_steps,
         "clocks": clock_info,
     }
     if world == 1 and not args.no_configs:
@@ -502,7 +523,7 @@ def run_gpu(args):
         result["cpu_baseline"] = cpu_baseline(w, Kh, Vh, rk, rv, res_end, qh)
     if world > 1:
         dist.barrier()
-        del g_step, g_attn, g_e2e
+        del g_step, g_attn, g_e2e, graph
         dist.destroy_process_group()
     return result if rank == 0 else None
 

@@ -140,14 +140,17 @@ class PagedKVCache:
                             self.res_len, out, self.workspace, sm_scale, self.err, stream)
 
     def step(self, q, k_new, v_new, out, sm_scale=None, stream=None):
-        """One decode step: append, flush full windows, attend.  The three small launches
-        (append, flush that exits at once unless a window is full, page-table commit) stay
-        out of the decode kernel's way; the single append_flush launch needs 41 KB of shared
-        memory per CTA and, chained before the decode, delays the decode's CTAs more than it
-        saves (measured on B200: 40.1 vs 34.3 us per layer of the 8B-shaped 32-layer step)."""
+        """One decode step: append, flush full windows, attend.  The host tracks every
+        window's length, so the flush (quantize of the full windows and the page-table
+        commit) is launched only on steps where some window fills: once every P steps
+        per sequence.  Append, flush and commit stay separate launches: the single
+        append_flush launch needs 41 KB of shared memory per CTA and, chained before the
+        decode, delays the decode's CTAs more than it saves (measured on B200: 40.1 vs
+        34.3 us per layer of the 8B-shaped 32-layer step)."""
         flushing = self.reserve_flush_pages()
         self.append(k_new, v_new, stream)
-        self.flush(stream)
+        if flushing:
+            self.flush(stream)
         self.attend(q, out, sm_scale, stream)
         self.commit_host(flushing)
 
