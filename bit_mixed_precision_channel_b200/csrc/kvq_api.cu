@@ -360,7 +360,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool, int64_t
 
 size_t kvq_prefill_workspace_bytes(const kvq_config* cfg, int32_t L) {
   if (kvq_check_config(cfg) != KVQ_OK || L < 0) return 0;
-  return (size_t(cfg->num_q_heads) * size_t(L) * sizeof(float) + 255) / 256 * 256;
+  return (2 * size_t(cfg->num_q_heads) * size_t(L) * sizeof(float) + 255) / 256 * 256;
 }
 
 kvq_status kvq_prefill_attention(const kvq_config* cfg, const void* q, const void* k, const void* v, int32_t L,

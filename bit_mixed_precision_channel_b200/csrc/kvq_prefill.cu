@@ -9,18 +9,19 @@
 //                          (tcgen05, accumulators in tensor memory), one CTA per (128
 //                          query rows, query head): the output rows and each row's
 //                          log2-sum-exp;
-//   pass 2 (prefill_score) one CTA per (64 key rows, KV head): recomputes K Q^T for the
-//                          query blocks at or after the key block and the query heads of
-//                          the KV head, turns it into probabilities with the rows'
-//                          log2-sum-exp, and sums them per key — no L x L matrix is kept;
+//   pass 2 (prefill_score_tc) one CTA per (128 key rows, query head), also on tcgen05:
+//                          recomputes K Q^T for the query blocks at or after the key
+//                          block, turns it into probabilities with the rows' log2-sum-exp
+//                          and sums them per key — no L x L matrix is kept; score_heads
+//                          adds the query heads of each KV head;
 //   retain_kernel          per KV head: the last n_recent positions plus the n_heavy
 //                          best-scored others (radix select on the fp32 scores, ties to the
 //                          lower position), ascending;
 //   gather_kernel          the kept tokens of every KV head, compacted token-major, ready
 //                          for the page quantizer.
-// Pass 1 runs on tcgen05 (M = N = 128 products, operands in the cache dtype, fp32
-// accumulators in tensor memory); pass 2 on mma.sync m16n8k16.  fp16 probabilities carry
-// 11 bits, bf16 ones are split into a high and a low bf16 part.
+// Both passes run on tcgen05 (M = N = 128 products, operands in the cache dtype, fp32
+// accumulators in tensor memory).  fp16 probabilities carry 11 bits, bf16 ones are split
+// into a high and a low bf16 part.
 #include <type_traits>
 
 #include "kvq_internal.cuh"
@@ -29,46 +30,9 @@
 namespace kvq {
 namespace pf {
 
-constexpr int kRows = 64;  // query rows (pass 1) or key rows (pass 2) per CTA
-constexpr int kThreads = 128;
-constexpr int kTile = kRows * 256;  // one [64][128] tile of the 16-bit dtype
-
-// Byte offset of 16-byte chunk c (0..15) of row r in a [rows][256 B] tile: the chunk
-// index is XOR-ed with r % 8, so that the eight rows an ldmatrix reads at one chunk
-// column fall into different banks.
-__device__ __forceinline__ uint32_t swz(int r, int c) { return uint32_t(r * 256 + ((c ^ (r & 7)) << 4)); }
-
-// Copies rows [0, valid) of a 64-row tile (row i at src + i * stride elements) into
-// shared memory with cp.async; rows at or past `valid` are zero-filled.
-__device__ __forceinline__ void load_tile(uint8_t* dst, const uint16_t* src, long long stride, int valid, int tid) {
-#pragma unroll
-  for (int i = tid; i < kRows * 16; i += kThreads) {
-    const int r = i >> 4, c = i & 15;
-    const bool ok = r < valid;
-    cp_async16(dst + swz(r, c), src + (ok ? r : 0) * stride + c * 8, ok ? 16u : 0u);
-  }
-}
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// A fragments (row-major 16 x 16) of rows r0 .. r0 + 15 of a tile, k-step ks.
-__device__ __forceinline__ void ld_a(uint32_t (&a)[4], const uint8_t* tile, int r0, int ks, int lane) {
-  const int mi = lane >> 3, r = lane & 7;
-  ldmatrix_x4(a, smem_addr(tile + swz(r0 + ((mi & 1) ? 8 : 0) + r, 2 * ks + (mi >> 1))));
-}
-// B fragments (k = channels, n = tile rows) of n-tiles (n0 .. n0 + 7) and (n0 + 8 .. n0 + 15), k-step ks:
-// b[0], b[1] for the first n-tile, b[2], b[3] for the second.
-__device__ __forceinline__ void ld_b_rows(uint32_t (&b)[4], const uint8_t* tile, int n0, int ks, int lane) {
-  const int mi = lane >> 3, r = lane & 7;
-  ldmatrix_x4(b, smem_addr(tile + swz(n0 + ((mi >> 1) ? 8 : 0) + r, 2 * ks + (mi & 1))));
-}
-// B fragments (k = tile rows, n = channels) of the k-step of rows k0 .. k0 + 15 and the
-// channel n-tiles (c0 .. c0 + 7), (c0 + 8 .. c0 + 15): b[0], b[1] and b[2], b[3].
-__device__ __forceinline__ void ld_b_trans(uint32_t (&b)[4], const uint8_t* tile, int k0, int c0, int lane) {
-  const int mi = lane >> 3, r = lane & 7;
-  ldmatrix_x4_trans(b, smem_addr(tile + swz(k0 + ((mi & 1) ? 8 : 0) + r, (c0 >> 3) + (mi >> 1))));
-}
 
 // Two floats as a pair of the 16-bit type (low half = a).
 __device__ __forceinline__ uint32_t pk(float a, float b, __half) {
@@ -94,6 +58,7 @@ struct PrefillParams {
   float c_log2;       // sm_scale * log2(e)
   float* out;         // [L][Hq][128]
   float* lse;         // [Hq][L]: log2-sum-exp of every row (log2 units)
+  float* part;        // [Hq][L]: cumulative scores per query head (pass 2)
   float* score;       // [Hkv][L]
 };
 
@@ -304,87 +269,130 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_fwd_tc(const __grid_con
   if (warp == 0) tc::dealloc(tmem_base, 256);
 }
 
-// ---------------------------------------------------------------- pass 2
+// ---------------------------------------------------------------- pass 2 (tcgen05)
 
+// Cumulative attention scores on the fifth-generation tensor cores: one CTA per (128 key
+// rows, query head), thread t owns key k0 + t (tensor-memory lane t).  For every query
+// block at or after the key block:
+//   S^T = K Q^T  M = keys, N = queries, K = 128: both tiles from shared memory (K-major),
+//               S^T in tensor memory;
+//   each thread reads its row of S^T and adds 2^(c s - lse[query]) over the queries that
+//   see its key (query >= key, query < L), with lse the row's log2-sum-exp from pass 1.
+// The products of the next query block run while the current block is summed (two S^T
+// buffers of 128 columns, two query tiles).  A CTA writes its head's sums to part[h];
+// score_heads then adds the query heads of each KV head in order, so the scores do not
+// depend on scheduling.  Every wait is bounded; a CTA whose wait gives up writes NaN.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) prefill_score(const __grid_constant__ PrefillParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];  // K tile | 2 x (Q tile, lse[64])
-  pdl_wait();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, qd = lane & 3;
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_score_tc(const __grid_constant__ PrefillParams p) {
+  constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
+  extern __shared__ __align__(128) uint8_t smem[];  // K tile, 2 query tiles, 3 x lse[128]
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tmem_base;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int kb = blockIdx.x;  // the first key blocks see the most query blocks: scheduled first
-  const int kvh = blockIdx.y;
-  const int k0 = kb * kRows;
+  const int h = blockIdx.y, kvh = h / p.gqa;
+  const int k0 = kb * kTcRows, key = k0 + tid;
   const long long qs = (long long)p.Hq * 128, ks_ = (long long)p.Hkv * 128;
-  const int nqb = (p.L + kRows - 1) / kRows;
+  const int n = (p.L + kTcRows - 1) / kTcRows - kb;  // query blocks kb .. nqb - 1
   uint8_t* Kt = smem;
-  float* lse_s = reinterpret_cast<float*>(smem + kTile + 2 * kTile);  // [2][64]
-  load_tile(Kt, p.k + (long long)k0 * ks_ + kvh * 128, ks_, min(kRows, p.L - k0), tid);
-  // work list: (head, query block) for the gqa heads and the query blocks kb .. nqb - 1
-  const int per_head = nqb - kb, total = per_head * p.gqa;
-  auto issue = [&](int it) {
-    const int h = kvh * p.gqa + it / per_head, qb = kb + it % per_head;
-    const int q0 = qb * kRows;
-    uint8_t* Qn = smem + kTile + (it & 1) * kTile;
-    load_tile(Qn, p.q + (long long)q0 * qs + h * 128, qs, min(kRows, p.L - q0), tid);
-    if (tid < kRows) lse_s[(it & 1) * kRows + tid] = q0 + tid < p.L ? p.lse[(long long)h * p.L + q0 + tid] : 0.0f;
+  float* lse_s = reinterpret_cast<float*>(smem + 3 * kTcTile);
+  if (warp == 0) tc::alloc(&tmem_base, 256);
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  pdl_wait();
+  // query block kb + i: its tile into buffer i % 2, its log2-sum-exp into slot i % 3
+  auto load_q = [&](int i) {
+    const int q0 = (kb + i) * kTcRows;
+    load_tile_tc(smem + (1 + (i & 1)) * kTcTile, p.q + (long long)q0 * qs + h * 128, qs, min(kTcRows, p.L - q0), tid,
+                 kTcThreads);
+    lse_s[(i % 3) * kTcRows + tid] = q0 + tid < p.L ? p.lse[(long long)h * p.L + q0 + tid] : 0.0f;
   };
-  issue(0);
+  load_tile_tc(Kt, p.k + (long long)k0 * ks_ + kvh * 128, ks_, min(kTcRows, p.L - k0), tid, kTcThreads);
+  load_q(0);
   cp_commit();
-  uint32_t ka[8][4];
-  float acc[2] = {0.0f, 0.0f};
-  const int r0 = warp * 16;
-  const int key_g = k0 + r0 + g, key_g8 = key_g + 8;
-  for (int it = 0; it < total; ++it) {
-    if (it + 1 < total) {
-      __syncthreads();  // the buffer of it + 1 was read at it - 1
-      issue(it + 1);
-      cp_commit();
-      cp_wait<1>();
-    } else {
+  if (n > 1) load_q(1);
+  cp_commit();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t sK = smem_addr(Kt), sQ = smem_addr(smem + kTcTile);
+  constexpr uint32_t kId = tc::idesc_f16(128, BF, false);
+  auto products = [&](int i) {  // one thread: S^T of query block i into buffer i % 2
+    tc::fence_after();
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      tc::mma_ss(tmem_base + (i & 1) * 128, tc::smem_desc(sK + s * 256, 128, 2048),
+                 tc::smem_desc(sQ + (i & 1) * kTcTile + s * 256, 128, 2048), kId, s > 0 ? 1u : 0u);
+    tc::commit(&bar[i & 1]);
+  };
+  cp_wait<1>();  // the key tile and query block 0 landed
+  tc::fence_async_smem();
+  tc::fence_before();
+  __syncthreads();
+  if (tid == 0) products(0);
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  bool ok = true;
+  for (int i = 0; i < n; ++i) {
+    if (i + 1 < n) {  // the next block's products run while this one is summed
       cp_wait<0>();
+      tc::fence_async_smem();
+      tc::fence_before();
+      __syncthreads();
+      if (tid == 0) products(i + 1);
     }
-    __syncthreads();
-    if (it == 0) {
+    ok = mbar_wait_bounded(&bar[i & 1], uint32_t(i >> 1) & 1u) && ok;
+    tc::fence_after();
+    // the products of block i are done: its query buffer takes block i + 2, which loads
+    // while this block is summed (its log2-sum-exp slot held block i - 1's, which every
+    // thread finished before the barrier that preceded the products of block i + 1)
+    if (i + 2 < n) load_q(i + 2);
+    cp_commit();
+    uint32_t sv[8][16];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) ld_a(ka[ks], Kt, r0, ks, lane);
+    for (int j = 0; j < 8; ++j) tc::ld<16>(tc::lane_addr(tmem_base + (i & 1) * 128, warp, 16 * j), sv[j]);
+    tc::wait_ld();
+    const float* lq = lse_s + (i % 3) * kTcRows;
+    const int q0 = (kb + i) * kTcRows;
+    if (i == 0 || q0 + kTcRows > p.L) {  // the diagonal block, or the last one: masks
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int query = q0 + 16 * j + c;
+          if (query >= key && query < p.L)
+            acc[c & 3] += ex2(__fmaf_rn(__uint_as_float(sv[j][c]), p.c_log2, -lq[16 * j + c]));
+        }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          acc[c & 3] += ex2(__fmaf_rn(__uint_as_float(sv[j][c]), p.c_log2, -lq[16 * j + c]));
     }
-    const uint8_t* Qt = smem + kTile + (it & 1) * kTile;
-    const float* lq = lse_s + (it & 1) * kRows;
-    const int q0 = (kb + it % per_head) * kRows;
-    float s[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) s[i][j] = 0.0f;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t b[4];
-        ld_b_rows(b, Qt, 16 * np, ks, lane);
-        mma_16816(s[2 * np], ka[ks], b[0], b[1], T());
-        mma_16816(s[2 * np + 1], ka[ks], b[2], b[3], T());
-      }
-    // P^T[key][query] = 2^(c s - lse[query]) for query >= key (and query < L)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float2 lv = *reinterpret_cast<const float2*>(lq + 8 * nt + 2 * qd);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int query = q0 + 8 * nt + 2 * qd + (j & 1);
-        const int key = (j >> 1) ? key_g8 : key_g;
-        if (query >= key && query < p.L) acc[j >> 1] += ex2(fmaf(s[nt][j], p.c_log2, -((j & 1) ? lv.y : lv.x)));
-      }
-    }
+    // S^T(i) is overwritten by the products of block i + 2, issued after the barrier at
+    // the top of the next iteration
   }
   pdl_trigger();
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    acc[r] += __shfl_xor_sync(kFull, acc[r], 1);
-    acc[r] += __shfl_xor_sync(kFull, acc[r], 2);
-    const int key = r ? key_g8 : key_g;
-    if (qd == 0 && key < p.L) p.score[(long long)kvh * p.L + key] = acc[r];
+  if (key < p.L)
+    p.part[(long long)h * p.L + key] = ok ? (acc[0] + acc[1]) + (acc[2] + acc[3]) : __int_as_float(0x7fc00000);
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::dealloc(tmem_base, 256);
+}
+
+// score[kvh][j] = sum over the query heads of kvh of part[h][j], in head order.
+__global__ void __launch_bounds__(256) score_heads(const __grid_constant__ PrefillParams p) {
+  pdl_wait();
+  const int j = blockIdx.x * 256 + threadIdx.x, kvh = blockIdx.y;
+  if (j < p.L) {
+    float s = 0.0f;
+    for (int g = 0; g < p.gqa; ++g) s += p.part[(long long)(kvh * p.gqa + g) * p.L + j];
+    p.score[(long long)kvh * p.L + j] = s;
   }
+  pdl_trigger();
 }
 
 // ---------------------------------------------------------------- retention
@@ -510,25 +518,33 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, int L, i
   p.c_log2 = sm_scale * 1.4426950408889634f;
   p.out = out;
   p.lse = lse;
+  p.part = lse + size_t(Hq) * L;
   p.score = score;
-  const int nb = (L + pf::kRows - 1) / pf::kRows;
-  const int nb_tc = (L + pf::kTcRows - 1) / pf::kTcRows;
-  const size_t smem_fwd = 3 * pf::kTcTile, smem_score = 3 * pf::kTile + 2 * pf::kRows * sizeof(float);
+  const int nb = (L + pf::kTcRows - 1) / pf::kTcRows;
+  const size_t smem_fwd = 3 * pf::kTcTile, smem_score = 3 * pf::kTcTile + 3 * pf::kTcRows * sizeof(float);
   static int seen[4][64];
   cudaError_t e;
   if (dtype == KVQ_BF16) {
     if ((e = ensure_dynamic_smem(pf::prefill_fwd_tc<__nv_bfloat16>, int(smem_fwd), seen[0])) != cudaSuccess) return e;
-    if ((e = ensure_dynamic_smem(pf::prefill_score<__nv_bfloat16>, int(smem_score), seen[1])) != cudaSuccess) return e;
-    if ((e = launch_pdl(pf::prefill_fwd_tc<__nv_bfloat16>, dim3(nb_tc, Hq), dim3(pf::kTcThreads), smem_fwd, stream, p)) !=
+    if ((e = ensure_dynamic_smem(pf::prefill_score_tc<__nv_bfloat16>, int(smem_score), seen[1])) != cudaSuccess)
+      return e;
+    if ((e = launch_pdl(pf::prefill_fwd_tc<__nv_bfloat16>, dim3(nb, Hq), dim3(pf::kTcThreads), smem_fwd, stream, p)) !=
         cudaSuccess)
       return e;
-    return launch_pdl(pf::prefill_score<__nv_bfloat16>, dim3(nb, Hkv), dim3(pf::kThreads), smem_score, stream, p);
+    if ((e = launch_pdl(pf::prefill_score_tc<__nv_bfloat16>, dim3(nb, Hq), dim3(pf::kTcThreads), smem_score, stream,
+                        p)) != cudaSuccess)
+      return e;
+  } else {
+    if ((e = ensure_dynamic_smem(pf::prefill_fwd_tc<__half>, int(smem_fwd), seen[2])) != cudaSuccess) return e;
+    if ((e = ensure_dynamic_smem(pf::prefill_score_tc<__half>, int(smem_score), seen[3])) != cudaSuccess) return e;
+    if ((e = launch_pdl(pf::prefill_fwd_tc<__half>, dim3(nb, Hq), dim3(pf::kTcThreads), smem_fwd, stream, p)) !=
+        cudaSuccess)
+      return e;
+    if ((e = launch_pdl(pf::prefill_score_tc<__half>, dim3(nb, Hq), dim3(pf::kTcThreads), smem_score, stream, p)) !=
+        cudaSuccess)
+      return e;
   }
-  if ((e = ensure_dynamic_smem(pf::prefill_fwd_tc<__half>, int(smem_fwd), seen[2])) != cudaSuccess) return e;
-  if ((e = ensure_dynamic_smem(pf::prefill_score<__half>, int(smem_score), seen[3])) != cudaSuccess) return e;
-  if ((e = launch_pdl(pf::prefill_fwd_tc<__half>, dim3(nb_tc, Hq), dim3(pf::kTcThreads), smem_fwd, stream, p)) != cudaSuccess)
-    return e;
-  return launch_pdl(pf::prefill_score<__half>, dim3(nb, Hkv), dim3(pf::kThreads), smem_score, stream, p);
+  return launch_pdl(pf::score_heads, dim3((L + 255) / 256, Hkv), dim3(256), 0, stream, p);
 }
 
 cudaError_t launch_retain(const float* score, int L, int Hkv, int n_heavy, int n_recent, int32_t* keep,

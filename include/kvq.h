@@ -351,7 +351,8 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_config* cfg, const void* pool,
  * j of KV head h is the attention it receives, summed over all query positions and over
  * the query heads of h. */
 
-/* Workspace bytes of kvq_prefill_attention (the log2-sum-exp of every query row). */
+/* Workspace bytes of kvq_prefill_attention: the log2-sum-exp of every query row and the
+ * cumulative scores of every query head (fp32 [num_q_heads][L] each). */
 KVQ_API size_t kvq_prefill_workspace_bytes(const kvq_config* cfg, int32_t L);
 
 /* q: dtype [L][num_q_heads][head_dim]; k, v: dtype [L][num_kv_heads][head_dim];
