@@ -96,6 +96,15 @@ def test_calls_reject_bad_arguments_before_any_launch(lib):
                                     None, None) == 2
 
 
+def test_prefill_workspace_holds_two_values_per_query_row(lib):
+    """The prefill workspace holds each query row's log2-sum-exp and each query head's
+    cumulative scores: 2 * Hq * L fp32, rounded up to 256 bytes; 0 for a bad config."""
+    cfg = kb.Config(num_q_heads=32, num_kv_heads=8, page_tokens=128, num_boost=32)
+    for L in (1, 255, 4096):
+        assert kb.prefill_workspace_bytes(cfg, L) == (2 * 32 * L * 4 + 255) // 256 * 256
+    assert lib.kvq_prefill_workspace_bytes(ctypes.byref(kb.Config(head_dim=64).c()), 16) == 0
+
+
 def test_status_strings(lib):
     for s in range(5):
         assert kb.status_string(s)
