@@ -60,3 +60,25 @@ def test_a_window_never_exceeds_a_page():
     c.host_res_len = [31, 0, 0]
     with pytest.raises(AssertionError):
         c.commit_host([])                 # sequence 0 reached P tokens without a flush
+
+
+def test_step_launches_the_flush_only_when_a_window_fills(monkeypatch):
+    """PagedKVCache.step: append, then the flush only on a step where the host mirror says
+    some window fills, then attention; the host lengths and pages advance either way."""
+    c = _cache(order=[5, 4, 3, 2, 1, 0])
+    calls = []
+    monkeypatch.setattr(kb, "append_token", lambda *a, **k: calls.append("append"))
+    monkeypatch.setattr(kb, "flush_residual", lambda *a, **k: calls.append("flush"))
+    monkeypatch.setattr(kb, "decode_attention", lambda *a, **k: calls.append("attend"))
+    q = torch.zeros(3, 4, 128, dtype=torch.float16)
+    kn = torch.zeros(3, 1, 128, dtype=torch.float16)
+    out = torch.zeros(3, 4, 128)
+    c.host_res_len = [29, 0, 5]
+    c.step(q, kn, kn, out)                 # 29 -> 30: nothing fills
+    assert calls == ["append", "attend"] and c.host_res_len == [30, 1, 6]
+    calls.clear()
+    c.step(q, kn, kn, out)                 # 30 -> 31: still nothing
+    c.step(q, kn, kn, out)                 # 31 -> 32 = P: sequence 0 flushes into page 5
+    assert calls == ["append", "attend", "append", "flush", "attend"]
+    assert c.host_res_len == [0, 3, 8] and c.host_pages == [[5], [], []]
+    assert c.new_page.tolist() == [5, -1, -1]
